@@ -1,0 +1,218 @@
+"""CPU oracle of the MRA-2 forward pass (fp64, plain C, OpenMP over heads).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this package.  The
+product path (``resolution_block_sparse_b200`` and its CUDA library) never
+imports, links or runs it; the two share no code.
+
+Source of the arithmetic: the page "深入解析 Transformers 中的 MRA 模型"
+(blog.gitcode.com), sections "MraConfig：四个专属参数与完整默认值" and
+"源码级原理：MRA 两级注意力到底怎么算" (steps one to four).  The C source
+``mra_oracle.c`` cites the step each function follows.
+
+What pins each function (tests marked ``not gpu``):
+
+* ``num_block``            - the page's worked example (512 tokens, 4 blocks per
+                             row -> 64 of 256), ``tests/golden/num_block.txt``.
+* ``block_counts``/``pool``- closed forms on one-hot and masked inputs.
+* ``lowres_logits``        - closed forms (orthogonal one-hot blocks; a
+                             transposed operand fails).
+* ``row_max``/``selection_keys`` - closed forms for penalties and priors; the
+                             row-argmax invariant.
+* ``select``               - brute-force rank counting on tiny maps; the
+                             priors-present invariant; the tie rule.
+* ``forward`` (hi-res part)- a budget that selects every block equals dense
+                             softmax attention computed by torch's
+                             scaled_dot_product_attention in fp64.
+* ``forward`` (low-res part) - block-constant Q and K make full mode equal
+                             dense attention for any budget; probes with
+                             one-hot V measure the count weighting.
+* padded-query outputs (0), the empty-row output (0), the prior band offsets
+  and the exact bias arithmetic are readings of the page, not fixed by it:
+  **parity unpinned** beyond internal consistency.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mra_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libmra_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+BLOCK = 32
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle's shared library in place (gcc -O2 -fopenmp)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            dp = ctypes.POINTER(ctypes.c_double)
+            ip = ctypes.POINTER(ctypes.c_int32)
+            c_int, c_long = ctypes.c_int, ctypes.c_long
+            lib.mra_oracle_num_block.restype = c_long
+            lib.mra_oracle_num_block.argtypes = [c_long, c_long]
+            lib.mra_oracle_block_counts.restype = None
+            lib.mra_oracle_block_counts.argtypes = [dp, c_int, c_int, dp]
+            lib.mra_oracle_pool.restype = None
+            lib.mra_oracle_pool.argtypes = [dp, dp, c_int, c_int, c_int, c_int, dp]
+            lib.mra_oracle_lowres_logits.restype = None
+            lib.mra_oracle_lowres_logits.argtypes = [dp, dp, c_int, c_int, c_int, dp]
+            lib.mra_oracle_row_max.restype = None
+            lib.mra_oracle_row_max.argtypes = [dp, dp, c_int, c_int, c_int, dp]
+            lib.mra_oracle_selection_keys.restype = None
+            lib.mra_oracle_selection_keys.argtypes = [dp, dp, dp, c_int, c_int, c_int, c_int, c_int, dp]
+            lib.mra_oracle_select.restype = None
+            lib.mra_oracle_select.argtypes = [dp, c_int, c_int, c_long, ip]
+            lib.mra_oracle_forward.restype = c_int
+            lib.mra_oracle_forward.argtypes = [dp, dp, dp, dp] + [c_int] * 8 + [dp, ip, dp, dp, dp, dp, c_int]
+            lib.mra_oracle_attend_with_selection.restype = c_int
+            lib.mra_oracle_attend_with_selection.argtypes = [dp, dp, dp, dp] + [c_int] * 5 + [ip, c_long, dp, c_int]
+            _lib = lib
+    return _lib
+
+
+def _d(a):
+    """Contiguous fp64 numpy view (None stays None) and its pointer."""
+    if a is None:
+        return None, None
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _i32(a):
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def _out(shape, dtype=np.float64):
+    a = np.zeros(shape, dtype=dtype)
+    ct = ctypes.c_double if dtype == np.float64 else ctypes.c_int32
+    return a, a.ctypes.data_as(ctypes.POINTER(ct))
+
+
+def num_block(N: int, block_per_row: int) -> int:
+    return int(_load().mra_oracle_num_block(N, block_per_row))
+
+
+def block_counts(mask, B: int, N: int):
+    m, mp = _d(mask)
+    out, op = _out((B, N // BLOCK))
+    _load().mra_oracle_block_counts(mp, B, N, op)
+    return out
+
+
+def pool(x, mask):
+    """x: [B,H,N,D]; mask: [B,N] or None -> [B*H, nbr, D]."""
+    B, H, N, D = x.shape
+    xa, xp = _d(x)
+    m, mp = _d(mask)
+    out, op = _out((B * H, N // BLOCK, D))
+    _load().mra_oracle_pool(xp, mp, B, H, N, D, op)
+    return out
+
+
+def lowres_logits(qhat, khat):
+    BH, nbr, D = qhat.shape
+    qa, qp = _d(qhat)
+    ka, kp = _d(khat)
+    out, op = _out((BH, nbr, nbr))
+    _load().mra_oracle_lowres_logits(qp, kp, BH, nbr, D, op)
+    return out
+
+
+def row_max(logit, cnt, B: int, H: int):
+    nbr = logit.shape[-1]
+    la, lp = _d(logit)
+    ca, cp = _d(cnt)
+    out, op = _out((B * H, nbr))
+    _load().mra_oracle_row_max(lp, cp, B, H, nbr, op)
+    return out
+
+
+def selection_keys(logit, mlo, cnt, B: int, H: int, first_n: int, diag_n: int):
+    nbr = logit.shape[-1]
+    la, lp = _d(logit)
+    ma, mp = _d(mlo)
+    ca, cp = _d(cnt)
+    out, op = _out((B * H, nbr, nbr))
+    _load().mra_oracle_selection_keys(lp, mp, cp, B, H, nbr, first_n, diag_n, op)
+    return out
+
+
+def select(key, k: int):
+    """key: [BH, nbr, nbr] -> [BH, k] selected flat indices, ascending."""
+    BH, nbr, _ = key.shape
+    ka, kp = _d(key)
+    out, op = _out((BH, k), np.int32)
+    _load().mra_oracle_select(kp, BH, nbr, k, op)
+    return out
+
+
+def forward(q, k, v, mask=None, *, block_per_row: int, approx_mode: int = 0, first_n: int = 0,
+            diag_n: int = 0, nthreads: int = 0, want_intermediates: bool = True):
+    """The whole forward pass in fp64.
+
+    q, k, v: [B,H,N,D] (any float dtype, widened exactly to fp64); mask: [B,N]
+    of 0/1 or None.  approx_mode 0 = full, 1 = sparse.  Returns a dict with
+    ``out`` [B,H,N,D] and, when asked, ``sel`` [BH,k], ``key`` and ``logit``
+    [BH,nbr,nbr], ``pooled`` [3,BH,nbr,D], ``cnt`` [B,nbr].
+    """
+    B, H, N, D = q.shape
+    nbr = N // BLOCK
+    kk = num_block(N, block_per_row) if (N % BLOCK == 0 and N >= BLOCK) else 0
+    qa, qp = _d(q)
+    ka, kp = _d(k)
+    va, vp = _d(v)
+    ma, mp = _d(mask)
+    out, op = _out((B, H, N, D))
+    res = {"out": out, "k": kk}
+    if want_intermediates:
+        sel, sp = _out((B * H, kk), np.int32)
+        key, keyp = _out((B * H, nbr, nbr))
+        logit, lp = _out((B * H, nbr, nbr))
+        pooled, pp = _out((3, B * H, nbr, D))
+        cnt, cp = _out((B, nbr))
+        res.update(sel=sel, key=key, logit=logit, pooled=pooled, cnt=cnt)
+    else:
+        sp = keyp = lp = pp = cp = None
+    rc = _load().mra_oracle_forward(qp, kp, vp, mp, B, H, N, D, block_per_row, approx_mode,
+                                    first_n, diag_n, op, sp, keyp, lp, pp, cp, nthreads)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return res
+
+
+def attend_with_selection(q, k, v, mask, sel, *, approx_mode: int = 0, nthreads: int = 0):
+    """Attention (steps three and four) for a given selected set sel [BH, k]."""
+    B, H, N, D = q.shape
+    qa, qp = _d(q)
+    ka, kp = _d(k)
+    va, vp = _d(v)
+    ma, mp = _d(mask)
+    sa, sp = _i32(sel)
+    out, op = _out((B, H, N, D))
+    rc = _load().mra_oracle_attend_with_selection(qp, kp, vp, mp, B, H, N, D, approx_mode, sp,
+                                                  sa.shape[-1], op, nthreads)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
