@@ -60,35 +60,78 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    c_int, c_long = ctypes.c_int, ctypes.c_long
+    lib.mra_oracle_num_block.restype = c_long
+    lib.mra_oracle_num_block.argtypes = [c_long, c_long]
+    lib.mra_oracle_block_counts.restype = None
+    lib.mra_oracle_block_counts.argtypes = [dp, c_int, c_int, dp]
+    lib.mra_oracle_pool.restype = None
+    lib.mra_oracle_pool.argtypes = [dp, dp, c_int, c_int, c_int, c_int, dp]
+    lib.mra_oracle_lowres_logits.restype = None
+    lib.mra_oracle_lowres_logits.argtypes = [dp, dp, c_int, c_int, c_int, dp]
+    lib.mra_oracle_row_max.restype = None
+    lib.mra_oracle_row_max.argtypes = [dp, dp, c_int, c_int, c_int, dp]
+    lib.mra_oracle_selection_keys.restype = None
+    lib.mra_oracle_selection_keys.argtypes = [dp, dp, dp, c_int, c_int, c_int, c_int, c_int, dp]
+    lib.mra_oracle_select.restype = None
+    lib.mra_oracle_select.argtypes = [dp, c_int, c_int, c_long, ip]
+    lib.mra_oracle_forward.restype = c_int
+    lib.mra_oracle_forward.argtypes = [dp, dp, dp, dp] + [c_int] * 8 + [dp, ip, dp, dp, dp, dp, c_int]
+    lib.mra_oracle_attend_with_selection.restype = c_int
+    lib.mra_oracle_attend_with_selection.argtypes = [dp, dp, dp, dp] + [c_int] * 5 + [ip, c_long, dp, c_int]
+    return lib
+
+
+_active = None      # a library bound by use_variant(), for planted-mistake tests
+
+
 def _load():
     global _lib
+    if _active is not None:
+        return _active
     with _lock:
         if _lib is None:
             build()
-            lib = ctypes.CDLL(_LIB_PATH)
-            dp = ctypes.POINTER(ctypes.c_double)
-            ip = ctypes.POINTER(ctypes.c_int32)
-            c_int, c_long = ctypes.c_int, ctypes.c_long
-            lib.mra_oracle_num_block.restype = c_long
-            lib.mra_oracle_num_block.argtypes = [c_long, c_long]
-            lib.mra_oracle_block_counts.restype = None
-            lib.mra_oracle_block_counts.argtypes = [dp, c_int, c_int, dp]
-            lib.mra_oracle_pool.restype = None
-            lib.mra_oracle_pool.argtypes = [dp, dp, c_int, c_int, c_int, c_int, dp]
-            lib.mra_oracle_lowres_logits.restype = None
-            lib.mra_oracle_lowres_logits.argtypes = [dp, dp, c_int, c_int, c_int, dp]
-            lib.mra_oracle_row_max.restype = None
-            lib.mra_oracle_row_max.argtypes = [dp, dp, c_int, c_int, c_int, dp]
-            lib.mra_oracle_selection_keys.restype = None
-            lib.mra_oracle_selection_keys.argtypes = [dp, dp, dp, c_int, c_int, c_int, c_int, c_int, dp]
-            lib.mra_oracle_select.restype = None
-            lib.mra_oracle_select.argtypes = [dp, c_int, c_int, c_long, ip]
-            lib.mra_oracle_forward.restype = c_int
-            lib.mra_oracle_forward.argtypes = [dp, dp, dp, dp] + [c_int] * 8 + [dp, ip, dp, dp, dp, dp, c_int]
-            lib.mra_oracle_attend_with_selection.restype = c_int
-            lib.mra_oracle_attend_with_selection.argtypes = [dp, dp, dp, dp] + [c_int] * 5 + [ip, c_long, dp, c_int]
-            _lib = lib
+            _lib = _bind(_LIB_PATH)
     return _lib
+
+
+def compile_variant(source_text: str, out_dir: str) -> str:
+    """Compile a modified copy of the oracle source (used only by tests that
+    plant a mistake in the oracle to show that a pin catches it)."""
+    src = os.path.join(out_dir, "mra_oracle_variant.c")
+    lib = os.path.join(out_dir, "libmra_oracle_variant.so")
+    with open(src, "w") as f:
+        f.write(source_text)
+    subprocess.check_call(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c99", "-o", lib, src, "-lm"])
+    return lib
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+class use_variant:
+    """Context manager: route every oracle call through the library at path."""
+
+    def __init__(self, path: str):
+        self.lib = _bind(path)
+
+    def __enter__(self):
+        global _active
+        self.prev = _active
+        _active = self.lib
+        return self
+
+    def __exit__(self, *exc):
+        global _active
+        _active = self.prev
+        return False
 
 
 def _d(a):
