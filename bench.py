@@ -1,0 +1,341 @@
+"""Benchmark of the MRA-2 forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 4] [--impl reference]
+
+One step = one whole forward pass (pool, low-resolution logits and keys,
+top-k selection, CSR build, [low-resolution PV], block-sparse attention and
+combine) over one batch of the seeded synthetic workload, inputs resident in
+HBM.  L2 is flushed (a 256 MiB write) before every timed step; each step is
+timed with CUDA events on the launching stream.  Under torchrun every rank
+runs its own copy of the workload (independent (batch, head) shards: weak
+scaling, no data-path collective); the reported time is the max over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle (the
+reference arm of this build) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from resolution_block_sparse_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MRA-2 attention fwd tokens/s and TFLOP/s (selected blocks) at N=4096; % of roofline"
+L2_FLUSH_BYTES = 256 << 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxs.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sms) if sms else None,
+                "sm_max_mhz": max(maxs) if maxs else None,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def traffic_for(kernel_phase: str, src_file: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel_phase)
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    with open(os.path.join(ROOT, "resolution_block_sparse_b200", "csrc", src_file), "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    if rec.get("source_sha256_16") != h:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def algorithmic(w):
+    """Selected-block FLOPs and compulsory bytes of one step (per workload)."""
+    esz = 2 if w.dtype == "bf16" else 4
+    BH = w.B * w.H
+    flops_hi = BH * w.num_block * 4 * 32 * 32 * w.D
+    qkvo = 4 * BH * w.N * w.D * esz             # Q, K, V read + O write
+    return flops_hi, qkvo
+
+
+def run_cuda(args, w, world, rank, local):
+    import resolution_block_sparse_b200 as mra
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    mra.load_library()
+    inputs = make_inputs(w)
+    q, k, v = (inputs[x].to(dev) for x in ("q", "k", "v"))
+    mask = None if inputs["mask"] is None else inputs["mask"].to(dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fwd = mra.mra_attention_fwd if w.dtype == "bf16" else mra.mra_attention_fwd_f32
+
+    def step():
+        fwd(q, k, v, mask, out, w.block_per_row, w.approx_mode, w.first_n, w.diag_n, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    status = mra.mra_get_device_status()
+    launches_per_step = mra.mra_last_launch_count()
+
+    if world > 1:
+        torch.distributed.barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    mra.mra_profile_enable(True)
+    mra.mra_profile_read()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        stops[i].record(stream)
+    torch.cuda.synchronize()
+    phases = mra.mra_profile_read()
+    mra.mra_profile_enable(False)
+    # same steps again without the per-phase events, for the headline number
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        stops[i].record(stream)
+    torch.cuda.synchronize()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, stops)]
+    if world > 1:
+        torch.distributed.barrier()
+
+    # end to end through the host-buffer entry point (pinned memory)
+    qh, kh, vh = (inputs[x].pin_memory() for x in ("q", "k", "v"))
+    mh = None if inputs["mask"] is None else inputs["mask"].pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    e2e_ms = []
+    for i in range(max(args.warmup, 3) + args.steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        mra.mra_attention_fwd_host(qh, kh, vh, mh, oh, w.block_per_row, w.approx_mode, w.first_n,
+                                   w.diag_n, stream)
+        b.record(stream)
+        b.synchronize()
+        if i >= max(args.warmup, 3):
+            e2e_ms.append(a.elapsed_time(b))
+    clocks = sampler.stop()
+
+    ms = statistics.mean(step_ms)
+    e2e = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([ms, e2e], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e = float(t[0]), float(t[1])
+    return {"ms": ms, "e2e_ms": e2e, "phases": phases, "status": status,
+            "launches_per_step": launches_per_step, "clocks": clocks,
+            "h2d": sum(x.numel() * x.element_size() for x in (qh, kh, vh)) +
+                   (0 if mh is None else mh.numel() * 4),
+            "d2h": oh.numel() * oh.element_size()}
+
+
+def oracle_sample(w, target_s: float = 15.0):
+    """Time the CPU oracle on a bounded sample of the workload: the first S
+    (batch, head) slices, S grown until the run takes a few seconds; return
+    (tokens/s of the whole workload at that rate, sample text, cores)."""
+    import oracle
+
+    inputs = make_inputs(w)
+    cores = os.cpu_count() or 1
+    BH = w.B * w.H
+    S = 1
+    while True:
+        q = inputs["q"].reshape(BH, 1, w.N, w.D)[:S].double().numpy()
+        k = inputs["k"].reshape(BH, 1, w.N, w.D)[:S].double().numpy()
+        v = inputs["v"].reshape(BH, 1, w.N, w.D)[:S].double().numpy()
+        m = None
+        if inputs["mask"] is not None:
+            m = inputs["mask"].repeat_interleave(w.H, dim=0)[:S].double().numpy()
+        t0 = time.perf_counter()
+        oracle.forward(q, k, v, m, block_per_row=w.block_per_row, approx_mode=w.approx_mode,
+                       first_n=w.first_n, diag_n=w.diag_n, nthreads=cores,
+                       want_intermediates=False)
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 4 or S >= BH:
+            break
+        S = min(BH, S * 2)
+    full_s = dt * BH / S
+    tokens = w.B * w.N
+    return tokens / full_s, f"{S} of {BH} (batch, head) slices, fp64, scaled to the full step", cores, dt
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=4)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_env()
+    w = WORKLOADS[args.workload]
+    flops_hi, qkvo = algorithmic(w)
+    tokens = w.B * w.N
+    config = {"workload": w.describe(), "B": w.B, "H": w.H, "N": w.N, "D": w.D,
+              "block_per_row": w.block_per_row, "num_block": w.num_block,
+              "approx_mode": "full" if w.approx_mode == 0 else "sparse",
+              "first_n": w.first_n, "diag_n": w.diag_n,
+              "l2": "flushed before every timed step (256 MiB write)",
+              "parallelism": f"replicas x{world} (independent (batch, head) shards)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps_s = []
+        val, sample, cores, _ = oracle_sample(w, target_s=4.0)
+        for _ in range(max(1, min(args.steps, 3))):
+            v2, _, _, dt = oracle_sample(w, target_s=4.0)
+            steps_s.append(v2)
+        value = statistics.mean(steps_s)
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+                "n_gpus": 1, "steps": len(steps_s), "warmup": 1,
+                "ms_per_step": 1000.0 * tokens / value, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": config,
+                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    res = run_cuda(args, w, world, rank, local)
+    peaks, peak_src = load_peaks()
+
+    ms = res["ms"]
+    value = world * tokens / (ms / 1e3)
+    tflops = world * flops_hi / (ms / 1e3) / 1e12
+    phases = {k: {"launches": n, "avg_us": 1000.0 * t / max(n, 1)} for k, (n, t) in res["phases"].items()}
+    # dominant kernel phase and its roofline
+    dom = max((k for k in phases if k != "memset"), key=lambda k: phases[k]["avg_us"])
+    dom_s = phases[dom]["avg_us"] * 1e-6
+    esz = 2 if w.dtype == "bf16" else 4
+    BH = w.B * w.H
+    kernel_src = {"attention": "mra_attn.cu", "pool": "mra_pool.cu", "lowres_keys": "mra_lowres.cu",
+                  "lowres_pv": "mra_lowres.cu", "select": "mra_select.cu"}
+    if dom == "attention":
+        # compulsory Q, K, V read + O write of the attended heads; intensity
+        # 16*block_per_row flop/B is below the bf16 ridge -> HBM bound
+        bytes_ = qkvo
+        bound, unit, achieved, peak = "hbm", "GB/s", bytes_ / dom_s / 1e9, peaks["hbm_gbs"]
+    elif dom == "pool":
+        ntens = 3 if w.approx_mode == 0 else 2
+        bytes_ = ntens * BH * w.N * w.D * esz + ntens * BH * w.nbr * w.D * 4
+        bound, unit, achieved, peak = "hbm", "GB/s", bytes_ / dom_s / 1e9, peaks["hbm_gbs"]
+    else:
+        bytes_ = 8 * BH * w.nbr * w.nbr * 2
+        bound, unit, achieved, peak = "hbm", "GB/s", bytes_ / dom_s / 1e9, peaks["hbm_gbs"]
+    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "peak_source": f"{peak_src} (burst)",
+                "algorithmic_bytes_per_launch": bytes_,
+                "traffic": traffic_for(dom, kernel_src.get(dom, "mra_attn.cu"))}
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic", "config": config,
+            "tflops_selected_blocks": tflops,
+            "tensor_frac_selected_blocks": tflops / peaks["bf16_tflops"],
+            "roofline": roofline, "phases_us": phases,
+            "e2e": {"value": world * tokens / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+            "gpu_launches": res["launches_per_step"] * args.steps,
+            "device_status": res["status"], "clocks": res["clocks"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, sample, cores, _ = oracle_sample(w)
+        line["cpu_baseline"] = {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,144 @@
+/*
+ * mra.h - C ABI of the B200 (sm_100a) MRA-2 approximate self-attention
+ * forward pass.
+ *
+ * The method is the mra2_attention path described on the page
+ * "深入解析 Transformers 中的 MRA 模型：多分辨率近似自注意力机制的架构、配置与实战"
+ * (blog.gitcode.com), cited here as [MRA page]:
+ *   step one   - 32-token block mean-pooling of Q and K (masked by valid-token
+ *                counts) and the low-resolution block-logit map;
+ *   step two   - global top-num_block selection over that map, with the
+ *                first-n and diagonal priors biased in;
+ *   step three - exact softmax attention on the selected 32x32 blocks only;
+ *   step four  - in "full" mode, the low-resolution correction for every
+ *                unselected block (block-pooled V weighted by low-resolution
+ *                attention), brought to a shared maximum and normaliser.
+ * The knobs block_per_row, approx_mode, initial_prior_first_n_blocks and
+ * initial_prior_diagonal_n_blocks are the four MraConfig parameters of the
+ * page's section "MraConfig：四个专属参数与完整默认值".
+ *
+ * Conventions shared by every entry point
+ *   - Tensors q, k, v, out are contiguous row-major [B][H][N][D] in DEVICE
+ *     memory, 16-byte aligned.  bf16 entry points read and write bfloat16,
+ *     the _f32 entry points float32.
+ *   - key_mask is a DEVICE float array [B][N] of 0/1 shared by all heads of a
+ *     batch entry (1 = valid token), or NULL for "every token valid".  It
+ *     masks keys, values and queries alike; outputs of padded queries are 0.
+ *   - N must be a positive multiple of 32 ([MRA page], paragraph on
+ *     engineering details: the sequence length must divide by the 32-token
+ *     block), N <= 65536; D must be 32 or 64 (callers with a smaller head
+ *     size zero-pad to 32, as the page's self-attention module does).
+ *   - num_block = min((N/32) * block_per_row, (N/32)^2) blocks are selected
+ *     per (batch, head) ([MRA page], num_block formula).
+ *   - approx_mode: MRA_FULL (0) or MRA_SPARSE (1).  0 <= first_n, diag_n <= N/32.
+ *   - Work is enqueued on `stream` and returns without synchronising.  The
+ *     caller owns every pointer; the library owns a per-device workspace that
+ *     it allocates on first use (and grows when a larger problem arrives),
+ *     so the first call of a given size should precede any stream capture.
+ *     Calls that share the workspace are serialised by the library's host
+ *     lock, but kernels of two calls on different streams may overlap on
+ *     the GPU and then race on the workspace: issue them on one stream.
+ *   - Errors are returned synchronously, before any launch, as mra_status
+ *     values; nothing aborts or prints.
+ */
+#ifndef MRA_B200_H
+#define MRA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#ifndef __CUDA_RUNTIME_H__
+struct CUstream_st;
+typedef struct CUstream_st *cudaStream_t;
+#endif
+
+#if defined(__GNUC__)
+#define MRA_API __attribute__((visibility("default")))
+#else
+#define MRA_API
+#endif
+
+typedef enum {
+    MRA_OK = 0,
+    MRA_ERR_INVALID_ARG = 1,     /* a size, mode, prior or pointer is invalid      */
+    MRA_ERR_UNSUPPORTED = 2,     /* D not in {32, 64}, or N above the maximum       */
+    MRA_ERR_CUDA = 3,            /* a CUDA call or launch failed                    */
+    MRA_ERR_ALLOC = 4,           /* workspace allocation failed                     */
+    MRA_ERR_DEVICE_TIMEOUT = 5   /* reserved: a bounded device wait gave up         */
+} mra_status;
+
+enum { MRA_FULL = 0, MRA_SPARSE = 1 };
+enum { MRA_DTYPE_BF16 = 0, MRA_DTYPE_F32 = 1 };
+
+/* Bits of the device status word read by mra_get_device_status. */
+enum {
+    MRA_DEV_KEY_RANGE = 1,   /* some |l - rowmax| >= 2500: the tier order may
+                                differ from exact additive biases              */
+    MRA_DEV_COUNT = 2        /* selected-block count per head differed from k  */
+};
+
+/* Forward pass, bf16 in/out, fp32 accumulation.  Steps one to four of the
+ * [MRA page]; see the conventions above for layout and errors. */
+MRA_API int mra_attention_fwd(const void *q, const void *k, const void *v, const float *key_mask,
+                      void *out, int B, int H, int N, int D, int block_per_row,
+                      int approx_mode, int first_n, int diag_n, cudaStream_t stream);
+
+/* Forward pass, fp32 in/out (no TF32 anywhere on this path). */
+MRA_API int mra_attention_fwd_f32(const float *q, const float *k, const float *v,
+                          const float *key_mask, float *out, int B, int H, int N, int D,
+                          int block_per_row, int approx_mode, int first_n, int diag_n,
+                          cudaStream_t stream);
+
+/* Forward pass that also exports intermediates (each pointer may be NULL):
+ *   sel_idx      int32 [B*H][num_block]  selected flat block indices r*(N/32)+c,
+ *                                        ascending (row-major order)
+ *   lowres_logit float [B*H][N/32][N/32] low-resolution logits qhat.khat/sqrt(D)
+ *   pooled       float [3][B*H][N/32][D] qhat, khat, vhat (vhat only in full mode;
+ *                                        zero in sparse mode)
+ * dtype is MRA_DTYPE_BF16 or MRA_DTYPE_F32; all pointers are device pointers. */
+MRA_API int mra_attention_fwd_ex(const void *q, const void *k, const void *v, const float *key_mask,
+                         void *out, int B, int H, int N, int D, int block_per_row,
+                         int approx_mode, int first_n, int diag_n, int dtype, int32_t *sel_idx,
+                         float *lowres_logit, float *pooled, cudaStream_t stream);
+
+/* End-to-end convenience call on HOST buffers: copies q, k, v (and the mask)
+ * from host memory to a library-owned device staging area on `stream`, runs
+ * the forward pass and copies `out` back, then synchronises `stream`.  Pinned
+ * host memory gives asynchronous copies; pageable memory works but is
+ * slower.  Same arguments as mra_attention_fwd_ex without intermediates. */
+MRA_API int mra_attention_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                           const float *key_mask_host, void *out_host, int B, int H, int N,
+                           int D, int block_per_row, int approx_mode, int first_n, int diag_n,
+                           int dtype, cudaStream_t stream);
+
+/* num_block = min((N/32) * block_per_row, (N/32)^2); 0 for invalid input. */
+MRA_API size_t mra_num_block(int N, int block_per_row);
+
+/* Static text for an mra_status value. */
+MRA_API const char *mra_status_string(int status);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device (a bitwise OR of MRA_DEV_* flags set by kernels since the
+ * previous read), or -MRA_ERR_CUDA on a CUDA error. */
+MRA_API int mra_get_device_status(cudaStream_t stream);
+
+/* Kernel timing for benchmarks.  When enabled, the library records CUDA events
+ * on `stream` around each kernel phase of every call; mra_profile_read
+ * synchronises on the last recorded event and returns, per phase, the number
+ * of launches and the summed milliseconds since the previous read.  Phase
+ * names are static strings.  Returns the number of phases written (<= max). */
+MRA_API void mra_profile_enable(int enable);
+MRA_API int mra_profile_read(const char **names, int *launches, double *total_ms, int max);
+
+/* Number of kernel launches issued by the most recent forward call. */
+MRA_API int mra_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MRA_B200_H */

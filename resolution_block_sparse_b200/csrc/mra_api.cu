@@ -1,0 +1,413 @@
+// mra_api.cu - the C ABI of include/mra.h: argument checks, the per-device
+// workspace, and the stream-ordered launch sequence of the forward pass.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "mra.h"
+#include "mra_internal.cuh"
+
+using namespace mra;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceCtx {
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    unsigned int *status = nullptr;  // persistent status word
+    void *stage = nullptr;           // host-entry staging buffers
+    size_t stage_bytes = 0;
+};
+
+std::mutex g_mutex;
+DeviceCtx g_dev[kMaxDevices];
+int g_last_launches = 0;
+
+// ---------------------------------------------------------------- profiling
+struct PhaseStat {
+    const char *name;
+    int launches;
+    double ms;
+};
+struct PendingEvent {
+    int phase;
+    cudaEvent_t start, stop;
+};
+bool g_prof = false;
+std::vector<PhaseStat> g_phase;
+std::vector<PendingEvent> g_pending;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+int phase_index(const char *name) {
+    for (size_t i = 0; i < g_phase.size(); ++i)
+        if (std::strcmp(g_phase[i].name, name) == 0) return (int)i;
+    g_phase.push_back({name, 0, 0.0});
+    return (int)g_phase.size() - 1;
+}
+
+struct PhaseScope {
+    bool on;
+    PendingEvent pe;
+    cudaStream_t s;
+    PhaseScope(const char *name, cudaStream_t st) : on(g_prof), s(st) {
+        if (!on) return;
+        pe.phase = phase_index(name);
+        pe.start = take_event();
+        pe.stop = take_event();
+        cudaEventRecord(pe.start, s);
+    }
+    ~PhaseScope() {
+        if (!on) return;
+        cudaEventRecord(pe.stop, s);
+        g_pending.push_back(pe);
+    }
+};
+
+// ---------------------------------------------------------------- planning
+size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int validate_sizes(int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n) {
+    if (B < 1 || H < 1 || N < kBlock || (N % kBlock) != 0 || bpr < 1) return MRA_ERR_INVALID_ARG;
+    if (mode != MRA_FULL && mode != MRA_SPARSE) return MRA_ERR_INVALID_ARG;
+    const int nbr = N / kBlock;
+    if (first_n < 0 || first_n > nbr || diag_n < 0 || diag_n > nbr) return MRA_ERR_INVALID_ARG;
+    if (D != 32 && D != 64) return MRA_ERR_UNSUPPORTED;
+    if (N > kMaxN) return MRA_ERR_UNSUPPORTED;
+    const long long BH = (long long)B * H;
+    if (BH > 65535) return MRA_ERR_UNSUPPORTED;
+    const long long kk = std::min<long long>((long long)nbr * bpr, (long long)nbr * nbr);
+    if (BH * kk > 0x7fffffffLL || BH * ((long long)nbr + kk / kChunk) > 0x7fffffffLL)
+        return MRA_ERR_UNSUPPORTED;
+    return MRA_OK;
+}
+
+int validate(const void *q, const void *k, const void *v, const void *out, int B, int H, int N,
+             int D, int bpr, int mode, int first_n, int diag_n) {
+    if (!q || !k || !v || !out) return MRA_ERR_INVALID_ARG;
+    if ((((uintptr_t)q) | ((uintptr_t)k) | ((uintptr_t)v) | ((uintptr_t)out)) & 15u)
+        return MRA_ERR_INVALID_ARG;
+    return validate_sizes(B, H, N, D, bpr, mode, first_n, diag_n);
+}
+
+Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n,
+                     int dtype) {
+    Problem p;
+    p.B = B;
+    p.H = H;
+    p.N = N;
+    p.D = D;
+    p.nbr = N / kBlock;
+    p.BH = B * H;
+    p.nbr2 = (long long)p.nbr * p.nbr;
+    p.k = (int)std::min<long long>((long long)p.nbr * bpr, p.nbr2);
+    p.mode = mode;
+    p.first_n = first_n;
+    p.diag_n = diag_n;
+    p.dtype = dtype;
+    p.cap = p.nbr + p.k / kChunk;
+    p.r_tile = p.nbr >= 2048 ? 8 : (p.nbr >= 1024 ? 16 : 32);
+    p.lowres_ctas = (p.nbr + p.r_tile - 1) / p.r_tile;
+    long long ctas = (p.nbr2 + 8191) / 8192;
+    if (ctas < 1) ctas = 1;
+    if (ctas > 256) ctas = 256;
+    p.radix_ctas = (int)ctas;
+    p.radix_chunk = (p.nbr2 + ctas - 1) / ctas;
+    return p;
+}
+
+// Carves the workspace; with base == nullptr only computes the size.
+size_t carve(const Problem &p, char *base, Workspace *w) {
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> char * {
+        char *ptr = base ? base + off : nullptr;
+        off += align_up(bytes);
+        return ptr;
+    };
+    const size_t BH = (size_t)p.BH, nbr = (size_t)p.nbr, D = (size_t)p.D;
+    Workspace t{};
+    // zeroed region
+    t.hist = (unsigned int *)take(sizeof(unsigned int) * BH * 3 * kHistBins);
+    t.arrive = (unsigned int *)take(sizeof(unsigned int) * BH * 4);
+    t.row_arrive = (int *)take(sizeof(int) * BH * nbr);
+    t.zero_base = t.hist;
+    t.zero_bytes = off;
+    t.cnt = (int *)take(sizeof(int) * (size_t)p.B * nbr);
+    t.pooled = (float *)take(sizeof(float) * 3 * BH * nbr * D);
+    t.keys = (unsigned long long *)take(sizeof(unsigned long long) * BH * (size_t)p.nbr2);
+    t.mlo = (float *)take(sizeof(float) * BH * nbr);
+    t.state = (SelState *)take(sizeof(SelState) * BH);
+    t.gt = (int *)take(sizeof(int) * BH * nbr);
+    t.eq = (int *)take(sizeof(int) * BH * nbr);
+    t.row_start = (int *)take(sizeof(int) * BH * nbr);
+    t.take_eq = (int *)take(sizeof(int) * BH * nbr);
+    t.cols = (int *)take(sizeof(int) * BH * (size_t)p.k);
+    t.words_per_row = (p.nbr + 31) / 32;
+    t.bitmap = (unsigned int *)take(sizeof(unsigned int) * BH * nbr * (size_t)t.words_per_row);
+    t.items = (WorkItem *)take(sizeof(WorkItem) * BH * (size_t)p.cap);
+    t.head_items = (int *)take(sizeof(int) * BH);
+    t.olo = (float *)take(sizeof(float) * BH * nbr * D);
+    t.llo = (float *)take(sizeof(float) * BH * nbr);
+    t.partial = (float *)take(sizeof(float) * BH * (size_t)p.cap * 32 * (D + 2));
+    if (w) *w = t;
+    return off;
+}
+
+int ensure_workspace(int dev, const Problem &p, Workspace *w) {
+    DeviceCtx &ctx = g_dev[dev];
+    if (!ctx.status) {
+        if (cudaMalloc(&ctx.status, 256) != cudaSuccess) return MRA_ERR_ALLOC;
+        if (cudaMemset(ctx.status, 0, 256) != cudaSuccess) return MRA_ERR_CUDA;
+    }
+    const size_t need = carve(p, nullptr, nullptr);
+    if (need > ctx.ws_bytes) {
+        if (ctx.ws) {
+            cudaDeviceSynchronize();
+            cudaFree(ctx.ws);
+            ctx.ws = nullptr;
+            ctx.ws_bytes = 0;
+        }
+        size_t bytes = need + need / 4;
+        if (cudaMalloc(&ctx.ws, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return MRA_ERR_ALLOC;
+        }
+        ctx.ws_bytes = bytes;
+    }
+    carve(p, static_cast<char *>(ctx.ws), w);
+    w->status = ctx.status;
+    return MRA_OK;
+}
+
+int current_device(int *dev) {
+    if (cudaGetDevice(dev) != cudaSuccess) return MRA_ERR_CUDA;
+    if (*dev < 0 || *dev >= kMaxDevices) return MRA_ERR_UNSUPPORTED;
+    return MRA_OK;
+}
+
+#define MRA_TRY(expr)                              \
+    do {                                           \
+        cudaError_t e_ = (expr);                   \
+        if (e_ != cudaSuccess) return MRA_ERR_CUDA; \
+    } while (0)
+
+// The forward pass proper; the caller holds g_mutex.
+int forward_locked(const void *q, const void *k, const void *v, const float *mask, void *out,
+                   int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n,
+                   int dtype, int32_t *sel_out, float *logit_out, float *pooled_out,
+                   cudaStream_t s) {
+    int rc = validate(q, k, v, out, B, H, N, D, bpr, mode, first_n, diag_n);
+    if (rc != MRA_OK) return rc;
+    if (dtype != MRA_DTYPE_BF16 && dtype != MRA_DTYPE_F32) return MRA_ERR_INVALID_ARG;
+    if (mask && (((uintptr_t)mask) & 3u)) return MRA_ERR_INVALID_ARG;
+    int dev;
+    rc = current_device(&dev);
+    if (rc != MRA_OK) return rc;
+    const Problem p = make_problem(B, H, N, D, bpr, mode, first_n, diag_n, dtype);
+    Workspace w;
+    rc = ensure_workspace(dev, p, &w);
+    if (rc != MRA_OK) return rc;
+
+    int launches = 0;
+    {
+        PhaseScope ps("memset", s);
+        MRA_TRY(cudaMemsetAsync(w.zero_base, 0, w.zero_bytes, s));
+    }
+    {
+        PhaseScope ps("pool", s);
+        MRA_TRY(launch_pool(p, w, q, k, v, mask, s));
+        ++launches;
+    }
+    {
+        PhaseScope ps("lowres_keys", s);
+        MRA_TRY(launch_lowres_keys(p, w, logit_out, s));
+        ++launches;
+    }
+    {
+        PhaseScope ps("select", s);
+        MRA_TRY(launch_radix_pass(p, w, 1, s));
+        MRA_TRY(launch_radix_pass(p, w, 2, s));
+        MRA_TRY(launch_row_counts(p, w, s));
+        MRA_TRY(launch_row_scan(p, w, s));
+        MRA_TRY(launch_cols(p, w, sel_out, s));
+        launches += 5;
+    }
+    if (p.mode == MRA_FULL) {
+        PhaseScope ps("lowres_pv", s);
+        MRA_TRY(launch_lowres_pv(p, w, s));
+        ++launches;
+    }
+    {
+        PhaseScope ps("attention", s);
+        MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s));
+        ++launches;
+    }
+    if (pooled_out) {
+        const size_t plane = sizeof(float) * (size_t)p.BH * p.nbr * p.D;
+        MRA_TRY(cudaMemcpyAsync(pooled_out, w.pooled, p.mode == MRA_FULL ? 3 * plane : 2 * plane,
+                                cudaMemcpyDeviceToDevice, s));
+        if (p.mode != MRA_FULL)
+            MRA_TRY(cudaMemsetAsync(reinterpret_cast<char *>(pooled_out) + 2 * plane, 0, plane, s));
+    }
+    g_last_launches = launches;
+    return MRA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mra_attention_fwd(const void *q, const void *k, const void *v, const float *key_mask,
+                      void *out, int B, int H, int N, int D, int block_per_row, int approx_mode,
+                      int first_n, int diag_n, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    return forward_locked(q, k, v, key_mask, out, B, H, N, D, block_per_row, approx_mode, first_n,
+                          diag_n, MRA_DTYPE_BF16, nullptr, nullptr, nullptr, stream);
+}
+
+int mra_attention_fwd_f32(const float *q, const float *k, const float *v, const float *key_mask,
+                          float *out, int B, int H, int N, int D, int block_per_row,
+                          int approx_mode, int first_n, int diag_n, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    return forward_locked(q, k, v, key_mask, out, B, H, N, D, block_per_row, approx_mode, first_n,
+                          diag_n, MRA_DTYPE_F32, nullptr, nullptr, nullptr, stream);
+}
+
+int mra_attention_fwd_ex(const void *q, const void *k, const void *v, const float *key_mask,
+                         void *out, int B, int H, int N, int D, int block_per_row,
+                         int approx_mode, int first_n, int diag_n, int dtype, int32_t *sel_idx,
+                         float *lowres_logit, float *pooled, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    return forward_locked(q, k, v, key_mask, out, B, H, N, D, block_per_row, approx_mode, first_n,
+                          diag_n, dtype, sel_idx, lowres_logit, pooled, stream);
+}
+
+int mra_attention_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                           const float *key_mask_host, void *out_host, int B, int H, int N, int D,
+                           int block_per_row, int approx_mode, int first_n, int diag_n, int dtype,
+                           cudaStream_t stream) {
+    if (!q_host || !k_host || !v_host || !out_host) return MRA_ERR_INVALID_ARG;
+    if (dtype != MRA_DTYPE_BF16 && dtype != MRA_DTYPE_F32) return MRA_ERR_INVALID_ARG;
+    int vrc = validate_sizes(B, H, N, D, block_per_row, approx_mode, first_n, diag_n);
+    if (vrc != MRA_OK) return vrc;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int dev;
+    int rc = current_device(&dev);
+    if (rc != MRA_OK) return rc;
+    const size_t esz = dtype == MRA_DTYPE_BF16 ? 2 : 4;
+    const size_t tensor = align_up(esz * (size_t)B * H * N * D);
+    const size_t mbytes = key_mask_host ? align_up(sizeof(float) * (size_t)B * N) : 0;
+    const size_t need = 4 * tensor + mbytes;
+    DeviceCtx &ctx = g_dev[dev];
+    if (need > ctx.stage_bytes) {
+        if (ctx.stage) {
+            cudaDeviceSynchronize();
+            cudaFree(ctx.stage);
+            ctx.stage = nullptr;
+            ctx.stage_bytes = 0;
+        }
+        if (cudaMalloc(&ctx.stage, need) != cudaSuccess) {
+            cudaGetLastError();
+            return MRA_ERR_ALLOC;
+        }
+        ctx.stage_bytes = need;
+    }
+    char *base = static_cast<char *>(ctx.stage);
+    char *qd = base, *kd = base + tensor, *vd = base + 2 * tensor, *od = base + 3 * tensor;
+    float *md = key_mask_host ? reinterpret_cast<float *>(base + 4 * tensor) : nullptr;
+    const size_t tb = esz * (size_t)B * H * N * D;
+    MRA_TRY(cudaMemcpyAsync(qd, q_host, tb, cudaMemcpyHostToDevice, stream));
+    MRA_TRY(cudaMemcpyAsync(kd, k_host, tb, cudaMemcpyHostToDevice, stream));
+    MRA_TRY(cudaMemcpyAsync(vd, v_host, tb, cudaMemcpyHostToDevice, stream));
+    if (md)
+        MRA_TRY(cudaMemcpyAsync(md, key_mask_host, sizeof(float) * (size_t)B * N,
+                                cudaMemcpyHostToDevice, stream));
+    rc = forward_locked(qd, kd, vd, md, od, B, H, N, D, block_per_row, approx_mode, first_n, diag_n,
+                        dtype, nullptr, nullptr, nullptr, stream);
+    if (rc != MRA_OK) return rc;
+    MRA_TRY(cudaMemcpyAsync(out_host, od, tb, cudaMemcpyDeviceToHost, stream));
+    MRA_TRY(cudaStreamSynchronize(stream));
+    return MRA_OK;
+}
+
+size_t mra_num_block(int N, int block_per_row) {
+    if (N < kBlock || (N % kBlock) != 0 || block_per_row < 1) return 0;
+    const long long nbr = N / kBlock;
+    return (size_t)std::min<long long>(nbr * block_per_row, nbr * nbr);
+}
+
+const char *mra_status_string(int status) {
+    switch (status) {
+        case MRA_OK: return "ok";
+        case MRA_ERR_INVALID_ARG: return "invalid argument";
+        case MRA_ERR_UNSUPPORTED: return "unsupported size or head dimension";
+        case MRA_ERR_CUDA: return "CUDA error";
+        case MRA_ERR_ALLOC: return "workspace allocation failed";
+        case MRA_ERR_DEVICE_TIMEOUT: return "bounded device wait gave up";
+        default: return "unknown status";
+    }
+}
+
+int mra_get_device_status(cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int dev;
+    if (current_device(&dev) != MRA_OK) return -MRA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return -MRA_ERR_CUDA;
+    DeviceCtx &ctx = g_dev[dev];
+    if (!ctx.status) return 0;
+    unsigned int word = 0;
+    if (cudaMemcpy(&word, ctx.status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return -MRA_ERR_CUDA;
+    if (cudaMemset(ctx.status, 0, sizeof(word)) != cudaSuccess) return -MRA_ERR_CUDA;
+    return (int)word;
+}
+
+void mra_profile_enable(int enable) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_prof = enable != 0;
+}
+
+int mra_profile_read(const char **names, int *launches, double *total_ms, int max) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_pending.empty()) cudaEventSynchronize(g_pending.back().stop);
+    for (const PendingEvent &pe : g_pending) {
+        float ms = 0.0f;
+        if (cudaEventElapsedTime(&ms, pe.start, pe.stop) == cudaSuccess) {
+            g_phase[pe.phase].ms += ms;
+            g_phase[pe.phase].launches += 1;
+        }
+        g_event_pool.push_back(pe.start);
+        g_event_pool.push_back(pe.stop);
+    }
+    g_pending.clear();
+    int n = 0;
+    for (PhaseStat &st : g_phase) {
+        if (n >= max) break;
+        if (names) names[n] = st.name;
+        if (launches) launches[n] = st.launches;
+        if (total_ms) total_ms[n] = st.ms;
+        st.launches = 0;
+        st.ms = 0.0;
+        ++n;
+    }
+    return n;
+}
+
+int mra_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

@@ -1,0 +1,515 @@
+// mra_attn.cu - exact softmax attention on the selected 32x32 blocks, merged
+// with the low-resolution part (full mode).
+//
+// Page "深入解析 Transformers 中的 MRA 模型", section "源码级原理":
+//   step three - Q.K^T only on the selected blocks (sampled dense matmul), the
+//                row max for a stable softmax, exp(.) times V, and the row sum
+//                of the weights as normaliser; no dense N x N matrix is formed;
+//   step four  - full mode adds the low-resolution output and normaliser after
+//                bringing both parts to a shared maximum; sparse mode divides
+//                the high-resolution output by its own normaliser.
+//
+// Work item = (batch*head, block row r, up to kChunk selected columns).  The
+// row max and sum are kept online (flash style) over the item's columns.  An
+// item that covers its whole row writes the final output; the items of a longer
+// row write (max, sum, output) partials and the last one to finish (arrival
+// counter, no waiting) merges them.  Padded queries (mask 0) output 0.
+//
+// bf16 kernel: two warps, each owning 16 query rows, mma.sync m16n8k16 with
+// fp32 accumulation; K/V blocks double-buffered in XOR-swizzled shared memory
+// by cp.async.  fp32 kernel: FFMA only (no TF32).
+#include <cuda_bf16.h>
+
+#include "mra_internal.cuh"
+
+namespace mra {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ unsigned smem_u32(const void *p) {
+    return (unsigned)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+__device__ __forceinline__ void ldsm_x4(unsigned &r0, unsigned &r1, unsigned &r2, unsigned &r3,
+                                        unsigned addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(unsigned &r0, unsigned &r1, unsigned &r2, unsigned &r3,
+                                          unsigned addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float *c, const unsigned *a, unsigned b0, unsigned b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ unsigned pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<unsigned *>(&v);
+}
+
+// Element offset of (row, 8-element chunk j) in a swizzled [32][D] bf16 tile:
+// chunk j of a row is stored at position j ^ f(row), which keeps the eight
+// rows read by one ldmatrix phase in distinct 16-byte bank groups.
+template <int D>
+__device__ __forceinline__ int swz(int row, int j) {
+    if constexpr (D == 64) return row * D + ((j ^ (row & 7)) << 3);
+    else return row * D + ((j ^ ((row >> 1) & 3)) << 3);
+}
+
+template <int D, int NT>
+__device__ __forceinline__ void load_tile_async(__nv_bfloat16 *tile, const __nv_bfloat16 *g, int tid) {
+    constexpr int kCpr = D / 8;
+    constexpr int kChunks = 32 * kCpr;
+#pragma unroll
+    for (int e = tid; e < kChunks; e += NT) {
+        const int row = e / kCpr, j = e % kCpr;
+        cp_async16(tile + swz<D>(row, j), g + (size_t)row * D + j * 8);
+    }
+}
+
+template <bool G>
+__device__ __forceinline__ float ldp(const float *p) {
+    if constexpr (G) return __ldcg(p);
+    else return *p;
+}
+
+template <typename T>
+__device__ __forceinline__ T to_out(float x);
+template <>
+__device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+template <>
+__device__ __forceinline__ float to_out<float>(float x) { return x; }
+
+struct MergeSmem {
+    float w[32][33];
+    float M[32], inv[32], beta[32];
+};
+
+// Merge nchunks partials (layout per slot: m[32], l[32], O[32][D]; m in log2
+// units, l and O relative to exp2(m)) with the low-resolution part of the row
+// (full mode) and write the 32 x D output block.
+template <int D, int NT, bool G, typename OutT>
+__device__ void merge_write(const float *src0, size_t slot_stride, int nchunks, int full,
+                            float m_lo2, float l_lo, const float *olo_row, const float *qmask,
+                            OutT *out_blk, MergeSmem &sm) {
+    const int tid = threadIdx.x;
+    if (tid < 32) {
+        const int q = tid;
+        float M = -INFINITY;
+        for (int c = 0; c < nchunks; ++c) {
+            const float *P = src0 + (size_t)c * slot_stride;
+            if (ldp<G>(P + 32 + q) > 0.0f) M = fmaxf(M, ldp<G>(P + q));
+        }
+        const bool lo = full && l_lo > 0.0f;
+        if (lo) M = fmaxf(M, m_lo2);
+        float inv = 0.0f, beta = 0.0f;
+        if (M != -INFINITY && (!qmask || qmask[q] > 0.0f)) {
+            float den = 0.0f;
+            for (int c = 0; c < nchunks; ++c) {
+                const float *P = src0 + (size_t)c * slot_stride;
+                const float l = ldp<G>(P + 32 + q);
+                if (l > 0.0f) den += exp2f(ldp<G>(P + q) - M) * l;
+            }
+            if (lo) {
+                beta = exp2f(m_lo2 - M);
+                den += beta * l_lo;
+            }
+            inv = den > 0.0f ? 1.0f / den : 0.0f;
+        }
+        sm.M[q] = (M == -INFINITY) ? 0.0f : M;
+        sm.inv[q] = inv;
+        sm.beta[q] = beta;
+    }
+    __syncthreads();
+    constexpr int E = 32 * D / NT;
+    float acc[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) acc[i] = 0.0f;
+    for (int cg = 0; cg < nchunks; cg += 32) {
+        const int nc = min(32, nchunks - cg);
+        for (int e = tid; e < nc * 32; e += NT) {
+            const int c = e / 32, q = e % 32;
+            const float *P = src0 + (size_t)(cg + c) * slot_stride;
+            sm.w[c][q] = ldp<G>(P + 32 + q) > 0.0f ? exp2f(ldp<G>(P + q) - sm.M[q]) : 0.0f;
+        }
+        __syncthreads();
+        for (int c = 0; c < nc; ++c) {
+            const float *O = src0 + (size_t)(cg + c) * slot_stride + 64;
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const int e = tid + i * NT;
+                acc[i] = fmaf(sm.w[c][e / D], ldp<G>(O + e), acc[i]);
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int e = tid + i * NT;
+        const int q = e / D, d = e % D;
+        float val = acc[i];
+        if (full) val = fmaf(sm.beta[q], olo_row[d], val);
+        out_blk[e] = to_out<OutT>(val * sm.inv[q]);
+    }
+}
+
+// Shared epilogue: the item's (m, l, O) sit in `stage` (shared, slot layout).
+template <int D, int NT, typename OutT>
+__device__ void finish_item(float *stage, int slot, int chunk, int nchunks, int row, int full,
+                            const float *mlo, const float *olo, const float *llo,
+                            float *partial, int *row_arrive, const float *qmask, OutT *out_blk,
+                            MergeSmem &sm, int *s_last) {
+    const int tid = threadIdx.x;
+    const size_t stride = (size_t)32 * (D + 2);
+    const float m_lo2 = full ? mlo[row] * kLog2e : 0.0f;
+    const float l_lo = full ? llo[row] : 0.0f;
+    const float *olo_row = full ? olo + (size_t)row * D : nullptr;
+    if (nchunks == 1) {
+        merge_write<D, NT, false, OutT>(stage, stride, 1, full, m_lo2, l_lo, olo_row, qmask, out_blk, sm);
+        return;
+    }
+    float *dst = partial + (size_t)slot * stride;
+    for (int e = tid; e < (int)stride; e += NT) dst[e] = stage[e];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) *s_last = (atomicAdd(&row_arrive[row], 1) == nchunks - 1);
+    __syncthreads();
+    if (!*s_last) return;
+    __threadfence();
+    merge_write<D, NT, true, OutT>(partial + (size_t)(slot - chunk) * stride, stride, nchunks, full,
+                                   m_lo2, l_lo, olo_row, qmask, out_blk, sm);
+    if (tid == 0) row_arrive[row] = 0;
+}
+
+struct AttnArgs {
+    const void *q, *k, *v;
+    const float *mask;
+    const WorkItem *items;
+    const int *head_items;
+    const int *cols;
+    int cap, H, N, nbr, full;
+    float scale_log2;
+    const float *mlo, *olo, *llo;
+    float *partial;
+    int *row_arrive;
+    void *out;
+};
+
+constexpr int kBf16Threads = 64;
+
+template <int D>
+__global__ void __launch_bounds__(kBf16Threads)
+attn_bf16_kernel(const AttnArgs a) {
+    constexpr int kTile = 32 * D;
+    __shared__ __align__(128) __nv_bfloat16 sQ[kTile];
+    __shared__ __align__(128) __nv_bfloat16 sKV[2][2][kTile];  // [buffer][K or V]
+    __shared__ float sKm[2][32];                                // key mask per buffer
+    __shared__ MergeSmem sm;
+    __shared__ int s_last;
+
+    const int slot = blockIdx.x;
+    const int bh = slot / a.cap, local = slot % a.cap;
+    if (local >= a.head_items[bh]) return;
+    const WorkItem it = a.items[slot];
+    const int r = it.row % a.nbr;
+    const int chunk = it.chunk_info & 0xffff, nchunks = it.chunk_info >> 16;
+    const int b = bh / a.H;
+    const size_t head_off = (size_t)bh * a.N * D;
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q) + head_off;
+    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k) + head_off;
+    const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(a.v) + head_off;
+    const float *mrow = a.mask ? a.mask + (size_t)b * a.N : nullptr;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, tq = lane & 3;
+
+    load_tile_async<D, kBf16Threads>(sQ, qg + (size_t)r * kTile, tid);
+    const int ncols = it.ncols;
+    if (ncols > 0) {
+        const int c0 = a.cols[it.col_start];
+        load_tile_async<D, kBf16Threads>(sKV[0][0], kg + (size_t)c0 * kTile, tid);
+        load_tile_async<D, kBf16Threads>(sKV[0][1], vg + (size_t)c0 * kTile, tid);
+        if (tid < 32) sKm[0][tid] = mrow ? mrow[c0 * 32 + tid] : 1.0f;
+    }
+    cp_async_commit();
+
+    float o[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;
+    unsigned qf[D / 16][4];
+
+    for (int j = 0; j < ncols; ++j) {
+        const int buf = j & 1;
+        if (j + 1 < ncols) {
+            const int c1 = a.cols[it.col_start + j + 1];
+            load_tile_async<D, kBf16Threads>(sKV[buf ^ 1][0], kg + (size_t)c1 * kTile, tid);
+            load_tile_async<D, kBf16Threads>(sKV[buf ^ 1][1], vg + (size_t)c1 * kTile, tid);
+            if (tid < 32) sKm[buf ^ 1][tid] = mrow ? mrow[c1 * 32 + tid] : 1.0f;
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        if (j == 0) {
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int row = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int ch = 2 * ks + (lane >> 4);
+                ldsm_x4(qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], smem_u32(sQ + swz<D>(row, ch)));
+            }
+        }
+        const __nv_bfloat16 *sK = sKV[buf][0];
+        const __nv_bfloat16 *sV = sKV[buf][1];
+
+        // S = Q K^T for this warp's 16 rows x 32 keys
+        float s[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ks += 2) {
+                const int key = nt * 8 + (lane & 7);
+                const int ch = 2 * ks + (lane >> 3);
+                unsigned b0, b1, b2, b3;
+                ldsm_x4(b0, b1, b2, b3, smem_u32(sK + swz<D>(key, ch)));
+                mma16816(s[nt], qf[ks], b0, b1);
+                mma16816(s[nt], qf[ks + 1], b2, b3);
+            }
+        }
+        // scale to log2 units, mask padded keys, online max / sum
+        float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const int c = nt * 8 + tq * 2;
+            const bool v0 = sKm[buf][c] > 0.0f, v1 = sKm[buf][c + 1] > 0.0f;
+            s[nt][0] = v0 ? s[nt][0] * a.scale_log2 : -INFINITY;
+            s[nt][1] = v1 ? s[nt][1] * a.scale_log2 : -INFINITY;
+            s[nt][2] = v0 ? s[nt][2] * a.scale_log2 : -INFINITY;
+            s[nt][3] = v1 ? s[nt][3] * a.scale_log2 : -INFINITY;
+            mx_a = fmaxf(mx_a, fmaxf(s[nt][0], s[nt][1]));
+            mx_b = fmaxf(mx_b, fmaxf(s[nt][2], s[nt][3]));
+        }
+#pragma unroll
+        for (int off = 1; off < 4; off <<= 1) {
+            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+        }
+        const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+        const float ref_a = (mn_a == -INFINITY) ? 0.0f : mn_a;
+        const float ref_b = (mn_b == -INFINITY) ? 0.0f : mn_b;
+        const float al_a = exp2f(m_a - ref_a), al_b = exp2f(m_b - ref_b);
+        m_a = mn_a;
+        m_b = mn_b;
+        float ps_a = 0.0f, ps_b = 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            s[nt][0] = exp2f(s[nt][0] - ref_a);
+            s[nt][1] = exp2f(s[nt][1] - ref_a);
+            s[nt][2] = exp2f(s[nt][2] - ref_b);
+            s[nt][3] = exp2f(s[nt][3] - ref_b);
+            ps_a += s[nt][0] + s[nt][1];
+            ps_b += s[nt][2] + s[nt][3];
+        }
+        l_a = l_a * al_a + ps_a;
+        l_b = l_b * al_b + ps_b;
+#pragma unroll
+        for (int nd = 0; nd < D / 8; ++nd) {
+            o[nd][0] *= al_a;
+            o[nd][1] *= al_a;
+            o[nd][2] *= al_b;
+            o[nd][3] *= al_b;
+        }
+        // O += P V
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            unsigned pf[4];
+            pf[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
+            pf[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
+            pf[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+            pf[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+#pragma unroll
+            for (int nd2 = 0; nd2 < D / 16; ++nd2) {
+                const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int ch = 2 * nd2 + (lane >> 4);
+                unsigned b0, b1, b2, b3;
+                ldsm_x4_t(b0, b1, b2, b3, smem_u32(sV + swz<D>(key, ch)));
+                mma16816(o[2 * nd2], pf, b0, b1);
+                mma16816(o[2 * nd2 + 1], pf, b2, b3);
+            }
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, off);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, off);
+    }
+    // stage (m, l, O) in shared memory, reusing the K/V buffers
+    __syncthreads();
+    float *stage = reinterpret_cast<float *>(&sKV[0][0][0]);
+    static_assert(sizeof(sKV) >= sizeof(float) * 32 * (D + 2), "stage does not fit");
+    const int ra = warp * 16 + g, rb = ra + 8;
+    if (tq == 0) {
+        stage[ra] = m_a;
+        stage[rb] = m_b;
+        stage[32 + ra] = l_a;
+        stage[32 + rb] = l_b;
+    }
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd) {
+        const int d = nd * 8 + tq * 2;
+        stage[64 + ra * D + d] = o[nd][0];
+        stage[64 + ra * D + d + 1] = o[nd][1];
+        stage[64 + rb * D + d] = o[nd][2];
+        stage[64 + rb * D + d + 1] = o[nd][3];
+    }
+    __syncthreads();
+    __nv_bfloat16 *out_blk = static_cast<__nv_bfloat16 *>(a.out) + head_off + (size_t)r * kTile;
+    finish_item<D, kBf16Threads, __nv_bfloat16>(stage, slot, chunk, nchunks, it.row, a.full, a.mlo,
+                                                a.olo, a.llo, a.partial, a.row_arrive,
+                                                mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
+}
+
+constexpr int kF32Threads = 128;
+
+// fp32: four threads per query row, each owning D/4 output dimensions.
+template <int D>
+__global__ void __launch_bounds__(kF32Threads)
+attn_f32_kernel(const AttnArgs a) {
+    constexpr int kTile = 32 * D;
+    constexpr int kDp = D / 4;
+    __shared__ __align__(16) float sK[kTile];
+    __shared__ __align__(16) float sV[kTile];
+    __shared__ float sKm[32];
+    __shared__ __align__(16) float stage[32 * (D + 2)];
+    __shared__ MergeSmem sm;
+    __shared__ int s_last;
+
+    const int slot = blockIdx.x;
+    const int bh = slot / a.cap, local = slot % a.cap;
+    if (local >= a.head_items[bh]) return;
+    const WorkItem it = a.items[slot];
+    const int r = it.row % a.nbr;
+    const int chunk = it.chunk_info & 0xffff, nchunks = it.chunk_info >> 16;
+    const int b = bh / a.H;
+    const size_t head_off = (size_t)bh * a.N * D;
+    const float *qg = static_cast<const float *>(a.q) + head_off;
+    const float *kg = static_cast<const float *>(a.k) + head_off;
+    const float *vg = static_cast<const float *>(a.v) + head_off;
+    const float *mrow = a.mask ? a.mask + (size_t)b * a.N : nullptr;
+    const int tid = threadIdx.x;
+    const int qrow = tid >> 2, part = tid & 3;
+    const int d0 = part * kDp;
+
+    float qv[kDp], o[kDp];
+#pragma unroll
+    for (int i = 0; i < kDp; ++i) {
+        qv[i] = qg[((size_t)r * 32 + qrow) * D + d0 + i];
+        o[i] = 0.0f;
+    }
+    float m = -INFINITY, l = 0.0f;
+    for (int j = 0; j < it.ncols; ++j) {
+        const int c = a.cols[it.col_start + j];
+        __syncthreads();
+        for (int e = tid; e < kTile / 4; e += kF32Threads) {
+            reinterpret_cast<float4 *>(sK)[e] = reinterpret_cast<const float4 *>(kg + (size_t)c * kTile)[e];
+            reinterpret_cast<float4 *>(sV)[e] = reinterpret_cast<const float4 *>(vg + (size_t)c * kTile)[e];
+        }
+        if (tid < 32) sKm[tid] = mrow ? mrow[c * 32 + tid] : 1.0f;
+        __syncthreads();
+        float sc[32];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int kj = 0; kj < 32; ++kj) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int i = 0; i < kDp; ++i) acc = fmaf(qv[i], sK[kj * D + d0 + i], acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            sc[kj] = sKm[kj] > 0.0f ? acc * a.scale_log2 : -INFINITY;
+            mx = fmaxf(mx, sc[kj]);
+        }
+        const float mn = fmaxf(m, mx);
+        const float ref = (mn == -INFINITY) ? 0.0f : mn;
+        const float al = exp2f(m - ref);
+        m = mn;
+        l *= al;
+#pragma unroll
+        for (int i = 0; i < kDp; ++i) o[i] *= al;
+#pragma unroll
+        for (int kj = 0; kj < 32; ++kj) {
+            const float p = exp2f(sc[kj] - ref);
+            l += p;
+#pragma unroll
+            for (int i = 0; i < kDp; ++i) o[i] = fmaf(p, sV[kj * D + d0 + i], o[i]);
+        }
+    }
+    __syncthreads();
+    if (part == 0) {
+        stage[qrow] = m;
+        stage[32 + qrow] = l;
+    }
+#pragma unroll
+    for (int i = 0; i < kDp; ++i) stage[64 + qrow * D + d0 + i] = o[i];
+    __syncthreads();
+    float *out_blk = static_cast<float *>(a.out) + head_off + (size_t)r * kTile;
+    finish_item<D, kF32Threads, float>(stage, slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
+                                       a.llo, a.partial, a.row_arrive,
+                                       mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
+                             const void *v, const float *mask, void *out, cudaStream_t s) {
+    AttnArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.mask = mask;
+    a.items = w.items;
+    a.head_items = w.head_items;
+    a.cols = w.cols;
+    a.cap = p.cap;
+    a.H = p.H;
+    a.N = p.N;
+    a.nbr = p.nbr;
+    a.full = p.mode == 0 ? 1 : 0;
+    a.scale_log2 = kLog2e / sqrtf((float)p.D);
+    a.mlo = w.mlo;
+    a.olo = w.olo;
+    a.llo = w.llo;
+    a.partial = w.partial;
+    a.row_arrive = w.row_arrive;
+    a.out = out;
+    const long long grid = (long long)p.BH * p.cap;
+    if (p.dtype == 0) {
+        if (p.D == 64) attn_bf16_kernel<64><<<(unsigned)grid, kBf16Threads, 0, s>>>(a);
+        else attn_bf16_kernel<32><<<(unsigned)grid, kBf16Threads, 0, s>>>(a);
+    } else {
+        if (p.D == 64) attn_f32_kernel<64><<<(unsigned)grid, kF32Threads, 0, s>>>(a);
+        else attn_f32_kernel<32><<<(unsigned)grid, kF32Threads, 0, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace mra

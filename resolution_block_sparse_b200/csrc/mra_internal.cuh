@@ -1,0 +1,115 @@
+// mra_internal.cuh - shared declarations of the B200 MRA-2 forward library.
+//
+// The forward pass of the page "深入解析 Transformers 中的 MRA 模型" (steps one
+// to four of "源码级原理：MRA 两级注意力到底怎么算") is split into these phases,
+// all enqueued on the caller's stream:
+//   pool        masked 32-token block means of Q, K (and V in full mode)
+//   lowres      low-resolution logits, row max, 64-bit selection keys, first
+//               radix histogram of the global top-k
+//   select      remaining radix passes, per-row counts, row scan with the
+//               attention work list, CSR column lists
+//   lowres_pv   (full mode) low-resolution weights times pooled V for the
+//               unselected blocks of every block row
+//   attention   exact softmax attention on the selected 32x32 blocks with an
+//               online max/sum, merged with the low-resolution part
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mra {
+
+constexpr int kBlock = 32;            // tokens per block (fixed by the method)
+constexpr int kChunk = 8;             // max selected blocks per attention work item
+constexpr int kHist0Bits = 11;        // radix digit widths over the 35-bit key
+constexpr int kHist1Bits = 12;
+constexpr int kHist2Bits = 12;
+constexpr int kHistBins = 4096;       // per-pass histogram stride per head
+constexpr int kMaxN = 65536;
+
+// Device status bits (mirrors of the public MRA_DEV_* values).
+constexpr unsigned kDevKeyRange = 1u;
+constexpr unsigned kDevCount = 2u;
+
+struct SelState {
+    unsigned long long prefix;  // key bits fixed so far (threshold after the last pass)
+    unsigned int need;          // elements still to take from the current bucket
+    unsigned int pad;
+};
+
+struct WorkItem {
+    int row;         // global block row id: bh * nbr + r
+    int col_start;   // offset into cols[] of the first column of this chunk
+    int ncols;       // number of selected columns in this chunk (0..kChunk)
+    int chunk_info;  // chunk | (nchunks << 16)
+};
+
+struct Problem {
+    int B, H, N, D, nbr, BH;
+    long long nbr2;
+    int k;            // num_block
+    int mode;         // 0 full, 1 sparse
+    int first_n, diag_n;
+    int dtype;        // 0 bf16, 1 f32
+    int cap;          // work-item slots per head: nbr + k / kChunk
+    int r_tile;       // rows per CTA of the low-res kernels
+    int lowres_ctas;  // CTAs per head of the low-res key kernel
+    int radix_ctas;   // CTAs per head of a radix pass
+    long long radix_chunk;  // keys per radix CTA
+};
+
+struct Workspace {
+    // zero-initialised every call (one memset)
+    unsigned int *hist;      // [BH][3][kHistBins]
+    unsigned int *arrive;    // [BH][4]
+    int *row_arrive;         // [BH*nbr]
+    size_t zero_bytes;
+    void *zero_base;
+    // written before read every call
+    int *cnt;                // [B][nbr]
+    float *pooled;           // [3][BH][nbr][D]
+    unsigned long long *keys;// [BH][nbr2]
+    float *mlo;              // [BH][nbr]
+    SelState *state;         // [BH]
+    int *gt, *eq;            // [BH*nbr]
+    int *row_start;          // [BH*nbr]
+    int *take_eq;            // [BH*nbr]
+    int *cols;               // [BH*k]
+    unsigned int *bitmap;    // [BH*nbr][words_per_row]
+    int words_per_row;
+    WorkItem *items;         // [BH*cap]
+    int *head_items;         // [BH]
+    float *olo;              // [BH*nbr][D]
+    float *llo;              // [BH*nbr]
+    float *partial;          // [BH*cap][32*(D+2)]
+    unsigned int *status;    // 1 word, persistent across calls
+};
+
+// Launchers (each returns cudaGetLastError() of its launches).
+cudaError_t launch_pool(const Problem &p, const Workspace &w, const void *q, const void *k,
+                        const void *v, const float *mask, cudaStream_t s);
+cudaError_t launch_lowres_keys(const Problem &p, const Workspace &w, float *logit_out,
+                               cudaStream_t s);
+cudaError_t launch_radix_pass(const Problem &p, const Workspace &w, int pass, cudaStream_t s);
+cudaError_t launch_row_counts(const Problem &p, const Workspace &w, cudaStream_t s);
+cudaError_t launch_row_scan(const Problem &p, const Workspace &w, cudaStream_t s);
+cudaError_t launch_cols(const Problem &p, const Workspace &w, int32_t *sel_out, cudaStream_t s);
+cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t s);
+cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
+                             const void *v, const float *mask, void *out, cudaStream_t s);
+
+// ---------------------------------------------------------------- device helpers
+#ifdef __CUDACC__
+// Order-preserving map of a float to an unsigned integer (larger float ->
+// larger integer); -0 is canonicalised to +0 before the call.
+__device__ __forceinline__ unsigned int float_order_bits(float x) {
+    unsigned int u = __float_as_uint(x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float float_from_order_bits(unsigned int u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+#endif
+
+}  // namespace mra

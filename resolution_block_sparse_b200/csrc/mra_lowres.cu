@@ -1,0 +1,276 @@
+// mra_lowres.cu - low-resolution logits, selection keys, and the
+// low-resolution correction of full mode.
+//
+// Page "深入解析 Transformers 中的 MRA 模型", section "源码级原理":
+//   step one  - a small full matmul of the pooled Q and K gives the block-logit
+//               map; blocks without valid tokens are pushed down in their rows
+//               and columns;
+//   step two  - a global top-k over that map, with a 5e3 bias on the first-n
+//               row/column blocks and on the band around the main diagonal;
+//   step four - in full mode the pooled V, weighted by the low-resolution
+//               attention of the unselected blocks, is added with its own
+//               maximum and normaliser.
+//
+// Selection key.  The top-k ranks, per (batch, head), the value
+//   x + 5e3 * tier,  x = l - rowmax (fp32), tier = #priors - 2*[empty row] - 2*[empty col],
+// which equals the page's additive biases (5e3 per prior, 1e4 per empty side).
+// Instead of adding 5e3 in fp32 (which would quantise x to ~5e-4), the key is
+// the exact lexicographic pair (tier, x) packed into 35 bits:
+//   key = (tier + 4) << 32 | order_bits(x).
+// For |x| < 2500 this order equals the order of the exact sum; a larger |x|
+// raises MRA_DEV_KEY_RANGE in the device status word.
+#include <cuda_bf16.h>
+
+#include "mra_internal.cuh"
+#include "mra_select_common.cuh"
+
+namespace mra {
+
+namespace {
+
+__device__ __forceinline__ int in_band(int r, int c, int g) {
+    if (g <= 0) return 0;
+    const int lo = -(g / 2);
+    const int hi = (g + 1) / 2 - 1;
+    const int off = c - r;
+    return (off >= lo && off <= hi) ? 1 : 0;
+}
+
+constexpr int kLowresThreads = 256;
+constexpr int kColTile = 64;
+
+// One CTA: R block rows of one (batch, head) against every block column.
+template <int D>
+__global__ void __launch_bounds__(kLowresThreads)
+lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ khat,
+                   const int *__restrict__ cnt, int H, int nbr, long long nbr2, int R, float scale,
+                   int first_n, int diag_n, int k, unsigned long long *__restrict__ keys,
+                   float *__restrict__ mlo, float *__restrict__ logit_out,
+                   unsigned int *__restrict__ hist, unsigned int *__restrict__ arrive,
+                   SelState *__restrict__ state, unsigned int *__restrict__ status) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    float *qs = reinterpret_cast<float *>(smem_raw);                 // [R][D]
+    float *ks = qs + R * D;                                           // [kColTile][D+1]
+    float *lt = ks + kColTile * (D + 1);                              // [R][nbr]
+    float *rmax = lt + (size_t)R * nbr;                               // [R]
+    int *cnts = reinterpret_cast<int *>(rmax + R);                    // [nbr]
+    unsigned int *h0 = reinterpret_cast<unsigned int *>(cnts + nbr);  // [2048]
+    __shared__ unsigned int s_tmp[256];
+    __shared__ int s_flag, s_last, s_bin;
+    __shared__ unsigned int s_need;
+
+    const int t = threadIdx.x;
+    const int bh = blockIdx.y;
+    const int b = bh / H;
+    const int r0 = blockIdx.x * R;
+    const float *qh = qhat + (size_t)bh * nbr * D;
+    const float *kh = khat + (size_t)bh * nbr * D;
+
+    if (t == 0) s_flag = 0;
+    for (int c = t; c < nbr; c += kLowresThreads) cnts[c] = cnt[(size_t)b * nbr + c];
+    for (int i = t; i < (1 << kHist0Bits); i += kLowresThreads) h0[i] = 0u;
+    for (int i = t; i < R * D; i += kLowresThreads) {
+        const int r = i / D;
+        qs[i] = (r0 + r < nbr) ? qh[(size_t)(r0 + r) * D + (i % D)] : 0.0f;
+    }
+
+    constexpr int kRowGroups = kLowresThreads / kColTile;  // 4
+    const int cl = t % kColTile;
+    const int rg = t / kColTile;
+    for (int ct = 0; ct < nbr; ct += kColTile) {
+        __syncthreads();
+        for (int i = t; i < kColTile * D; i += kLowresThreads) {
+            const int c = i / D, d = i % D;
+            ks[c * (D + 1) + d] = (ct + c < nbr) ? kh[(size_t)(ct + c) * D + d] : 0.0f;
+        }
+        __syncthreads();
+        const float *kr = ks + cl * (D + 1);
+        for (int r = rg; r < R; r += kRowGroups) {
+            const float *qr = qs + r * D;
+            float acc = 0.0f;
+#pragma unroll 16
+            for (int d = 0; d < D; ++d) acc = fmaf(qr[d], kr[d], acc);
+            if (ct + cl < nbr) lt[(size_t)r * nbr + ct + cl] = acc * scale;
+        }
+    }
+    __syncthreads();
+
+    // row max over valid columns (0 when the row has none)
+    const int warp = t >> 5, lane = t & 31;
+    for (int r = warp; r < R; r += kLowresThreads / 32) {
+        float m = -INFINITY;
+        for (int c = lane; c < nbr; c += 32)
+            if (cnts[c] > 0) m = fmaxf(m, lt[(size_t)r * nbr + c]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (m == -INFINITY) m = 0.0f;
+        if (lane == 0) {
+            rmax[r] = m;
+            if (r0 + r < nbr) mlo[(size_t)bh * nbr + r0 + r] = m;
+        }
+    }
+    __syncthreads();
+
+    // keys, exported logits, first radix histogram (bits 24..34)
+    const int rows_here = min(R, nbr - r0);
+    const long long n_here = (long long)rows_here * nbr;
+    unsigned long long *kout = keys + (size_t)bh * nbr2 + (size_t)r0 * nbr;
+    int flag = 0;
+    for (long long e = t; e < n_here; e += kLowresThreads) {
+        const int r = (int)(e / nbr), c = (int)(e % nbr);
+        const int gr = r0 + r;
+        const float l = lt[(size_t)r * nbr + c];
+        float x = l - rmax[r];
+        if (x == 0.0f) x = 0.0f;  // canonical +0
+        if (!(fabsf(x) < 2500.0f)) flag = 1;
+        int tier = 0;
+        if (first_n > 0 && (gr < first_n || c < first_n)) ++tier;
+        tier += in_band(gr, c, diag_n);
+        if (cnts[gr] <= 0) tier -= 2;
+        if (cnts[c] <= 0) tier -= 2;
+        const unsigned long long key =
+            ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
+        kout[e] = key;
+        if (logit_out) logit_out[(size_t)bh * nbr2 + (size_t)gr * nbr + c] = l;
+        atomicAdd(&h0[(unsigned)(key >> 24)], 1u);
+    }
+    if (flag) s_flag = 1;
+    __syncthreads();
+    if (t == 0 && s_flag) atomicOr(status, kDevKeyRange);
+    unsigned int *gh = hist + (size_t)bh * 3 * kHistBins;
+    for (int i = t; i < (1 << kHist0Bits); i += kLowresThreads)
+        if (h0[i]) atomicAdd(&gh[i], h0[i]);
+
+    // the last CTA of this head locates the bucket of the k-th key
+    __threadfence();
+    __syncthreads();
+    if (t == 0) s_last = (atomicAdd(&arrive[(size_t)bh * 4 + 0], 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    find_bucket_256(gh, 1 << kHist0Bits, (unsigned)k, s_tmp, &s_bin, &s_need);
+    if (t == 0) {
+        SelState st;
+        st.prefix = (unsigned long long)s_bin << (kHist1Bits + kHist2Bits);
+        st.need = s_need;
+        st.pad = 0;
+        state[bh] = st;
+    }
+}
+
+// Low-resolution part of full mode for R block rows of one (batch, head):
+//   w_rc = cnt_c * exp(l_rc - rowmax_r) for every unselected c with cnt_c > 0,
+//   olo_r = sum_c w_rc * vhat_c,   llo_r = sum_c w_rc.
+template <int D>
+__global__ void __launch_bounds__(kLowresThreads)
+lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int *__restrict__ bitmap,
+                 int wpr, const int *__restrict__ cnt, const float *__restrict__ vhat, int H,
+                 int nbr, long long nbr2, float *__restrict__ olo, float *__restrict__ llo) {
+    constexpr int R = 32;
+    constexpr int kCt = 32;
+    __shared__ float vs[kCt][D];
+    __shared__ float ws[R][kCt + 1];
+    __shared__ int cc[kCt];
+    const int t = threadIdx.x;
+    const int bh = blockIdx.y;
+    const int b = bh / H;
+    const int r0 = blockIdx.x * R;
+    const float *vh = vhat + (size_t)bh * nbr * D;
+    constexpr int kStride = kLowresThreads / D;   // rows per thread step
+    constexpr int kPer = R / kStride;             // rows per thread
+    const int d = t % D;
+    const int rb = t / D;
+    float acc[kPer], lsum[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = lsum[i] = 0.0f;
+
+    for (int ct = 0; ct < nbr; ct += kCt) {
+        __syncthreads();
+        for (int i = t; i < kCt * D; i += kLowresThreads) {
+            const int c = i / D;
+            vs[c][i % D] = (ct + c < nbr) ? vh[(size_t)(ct + c) * D + (i % D)] : 0.0f;
+        }
+        if (t < kCt) cc[t] = (ct + t < nbr) ? cnt[(size_t)b * nbr + ct + t] : 0;
+        __syncthreads();
+        for (int e = t; e < R * kCt; e += kLowresThreads) {
+            const int r = e / kCt, c = e % kCt;
+            const int gr = r0 + r, gc = ct + c;
+            float wv = 0.0f;
+            if (gr < nbr && gc < nbr && cc[c] > 0) {
+                const unsigned int word = bitmap[((size_t)bh * nbr + gr) * wpr + (gc >> 5)];
+                if (!((word >> (gc & 31)) & 1u)) {
+                    const unsigned long long key = keys[(size_t)bh * nbr2 + (size_t)gr * nbr + gc];
+                    const float x = float_from_order_bits((unsigned int)(key & 0xffffffffull));
+                    wv = (float)cc[c] * expf(x);
+                }
+            }
+            ws[r][c] = wv;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int r = rb + i * kStride;
+#pragma unroll 8
+            for (int c = 0; c < kCt; ++c) {
+                const float wv = ws[r][c];
+                acc[i] = fmaf(wv, vs[c][d], acc[i]);
+                lsum[i] += wv;
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int gr = r0 + rb + i * kStride;
+        if (gr < nbr) {
+            olo[((size_t)bh * nbr + gr) * D + d] = acc[i];
+            if (d == 0) llo[(size_t)bh * nbr + gr] = lsum[i];
+        }
+    }
+}
+
+template <int D>
+size_t lowres_smem_bytes(int R, int nbr) {
+    return sizeof(float) * ((size_t)R * D + (size_t)kColTile * (D + 1) + (size_t)R * nbr + R) +
+           sizeof(int) * (size_t)nbr + sizeof(unsigned int) * (1u << kHist0Bits);
+}
+
+template <int D>
+cudaError_t launch_keys_typed(const Problem &p, const Workspace &w, float *logit_out,
+                              cudaStream_t s) {
+    const size_t smem = lowres_smem_bytes<D>(p.r_tile, p.nbr);
+    cudaError_t e = cudaFuncSetAttribute(lowres_keys_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.lowres_ctas, p.BH);
+    const float scale = 1.0f / sqrtf((float)p.D);
+    const float *qhat = w.pooled;
+    const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;
+    lowres_keys_kernel<D><<<grid, kLowresThreads, smem, s>>>(
+        qhat, khat, w.cnt, p.H, p.nbr, p.nbr2, p.r_tile, scale, p.first_n, p.diag_n, p.k, w.keys,
+        w.mlo, logit_out, w.hist, w.arrive, w.state, w.status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_lowres_keys(const Problem &p, const Workspace &w, float *logit_out,
+                               cudaStream_t s) {
+    return p.D == 64 ? launch_keys_typed<64>(p, w, logit_out, s)
+                     : launch_keys_typed<32>(p, w, logit_out, s);
+}
+
+cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t s) {
+    dim3 grid((p.nbr + 31) / 32, p.BH);
+    const float *vhat = w.pooled + (size_t)2 * p.BH * p.nbr * p.D;
+    if (p.D == 64)
+        lowres_pv_kernel<64><<<grid, kLowresThreads, 0, s>>>(w.keys, w.bitmap, w.words_per_row,
+                                                             w.cnt, vhat, p.H, p.nbr, p.nbr2,
+                                                             w.olo, w.llo);
+    else
+        lowres_pv_kernel<32><<<grid, kLowresThreads, 0, s>>>(w.keys, w.bitmap, w.words_per_row,
+                                                             w.cnt, vhat, p.H, p.nbr, p.nbr2,
+                                                             w.olo, w.llo);
+    return cudaGetLastError();
+}
+
+}  // namespace mra

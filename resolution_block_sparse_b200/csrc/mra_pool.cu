@@ -1,0 +1,142 @@
+// mra_pool.cu - masked 32-token block means of Q, K and V.
+//
+// Page "深入解析 Transformers 中的 MRA 模型", section "源码级原理", step one: the
+// sequence is cut into 32-token blocks and each block is replaced by the mean
+// of its valid tokens (count-weighted when a mask is given), giving the
+// low-resolution Q and K (and, in full mode, the block-pooled V of step four).
+//
+// One warp per (tensor, head, block).  A block of 32 rows is one contiguous
+// 32*D-element span, so the warp streams it with 16-byte loads, every lane
+// holding one 16-byte column slice of several rows; partial sums are folded
+// across the lanes that share a slice.  HBM-bound: the algorithmic traffic is
+// the bytes of Q, K (, V) read plus 4*D bytes written per block and tensor.
+#include <cuda_bf16.h>
+
+#include "mra_internal.cuh"
+
+namespace mra {
+namespace {
+
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+    static constexpr int kElems = 8;
+    __device__ __forceinline__ static void to_float(const uint4 &r, float *f) {
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 t = __bfloat1622float2(h[i]);
+            f[2 * i] = t.x;
+            f[2 * i + 1] = t.y;
+        }
+    }
+};
+template <>
+struct Vec16<float> {
+    static constexpr int kElems = 4;
+    __device__ __forceinline__ static void to_float(const uint4 &r, float *f) {
+        f[0] = __uint_as_float(r.x);
+        f[1] = __uint_as_float(r.y);
+        f[2] = __uint_as_float(r.z);
+        f[3] = __uint_as_float(r.w);
+    }
+};
+
+constexpr int kPoolWarps = 4;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kPoolWarps * 32)
+pool_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+            const float *__restrict__ mask, int H, int N, int nbr, int BH, int ntensors,
+            float *__restrict__ pooled, int *__restrict__ cnt_out) {
+    constexpr int kEpc = Vec16<T>::kElems;          // elements per 16-byte slice
+    constexpr int kCpr = D / kEpc;                  // slices per row
+    constexpr int kRpp = 32 / kCpr;                 // rows per warp pass
+    constexpr int kPasses = kBlock / kRpp;
+    static_assert(kCpr >= 1 && kCpr <= 32 && 32 % kCpr == 0, "unsupported D");
+
+    const int lane = threadIdx.x & 31;
+    const long long gw = (long long)blockIdx.x * kPoolWarps + (threadIdx.x >> 5);
+    const long long total = (long long)ntensors * BH * nbr;
+    if (gw >= total) return;
+    const int blk = (int)(gw % nbr);
+    const int bh = (int)((gw / nbr) % BH);
+    const int t = (int)(gw / ((long long)nbr * BH));
+    const int b = bh / H;
+    const T *x = (t == 0) ? q : (t == 1 ? k : v);
+    const T *base = x + ((size_t)bh * N + (size_t)blk * kBlock) * D;
+    const float *mrow = mask ? mask + (size_t)b * N + (size_t)blk * kBlock : nullptr;
+
+    // valid-token count of the block
+    float mine = mrow ? mrow[lane] : 1.0f;
+    float c = mine;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+
+    const int slice = lane % kCpr;
+    const int row0 = lane / kCpr;
+    uint4 raw[kPasses];
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+        const int row = p * kRpp + row0;
+        raw[p] = __ldg(reinterpret_cast<const uint4 *>(base + (size_t)row * D) + slice);
+    }
+    float acc[kEpc];
+#pragma unroll
+    for (int e = 0; e < kEpc; ++e) acc[e] = 0.0f;
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+        const int row = p * kRpp + row0;
+        const float m = mrow ? __shfl_sync(0xffffffffu, mine, row) : 1.0f;
+        float f[kEpc];
+        Vec16<T>::to_float(raw[p], f);
+#pragma unroll
+        for (int e = 0; e < kEpc; ++e) acc[e] = fmaf(m, f[e], acc[e]);
+    }
+    // fold the lanes that hold the same slice
+#pragma unroll
+    for (int o = kCpr; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < kEpc; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+
+    if (lane < kCpr) {
+        float *dst = pooled + (size_t)t * BH * nbr * D + ((size_t)bh * nbr + blk) * D + lane * kEpc;
+#pragma unroll
+        for (int e = 0; e < kEpc; e += 4) {
+            float4 o4;
+            o4.x = c > 0.0f ? acc[e + 0] / c : 0.0f;
+            o4.y = c > 0.0f ? acc[e + 1] / c : 0.0f;
+            o4.z = c > 0.0f ? acc[e + 2] / c : 0.0f;
+            o4.w = c > 0.0f ? acc[e + 3] / c : 0.0f;
+            *reinterpret_cast<float4 *>(dst + e) = o4;
+        }
+    }
+    if (t == 0 && (bh % H) == 0 && lane == 0) cnt_out[(size_t)b * nbr + blk] = (int)c;
+}
+
+template <typename T, int D>
+cudaError_t launch_typed(const Problem &p, const Workspace &w, const void *q, const void *k,
+                         const void *v, const float *mask, cudaStream_t s) {
+    const int ntensors = (p.mode == 0) ? 3 : 2;
+    const long long warps = (long long)ntensors * p.BH * p.nbr;
+    const long long grid = (warps + kPoolWarps - 1) / kPoolWarps;
+    pool_kernel<T, D><<<(unsigned)grid, kPoolWarps * 32, 0, s>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), mask,
+        p.H, p.N, p.nbr, p.BH, ntensors, w.pooled, w.cnt);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Problem &p, const Workspace &w, const void *q, const void *k,
+                        const void *v, const float *mask, cudaStream_t s) {
+    if (p.dtype == 0) {
+        return p.D == 64 ? launch_typed<__nv_bfloat16, 64>(p, w, q, k, v, mask, s)
+                         : launch_typed<__nv_bfloat16, 32>(p, w, q, k, v, mask, s);
+    }
+    return p.D == 64 ? launch_typed<float, 64>(p, w, q, k, v, mask, s)
+                     : launch_typed<float, 32>(p, w, q, k, v, mask, s);
+}
+
+}  // namespace mra

@@ -1,0 +1,261 @@
+// mra_select.cu - global top-num_block selection and the CSR / work-list build.
+//
+// Page "深入解析 Transformers 中的 MRA 模型", section "源码级原理", step two: a
+// global top-k over each (batch, head)'s low-resolution map, k = num_block,
+// returning the selected block coordinates.  Equal keys go to the smaller flat
+// index r*nbr + c.
+//
+// Radix select over the 35-bit keys: the first 11-bit digit is histogrammed by
+// the low-resolution kernel, two 12-bit digits here.  After each pass the last
+// CTA of a head (threadfence + arrival counter, no waiting) locates the bucket
+// of the k-th key; after the third pass the threshold key T is exact and
+// `need` says how many keys equal to T are taken (the smallest indices).
+// Then, per block row, counts of keys above / equal to T, a per-head scan that
+// assigns CSR offsets and attention work items (chunks of at most kChunk
+// columns), and the column lists in ascending column order.
+#include "mra_internal.cuh"
+#include "mra_select_common.cuh"
+
+namespace mra {
+namespace {
+
+constexpr int kThreads = 256;
+
+__global__ void __launch_bounds__(kThreads)
+radix_pass_kernel(const unsigned long long *__restrict__ keys, long long nbr2, long long chunk,
+                  int pass, int shift, int bits, unsigned int *__restrict__ hist,
+                  unsigned int *__restrict__ arrive, SelState *__restrict__ state) {
+    __shared__ unsigned int h[kHistBins];
+    __shared__ unsigned int s_tmp[256];
+    __shared__ int s_last, s_bin;
+    __shared__ unsigned int s_need;
+    const int t = threadIdx.x;
+    const int bh = blockIdx.y;
+    const SelState st = state[bh];
+    const int hi = shift + bits;
+    const unsigned long long want = st.prefix >> hi;
+    const unsigned int dmask = (1u << bits) - 1u;
+    for (int i = t; i < (1 << bits); i += kThreads) h[i] = 0u;
+    __syncthreads();
+    const long long start = (long long)blockIdx.x * chunk;
+    const long long end = min(start + chunk, nbr2);
+    const unsigned long long *kb = keys + (size_t)bh * nbr2;
+    for (long long i = start + t; i < end; i += kThreads) {
+        const unsigned long long key = kb[i];
+        if ((key >> hi) == want) atomicAdd(&h[(unsigned)(key >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    unsigned int *gh = hist + ((size_t)bh * 3 + pass) * kHistBins;
+    for (int i = t; i < (1 << bits); i += kThreads)
+        if (h[i]) atomicAdd(&gh[i], h[i]);
+    __threadfence();
+    __syncthreads();
+    if (t == 0) s_last = (atomicAdd(&arrive[(size_t)bh * 4 + pass], 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    find_bucket_256(gh, 1 << bits, st.need, s_tmp, &s_bin, &s_need);
+    if (t == 0) {
+        SelState ns;
+        ns.prefix = st.prefix | ((unsigned long long)s_bin << shift);
+        ns.need = s_need;
+        ns.pad = 0;
+        state[bh] = ns;
+    }
+}
+
+// One warp per block row: number of keys above and equal to the threshold.
+__global__ void __launch_bounds__(kThreads)
+row_counts_kernel(const unsigned long long *__restrict__ keys, const SelState *__restrict__ state,
+                  int nbr, long long nbr2, int rows, int *__restrict__ gt, int *__restrict__ eq) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const int bh = row / nbr, r = row % nbr;
+    const unsigned long long T = state[bh].prefix;
+    const unsigned long long *kr = keys + (size_t)bh * nbr2 + (size_t)r * nbr;
+    int g = 0, e = 0;
+    for (int c = lane; c < nbr; c += 32) {
+        const unsigned long long key = kr[c];
+        g += key > T;
+        e += key == T;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        g += __shfl_xor_sync(0xffffffffu, g, o);
+        e += __shfl_xor_sync(0xffffffffu, e, o);
+    }
+    if (lane == 0) {
+        gt[row] = g;
+        eq[row] = e;
+    }
+}
+
+constexpr int kScanThreads = 1024;
+
+// Exclusive scan of one int per thread over the block; returns the prefix and
+// writes the block total to *total.
+__device__ int block_exclusive_scan(int v, int *s_warp, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = (lane < kScanThreads / 32) ? s_warp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        s_warp[lane] = w;  // inclusive prefix of warp totals
+    }
+    __syncthreads();
+    const int before = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
+    *total = s_warp[kScanThreads / 32 - 1];
+    __syncthreads();
+    return before;
+}
+
+// One CTA per (batch, head): CSR row offsets and the attention work list.
+__global__ void __launch_bounds__(kScanThreads)
+row_scan_kernel(const int *__restrict__ gt, const int *__restrict__ eq,
+                const SelState *__restrict__ state, int nbr, int k, int cap,
+                int *__restrict__ row_start, int *__restrict__ take_eq, WorkItem *__restrict__ items,
+                int *__restrict__ head_items, unsigned int *__restrict__ status) {
+    __shared__ int s_warp[32];
+    const int bh = blockIdx.x;
+    const int t = threadIdx.x;
+    const int per = (nbr + kScanThreads - 1) / kScanThreads;   // rows per thread (<= 2)
+    const int rbeg = min(t * per, nbr), rend = min(rbeg + per, nbr);
+    const int base = bh * nbr;
+    const unsigned int need = state[bh].need;
+
+    int eq_local = 0;
+    for (int r = rbeg; r < rend; ++r) eq_local += eq[base + r];
+    int tot;
+    int eq_before = block_exclusive_scan(eq_local, s_warp, &tot);
+
+    int sel[2] = {0, 0}, tk[2] = {0, 0};
+    int sel_local = 0;
+    for (int r = rbeg, i = 0; r < rend; ++r, ++i) {
+        const int e = eq[base + r];
+        int take = (int)need - eq_before;
+        take = take < 0 ? 0 : (take > e ? e : take);
+        tk[i] = take;
+        sel[i] = gt[base + r] + take;
+        sel_local += sel[i];
+        eq_before += e;
+    }
+    int sel_total;
+    int sel_before = block_exclusive_scan(sel_local, s_warp, &sel_total);
+    int it_local = 0;
+    for (int r = rbeg, i = 0; r < rend; ++r, ++i) it_local += sel[i] > 0 ? (sel[i] + kChunk - 1) / kChunk : 1;
+    int it_total;
+    int it_before = block_exclusive_scan(it_local, s_warp, &it_total);
+
+    for (int r = rbeg, i = 0; r < rend; ++r, ++i) {
+        const int rs = bh * k + sel_before;
+        row_start[base + r] = rs;
+        take_eq[base + r] = tk[i];
+        const int n = sel[i] > 0 ? (sel[i] + kChunk - 1) / kChunk : 1;
+        for (int j = 0; j < n && it_before + j < cap; ++j) {
+            WorkItem w;
+            w.row = base + r;
+            w.col_start = rs + j * kChunk;
+            w.ncols = min(kChunk, sel[i] - j * kChunk);
+            if (w.ncols < 0) w.ncols = 0;
+            w.chunk_info = j | (n << 16);
+            items[(size_t)bh * cap + it_before + j] = w;
+        }
+        sel_before += sel[i];
+        it_before += n;
+    }
+    if (t == 0) {
+        // a head whose selection does not add up to k is skipped (never read
+        // out of bounds) and flagged in the status word
+        const bool ok = (sel_total == k && it_total <= cap);
+        head_items[bh] = ok ? it_total : 0;
+        if (!ok) atomicOr(status, kDevCount);
+    }
+}
+
+// One warp per block row: the selected columns in ascending order, the
+// exported flat indices, and (full mode) the row's selection bitmap.
+__global__ void __launch_bounds__(kThreads)
+cols_kernel(const unsigned long long *__restrict__ keys, const SelState *__restrict__ state,
+            const int *__restrict__ row_start, const int *__restrict__ take_eq, int nbr,
+            long long nbr2, int rows, int k, int *__restrict__ cols, int32_t *__restrict__ sel_out,
+            unsigned int *__restrict__ bitmap, int wpr) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const int bh = row / nbr, r = row % nbr;
+    const unsigned long long T = state[bh].prefix;
+    const unsigned long long *kr = keys + (size_t)bh * nbr2 + (size_t)r * nbr;
+    const int rs = row_start[row];
+    const int take = take_eq[row];
+    const int limit = (bh + 1) * k;   // this head's slice of cols[] ends here
+    const unsigned int lt_mask = (1u << lane) - 1u;
+    int eq_seen = 0, sel_seen = 0;
+    for (int c0 = 0; c0 < nbr; c0 += 32) {
+        const int c = c0 + lane;
+        unsigned long long key = 0;
+        if (c < nbr) key = kr[c];
+        const bool is_gt = (c < nbr) && key > T;
+        const bool is_eq = (c < nbr) && key == T;
+        const unsigned int eqb = __ballot_sync(0xffffffffu, is_eq);
+        const int eq_rank = eq_seen + __popc(eqb & lt_mask);
+        const bool sel = is_gt || (is_eq && eq_rank < take);
+        const unsigned int sb = __ballot_sync(0xffffffffu, sel);
+        if (sel && rs + sel_seen + __popc(sb & lt_mask) < limit) {
+            const int pos = rs + sel_seen + __popc(sb & lt_mask);
+            cols[pos] = c;
+            if (sel_out) sel_out[pos] = r * nbr + c;
+        }
+        if (bitmap && lane == 0) bitmap[(size_t)row * wpr + (c0 >> 5)] = sb;
+        eq_seen += __popc(eqb);
+        sel_seen += __popc(sb);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_radix_pass(const Problem &p, const Workspace &w, int pass, cudaStream_t s) {
+    // pass 1: bits 12..23, pass 2: bits 0..11
+    const int shift = (pass == 1) ? kHist2Bits : 0;
+    const int bits = (pass == 1) ? kHist1Bits : kHist2Bits;
+    dim3 grid(p.radix_ctas, p.BH);
+    radix_pass_kernel<<<grid, kThreads, 0, s>>>(w.keys, p.nbr2, p.radix_chunk, pass, shift, bits,
+                                                w.hist, w.arrive, w.state);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_row_counts(const Problem &p, const Workspace &w, cudaStream_t s) {
+    const int rows = p.BH * p.nbr;
+    const int grid = (rows + kThreads / 32 - 1) / (kThreads / 32);
+    row_counts_kernel<<<grid, kThreads, 0, s>>>(w.keys, w.state, p.nbr, p.nbr2, rows, w.gt, w.eq);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_row_scan(const Problem &p, const Workspace &w, cudaStream_t s) {
+    row_scan_kernel<<<p.BH, kScanThreads, 0, s>>>(w.gt, w.eq, w.state, p.nbr, p.k, p.cap,
+                                                  w.row_start, w.take_eq, w.items, w.head_items,
+                                                  w.status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cols(const Problem &p, const Workspace &w, int32_t *sel_out, cudaStream_t s) {
+    const int rows = p.BH * p.nbr;
+    const int grid = (rows + kThreads / 32 - 1) / (kThreads / 32);
+    cols_kernel<<<grid, kThreads, 0, s>>>(w.keys, w.state, w.row_start, w.take_eq, p.nbr, p.nbr2,
+                                          rows, p.k, w.cols, sel_out, p.mode == 0 ? w.bitmap : nullptr,
+                                          w.words_per_row);
+    return cudaGetLastError();
+}
+
+}  // namespace mra
