@@ -112,13 +112,15 @@ def make_inputs(w: Workload, seed: Optional[int] = None):
 
 
 def random_inputs(B: int, H: int, N: int, D: int, dtype=torch.float32, seed: int = 0,
-                  scale: float = 1.0, pad_tokens=None):
-    """Generic seeded inputs for tests.  pad_tokens: None, or a list of B
-    counts of trailing padded tokens (any count, not only whole blocks)."""
+                  scale: float = 1.0, pad_tokens=None, v_scale=None):
+    """Generic seeded inputs for tests.  Q and K are N(0, scale^2), V is
+    N(0, v_scale^2) (v_scale defaults to scale).  pad_tokens: None, or a list
+    of B counts of trailing padded tokens (any count, not only whole blocks)."""
     gen = torch.Generator("cpu").manual_seed(seed)
+    vs = scale if v_scale is None else v_scale
     q = (torch.randn(B, H, N, D, generator=gen) * scale).to(dtype).contiguous()
     k = (torch.randn(B, H, N, D, generator=gen) * scale).to(dtype).contiguous()
-    v = (torch.randn(B, H, N, D, generator=gen) * scale).to(dtype).contiguous()
+    v = (torch.randn(B, H, N, D, generator=gen) * vs).to(dtype).contiguous()
     mask = None
     if pad_tokens is not None:
         mask = torch.ones(B, N, dtype=torch.float32)
