@@ -29,6 +29,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from resolution_block_sparse_b200.sharding import max_over_ranks, weak_scaling_seed  # noqa: E402
 from resolution_block_sparse_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "MRA-2 attention fwd tokens/s and TFLOP/s (selected blocks) at N=4096; % of roofline"
@@ -134,7 +135,9 @@ def run_cuda(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     mra.load_library()
-    inputs = make_inputs(w)
+    # weak scaling: every rank owns a full-size batch of independent
+    # (batch, head) slices of its own (rank 0 holds the seeded workload itself)
+    inputs = make_inputs(w, seed=None if rank == 0 else weak_scaling_seed(1000 + w.index, rank))
     q, k, v = (inputs[x].to(dev) for x in ("q", "k", "v"))
     mask = None if inputs["mask"] is None else inputs["mask"].to(dev)
     out = torch.empty_like(q)
@@ -201,10 +204,7 @@ def run_cuda(args, w, world, rank, local):
 
     ms = statistics.mean(step_ms)
     e2e = statistics.mean(e2e_ms)
-    if world > 1:
-        t = torch.tensor([ms, e2e], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e = float(t[0]), float(t[1])
+    ms, e2e = max_over_ranks([ms, e2e], device=dev)
     return {"ms": ms, "e2e_ms": e2e, "phases": phases, "status": status,
             "launches_per_step": launches_per_step, "clocks": clocks,
             "h2d": sum(x.numel() * x.element_size() for x in (qh, kh, vh)) +
