@@ -68,7 +68,9 @@ typedef enum {
     MRA_ERR_UNSUPPORTED = 2,     /* D not in {32, 64}, or N above the maximum       */
     MRA_ERR_CUDA = 3,            /* a CUDA call or launch failed                    */
     MRA_ERR_ALLOC = 4,           /* workspace allocation failed                     */
-    MRA_ERR_DEVICE_TIMEOUT = 5   /* reserved: a bounded device wait gave up         */
+    MRA_ERR_DEVICE_TIMEOUT = 5,  /* reserved: a bounded device wait gave up         */
+    MRA_ERR_TOO_LARGE = 6        /* the problem needs more scratch than the static
+                                    array of mra_attention_fwd_noalloc holds         */
 } mra_status;
 
 enum { MRA_FULL = 0, MRA_SPARSE = 1 };
@@ -114,6 +116,39 @@ MRA_API int mra_attention_fwd_host(const void *q_host, const void *k_host, const
                            const float *key_mask_host, void *out_host, int B, int H, int N,
                            int D, int block_per_row, int approx_mode, int first_n, int diag_n,
                            int dtype, cudaStream_t stream);
+
+/* Size of the static device array behind mra_attention_fwd_noalloc. */
+#define MRA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* Forward pass, bf16, for callers that cannot allocate device memory.
+ *
+ * The method's pages have no counterpart of this entry point; it exists for
+ * callers that are not allowed to call cudaMalloc or any allocating routine:
+ * code running under another framework's caching allocator, plugins that
+ * must not allocate, and hosts that enqueue work where an allocation could
+ * block or fail.  The caller passes q, k, v, key_mask and out exactly as for
+ * mra_attention_fwd (device memory, same layout); all scratch memory comes
+ * from one static __device__ array of MRA_NOALLOC_SCRATCH_BYTES (16 MiB) that
+ * every GPU loading the library holds until the process exits.  Nothing here
+ * calls cudaMalloc, cudaFree or an allocating library routine.
+ *
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, that device current) and clears its status
+ *     word; make that first call before any stream capture.
+ *   - Problems whose scratch does not fit return MRA_ERR_TOO_LARGE before any
+ *     launch (for example B*H = 4, N = 1024, block_per_row = 4 fits; the
+ *     N = 4096 benchmark workload does not).
+ *   - Every call reuses the same array and leaves its contents behind; each
+ *     call clears what must start at zero.  Calls whose kernels overlap on the
+ *     GPU (different streams, or several host threads with different streams)
+ *     race on the array and give wrong results: issue them on one stream.
+ *   - Device status flags of these calls are not reported by
+ *     mra_get_device_status.
+ * Returns mra_status values like mra_attention_fwd. */
+MRA_API int mra_attention_fwd_noalloc(const void *q, const void *k, const void *v,
+                                      const float *key_mask, void *out, int B, int H, int N,
+                                      int D, int block_per_row, int approx_mode, int first_n,
+                                      int diag_n, cudaStream_t stream);
 
 /* num_block = min((N/32) * block_per_row, (N/32)^2); 0 for invalid input. */
 MRA_API size_t mra_num_block(int N, int block_per_row);

@@ -19,6 +19,7 @@ from ._binding import (  # noqa: F401
     mra_attention_fwd_ex,
     mra_attention_fwd_f32,
     mra_attention_fwd_host,
+    mra_attention_fwd_noalloc,
     mra_get_device_status,
     mra_last_launch_count,
     mra_num_block,

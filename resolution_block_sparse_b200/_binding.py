@@ -15,7 +15,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmra_b200.so")
 
-MRA_OK, MRA_ERR_INVALID_ARG, MRA_ERR_UNSUPPORTED, MRA_ERR_CUDA, MRA_ERR_ALLOC, MRA_ERR_DEVICE_TIMEOUT = range(6)
+(MRA_OK, MRA_ERR_INVALID_ARG, MRA_ERR_UNSUPPORTED, MRA_ERR_CUDA, MRA_ERR_ALLOC,
+ MRA_ERR_DEVICE_TIMEOUT, MRA_ERR_TOO_LARGE) = range(7)
+MRA_NOALLOC_SCRATCH_BYTES = 16 << 20
 MRA_FULL, MRA_SPARSE = 0, 1
 MRA_DTYPE_BF16, MRA_DTYPE_F32 = 0, 1
 MRA_DEV_KEY_RANGE, MRA_DEV_COUNT = 1, 2
@@ -23,7 +25,7 @@ MRA_DEV_KEY_RANGE, MRA_DEV_COUNT = 1, 2
 EXPORTED = (
     "mra_attention_fwd", "mra_attention_fwd_f32", "mra_attention_fwd_ex", "mra_attention_fwd_host",
     "mra_num_block", "mra_status_string", "mra_get_device_status", "mra_profile_enable",
-    "mra_profile_read", "mra_last_launch_count",
+    "mra_profile_read", "mra_last_launch_count", "mra_attention_fwd_noalloc",
 )
 
 _lock = threading.Lock()
@@ -53,6 +55,8 @@ def load_library(path: str = LIB_PATH):
         lib.mra_attention_fwd.restype = c_int
         lib.mra_attention_fwd_f32.argtypes = fwd_args
         lib.mra_attention_fwd_f32.restype = c_int
+        lib.mra_attention_fwd_noalloc.argtypes = fwd_args
+        lib.mra_attention_fwd_noalloc.restype = c_int
         lib.mra_attention_fwd_ex.argtypes = [vp, vp, vp, vp, vp] + [c_int] * 9 + [vp, vp, vp, vp]
         lib.mra_attention_fwd_ex.restype = c_int
         lib.mra_attention_fwd_host.argtypes = [vp, vp, vp, vp, vp] + [c_int] * 9 + [vp]
@@ -123,6 +127,19 @@ def mra_attention_fwd_f32(q, k, v, key_mask, out, block_per_row, approx_mode, fi
                                               B, H, N, D, block_per_row, _mode(approx_mode),
                                               first_n, diag_n, _stream(stream))
     _check(st, "mra_attention_fwd_f32")
+    return out
+
+
+def mra_attention_fwd_noalloc(q, k, v, key_mask, out, block_per_row, approx_mode, first_n,
+                              diag_n, stream=None):
+    """bf16 forward that allocates no device memory (static 16 MiB scratch);
+    raises MraError(MRA_ERR_TOO_LARGE) when the problem does not fit."""
+    B, H, N, D = _shape(q)
+    st = load_library().mra_attention_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(key_mask),
+                                                  _ptr(out), B, H, N, D, block_per_row,
+                                                  _mode(approx_mode), first_n, diag_n,
+                                                  _stream(stream))
+    _check(st, "mra_attention_fwd_noalloc")
     return out
 
 

@@ -12,72 +12,7 @@
 
 using namespace mra;
 
-namespace {
-
-constexpr int kMaxDevices = 64;
-
-struct DeviceCtx {
-    void *ws = nullptr;
-    size_t ws_bytes = 0;
-    unsigned int *status = nullptr;  // persistent status word
-    void *stage = nullptr;           // host-entry staging buffers
-    size_t stage_bytes = 0;
-};
-
-std::mutex g_mutex;
-DeviceCtx g_dev[kMaxDevices];
-int g_last_launches = 0;
-
-// ---------------------------------------------------------------- profiling
-struct PhaseStat {
-    const char *name;
-    int launches;
-    double ms;
-};
-struct PendingEvent {
-    int phase;
-    cudaEvent_t start, stop;
-};
-bool g_prof = false;
-std::vector<PhaseStat> g_phase;
-std::vector<PendingEvent> g_pending;
-std::vector<cudaEvent_t> g_event_pool;
-
-cudaEvent_t take_event() {
-    if (!g_event_pool.empty()) {
-        cudaEvent_t e = g_event_pool.back();
-        g_event_pool.pop_back();
-        return e;
-    }
-    cudaEvent_t e = nullptr;
-    cudaEventCreate(&e);
-    return e;
-}
-
-int phase_index(const char *name) {
-    for (size_t i = 0; i < g_phase.size(); ++i)
-        if (std::strcmp(g_phase[i].name, name) == 0) return (int)i;
-    g_phase.push_back({name, 0, 0.0});
-    return (int)g_phase.size() - 1;
-}
-
-struct PhaseScope {
-    bool on;
-    PendingEvent pe;
-    cudaStream_t s;
-    PhaseScope(const char *name, cudaStream_t st) : on(g_prof), s(st) {
-        if (!on) return;
-        pe.phase = phase_index(name);
-        pe.start = take_event();
-        pe.stop = take_event();
-        cudaEventRecord(pe.start, s);
-    }
-    ~PhaseScope() {
-        if (!on) return;
-        cudaEventRecord(pe.stop, s);
-        g_pending.push_back(pe);
-    }
-};
+namespace mra {
 
 // ---------------------------------------------------------------- planning
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -132,7 +67,7 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
 }
 
 // Carves the workspace; with base == nullptr only computes the size.
-size_t carve(const Problem &p, char *base, Workspace *w) {
+size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     size_t off = 0;
     auto take = [&](size_t bytes) -> char * {
         char *ptr = base ? base + off : nullptr;
@@ -168,13 +103,82 @@ size_t carve(const Problem &p, char *base, Workspace *w) {
     return off;
 }
 
+}  // namespace mra
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceCtx {
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    unsigned int *status = nullptr;  // persistent status word
+    void *stage = nullptr;           // host-entry staging buffers
+    size_t stage_bytes = 0;
+};
+
+std::mutex g_mutex;
+DeviceCtx g_dev[kMaxDevices];
+int g_last_launches = 0;
+
+// ---------------------------------------------------------------- profiling
+struct PhaseStat {
+    const char *name;
+    int launches;
+    double ms;
+};
+struct PendingEvent {
+    int phase;
+    cudaEvent_t start, stop;
+};
+bool g_prof = false;
+std::vector<PhaseStat> g_phase;
+std::vector<PendingEvent> g_pending;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+int phase_index(const char *name) {
+    for (size_t i = 0; i < g_phase.size(); ++i)
+        if (std::strcmp(g_phase[i].name, name) == 0) return (int)i;
+    g_phase.push_back({name, 0, 0.0});
+    return (int)g_phase.size() - 1;
+}
+
+struct PhaseScope {
+    bool on;
+    PendingEvent pe;
+    cudaStream_t s;
+    PhaseScope(const char *name, cudaStream_t st, bool enabled) : on(enabled), s(st) {
+        if (!on) return;
+        pe.phase = phase_index(name);
+        pe.start = take_event();
+        pe.stop = take_event();
+        cudaEventRecord(pe.start, s);
+    }
+    ~PhaseScope() {
+        if (!on) return;
+        cudaEventRecord(pe.stop, s);
+        g_pending.push_back(pe);
+    }
+};
+
 int ensure_workspace(int dev, const Problem &p, Workspace *w) {
     DeviceCtx &ctx = g_dev[dev];
     if (!ctx.status) {
         if (cudaMalloc(&ctx.status, 256) != cudaSuccess) return MRA_ERR_ALLOC;
         if (cudaMemset(ctx.status, 0, 256) != cudaSuccess) return MRA_ERR_CUDA;
     }
-    const size_t need = carve(p, nullptr, nullptr);
+    const size_t need = carve_workspace(p, nullptr, nullptr);
     if (need > ctx.ws_bytes) {
         if (ctx.ws) {
             cudaDeviceSynchronize();
@@ -189,7 +193,7 @@ int ensure_workspace(int dev, const Problem &p, Workspace *w) {
         }
         ctx.ws_bytes = bytes;
     }
-    carve(p, static_cast<char *>(ctx.ws), w);
+    carve_workspace(p, static_cast<char *>(ctx.ws), w);
     w->status = ctx.status;
     return MRA_OK;
 }
@@ -205,6 +209,67 @@ int current_device(int *dev) {
         cudaError_t e_ = (expr);                   \
         if (e_ != cudaSuccess) return MRA_ERR_CUDA; \
     } while (0)
+
+}  // namespace
+
+namespace mra {
+
+// The stream-ordered launch sequence of one forward pass on a prepared
+// workspace (shared by every entry point).  profile enables the per-phase
+// CUDA events of mra_profile_enable.
+int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const void *k,
+                    const void *v, const float *mask, void *out, int32_t *sel_out,
+                    float *logit_out, float *pooled_out, cudaStream_t s, bool profile,
+                    int *launch_count) {
+    const bool prof = profile && g_prof;
+    int launches = 0;
+    {
+        PhaseScope ps("memset", s, prof);
+        MRA_TRY(cudaMemsetAsync(w.zero_base, 0, w.zero_bytes, s));
+    }
+    {
+        PhaseScope ps("pool", s, prof);
+        MRA_TRY(launch_pool(p, w, q, k, v, mask, s));
+        ++launches;
+    }
+    {
+        PhaseScope ps("lowres_keys", s, prof);
+        MRA_TRY(launch_lowres_keys(p, w, logit_out, s));
+        ++launches;
+    }
+    {
+        PhaseScope ps("select", s, prof);
+        MRA_TRY(launch_radix_pass(p, w, 1, s));
+        MRA_TRY(launch_radix_pass(p, w, 2, s));
+        MRA_TRY(launch_row_counts(p, w, s));
+        MRA_TRY(launch_row_scan(p, w, s));
+        MRA_TRY(launch_cols(p, w, sel_out, s));
+        launches += 5;
+    }
+    if (p.mode == MRA_FULL) {
+        PhaseScope ps("lowres_pv", s, prof);
+        MRA_TRY(launch_lowres_pv(p, w, s));
+        ++launches;
+    }
+    {
+        PhaseScope ps("attention", s, prof);
+        MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s));
+        ++launches;
+    }
+    if (pooled_out) {
+        const size_t plane = sizeof(float) * (size_t)p.BH * p.nbr * p.D;
+        MRA_TRY(cudaMemcpyAsync(pooled_out, w.pooled, p.mode == MRA_FULL ? 3 * plane : 2 * plane,
+                                cudaMemcpyDeviceToDevice, s));
+        if (p.mode != MRA_FULL)
+            MRA_TRY(cudaMemsetAsync(reinterpret_cast<char *>(pooled_out) + 2 * plane, 0, plane, s));
+    }
+    *launch_count = launches;
+    return MRA_OK;
+}
+
+}  // namespace mra
+
+namespace {
 
 // The forward pass proper; the caller holds g_mutex.
 int forward_locked(const void *q, const void *k, const void *v, const float *mask, void *out,
@@ -224,46 +289,9 @@ int forward_locked(const void *q, const void *k, const void *v, const float *mas
     if (rc != MRA_OK) return rc;
 
     int launches = 0;
-    {
-        PhaseScope ps("memset", s);
-        MRA_TRY(cudaMemsetAsync(w.zero_base, 0, w.zero_bytes, s));
-    }
-    {
-        PhaseScope ps("pool", s);
-        MRA_TRY(launch_pool(p, w, q, k, v, mask, s));
-        ++launches;
-    }
-    {
-        PhaseScope ps("lowres_keys", s);
-        MRA_TRY(launch_lowres_keys(p, w, logit_out, s));
-        ++launches;
-    }
-    {
-        PhaseScope ps("select", s);
-        MRA_TRY(launch_radix_pass(p, w, 1, s));
-        MRA_TRY(launch_radix_pass(p, w, 2, s));
-        MRA_TRY(launch_row_counts(p, w, s));
-        MRA_TRY(launch_row_scan(p, w, s));
-        MRA_TRY(launch_cols(p, w, sel_out, s));
-        launches += 5;
-    }
-    if (p.mode == MRA_FULL) {
-        PhaseScope ps("lowres_pv", s);
-        MRA_TRY(launch_lowres_pv(p, w, s));
-        ++launches;
-    }
-    {
-        PhaseScope ps("attention", s);
-        MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s));
-        ++launches;
-    }
-    if (pooled_out) {
-        const size_t plane = sizeof(float) * (size_t)p.BH * p.nbr * p.D;
-        MRA_TRY(cudaMemcpyAsync(pooled_out, w.pooled, p.mode == MRA_FULL ? 3 * plane : 2 * plane,
-                                cudaMemcpyDeviceToDevice, s));
-        if (p.mode != MRA_FULL)
-            MRA_TRY(cudaMemsetAsync(reinterpret_cast<char *>(pooled_out) + 2 * plane, 0, plane, s));
-    }
+    rc = enqueue_forward(p, w, q, k, v, mask, out, sel_out, logit_out, pooled_out, s, true,
+                         &launches);
+    if (rc != MRA_OK) return rc;
     g_last_launches = launches;
     return MRA_OK;
 }
@@ -359,6 +387,8 @@ const char *mra_status_string(int status) {
         case MRA_ERR_CUDA: return "CUDA error";
         case MRA_ERR_ALLOC: return "workspace allocation failed";
         case MRA_ERR_DEVICE_TIMEOUT: return "bounded device wait gave up";
+        case MRA_ERR_TOO_LARGE:
+            return "problem needs more scratch than the no-allocation entry point's static array";
         default: return "unknown status";
     }
 }

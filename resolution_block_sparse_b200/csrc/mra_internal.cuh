@@ -86,6 +86,19 @@ struct Workspace {
     unsigned int *status;    // 1 word, persistent across calls
 };
 
+// Planning and the launch sequence shared by the entry points (mra_api.cu).
+int validate_sizes(int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n);
+int validate(const void *q, const void *k, const void *v, const void *out, int B, int H, int N,
+             int D, int bpr, int mode, int first_n, int diag_n);
+Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n,
+                     int dtype);
+// Carves the workspace out of base (size only when base is null); returns bytes.
+size_t carve_workspace(const Problem &p, char *base, Workspace *w);
+int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const void *k,
+                    const void *v, const float *mask, void *out, int32_t *sel_out,
+                    float *logit_out, float *pooled_out, cudaStream_t s, bool profile,
+                    int *launch_count);
+
 // Launchers (each returns cudaGetLastError() of its launches).
 cudaError_t launch_pool(const Problem &p, const Workspace &w, const void *q, const void *k,
                         const void *v, const float *mask, cudaStream_t s);
