@@ -80,7 +80,9 @@ enum { MRA_DTYPE_BF16 = 0, MRA_DTYPE_F32 = 1 };
 enum {
     MRA_DEV_KEY_RANGE = 1,   /* some |l - rowmax| >= 2500: the tier order may
                                 differ from exact additive biases              */
-    MRA_DEV_COUNT = 2        /* selected-block count per head differed from k  */
+    MRA_DEV_COUNT = 2,       /* selected-block count per head differed from k  */
+    MRA_DEV_TIMEOUT = 4      /* a bounded wait inside a kernel gave up; that
+                                kernel's output is incomplete                  */
 };
 
 /* Forward pass, bf16 in/out, fp32 accumulation.  Steps one to four of the

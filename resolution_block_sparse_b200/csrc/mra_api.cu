@@ -56,11 +56,15 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
     p.diag_n = diag_n;
     p.dtype = dtype;
     p.cap = p.nbr + p.k / kChunk;
-    p.r_tile = p.nbr >= 2048 ? 8 : (p.nbr >= 1024 ? 16 : 32);
+    // low-res rows per CTA: at most 64 KB of logits per CTA, and enough CTAs
+    // to cover the SMs twice when the problem allows
+    // low-res rows per CTA: the logits of a CTA's rows stay in shared memory
+    // (at most 64 KB), so longer maps take fewer rows per CTA
+    p.r_tile = p.nbr > 1024 ? 8 : (p.nbr > 512 ? 16 : 32);
     p.lowres_ctas = (p.nbr + p.r_tile - 1) / p.r_tile;
-    long long ctas = (p.nbr2 + 8191) / 8192;
+    long long ctas = (p.nbr2 + 4095) / 4096;
     if (ctas < 1) ctas = 1;
-    if (ctas > 256) ctas = 256;
+    if (ctas > 1024) ctas = 1024;
     p.radix_ctas = (int)ctas;
     p.radix_chunk = (p.nbr2 + ctas - 1) / ctas;
     return p;
@@ -224,10 +228,7 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
     const bool prof = profile && g_prof;
     int launches = 0;
     {
-        PhaseScope ps("memset", s, prof);
-        MRA_TRY(cudaMemsetAsync(w.zero_base, 0, w.zero_bytes, s));
-    }
-    {
+        // the pool kernel also clears the per-call counters and histograms
         PhaseScope ps("pool", s, prof);
         MRA_TRY(launch_pool(p, w, q, k, v, mask, s));
         ++launches;
@@ -239,12 +240,17 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
     }
     {
         PhaseScope ps("select", s, prof);
-        MRA_TRY(launch_radix_pass(p, w, 1, s));
-        MRA_TRY(launch_radix_pass(p, w, 2, s));
-        MRA_TRY(launch_row_counts(p, w, s));
-        MRA_TRY(launch_row_scan(p, w, s));
-        MRA_TRY(launch_cols(p, w, sel_out, s));
-        launches += 5;
+        if (p.nbr <= kSmallMaxRows) {
+            MRA_TRY(launch_select_small(p, w, sel_out, s));
+            launches += 1;
+        } else {
+            MRA_TRY(launch_radix_pass(p, w, 1, s));
+            MRA_TRY(launch_radix_pass(p, w, 2, s));
+            MRA_TRY(launch_row_counts(p, w, s));
+            MRA_TRY(launch_row_scan(p, w, s));
+            MRA_TRY(launch_cols(p, w, sel_out, s));
+            launches += 5;
+        }
     }
     if (p.mode == MRA_FULL) {
         PhaseScope ps("lowres_pv", s, prof);

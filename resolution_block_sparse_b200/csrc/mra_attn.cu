@@ -20,12 +20,15 @@
 // by cp.async.  fp32 kernel: FFMA only (no TF32).
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+
+#include "mra_attn_common.cuh"
 #include "mra_internal.cuh"
 
 namespace mra {
 namespace {
 
-constexpr float kLog2e = 1.4426950408889634f;
+using namespace attn;
 
 __device__ __forceinline__ unsigned smem_u32(const void *p) {
     return (unsigned)__cvta_generic_to_shared(p);
@@ -82,120 +85,6 @@ __device__ __forceinline__ void load_tile_async(__nv_bfloat16 *tile, const __nv_
     }
 }
 
-template <bool G>
-__device__ __forceinline__ float ldp(const float *p) {
-    if constexpr (G) return __ldcg(p);
-    else return *p;
-}
-
-template <typename T>
-__device__ __forceinline__ T to_out(float x);
-template <>
-__device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
-template <>
-__device__ __forceinline__ float to_out<float>(float x) { return x; }
-
-struct MergeSmem {
-    float w[32][33];
-    float M[32], inv[32], beta[32];
-};
-
-// Merge nchunks partials (layout per slot: m[32], l[32], O[32][D]; m in log2
-// units, l and O relative to exp2(m)) with the low-resolution part of the row
-// (full mode) and write the 32 x D output block.
-template <int D, int NT, bool G, typename OutT>
-__device__ void merge_write(const float *src0, size_t slot_stride, int nchunks, int full,
-                            float m_lo2, float l_lo, const float *olo_row, const float *qmask,
-                            OutT *out_blk, MergeSmem &sm) {
-    const int tid = threadIdx.x;
-    if (tid < 32) {
-        const int q = tid;
-        float M = -INFINITY;
-        for (int c = 0; c < nchunks; ++c) {
-            const float *P = src0 + (size_t)c * slot_stride;
-            if (ldp<G>(P + 32 + q) > 0.0f) M = fmaxf(M, ldp<G>(P + q));
-        }
-        const bool lo = full && l_lo > 0.0f;
-        if (lo) M = fmaxf(M, m_lo2);
-        float inv = 0.0f, beta = 0.0f;
-        if (M != -INFINITY && (!qmask || qmask[q] > 0.0f)) {
-            float den = 0.0f;
-            for (int c = 0; c < nchunks; ++c) {
-                const float *P = src0 + (size_t)c * slot_stride;
-                const float l = ldp<G>(P + 32 + q);
-                if (l > 0.0f) den += exp2f(ldp<G>(P + q) - M) * l;
-            }
-            if (lo) {
-                beta = exp2f(m_lo2 - M);
-                den += beta * l_lo;
-            }
-            inv = den > 0.0f ? 1.0f / den : 0.0f;
-        }
-        sm.M[q] = (M == -INFINITY) ? 0.0f : M;
-        sm.inv[q] = inv;
-        sm.beta[q] = beta;
-    }
-    __syncthreads();
-    constexpr int E = 32 * D / NT;
-    float acc[E];
-#pragma unroll
-    for (int i = 0; i < E; ++i) acc[i] = 0.0f;
-    for (int cg = 0; cg < nchunks; cg += 32) {
-        const int nc = min(32, nchunks - cg);
-        for (int e = tid; e < nc * 32; e += NT) {
-            const int c = e / 32, q = e % 32;
-            const float *P = src0 + (size_t)(cg + c) * slot_stride;
-            sm.w[c][q] = ldp<G>(P + 32 + q) > 0.0f ? exp2f(ldp<G>(P + q) - sm.M[q]) : 0.0f;
-        }
-        __syncthreads();
-        for (int c = 0; c < nc; ++c) {
-            const float *O = src0 + (size_t)(cg + c) * slot_stride + 64;
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                const int e = tid + i * NT;
-                acc[i] = fmaf(sm.w[c][e / D], ldp<G>(O + e), acc[i]);
-            }
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-        const int e = tid + i * NT;
-        const int q = e / D, d = e % D;
-        float val = acc[i];
-        if (full) val = fmaf(sm.beta[q], olo_row[d], val);
-        out_blk[e] = to_out<OutT>(val * sm.inv[q]);
-    }
-}
-
-// Shared epilogue: the item's (m, l, O) sit in `stage` (shared, slot layout).
-template <int D, int NT, typename OutT>
-__device__ void finish_item(float *stage, int slot, int chunk, int nchunks, int row, int full,
-                            const float *mlo, const float *olo, const float *llo,
-                            float *partial, int *row_arrive, const float *qmask, OutT *out_blk,
-                            MergeSmem &sm, int *s_last) {
-    const int tid = threadIdx.x;
-    const size_t stride = (size_t)32 * (D + 2);
-    const float m_lo2 = full ? mlo[row] * kLog2e : 0.0f;
-    const float l_lo = full ? llo[row] : 0.0f;
-    const float *olo_row = full ? olo + (size_t)row * D : nullptr;
-    if (nchunks == 1) {
-        merge_write<D, NT, false, OutT>(stage, stride, 1, full, m_lo2, l_lo, olo_row, qmask, out_blk, sm);
-        return;
-    }
-    float *dst = partial + (size_t)slot * stride;
-    for (int e = tid; e < (int)stride; e += NT) dst[e] = stage[e];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) *s_last = (atomicAdd(&row_arrive[row], 1) == nchunks - 1);
-    __syncthreads();
-    if (!*s_last) return;
-    __threadfence();
-    merge_write<D, NT, true, OutT>(partial + (size_t)(slot - chunk) * stride, stride, nchunks, full,
-                                   m_lo2, l_lo, olo_row, qmask, out_blk, sm);
-    if (tid == 0) row_arrive[row] = 0;
-}
-
 struct AttnArgs {
     const void *q, *k, *v;
     const float *mask;
@@ -239,8 +128,12 @@ attn_bf16_kernel(const AttnArgs a) {
 
     load_tile_async<D, kBf16Threads>(sQ, qg + (size_t)r * kTile, tid);
     const int ncols = it.ncols;
+    // the item's column list, read once (the loads below depend on it)
+    __shared__ int s_cols[kChunk];
+    for (int j = tid; j < ncols; j += kBf16Threads) s_cols[j] = a.cols[it.col_start + j];
+    __syncthreads();
     if (ncols > 0) {
-        const int c0 = a.cols[it.col_start];
+        const int c0 = s_cols[0];
         load_tile_async<D, kBf16Threads>(sKV[0][0], kg + (size_t)c0 * kTile, tid);
         load_tile_async<D, kBf16Threads>(sKV[0][1], vg + (size_t)c0 * kTile, tid);
         if (tid < 32) sKm[0][tid] = mrow ? mrow[c0 * 32 + tid] : 1.0f;
@@ -256,7 +149,7 @@ attn_bf16_kernel(const AttnArgs a) {
     for (int j = 0; j < ncols; ++j) {
         const int buf = j & 1;
         if (j + 1 < ncols) {
-            const int c1 = a.cols[it.col_start + j + 1];
+            const int c1 = s_cols[j + 1];
             load_tile_async<D, kBf16Threads>(sKV[buf ^ 1][0], kg + (size_t)c1 * kTile, tid);
             load_tile_async<D, kBf16Threads>(sKV[buf ^ 1][1], vg + (size_t)c1 * kTile, tid);
             if (tid < 32) sKm[buf ^ 1][tid] = mrow ? mrow[c1 * 32 + tid] : 1.0f;
@@ -384,7 +277,7 @@ attn_bf16_kernel(const AttnArgs a) {
     }
     __syncthreads();
     __nv_bfloat16 *out_blk = static_cast<__nv_bfloat16 *>(a.out) + head_off + (size_t)r * kTile;
-    finish_item<D, kBf16Threads, __nv_bfloat16>(stage, slot, chunk, nchunks, it.row, a.full, a.mlo,
+    finish_item<D, kBf16Threads, __nv_bfloat16, SyncAll>(stage, slot, chunk, nchunks, it.row, a.full, a.mlo,
                                                 a.olo, a.llo, a.partial, a.row_arrive,
                                                 mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
 }
@@ -472,7 +365,7 @@ attn_f32_kernel(const AttnArgs a) {
     for (int i = 0; i < kDp; ++i) stage[64 + qrow * D + d0 + i] = o[i];
     __syncthreads();
     float *out_blk = static_cast<float *>(a.out) + head_off + (size_t)r * kTile;
-    finish_item<D, kF32Threads, float>(stage, slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
+    finish_item<D, kF32Threads, float, SyncAll>(stage, slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
                                        a.llo, a.partial, a.row_arrive,
                                        mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
 }
@@ -502,6 +395,12 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
     a.row_arrive = w.row_arrive;
     a.out = out;
     const long long grid = (long long)p.BH * p.cap;
+    // MRA_ATTN_IMPL=tc selects the tcgen05/TMA kernel (bf16, head size 64);
+    // the default is the warp-level kernel below, which measures faster on
+    // the sparse workloads (a few 32x32 blocks per block row)
+    static const char *impl = getenv("MRA_ATTN_IMPL");
+    const bool want_tc = impl && impl[0] == 't';
+    if (want_tc && attention_tc_supported(p)) return launch_attention_tc(p, w, q, k, v, mask, out, s);
     if (p.dtype == 0) {
         if (p.D == 64) attn_bf16_kernel<64><<<(unsigned)grid, kBf16Threads, 0, s>>>(a);
         else attn_bf16_kernel<32><<<(unsigned)grid, kBf16Threads, 0, s>>>(a);

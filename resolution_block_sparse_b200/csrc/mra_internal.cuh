@@ -21,16 +21,19 @@
 namespace mra {
 
 constexpr int kBlock = 32;            // tokens per block (fixed by the method)
-constexpr int kChunk = 8;             // max selected blocks per attention work item
+constexpr int kChunk = 32;            // max selected blocks per attention work item
 constexpr int kHist0Bits = 11;        // radix digit widths over the 35-bit key
 constexpr int kHist1Bits = 12;
 constexpr int kHist2Bits = 12;
 constexpr int kHistBins = 4096;       // per-pass histogram stride per head
 constexpr int kMaxN = 65536;
+constexpr int kSmallMaxRows = 128;               // one-CTA selection up to 128 x 128 blocks
+constexpr int kSmallMaxKeys = kSmallMaxRows * kSmallMaxRows;
 
 // Device status bits (mirrors of the public MRA_DEV_* values).
 constexpr unsigned kDevKeyRange = 1u;
 constexpr unsigned kDevCount = 2u;
+constexpr unsigned kDevTimeout = 4u;
 
 struct SelState {
     unsigned long long prefix;  // key bits fixed so far (threshold after the last pass)
@@ -108,9 +111,17 @@ cudaError_t launch_radix_pass(const Problem &p, const Workspace &w, int pass, cu
 cudaError_t launch_row_counts(const Problem &p, const Workspace &w, cudaStream_t s);
 cudaError_t launch_row_scan(const Problem &p, const Workspace &w, cudaStream_t s);
 cudaError_t launch_cols(const Problem &p, const Workspace &w, int32_t *sel_out, cudaStream_t s);
+// Whole selection (radix passes 2-3, counts, scan, work list, cols) in one CTA
+// per head, for nbr <= kSmallMaxRows.
+cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *sel_out,
+                                cudaStream_t s);
 cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t s);
 cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
                              const void *v, const float *mask, void *out, cudaStream_t s);
+// tcgen05 / TMA attention (bf16, D = 64); used by launch_attention when supported.
+bool attention_tc_supported(const Problem &p);
+cudaError_t launch_attention_tc(const Problem &p, const Workspace &w, const void *q, const void *k,
+                                const void *v, const float *mask, void *out, cudaStream_t s);
 
 // ---------------------------------------------------------------- device helpers
 #ifdef __CUDACC__

@@ -37,24 +37,28 @@ __device__ __forceinline__ int in_band(int r, int c, int g) {
 }
 
 constexpr int kLowresThreads = 256;
-constexpr int kColTile = 64;
 
 // One CTA: R block rows of one (batch, head) against every block column.
-template <int D>
+// Thread tile: 4 rows x 4 consecutive columns, fp32 FFMA; Q-hat rows and a
+// transposed K-hat column tile sit in shared memory and are read as float4.
+template <int D, int R>
 __global__ void __launch_bounds__(kLowresThreads)
 lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ khat,
-                   const int *__restrict__ cnt, int H, int nbr, long long nbr2, int R, float scale,
+                   const int *__restrict__ cnt, int H, int nbr, long long nbr2, float scale,
                    int first_n, int diag_n, int k, unsigned long long *__restrict__ keys,
                    float *__restrict__ mlo, float *__restrict__ logit_out,
                    unsigned int *__restrict__ hist, unsigned int *__restrict__ arrive,
                    SelState *__restrict__ state, unsigned int *__restrict__ status) {
+    constexpr int RG = R / 4;                  // row groups
+    constexpr int CG = kLowresThreads / RG;    // column groups
+    constexpr int CT = 4 * CG;                 // columns per tile
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    float *qs = reinterpret_cast<float *>(smem_raw);                 // [R][D]
-    float *ks = qs + R * D;                                           // [kColTile][D+1]
-    float *lt = ks + kColTile * (D + 1);                              // [R][nbr]
-    float *rmax = lt + (size_t)R * nbr;                               // [R]
-    int *cnts = reinterpret_cast<int *>(rmax + R);                    // [nbr]
-    unsigned int *h0 = reinterpret_cast<unsigned int *>(cnts + nbr);  // [2048]
+    float *qs = reinterpret_cast<float *>(smem_raw);                  // [R][D]
+    float *kT = qs + R * D;                                            // [D][CT]
+    float *lt = kT + D * CT;                                           // [R][nbr]
+    float *rmax = lt + (size_t)R * nbr;                                // [R]
+    int *cnts = reinterpret_cast<int *>(rmax + R);                     // [nbr]
+    unsigned int *h0 = reinterpret_cast<unsigned int *>(cnts + nbr);   // [2048]
     __shared__ unsigned int s_tmp[256];
     __shared__ int s_flag, s_last, s_bin;
     __shared__ unsigned int s_need;
@@ -69,29 +73,79 @@ lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ kha
     if (t == 0) s_flag = 0;
     for (int c = t; c < nbr; c += kLowresThreads) cnts[c] = cnt[(size_t)b * nbr + c];
     for (int i = t; i < (1 << kHist0Bits); i += kLowresThreads) h0[i] = 0u;
-    for (int i = t; i < R * D; i += kLowresThreads) {
-        const int r = i / D;
-        qs[i] = (r0 + r < nbr) ? qh[(size_t)(r0 + r) * D + (i % D)] : 0.0f;
+    {
+        // all loads in flight before the first shared-memory store
+        constexpr int kQ = (R * D / 4 + kLowresThreads - 1) / kLowresThreads;
+        float4 v[kQ];
+#pragma unroll
+        for (int u = 0; u < kQ; ++u) {
+            const int i = t + u * kLowresThreads;
+            const int r = (4 * i) / D;
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < R * D / 4 && r0 + r < nbr)
+                v[u] = reinterpret_cast<const float4 *>(qh + (size_t)(r0 + r) * D)[(4 * i) % D / 4];
+        }
+#pragma unroll
+        for (int u = 0; u < kQ; ++u) {
+            const int i = t + u * kLowresThreads;
+            if (i < R * D / 4) reinterpret_cast<float4 *>(qs)[i] = v[u];
+        }
     }
 
-    constexpr int kRowGroups = kLowresThreads / kColTile;  // 4
-    const int cl = t % kColTile;
-    const int rg = t / kColTile;
-    for (int ct = 0; ct < nbr; ct += kColTile) {
+    const int rg = t / CG, cg = t % CG;
+    for (int ct = 0; ct < nbr; ct += CT) {
         __syncthreads();
-        for (int i = t; i < kColTile * D; i += kLowresThreads) {
-            const int c = i / D, d = i % D;
-            ks[c * (D + 1) + d] = (ct + c < nbr) ? kh[(size_t)(ct + c) * D + d] : 0.0f;
+        // transposed column tile: kT[d][c] = khat[ct + c][d]
+        {
+            constexpr int kL = CT * D / 4 / kLowresThreads;   // float4 loads per thread
+            float4 v[kL];
+#pragma unroll
+            for (int u = 0; u < kL; ++u) {
+                const int e = t + u * kLowresThreads;
+                const int c = e % CT, d4 = e / CT;
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (ct + c < nbr) v[u] = reinterpret_cast<const float4 *>(kh + (size_t)(ct + c) * D)[d4];
+            }
+#pragma unroll
+            for (int u = 0; u < kL; ++u) {
+                const int e = t + u * kLowresThreads;
+                const int c = e % CT, d4 = e / CT;
+                kT[(4 * d4 + 0) * CT + c] = v[u].x;
+                kT[(4 * d4 + 1) * CT + c] = v[u].y;
+                kT[(4 * d4 + 2) * CT + c] = v[u].z;
+                kT[(4 * d4 + 3) * CT + c] = v[u].w;
+            }
         }
         __syncthreads();
-        const float *kr = ks + cl * (D + 1);
-        for (int r = rg; r < R; r += kRowGroups) {
-            const float *qr = qs + r * D;
-            float acc = 0.0f;
-#pragma unroll 16
-            for (int d = 0; d < D; ++d) acc = fmaf(qr[d], kr[d], acc);
-            if (ct + cl < nbr) lt[(size_t)r * nbr + ct + cl] = acc * scale;
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+#pragma unroll 4
+        for (int d = 0; d < D; d += 4) {
+            float4 qv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const float4 *>(qs + (4 * rg + i) * D + d);
+#pragma unroll
+            for (int dd = 0; dd < 4; ++dd) {
+                const float4 kv = *reinterpret_cast<const float4 *>(kT + (d + dd) * CT + 4 * cg);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float qd = dd == 0 ? qv[i].x : dd == 1 ? qv[i].y : dd == 2 ? qv[i].z : qv[i].w;
+                    acc[i][0] = fmaf(qd, kv.x, acc[i][0]);
+                    acc[i][1] = fmaf(qd, kv.y, acc[i][1]);
+                    acc[i][2] = fmaf(qd, kv.z, acc[i][2]);
+                    acc[i][3] = fmaf(qd, kv.w, acc[i][3]);
+                }
+            }
         }
+        const int c0 = ct + 4 * cg;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (c0 + j < nbr) lt[(size_t)(4 * rg + i) * nbr + c0 + j] = acc[i][j] * scale;
     }
     __syncthreads();
 
@@ -113,26 +167,31 @@ lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ kha
 
     // keys, exported logits, first radix histogram (bits 24..34)
     const int rows_here = min(R, nbr - r0);
-    const long long n_here = (long long)rows_here * nbr;
+    const int n_here = rows_here * nbr;
     unsigned long long *kout = keys + (size_t)bh * nbr2 + (size_t)r0 * nbr;
     int flag = 0;
-    for (long long e = t; e < n_here; e += kLowresThreads) {
-        const int r = (int)(e / nbr), c = (int)(e % nbr);
-        const int gr = r0 + r;
-        const float l = lt[(size_t)r * nbr + c];
-        float x = l - rmax[r];
-        if (x == 0.0f) x = 0.0f;  // canonical +0
-        if (!(fabsf(x) < 2500.0f)) flag = 1;
-        int tier = 0;
-        if (first_n > 0 && (gr < first_n || c < first_n)) ++tier;
-        tier += in_band(gr, c, diag_n);
-        if (cnts[gr] <= 0) tier -= 2;
-        if (cnts[c] <= 0) tier -= 2;
-        const unsigned long long key =
-            ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
-        kout[e] = key;
-        if (logit_out) logit_out[(size_t)bh * nbr2 + (size_t)gr * nbr + c] = l;
-        atomicAdd(&h0[(unsigned)(key >> 24)], 1u);
+    // warp-uniform trip count so that the histogram update can aggregate lanes
+    for (int e0 = (t & ~31); e0 < n_here; e0 += kLowresThreads) {
+        const int e = e0 + lane;
+        const bool act = e < n_here;
+        unsigned long long key = 0;
+        if (act) {
+            const int r = e / nbr, c = e - r * nbr;
+            const int gr = r0 + r;
+            const float l = lt[e];
+            float x = l - rmax[r];
+            if (x == 0.0f) x = 0.0f;  // canonical +0
+            if (!(fabsf(x) < 2500.0f)) flag = 1;
+            int tier = 0;
+            if (first_n > 0 && (gr < first_n || c < first_n)) ++tier;
+            tier += in_band(gr, c, diag_n);
+            if (cnts[gr] <= 0) tier -= 2;
+            if (cnts[c] <= 0) tier -= 2;
+            key = ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
+            kout[e] = key;
+            if (logit_out) logit_out[(size_t)bh * nbr2 + (size_t)gr * nbr + c] = l;
+        }
+        warp_hist_add(h0, (unsigned)(key >> 24), act);
     }
     if (flag) s_flag = 1;
     __syncthreads();
@@ -168,9 +227,10 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
                  int nbr, long long nbr2, float *__restrict__ olo, float *__restrict__ llo) {
     constexpr int R = 32;
     constexpr int kCt = 32;
-    __shared__ float vs[kCt][D];
+    constexpr int kVL = kCt * D / 4 / kLowresThreads;      // float4 loads of the V-hat tile
+    constexpr int kWL = R * kCt / kLowresThreads;          // weights per thread and tile
+    __shared__ __align__(16) float vs[kCt][D];
     __shared__ float ws[R][kCt + 1];
-    __shared__ int cc[kCt];
     const int t = threadIdx.x;
     const int bh = blockIdx.y;
     const int b = bh / H;
@@ -185,24 +245,47 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
     for (int i = 0; i < kPer; ++i) acc[i] = lsum[i] = 0.0f;
 
     for (int ct = 0; ct < nbr; ct += kCt) {
-        __syncthreads();
-        for (int i = t; i < kCt * D; i += kLowresThreads) {
-            const int c = i / D;
-            vs[c][i % D] = (ct + c < nbr) ? vh[(size_t)(ct + c) * D + (i % D)] : 0.0f;
+        // issue every global load of this tile before touching shared memory
+        float4 vv[kVL];
+#pragma unroll
+        for (int u = 0; u < kVL; ++u) {
+            const int i = t + u * kLowresThreads;
+            const int c = (4 * i) / D;
+            vv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (ct + c < nbr) vv[u] = reinterpret_cast<const float4 *>(vh + (size_t)(ct + c) * D)[(4 * i) % D / 4];
         }
-        if (t < kCt) cc[t] = (ct + t < nbr) ? cnt[(size_t)b * nbr + ct + t] : 0;
-        __syncthreads();
-        for (int e = t; e < R * kCt; e += kLowresThreads) {
+        unsigned long long kv[kWL];
+        unsigned int bw[kWL];
+        int cc[kWL];
+#pragma unroll
+        for (int u = 0; u < kWL; ++u) {
+            const int e = t + u * kLowresThreads;
             const int r = e / kCt, c = e % kCt;
             const int gr = r0 + r, gc = ct + c;
+            kv[u] = 0ull;
+            bw[u] = 0xffffffffu;
+            cc[u] = 0;
+            if (gr < nbr && gc < nbr) {
+                cc[u] = cnt[(size_t)b * nbr + gc];
+                bw[u] = bitmap[((size_t)bh * nbr + gr) * wpr + (gc >> 5)];
+                kv[u] = keys[(size_t)bh * nbr2 + (size_t)gr * nbr + gc];
+            }
+        }
+        __syncthreads();   // previous tile fully consumed
+#pragma unroll
+        for (int u = 0; u < kVL; ++u) {
+            const int i = t + u * kLowresThreads;
+            reinterpret_cast<float4 *>(&vs[0][0])[i] = vv[u];
+        }
+#pragma unroll
+        for (int u = 0; u < kWL; ++u) {
+            const int e = t + u * kLowresThreads;
+            const int r = e / kCt, c = e % kCt;
+            const int gc = ct + c;
             float wv = 0.0f;
-            if (gr < nbr && gc < nbr && cc[c] > 0) {
-                const unsigned int word = bitmap[((size_t)bh * nbr + gr) * wpr + (gc >> 5)];
-                if (!((word >> (gc & 31)) & 1u)) {
-                    const unsigned long long key = keys[(size_t)bh * nbr2 + (size_t)gr * nbr + gc];
-                    const float x = float_from_order_bits((unsigned int)(key & 0xffffffffull));
-                    wv = (float)cc[c] * expf(x);
-                }
+            if (cc[u] > 0 && !((bw[u] >> (gc & 31)) & 1u)) {
+                const float x = float_from_order_bits((unsigned int)(kv[u] & 0xffffffffull));
+                wv = (float)cc[u] * expf(x);
             }
             ws[r][c] = wv;
         }
@@ -228,27 +311,30 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
     }
 }
 
-template <int D>
-size_t lowres_smem_bytes(int R, int nbr) {
-    return sizeof(float) * ((size_t)R * D + (size_t)kColTile * (D + 1) + (size_t)R * nbr + R) +
-           sizeof(int) * (size_t)nbr + sizeof(unsigned int) * (1u << kHist0Bits);
+template <int D, int R>
+cudaError_t launch_keys_rt(const Problem &p, const Workspace &w, float *logit_out, cudaStream_t s) {
+    constexpr int CT = 4 * (kLowresThreads / (R / 4));
+    const size_t smem = sizeof(float) * ((size_t)R * D + (size_t)D * CT + (size_t)R * p.nbr + R) +
+                        sizeof(int) * (size_t)p.nbr + sizeof(unsigned int) * (1u << kHist0Bits);
+    cudaError_t e = cudaFuncSetAttribute(lowres_keys_kernel<D, R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((p.nbr + R - 1) / R, p.BH);
+    const float scale = 1.0f / sqrtf((float)p.D);
+    const float *qhat = w.pooled;
+    const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;
+    lowres_keys_kernel<D, R><<<grid, kLowresThreads, smem, s>>>(
+        qhat, khat, w.cnt, p.H, p.nbr, p.nbr2, scale, p.first_n, p.diag_n, p.k, w.keys, w.mlo,
+        logit_out, w.hist, w.arrive, w.state, w.status);
+    return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_keys_typed(const Problem &p, const Workspace &w, float *logit_out,
                               cudaStream_t s) {
-    const size_t smem = lowres_smem_bytes<D>(p.r_tile, p.nbr);
-    cudaError_t e = cudaFuncSetAttribute(lowres_keys_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(p.lowres_ctas, p.BH);
-    const float scale = 1.0f / sqrtf((float)p.D);
-    const float *qhat = w.pooled;
-    const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;
-    lowres_keys_kernel<D><<<grid, kLowresThreads, smem, s>>>(
-        qhat, khat, w.cnt, p.H, p.nbr, p.nbr2, p.r_tile, scale, p.first_n, p.diag_n, p.k, w.keys,
-        w.mlo, logit_out, w.hist, w.arrive, w.state, w.status);
-    return cudaGetLastError();
+    if (p.r_tile == 32) return launch_keys_rt<D, 32>(p, w, logit_out, s);
+    if (p.r_tile == 16) return launch_keys_rt<D, 16>(p, w, logit_out, s);
+    return launch_keys_rt<D, 8>(p, w, logit_out, s);
 }
 
 }  // namespace

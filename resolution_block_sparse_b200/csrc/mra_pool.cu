@@ -43,65 +43,38 @@ struct Vec16<float> {
     }
 };
 
-constexpr int kPoolWarps = 4;
+constexpr int kPoolWarps = 8;
+constexpr int kUnitsPerWarp = 1;   // (tensor, head, block) units per warp
 
+// Masked mean of one 32-row block held in registers (raw: the warp's 16-byte
+// slices) and the valid-token count; lanes < kCpr store the D means.
 template <typename T, int D>
-__global__ void __launch_bounds__(kPoolWarps * 32)
-pool_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-            const float *__restrict__ mask, int H, int N, int nbr, int BH, int ntensors,
-            float *__restrict__ pooled, int *__restrict__ cnt_out) {
-    constexpr int kEpc = Vec16<T>::kElems;          // elements per 16-byte slice
-    constexpr int kCpr = D / kEpc;                  // slices per row
-    constexpr int kRpp = 32 / kCpr;                 // rows per warp pass
+__device__ __forceinline__ void reduce_block(const uint4 (&raw)[kBlock / (32 / (D / Vec16<T>::kElems))],
+                                             float mine, float *dst, int lane) {
+    constexpr int kEpc = Vec16<T>::kElems;
+    constexpr int kCpr = D / kEpc;
+    constexpr int kRpp = 32 / kCpr;
     constexpr int kPasses = kBlock / kRpp;
-    static_assert(kCpr >= 1 && kCpr <= 32 && 32 % kCpr == 0, "unsupported D");
-
-    const int lane = threadIdx.x & 31;
-    const long long gw = (long long)blockIdx.x * kPoolWarps + (threadIdx.x >> 5);
-    const long long total = (long long)ntensors * BH * nbr;
-    if (gw >= total) return;
-    const int blk = (int)(gw % nbr);
-    const int bh = (int)((gw / nbr) % BH);
-    const int t = (int)(gw / ((long long)nbr * BH));
-    const int b = bh / H;
-    const T *x = (t == 0) ? q : (t == 1 ? k : v);
-    const T *base = x + ((size_t)bh * N + (size_t)blk * kBlock) * D;
-    const float *mrow = mask ? mask + (size_t)b * N + (size_t)blk * kBlock : nullptr;
-
-    // valid-token count of the block
-    float mine = mrow ? mrow[lane] : 1.0f;
+    const int row0 = lane / kCpr;
     float c = mine;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-
-    const int slice = lane % kCpr;
-    const int row0 = lane / kCpr;
-    uint4 raw[kPasses];
-#pragma unroll
-    for (int p = 0; p < kPasses; ++p) {
-        const int row = p * kRpp + row0;
-        raw[p] = __ldg(reinterpret_cast<const uint4 *>(base + (size_t)row * D) + slice);
-    }
     float acc[kEpc];
 #pragma unroll
     for (int e = 0; e < kEpc; ++e) acc[e] = 0.0f;
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
-        const int row = p * kRpp + row0;
-        const float m = mrow ? __shfl_sync(0xffffffffu, mine, row) : 1.0f;
+        const float m = __shfl_sync(0xffffffffu, mine, p * kRpp + row0);
         float f[kEpc];
         Vec16<T>::to_float(raw[p], f);
 #pragma unroll
         for (int e = 0; e < kEpc; ++e) acc[e] = fmaf(m, f[e], acc[e]);
     }
-    // fold the lanes that hold the same slice
 #pragma unroll
     for (int o = kCpr; o < 32; o <<= 1)
 #pragma unroll
         for (int e = 0; e < kEpc; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
-
     if (lane < kCpr) {
-        float *dst = pooled + (size_t)t * BH * nbr * D + ((size_t)bh * nbr + blk) * D + lane * kEpc;
 #pragma unroll
         for (int e = 0; e < kEpc; e += 4) {
             float4 o4;
@@ -109,21 +82,88 @@ pool_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restric
             o4.y = c > 0.0f ? acc[e + 1] / c : 0.0f;
             o4.z = c > 0.0f ? acc[e + 2] / c : 0.0f;
             o4.w = c > 0.0f ? acc[e + 3] / c : 0.0f;
-            *reinterpret_cast<float4 *>(dst + e) = o4;
+            *reinterpret_cast<float4 *>(dst + lane * kEpc + e) = o4;
         }
     }
-    if (t == 0 && (bh % H) == 0 && lane == 0) cnt_out[(size_t)b * nbr + blk] = (int)c;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kPoolWarps * 32)
+pool_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+            const float *__restrict__ mask, int H, int N, int nbr, int BH, int ntensors,
+            float *__restrict__ pooled, int *__restrict__ cnt_out, uint4 *__restrict__ zero,
+            long long zero_n16) {
+    constexpr int kEpc = Vec16<T>::kElems;          // elements per 16-byte slice
+    constexpr int kCpr = D / kEpc;                  // slices per row
+    constexpr int kRpp = 32 / kCpr;                 // rows per warp pass
+    constexpr int kPasses = kBlock / kRpp;
+    static_assert(kCpr >= 1 && kCpr <= 32 && 32 % kCpr == 0, "unsupported D");
+
+    // clear the per-call counters and histograms of the later phases
+    const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long gs = (long long)gridDim.x * blockDim.x;
+    for (long long i = gt; i < zero_n16; i += gs) zero[i] = make_uint4(0u, 0u, 0u, 0u);
+
+    const int lane = threadIdx.x & 31;
+    const long long total = (long long)ntensors * BH * nbr;
+    const long long u0 = ((long long)blockIdx.x * kPoolWarps + (threadIdx.x >> 5)) * kUnitsPerWarp;
+    const int slice = lane % kCpr;
+    const int row0 = lane / kCpr;
+    uint4 raw[kUnitsPerWarp][kPasses];
+    float mine[kUnitsPerWarp];
+#pragma unroll
+    for (int u = 0; u < kUnitsPerWarp; ++u) {
+        const long long gw = u0 + u;
+        mine[u] = 0.0f;
+        if (gw >= total) continue;
+        const int blk = (int)(gw % nbr);
+        const int bh = (int)((gw / nbr) % BH);
+        const int t = (int)(gw / ((long long)nbr * BH));
+        const T *x = (t == 0) ? q : (t == 1 ? k : v);
+        const T *base = x + ((size_t)bh * N + (size_t)blk * kBlock) * D;
+        const float *mrow = mask ? mask + (size_t)(bh / H) * N + (size_t)blk * kBlock : nullptr;
+        mine[u] = mrow ? mrow[lane] : 1.0f;
+#pragma unroll
+        for (int p = 0; p < kPasses; ++p)
+            raw[u][p] = __ldg(reinterpret_cast<const uint4 *>(base + (size_t)(p * kRpp + row0) * D) + slice);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnitsPerWarp; ++u) {
+        const long long gw = u0 + u;
+        if (gw >= total) continue;
+        const int blk = (int)(gw % nbr);
+        const int bh = (int)((gw / nbr) % BH);
+        const int t = (int)(gw / ((long long)nbr * BH));
+        float *dst = pooled + (size_t)t * BH * nbr * D + ((size_t)bh * nbr + blk) * D;
+        reduce_block<T, D>(raw[u], mine[u], dst, lane);
+    }
+    // block valid-token counts (one writer per (batch, block))
+#pragma unroll
+    for (int u = 0; u < kUnitsPerWarp; ++u) {
+        const long long gw = u0 + u;
+        if (gw >= total) continue;
+        const int blk = (int)(gw % nbr);
+        const int bh = (int)((gw / nbr) % BH);
+        const int t = (int)(gw / ((long long)nbr * BH));
+        if (t != 0 || (bh % H) != 0) continue;
+        float c = mine[u];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (lane == 0) cnt_out[(size_t)(bh / H) * nbr + blk] = (int)c;
+    }
 }
 
 template <typename T, int D>
 cudaError_t launch_typed(const Problem &p, const Workspace &w, const void *q, const void *k,
                          const void *v, const float *mask, cudaStream_t s) {
     const int ntensors = (p.mode == 0) ? 3 : 2;
-    const long long warps = (long long)ntensors * p.BH * p.nbr;
-    const long long grid = (warps + kPoolWarps - 1) / kPoolWarps;
+    const long long units = (long long)ntensors * p.BH * p.nbr;
+    const long long per_cta = (long long)kPoolWarps * kUnitsPerWarp;
+    const long long grid = (units + per_cta - 1) / per_cta;
     pool_kernel<T, D><<<(unsigned)grid, kPoolWarps * 32, 0, s>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), mask,
-        p.H, p.N, p.nbr, p.BH, ntensors, w.pooled, w.cnt);
+        p.H, p.N, p.nbr, p.BH, ntensors, w.pooled, w.cnt, static_cast<uint4 *>(w.zero_base),
+        (long long)(w.zero_bytes / 16));
     return cudaGetLastError();
 }
 

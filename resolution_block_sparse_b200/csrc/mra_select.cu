@@ -40,9 +40,20 @@ radix_pass_kernel(const unsigned long long *__restrict__ keys, long long nbr2, l
     const long long start = (long long)blockIdx.x * chunk;
     const long long end = min(start + chunk, nbr2);
     const unsigned long long *kb = keys + (size_t)bh * nbr2;
-    for (long long i = start + t; i < end; i += kThreads) {
-        const unsigned long long key = kb[i];
-        if ((key >> hi) == want) atomicAdd(&h[(unsigned)(key >> shift) & dmask], 1u);
+    constexpr int kUnroll = 4;
+    for (long long i0 = start + (t & ~31) * kUnroll; i0 < end; i0 += (long long)kThreads * kUnroll) {
+        unsigned long long kv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const long long i = i0 + u * 32 + (t & 31);
+            kv[u] = i < end ? __ldcg(kb + i) : ~0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const long long i = i0 + u * 32 + (t & 31);
+            const bool act = i < end && (kv[u] >> hi) == want;
+            warp_hist_add(h, (unsigned)(kv[u] >> shift) & dmask, act);
+        }
     }
     __syncthreads();
     unsigned int *gh = hist + ((size_t)bh * 3 + pass) * kHistBins;
@@ -223,6 +234,200 @@ cols_kernel(const unsigned long long *__restrict__ keys, const SelState *__restr
     }
 }
 
+constexpr int kSmallThreads = 1024;
+
+// Whole selection of one (batch, head) in one CTA, for maps of at most
+// kSmallMaxKeys keys (nbr <= 128): the keys stay in shared memory for the
+// two remaining radix passes, the per-row counts, the row scan, the work
+// list and the column lists.
+__global__ void __launch_bounds__(kSmallThreads)
+select_small_kernel(const unsigned long long *__restrict__ keys, SelState *__restrict__ state,
+                    int nbr, int k, int cap, int *__restrict__ cols, int32_t *__restrict__ sel_out,
+                    unsigned int *__restrict__ bitmap, int wpr, WorkItem *__restrict__ items,
+                    int *__restrict__ head_items, unsigned int *__restrict__ status) {
+    extern __shared__ __align__(16) unsigned long long sk[];   // [nbr * nbr]
+    __shared__ unsigned int h[kHistBins];
+    __shared__ unsigned int s_tmp[kSmallThreads];
+    __shared__ int s_gt[kSmallMaxRows], s_eq[kSmallMaxRows], s_sel[kSmallMaxRows];
+    __shared__ int s_start[kSmallMaxRows], s_take[kSmallMaxRows], s_item[kSmallMaxRows];
+    __shared__ int s_bin, s_total_sel, s_total_items;
+    __shared__ unsigned int s_need;
+    const int bh = blockIdx.x;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int n = nbr * nbr;
+    const unsigned long long *kb = keys + (size_t)bh * n;
+    {
+        // all (up to 16) loads of this thread in flight before the stores
+        constexpr int kL = kSmallMaxKeys / kSmallThreads;
+        unsigned long long v[kL];
+#pragma unroll
+        for (int u = 0; u < kL; ++u) {
+            const int i = t + u * kSmallThreads;
+            v[u] = i < n ? __ldcg(kb + i) : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < kL; ++u) {
+            const int i = t + u * kSmallThreads;
+            if (i < n) sk[i] = v[u];
+        }
+    }
+    const SelState st = state[bh];
+    unsigned long long prefix = st.prefix;
+    unsigned int need = st.need;
+    __syncthreads();
+
+    for (int pass = 1; pass <= 2; ++pass) {
+        const int shift = (pass == 1) ? kHist2Bits : 0;
+        const int bits = (pass == 1) ? kHist1Bits : kHist2Bits;
+        const int hi = shift + bits;
+        const unsigned long long want = prefix >> hi;
+        const unsigned int dmask = (1u << bits) - 1u;
+        for (int i = t; i < (1 << bits); i += kSmallThreads) h[i] = 0u;
+        __syncthreads();
+        for (int i0 = (t & ~31); i0 < n; i0 += kSmallThreads) {
+            const int i = i0 + lane;
+            const unsigned long long key = i < n ? sk[i] : ~0ull;
+            warp_hist_add(h, (unsigned)(key >> shift) & dmask, i < n && (key >> hi) == want);
+        }
+        __syncthreads();
+        find_bucket<kSmallThreads>([](int i) { return h[i]; }, 1 << bits, need, s_tmp, &s_bin,
+                                   &s_need);
+        prefix |= (unsigned long long)s_bin << shift;
+        need = s_need;
+        __syncthreads();
+    }
+    const unsigned long long T = prefix;
+    if (t == 0) {
+        SelState ns;
+        ns.prefix = T;
+        ns.need = need;
+        ns.pad = 0;
+        state[bh] = ns;
+    }
+
+    // keys above / equal to the threshold, per block row
+    for (int r = warp; r < nbr; r += kSmallThreads / 32) {
+        int g = 0, e = 0;
+        for (int c = lane; c < nbr; c += 32) {
+            const unsigned long long key = sk[r * nbr + c];
+            g += key > T;
+            e += key == T;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            e += __shfl_xor_sync(0xffffffffu, e, o);
+        }
+        if (lane == 0) {
+            s_gt[r] = g;
+            s_eq[r] = e;
+        }
+    }
+    __syncthreads();
+    // row scan on warp 0: rows 4*lane .. 4*lane+3
+    if (warp == 0) {
+        int eqv[4], sel[4], itm[4];
+        int eq_local = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int r = 4 * lane + j;
+            eqv[j] = r < nbr ? s_eq[r] : 0;
+            eq_local += eqv[j];
+        }
+        int x = eq_local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        int eq_before = x - eq_local;
+        int sel_local = 0, it_local = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int r = 4 * lane + j;
+            int take = (int)need - eq_before;
+            take = take < 0 ? 0 : (take > eqv[j] ? eqv[j] : take);
+            sel[j] = r < nbr ? s_gt[r] + take : 0;
+            itm[j] = r < nbr ? (sel[j] > 0 ? (sel[j] + kChunk - 1) / kChunk : 1) : 0;
+            if (r < nbr) s_take[r] = take;
+            eq_before += eqv[j];
+            sel_local += sel[j];
+            it_local += itm[j];
+        }
+        int xs = sel_local, xi = it_local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int ys = __shfl_up_sync(0xffffffffu, xs, o);
+            const int yi = __shfl_up_sync(0xffffffffu, xi, o);
+            if (lane >= o) {
+                xs += ys;
+                xi += yi;
+            }
+        }
+        int sb = xs - sel_local, ib = xi - it_local;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int r = 4 * lane + j;
+            if (r < nbr) {
+                s_sel[r] = sel[j];
+                s_start[r] = sb;
+                s_item[r] = ib;
+            }
+            sb += sel[j];
+            ib += itm[j];
+        }
+        if (lane == 31) {
+            s_total_sel = xs;
+            s_total_items = xi;
+        }
+    }
+    __syncthreads();
+    const bool ok = (s_total_sel == k && s_total_items <= cap);
+    if (t == 0) {
+        head_items[bh] = ok ? s_total_items : 0;
+        if (!ok) atomicOr(status, kDevCount);
+    }
+    if (!ok) return;
+    // work items: one thread per row
+    for (int r = t; r < nbr; r += kSmallThreads) {
+        const int sel = s_sel[r];
+        const int nit = sel > 0 ? (sel + kChunk - 1) / kChunk : 1;
+        const int rs = bh * k + s_start[r];
+        for (int j = 0; j < nit; ++j) {
+            WorkItem w;
+            w.row = bh * nbr + r;
+            w.col_start = rs + j * kChunk;
+            w.ncols = max(0, min(kChunk, sel - j * kChunk));
+            w.chunk_info = j | (nit << 16);
+            items[(size_t)bh * cap + s_item[r] + j] = w;
+        }
+    }
+    // column lists: one warp per row, ascending columns
+    const unsigned int lt_mask = (1u << lane) - 1u;
+    for (int r = warp; r < nbr; r += kSmallThreads / 32) {
+        const int rs = bh * k + s_start[r];
+        const int take = s_take[r];
+        int eq_seen = 0, sel_seen = 0;
+        for (int c0 = 0; c0 < nbr; c0 += 32) {
+            const int c = c0 + lane;
+            const unsigned long long key = c < nbr ? sk[r * nbr + c] : 0ull;
+            const bool is_gt = c < nbr && key > T;
+            const bool is_eq = c < nbr && key == T;
+            const unsigned int eqb = __ballot_sync(0xffffffffu, is_eq);
+            const bool sel = is_gt || (is_eq && eq_seen + __popc(eqb & lt_mask) < take);
+            const unsigned int sb = __ballot_sync(0xffffffffu, sel);
+            if (sel) {
+                const int pos = rs + sel_seen + __popc(sb & lt_mask);
+                cols[pos] = c;
+                if (sel_out) sel_out[pos] = r * nbr + c;
+            }
+            if (bitmap && lane == 0) bitmap[((size_t)bh * nbr + r) * wpr + (c0 >> 5)] = sb;
+            eq_seen += __popc(eqb);
+            sel_seen += __popc(sb);
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_radix_pass(const Problem &p, const Workspace &w, int pass, cudaStream_t s) {
@@ -246,6 +451,18 @@ cudaError_t launch_row_scan(const Problem &p, const Workspace &w, cudaStream_t s
     row_scan_kernel<<<p.BH, kScanThreads, 0, s>>>(w.gt, w.eq, w.state, p.nbr, p.k, p.cap,
                                                   w.row_start, w.take_eq, w.items, w.head_items,
                                                   w.status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *sel_out,
+                                cudaStream_t s) {
+    const size_t smem = sizeof(unsigned long long) * (size_t)p.nbr2;
+    cudaError_t e = cudaFuncSetAttribute(select_small_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    select_small_kernel<<<p.BH, kSmallThreads, smem, s>>>(
+        w.keys, w.state, p.nbr, p.k, p.cap, w.cols, sel_out, p.mode == 0 ? w.bitmap : nullptr,
+        w.words_per_row, w.items, w.head_items, w.status);
     return cudaGetLastError();
 }
 

@@ -1,41 +1,56 @@
-// mra_select_common.cuh - device helper shared by the kernels that locate
-// the bucket of the k-th largest selection key (radix select over per-head
-// histograms, page "深入解析 Transformers 中的 MRA 模型", step two: global top-k).
+// mra_select_common.cuh - device helpers shared by the kernels of the global
+// top-k (radix select over per-head histograms; page "深入解析 Transformers 中
+// 的 MRA 模型", section "源码级原理", step two: global top-k, k = num_block).
 #pragma once
 
 #include "mra_internal.cuh"
 
 namespace mra {
 
-// Finds, in the global histogram gh[0..nbins) of one head (read through L2),
-// the bucket that holds the need-th largest element counted from the top.
-// Runs on all 256 threads of the block; writes the bucket and the count still
-// needed inside it to *out_bin / *out_need (shared memory).
-static __device__ __noinline__ void find_bucket_256(const unsigned int *gh, int nbins, unsigned int need,
-                                unsigned int *s_tmp /* >= 256 */, int *out_bin,
-                                unsigned int *out_need) {
+// Histogram increment aggregated over the lanes of a warp that carry the same
+// bin: one shared-memory atomic per distinct bin instead of one per lane (the
+// keys of one row concentrate in few buckets).  Must be called by all 32
+// lanes; inactive lanes pass active = false.
+static __device__ __forceinline__ void warp_hist_add(unsigned int *h, unsigned int bin,
+                                                     bool active) {
+    if (!__any_sync(0xffffffffu, active)) return;   // warp-uniform early exit
+    const unsigned int key = active ? bin : 0xffffffffu;
+    const unsigned int peers = __match_any_sync(0xffffffffu, key);
+    const int leader = __ffs(peers) - 1;
+    if (active && (int)(threadIdx.x & 31) == leader) atomicAdd(&h[bin], (unsigned)__popc(peers));
+}
+
+// Finds, in the histogram h[0..nbins) of one head, the bucket that holds the
+// need-th largest element counted from the top.  Runs on all NT threads of
+// the block; `load` reads one bin (global memory through L2, or shared).
+// Writes the bucket and the count still needed inside it to *out_bin /
+// *out_need (shared memory).
+template <int NT, typename Load>
+static __device__ __forceinline__ void find_bucket(Load load, int nbins, unsigned int need,
+                                                   unsigned int *s_tmp /* >= NT */,
+                                                   int *out_bin, unsigned int *out_need) {
     const int t = threadIdx.x;
-    const int per = nbins / 256;
+    const int per = nbins / NT;
     if (t == 0) {  // defined result even if no bucket qualifies (cannot happen when need <= total)
         *out_bin = 0;
         *out_need = 1;
     }
     unsigned int local = 0;
-    for (int i = 0; i < per; ++i) local += __ldcg(gh + t * per + i);
+    for (int i = 0; i < per; ++i) local += load(t * per + i);
     s_tmp[t] = local;
     __syncthreads();
-    // inclusive suffix sum over threads (Hillis-Steele, 8 steps)
-    for (int off = 1; off < 256; off <<= 1) {
-        unsigned int add = (t + off < 256) ? s_tmp[t + off] : 0u;
+    // inclusive suffix sum over threads (Hillis-Steele)
+    for (int off = 1; off < NT; off <<= 1) {
+        const unsigned int add = (t + off < NT) ? s_tmp[t + off] : 0u;
         __syncthreads();
         s_tmp[t] += add;
         __syncthreads();
     }
-    const unsigned int above = (t + 1 < 256) ? s_tmp[t + 1] : 0u;  // bins above my range
+    const unsigned int above = (t + 1 < NT) ? s_tmp[t + 1] : 0u;  // bins above my range
     if (above < need && need <= above + local) {
         unsigned int cum = above;
         for (int i = per - 1; i >= 0; --i) {
-            unsigned int hb = __ldcg(gh + t * per + i);
+            const unsigned int hb = load(t * per + i);
             if (cum + hb >= need) {
                 *out_bin = t * per + i;
                 *out_need = need - cum;
@@ -45,6 +60,13 @@ static __device__ __noinline__ void find_bucket_256(const unsigned int *gh, int 
         }
     }
     __syncthreads();
+}
+
+// The global-memory form used by the multi-CTA passes (histogram in L2).
+static __device__ __forceinline__ void find_bucket_256(const unsigned int *gh, int nbins,
+                                                       unsigned int need, unsigned int *s_tmp,
+                                                       int *out_bin, unsigned int *out_need) {
+    find_bucket<256>([gh](int i) { return __ldcg(gh + i); }, nbins, need, s_tmp, out_bin, out_need);
 }
 
 }  // namespace mra

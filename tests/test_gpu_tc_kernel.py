@@ -1,0 +1,53 @@
+"""Parity of the tcgen05/TMA attention kernel (selected with MRA_ATTN_IMPL=tc).
+
+The kernel choice is read once per process, so each case runs in a child
+process with the variable set; the child compares the CUDA output with the
+oracle on the same seeded inputs and reports the error.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = r'''
+import json, sys
+sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + "/tests")
+import numpy as np, torch
+import mra_testlib as tl
+from resolution_block_sparse_b200.workloads import WORKLOADS, make_inputs, random_inputs
+case = json.loads(sys.argv[2])
+if "workload" in case:
+    w = WORKLOADS[case["workload"]]
+    inputs = make_inputs(w)
+    kw = dict(block_per_row=w.block_per_row, approx_mode=w.approx_mode, first_n=w.first_n, diag_n=w.diag_n)
+else:
+    inputs = random_inputs(case["B"], case["H"], case["N"], 64, dtype=torch.bfloat16, seed=case["seed"],
+                           pad_tokens=case.get("pad"), v_scale=1.0)
+    kw = dict(block_per_row=case["bpr"], approx_mode=case["mode"], first_n=case["f"], diag_n=case["g"])
+gpu = tl.run_gpu(inputs, **kw)
+ora = tl.run_oracle(inputs, **kw)
+stats = tl.compare(inputs, gpu, ora)
+print("RESULT " + json.dumps(stats))
+'''
+
+CASES = [
+    {"workload": 4},
+    {"workload": 2},
+    {"workload": 5},
+    {"B": 1, "H": 2, "N": 1024, "bpr": 4, "mode": 0, "f": 1, "g": 1, "seed": 3, "pad": [100]},
+    {"B": 1, "H": 2, "N": 2048, "bpr": 40, "mode": 1, "f": 1, "g": 1, "seed": 4},
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[json.dumps(c, sort_keys=True) for c in CASES])
+def test_tc_kernel_parity(case):
+    env = dict(os.environ, MRA_ATTN_IMPL="tc")
+    r = subprocess.run([sys.executable, "-c", CHILD, ROOT, json.dumps(case)], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-3000:]
+    assert "RESULT" in r.stdout
