@@ -233,12 +233,16 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
         MRA_TRY(launch_pool(p, w, q, k, v, mask, s));
         ++launches;
     }
-    {
-        PhaseScope ps("lowres_keys", s, prof);
-        MRA_TRY(launch_lowres_keys(p, w, logit_out, s));
+    if (lowres_select_fused_supported(p)) {
+        PhaseScope ps("lowres_select", s, prof);
+        MRA_TRY(launch_lowres_select_fused(p, w, logit_out, sel_out, s));
         ++launches;
-    }
-    {
+    } else {
+        {
+            PhaseScope ps("lowres_keys", s, prof);
+            MRA_TRY(launch_lowres_keys(p, w, logit_out, s));
+            ++launches;
+        }
         PhaseScope ps("select", s, prof);
         if (p.nbr <= kSmallMaxRows) {
             MRA_TRY(launch_select_small(p, w, sel_out, s));

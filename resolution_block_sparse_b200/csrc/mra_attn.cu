@@ -60,6 +60,12 @@ __device__ __forceinline__ void mma16816(float *c, const unsigned *a, unsigned b
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// 2^x on the special-function unit (ex2.approx.ftz, about 2 ulp)
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ unsigned pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<unsigned *>(&v);
@@ -102,13 +108,17 @@ struct AttnArgs {
 constexpr int kBf16Threads = 64;
 
 template <int D>
-__global__ void __launch_bounds__(kBf16Threads)
+__global__ void __launch_bounds__(kBf16Threads, 11)
 attn_bf16_kernel(const AttnArgs a) {
     constexpr int kTile = 32 * D;
     __shared__ __align__(128) __nv_bfloat16 sQ[kTile];
-    __shared__ __align__(128) __nv_bfloat16 sKV[2][2][kTile];  // [buffer][K or V]
-    __shared__ float sKm[2][32];                                // key mask per buffer
-    __shared__ MergeSmem sm;
+    // K/V double buffer; after the block loop the same bytes hold the output
+    // staging or, for split rows, the partial and the merge scratch
+    constexpr size_t kKvBytes = sizeof(__nv_bfloat16) * 4 * kTile;
+    constexpr size_t kMergeBytes = sizeof(float) * 32 * (D + 2) + sizeof(MergeSmem);
+    __shared__ __align__(128) unsigned char kv_raw[kKvBytes > kMergeBytes ? kKvBytes : kMergeBytes];
+    auto sKV = reinterpret_cast<__nv_bfloat16(*)[2][kTile]>(kv_raw);   // [buffer][K or V]
+    __shared__ float sKm[2][32];                                        // key mask per buffer
     __shared__ int s_last;
 
     const int slot = blockIdx.x;
@@ -186,16 +196,19 @@ attn_bf16_kernel(const AttnArgs a) {
                 mma16816(s[nt], qf[ks + 1], b2, b3);
             }
         }
-        // scale to log2 units, mask padded keys, online max / sum
+        // online max / sum; scores stay raw (the scale is folded into exp2)
+        if (mrow) {
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int c = nt * 8 + tq * 2;
+                const bool v0 = sKm[buf][c] > 0.0f, v1 = sKm[buf][c + 1] > 0.0f;
+                if (!v0) s[nt][0] = s[nt][2] = -INFINITY;
+                if (!v1) s[nt][1] = s[nt][3] = -INFINITY;
+            }
+        }
         float mx_a = -INFINITY, mx_b = -INFINITY;
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
-            const int c = nt * 8 + tq * 2;
-            const bool v0 = sKm[buf][c] > 0.0f, v1 = sKm[buf][c + 1] > 0.0f;
-            s[nt][0] = v0 ? s[nt][0] * a.scale_log2 : -INFINITY;
-            s[nt][1] = v1 ? s[nt][1] * a.scale_log2 : -INFINITY;
-            s[nt][2] = v0 ? s[nt][2] * a.scale_log2 : -INFINITY;
-            s[nt][3] = v1 ? s[nt][3] * a.scale_log2 : -INFINITY;
             mx_a = fmaxf(mx_a, fmaxf(s[nt][0], s[nt][1]));
             mx_b = fmaxf(mx_b, fmaxf(s[nt][2], s[nt][3]));
         }
@@ -204,30 +217,33 @@ attn_bf16_kernel(const AttnArgs a) {
             mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
             mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
         }
-        const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-        const float ref_a = (mn_a == -INFINITY) ? 0.0f : mn_a;
-        const float ref_b = (mn_b == -INFINITY) ? 0.0f : mn_b;
-        const float al_a = exp2f(m_a - ref_a), al_b = exp2f(m_b - ref_b);
-        m_a = mn_a;
-        m_b = mn_b;
-        float ps_a = 0.0f, ps_b = 0.0f;
+        // running maxima in log2 units
+        const float mn_a = fmaxf(m_a, mx_a * a.scale_log2), mn_b = fmaxf(m_b, mx_b * a.scale_log2);
+        if (__any_sync(0xffffffffu, mn_a != m_a || mn_b != m_b)) {
+            const float al_a = (m_a == -INFINITY) ? 0.0f : fast_exp2(m_a - mn_a);
+            const float al_b = (m_b == -INFINITY) ? 0.0f : fast_exp2(m_b - mn_b);
+            l_a *= al_a;
+            l_b *= al_b;
+#pragma unroll
+            for (int nd = 0; nd < D / 8; ++nd) {
+                o[nd][0] *= al_a;
+                o[nd][1] *= al_a;
+                o[nd][2] *= al_b;
+                o[nd][3] *= al_b;
+            }
+            m_a = mn_a;
+            m_b = mn_b;
+        }
+        const float ref_a = (m_a == -INFINITY) ? 0.0f : m_a;
+        const float ref_b = (m_b == -INFINITY) ? 0.0f : m_b;
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
-            s[nt][0] = exp2f(s[nt][0] - ref_a);
-            s[nt][1] = exp2f(s[nt][1] - ref_a);
-            s[nt][2] = exp2f(s[nt][2] - ref_b);
-            s[nt][3] = exp2f(s[nt][3] - ref_b);
-            ps_a += s[nt][0] + s[nt][1];
-            ps_b += s[nt][2] + s[nt][3];
-        }
-        l_a = l_a * al_a + ps_a;
-        l_b = l_b * al_b + ps_b;
-#pragma unroll
-        for (int nd = 0; nd < D / 8; ++nd) {
-            o[nd][0] *= al_a;
-            o[nd][1] *= al_a;
-            o[nd][2] *= al_b;
-            o[nd][3] *= al_b;
+            s[nt][0] = fast_exp2(fmaf(s[nt][0], a.scale_log2, -ref_a));
+            s[nt][1] = fast_exp2(fmaf(s[nt][1], a.scale_log2, -ref_a));
+            s[nt][2] = fast_exp2(fmaf(s[nt][2], a.scale_log2, -ref_b));
+            s[nt][3] = fast_exp2(fmaf(s[nt][3], a.scale_log2, -ref_b));
+            l_a += s[nt][0] + s[nt][1];
+            l_b += s[nt][2] + s[nt][3];
         }
         // O += P V
 #pragma unroll
@@ -256,11 +272,53 @@ attn_bf16_kernel(const AttnArgs a) {
         l_a += __shfl_xor_sync(0xffffffffu, l_a, off);
         l_b += __shfl_xor_sync(0xffffffffu, l_b, off);
     }
-    // stage (m, l, O) in shared memory, reusing the K/V buffers
-    __syncthreads();
-    float *stage = reinterpret_cast<float *>(&sKV[0][0][0]);
-    static_assert(sizeof(sKV) >= sizeof(float) * 32 * (D + 2), "stage does not fit");
+    __nv_bfloat16 *out_blk = static_cast<__nv_bfloat16 *>(a.out) + head_off + (size_t)r * kTile;
     const int ra = warp * 16 + g, rb = ra + 8;
+    __syncthreads();   // every warp is done with the K/V buffers
+    if (nchunks == 1) {
+        // whole row in this item: combine with the low-resolution part and
+        // write the final output straight from the accumulators
+        const float m_lo2 = a.full ? a.mlo[it.row] * kLog2e : 0.0f;
+        const float l_lo = a.full ? a.llo[it.row] : 0.0f;
+        const bool lo = a.full && l_lo > 0.0f;
+        float fa_a, fb_a, fa_b, fb_b;   // output = O * fa + O_lo * fb, per row
+        {
+            auto factors = [&](float m, float l, int row, float &fa, float &fb) {
+                fa = fb = 0.0f;
+                const bool hi = l > 0.0f;
+                float M = hi ? m : -INFINITY;
+                if (lo) M = fmaxf(M, m_lo2);
+                if (M == -INFINITY || (mrow && !(mrow[r * 32 + row] > 0.0f))) return;
+                const float al = hi ? fast_exp2(m - M) : 0.0f;
+                const float be = lo ? fast_exp2(m_lo2 - M) : 0.0f;
+                const float den = al * l + be * l_lo;
+                if (den > 0.0f) {
+                    fa = al / den;
+                    fb = be / den;
+                }
+            };
+            factors(m_a, l_a, ra, fa_a, fb_a);
+            factors(m_b, l_b, rb, fa_b, fb_b);
+        }
+        __nv_bfloat16 *ostage = &sKV[0][0][0];   // [32][D] bf16 staging
+#pragma unroll
+        for (int nd = 0; nd < D / 8; ++nd) {
+            const int d = nd * 8 + tq * 2;
+            float2 ol = make_float2(0.0f, 0.0f);
+            if (lo) ol = *reinterpret_cast<const float2 *>(a.olo + (size_t)it.row * D + d);
+            *reinterpret_cast<__nv_bfloat162 *>(ostage + ra * D + d) =
+                __floats2bfloat162_rn(fmaf(o[nd][0], fa_a, ol.x * fb_a), fmaf(o[nd][1], fa_a, ol.y * fb_a));
+            *reinterpret_cast<__nv_bfloat162 *>(ostage + rb * D + d) =
+                __floats2bfloat162_rn(fmaf(o[nd][2], fa_b, ol.x * fb_b), fmaf(o[nd][3], fa_b, ol.y * fb_b));
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = tid; e < kTile / 8; e += kBf16Threads)
+            reinterpret_cast<uint4 *>(out_blk)[e] = reinterpret_cast<const uint4 *>(ostage)[e];
+        return;
+    }
+    // row split across work items: (m, l, O) partial, merged by the last one
+    float *stage = reinterpret_cast<float *>(&sKV[0][0][0]);
     if (tq == 0) {
         stage[ra] = m_a;
         stage[rb] = m_b;
@@ -276,7 +334,7 @@ attn_bf16_kernel(const AttnArgs a) {
         stage[64 + rb * D + d + 1] = o[nd][3];
     }
     __syncthreads();
-    __nv_bfloat16 *out_blk = static_cast<__nv_bfloat16 *>(a.out) + head_off + (size_t)r * kTile;
+    MergeSmem &sm = *reinterpret_cast<MergeSmem *>(stage + 32 * (D + 2));
     finish_item<D, kBf16Threads, __nv_bfloat16, SyncAll>(stage, slot, chunk, nchunks, it.row, a.full, a.mlo,
                                                 a.olo, a.llo, a.partial, a.row_arrive,
                                                 mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);

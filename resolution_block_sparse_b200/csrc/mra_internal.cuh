@@ -111,6 +111,11 @@ cudaError_t launch_radix_pass(const Problem &p, const Workspace &w, int pass, cu
 cudaError_t launch_row_counts(const Problem &p, const Workspace &w, cudaStream_t s);
 cudaError_t launch_row_scan(const Problem &p, const Workspace &w, cudaStream_t s);
 cudaError_t launch_cols(const Problem &p, const Workspace &w, int32_t *sel_out, cudaStream_t s);
+// Low-resolution logits, keys and the whole selection in one kernel: one
+// thread-block cluster per head (nbr <= 128).
+bool lowres_select_fused_supported(const Problem &p);
+cudaError_t launch_lowres_select_fused(const Problem &p, const Workspace &w, float *logit_out,
+                                       int32_t *sel_out, cudaStream_t s);
 // Whole selection (radix passes 2-3, counts, scan, work list, cols) in one CTA
 // per head, for nbr <= kSmallMaxRows.
 cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *sel_out,
