@@ -27,7 +27,7 @@ int validate_sizes(int B, int H, int N, int D, int bpr, int mode, int first_n, i
     const long long BH = (long long)B * H;
     if (BH > 65535) return MRA_ERR_UNSUPPORTED;
     const long long kk = std::min<long long>((long long)nbr * bpr, (long long)nbr * nbr);
-    if (BH * kk > 0x7fffffffLL || BH * ((long long)nbr + kk / kChunk) > 0x7fffffffLL)
+    if (BH * kk > 0x7fffffffLL || BH * ((long long)nbr + kk / 8) > 0x7fffffffLL)
         return MRA_ERR_UNSUPPORTED;
     return MRA_OK;
 }
@@ -55,7 +55,12 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
     p.first_n = first_n;
     p.diag_n = diag_n;
     p.dtype = dtype;
-    p.cap = p.nbr + p.k / kChunk;
+    // work items of at most `chunk` blocks: short items keep the critical path
+    // of the long (prior) rows short when rows hold few blocks on average;
+    // longer items amortise the split-row merge when rows are dense
+    const int per_row = (p.k + p.nbr - 1) / p.nbr;
+    p.chunk = per_row <= 4 ? 8 : (per_row <= 16 ? 16 : kChunk);
+    p.cap = p.nbr + p.k / p.chunk;
     // low-res rows per CTA: at most 64 KB of logits per CTA, and enough CTAs
     // to cover the SMs twice when the problem allows
     // low-res rows per CTA: the logits of a CTA's rows stay in shared memory

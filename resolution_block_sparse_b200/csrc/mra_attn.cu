@@ -9,7 +9,7 @@
 //                bringing both parts to a shared maximum; sparse mode divides
 //                the high-resolution output by its own normaliser.
 //
-// Work item = (batch*head, block row r, up to kChunk selected columns).  The
+// Work item = (batch*head, block row r, up to `chunk` selected columns).  The
 // row max and sum are kept online (flash style) over the item's columns.  An
 // item that covers its whole row writes the final output; the items of a longer
 // row write (max, sum, output) partials and the last one to finish (arrival
@@ -20,6 +20,7 @@
 // by cp.async.  fp32 kernel: FFMA only (no TF32).
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cstdlib>
 
 #include "mra_attn_common.cuh"
@@ -108,20 +109,27 @@ struct AttnArgs {
 constexpr int kBf16Threads = 64;
 
 template <int D>
-__global__ void __launch_bounds__(kBf16Threads, 11)
-attn_bf16_kernel(const AttnArgs a) {
-    constexpr int kTile = 32 * D;
-    __shared__ __align__(128) __nv_bfloat16 sQ[kTile];
+struct Bf16Smem {
+    static constexpr int kTile = 32 * D;
+    static constexpr size_t kKvBytes = sizeof(__nv_bfloat16) * 4 * kTile;
+    static constexpr size_t kMergeBytes = sizeof(float) * 32 * (D + 2) + sizeof(MergeSmem);
+    __nv_bfloat16 q[kTile];
     // K/V double buffer; after the block loop the same bytes hold the output
     // staging or, for split rows, the partial and the merge scratch
-    constexpr size_t kKvBytes = sizeof(__nv_bfloat16) * 4 * kTile;
-    constexpr size_t kMergeBytes = sizeof(float) * 32 * (D + 2) + sizeof(MergeSmem);
-    __shared__ __align__(128) unsigned char kv_raw[kKvBytes > kMergeBytes ? kKvBytes : kMergeBytes];
-    auto sKV = reinterpret_cast<__nv_bfloat16(*)[2][kTile]>(kv_raw);   // [buffer][K or V]
-    __shared__ float sKm[2][32];                                        // key mask per buffer
-    __shared__ int s_last;
+    alignas(128) unsigned char kv_raw[kKvBytes > kMergeBytes ? kKvBytes : kMergeBytes];
+    float km[2][32];   // key mask per buffer
+    int cols[kChunk];
+    int last;
+};
 
-    const int slot = blockIdx.x;
+// One work item (block row, chunk of selected columns) on a 64-thread CTA.
+template <int D>
+__device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<D> &sh) {
+    constexpr int kTile = 32 * D;
+    __nv_bfloat16 *sQ = sh.q;
+    auto sKV = reinterpret_cast<__nv_bfloat16(*)[2][kTile]>(sh.kv_raw);   // [buffer][K or V]
+    auto &sKm = sh.km;
+    int &s_last = sh.last;
     const int bh = slot / a.cap, local = slot % a.cap;
     if (local >= a.head_items[bh]) return;
     const WorkItem it = a.items[slot];
@@ -139,7 +147,7 @@ attn_bf16_kernel(const AttnArgs a) {
     load_tile_async<D, kBf16Threads>(sQ, qg + (size_t)r * kTile, tid);
     const int ncols = it.ncols;
     // the item's column list, read once (the loads below depend on it)
-    __shared__ int s_cols[kChunk];
+    int *s_cols = sh.cols;
     for (int j = tid; j < ncols; j += kBf16Threads) s_cols[j] = a.cols[it.col_start + j];
     __syncthreads();
     if (ncols > 0) {
@@ -340,6 +348,21 @@ attn_bf16_kernel(const AttnArgs a) {
                                                 mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
 }
 
+// Persistent: each CTA walks the work items with a grid stride, in the order
+// (item index within its head) major, head minor.  The long rows of every
+// head (the first-n prior rows) come first in their head's list, so they
+// start in the first wave instead of forming the tail.
+template <int D>
+__global__ void __launch_bounds__(kBf16Threads, 10)
+attn_bf16_kernel(const AttnArgs a, int total_slots, int heads) {
+    __shared__ __align__(128) Bf16Smem<D> sh;
+    for (int i = blockIdx.x; i < total_slots; i += gridDim.x) {
+        const int slot = (i % heads) * a.cap + i / heads;
+        bf16_item<D>(a, slot, sh);
+        __syncthreads();   // shared buffers are free for the next item
+    }
+}
+
 constexpr int kF32Threads = 128;
 
 // fp32: four threads per query row, each owning D/4 output dimensions.
@@ -460,8 +483,16 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
     const bool want_tc = impl && impl[0] == 't';
     if (want_tc && attention_tc_supported(p)) return launch_attention_tc(p, w, q, k, v, mask, out, s);
     if (p.dtype == 0) {
-        if (p.D == 64) attn_bf16_kernel<64><<<(unsigned)grid, kBf16Threads, 0, s>>>(a);
-        else attn_bf16_kernel<32><<<(unsigned)grid, kBf16Threads, 0, s>>>(a);
+        static int sms = 0;
+        if (sms == 0) {
+            int dev = 0;
+            cudaGetDevice(&dev);
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (sms <= 0) sms = 148;
+        }
+        const long long pgrid = std::min<long long>(grid, 10LL * sms);
+        if (p.D == 64) attn_bf16_kernel<64><<<(unsigned)pgrid, kBf16Threads, 0, s>>>(a, (int)grid, p.BH);
+        else attn_bf16_kernel<32><<<(unsigned)pgrid, kBf16Threads, 0, s>>>(a, (int)grid, p.BH);
     } else {
         if (p.D == 64) attn_f32_kernel<64><<<(unsigned)grid, kF32Threads, 0, s>>>(a);
         else attn_f32_kernel<32><<<(unsigned)grid, kF32Threads, 0, s>>>(a);

@@ -188,16 +188,21 @@ struct TcArgs {
     unsigned int *status;
 };
 
-// The work items of this CTA, in order (the same walk for every role).
+// The work items of this CTA, in order (the same walk for every role):
+// grid stride over (item index within its head) major, head minor, so that
+// the long first-n rows of every head start first.
 struct ItemWalk {
-    int slot;
-    __device__ __forceinline__ explicit ItemWalk(int first) : slot(first) {}
+    int idx;
+    int slot;   // slot of the item returned by the last next()
+    __device__ __forceinline__ explicit ItemWalk(int first) : idx(first), slot(-1) {}
     __device__ __forceinline__ bool next(const TcArgs &a, WorkItem &it) {
-        for (; slot < a.total_slots; slot += gridDim.x) {
-            const int bh = slot / a.cap, local = slot % a.cap;
+        const int heads = a.total_slots / a.cap;
+        for (; idx < a.total_slots; idx += gridDim.x) {
+            const int bh = idx % heads, local = idx / heads;
             if (local < a.head_items[bh]) {
+                slot = bh * a.cap + local;
                 it = a.items[slot];
-                slot += gridDim.x;
+                idx += gridDim.x;
                 return true;
             }
         }
@@ -619,7 +624,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 // row split across work items: (max, sum, O) partial, the last
                 // item of the row merges (shared epilogue)
                 const size_t stride = (size_t)32 * (64 + 2);
-                const int slot = walk.slot - gridDim.x;
+                const int slot = walk.slot;
                 float *dst = a.partial + (size_t)slot * stride;
                 if (warp == 0) {
                     dst[lane] = m_hi;

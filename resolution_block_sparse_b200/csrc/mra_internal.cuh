@@ -21,7 +21,7 @@
 namespace mra {
 
 constexpr int kBlock = 32;            // tokens per block (fixed by the method)
-constexpr int kChunk = 32;            // max selected blocks per attention work item
+constexpr int kChunk = 32;            // upper bound of the blocks per attention work item
 constexpr int kHist0Bits = 11;        // radix digit widths over the 35-bit key
 constexpr int kHist1Bits = 12;
 constexpr int kHist2Bits = 12;
@@ -55,7 +55,8 @@ struct Problem {
     int mode;         // 0 full, 1 sparse
     int first_n, diag_n;
     int dtype;        // 0 bf16, 1 f32
-    int cap;          // work-item slots per head: nbr + k / kChunk
+    int chunk;        // selected blocks per attention work item (8, 16 or 32)
+    int cap;          // work-item slots per head: nbr + k / chunk
     int r_tile;       // rows per CTA of the low-res kernels
     int lowres_ctas;  // CTAs per head of the low-res key kernel
     int radix_ctas;   // CTAs per head of a radix pass

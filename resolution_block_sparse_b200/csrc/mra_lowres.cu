@@ -236,13 +236,19 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
     const int b = bh / H;
     const int r0 = blockIdx.x * R;
     const float *vh = vhat + (size_t)bh * nbr * D;
-    constexpr int kStride = kLowresThreads / D;   // rows per thread step
-    constexpr int kPer = R / kStride;             // rows per thread
-    const int d = t % D;
-    const int rb = t / D;
-    float acc[kPer], lsum[kPer];
+    // thread tile: kRpt rows x 4 head dims
+    constexpr int kDG = D / 4;                    // dim groups
+    constexpr int kRG = kLowresThreads / kDG;     // row groups
+    constexpr int kRpt = R / kRG;                 // rows per thread
+    static_assert(kRpt >= 1 && kRG * kRpt == R, "tile shape");
+    const int dg = t % kDG, rg = t / kDG;
+    float4 acc[kRpt];
+    float lsum[kRpt];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) acc[i] = lsum[i] = 0.0f;
+    for (int i = 0; i < kRpt; ++i) {
+        acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        lsum[i] = 0.0f;
+    }
 
     for (int ct = 0; ct < nbr; ct += kCt) {
         // issue every global load of this tile before touching shared memory
@@ -290,23 +296,26 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
             ws[r][c] = wv;
         }
         __syncthreads();
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const int r = rb + i * kStride;
 #pragma unroll 8
-            for (int c = 0; c < kCt; ++c) {
-                const float wv = ws[r][c];
-                acc[i] = fmaf(wv, vs[c][d], acc[i]);
+        for (int c = 0; c < kCt; ++c) {
+            const float4 v4 = *reinterpret_cast<const float4 *>(&vs[c][4 * dg]);
+#pragma unroll
+            for (int i = 0; i < kRpt; ++i) {
+                const float wv = ws[rg * kRpt + i][c];
+                acc[i].x = fmaf(wv, v4.x, acc[i].x);
+                acc[i].y = fmaf(wv, v4.y, acc[i].y);
+                acc[i].z = fmaf(wv, v4.z, acc[i].z);
+                acc[i].w = fmaf(wv, v4.w, acc[i].w);
                 lsum[i] += wv;
             }
         }
     }
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        const int gr = r0 + rb + i * kStride;
+    for (int i = 0; i < kRpt; ++i) {
+        const int gr = r0 + rg * kRpt + i;
         if (gr < nbr) {
-            olo[((size_t)bh * nbr + gr) * D + d] = acc[i];
-            if (d == 0) llo[(size_t)bh * nbr + gr] = lsum[i];
+            *reinterpret_cast<float4 *>(olo + ((size_t)bh * nbr + gr) * D + 4 * dg) = acc[i];
+            if (dg == 0) llo[(size_t)bh * nbr + gr] = lsum[i];
         }
     }
 }

@@ -10,10 +10,11 @@
 // One thread-block cluster per (batch, head): each CTA computes 16 block rows
 // of the map (fp32 FFMA, 2x4 register tiles), keeps their 35-bit keys in
 // shared memory, and the cluster runs the three radix passes of the top-k
-// together: local histograms are added into the rank-0 CTA's histogram
-// through distributed shared memory, rank 0 locates the bucket of the k-th
-// key, and every CTA reads the result back.  Cluster barriers separate the
-// steps (hardware barriers, no spinning).  The per-row counts, the scan that
+// together: local histograms are added into the rank-0 CTA's histogram of
+// the pass through distributed shared memory, rank 0 locates the bucket of
+// the k-th key and publishes it, and a pass whose bucket is taken whole ends
+// the search.  Cluster barriers (hardware barriers, no spinning) separate the
+// steps.  The per-row counts, the scan that
 // assigns CSR offsets and attention work items across the cluster, and the
 // column lists follow in the same kernel.  The key encoding and the tie rule
 // are those of the multi-kernel path (mra_lowres.cu, mra_select.cu).
@@ -34,6 +35,11 @@ constexpr int kMR = kRows / kRG;          // rows per thread tile (2)
 constexpr int kCT = 4 * kCG;              // columns per tile (128)
 constexpr int kMaxCta = 8;                // portable cluster size
 
+// Floats of the region that holds the transposed K-hat tile during the GEMM
+// and the histograms of the first two radix passes afterwards.
+template <int D>
+constexpr int region_floats() { return D * kCT > 2 * kHistBins ? D * kCT : 2 * kHistBins; }
+
 __device__ __forceinline__ int band_of(int r, int c, int g) {
     if (g <= 0) return 0;
     const int lo = -(g / 2);
@@ -43,15 +49,17 @@ __device__ __forceinline__ int band_of(int r, int c, int g) {
 }
 
 struct ClusterShared {
-    unsigned int hist[kHistBins];   // rank 0: the cluster histogram of the current pass
+    unsigned int hist2[kHistBins];  // rank 0: cluster histogram of the third pass
     unsigned int lh[kHistBins];     // this CTA's histogram
     unsigned int s_tmp[kThreads];
-    unsigned long long prefix;      // rank 0: threshold bits fixed so far
-    unsigned int need;
     int bin;
     unsigned int bin_need;
-    int tot_eq[kMaxCta], tot_sel[kMaxCta], tot_items[kMaxCta];   // rank 0: per-CTA totals
-    int row_gt[kRows], row_eq[kRows], row_sel[kRows], row_take[kRows], row_start[kRows], row_item[kRows];
+    unsigned long long pub_prefix;   // rank 0: result of the pass
+    unsigned int pub_need;
+    int pub_done;
+    int all_gt[kMaxCta * kRows], all_eq[kMaxCta * kRows];   // rank 0: per-row counts of the head
+    int row_take[kRows], row_start[kRows], row_item[kRows], row_sel[kRows];
+    int total_sel, total_items;
     int flag;
 };
 
@@ -59,7 +67,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads)
 lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__restrict__ khat,
                              const int *__restrict__ cnt, int H, int nbr, float scale, int first_n,
-                             int diag_n, int k, int cap, unsigned long long *__restrict__ keys_out,
+                             int diag_n, int k, int cap, int chunk,
+                             unsigned long long *__restrict__ keys_out,
                              float *__restrict__ mlo, float *__restrict__ logit_out,
                              int *__restrict__ cols, int32_t *__restrict__ sel_out,
                              unsigned int *__restrict__ bitmap, int wpr, WorkItem *__restrict__ items,
@@ -67,11 +76,10 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                              unsigned int *__restrict__ status) {
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
-    const int ncta = (int)cluster.num_blocks();
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *qs = reinterpret_cast<float *>(smem_raw);                     // [kRows][D]
     float *kT = qs + kRows * D;                                           // [D][kCT]
-    float *lt = kT + D * kCT;                                             // [kRows][nbr]
+    float *lt = kT + region_floats<D>();                                  // [kRows][nbr]
     unsigned long long *sk = reinterpret_cast<unsigned long long *>(lt + kRows * nbr);  // [kRows][nbr]
     int *cnts = reinterpret_cast<int *>(sk + kRows * nbr);                // [nbr]
     __shared__ ClusterShared cs;
@@ -88,7 +96,7 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
     const float *kh = khat + (size_t)bh * nbr * D;
 
     if (rank == 0)
-        for (int i = t; i < kHistBins; i += kThreads) cs.hist[i] = 0u;
+        for (int i = t; i < kHistBins; i += kThreads) cs.hist2[i] = 0u;
     if (t == 0) cs.flag = 0;
     // ------------------------------------------------------------ logits
     {
@@ -210,13 +218,25 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
         if (logit_out) logit_out[(size_t)bh * nbr2 + (size_t)gr * nbr + c] = l;
     }
     if (flag) atomicOr(&cs.flag, 1);
-    cluster.sync();   // rank 0's histogram is clear; every CTA of the cluster is running
+    // the histograms of the first two passes reuse the K-hat tile (rank 0's
+    // copy is cleared here, before any CTA adds into it)
+    unsigned int *hist01 = reinterpret_cast<unsigned int *>(kT);
+    if (rank == 0)
+        for (int i = t; i < 2 * kHistBins; i += kThreads) hist01[i] = 0u;
+    cluster.sync();   // histograms clear; every CTA of the cluster is running
     if (t == 0 && cs.flag) atomicOr(status, kDevKeyRange);
 
     // ------------------------------------------------------------ radix passes
+    // Every CTA adds its histogram into rank 0's buffer of the pass; rank 0
+    // locates the bucket of the k-th key in its own shared memory and
+    // publishes it.  A pass whose bucket is taken whole ends the search early:
+    // the threshold is then compared at that digit's bit.
+    unsigned int *hist_local[3] = {hist01, hist01 + kHistBins, cs.hist2};
     unsigned long long prefix = 0ull;
     unsigned int need = (unsigned)k;
-    for (int pass = 0; pass < 3; ++pass) {
+    int sh = 0;            // comparisons against the threshold use key >> sh
+    bool done = false;
+    for (int pass = 0; pass < 3 && !done; ++pass) {
         const int shift = pass == 0 ? (kHist1Bits + kHist2Bits) : (pass == 1 ? kHist2Bits : 0);
         const int bits = pass == 0 ? kHist0Bits : (pass == 1 ? kHist1Bits : kHist2Bits);
         const int hi = shift + bits;
@@ -230,29 +250,33 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
             warp_hist_add(cs.lh, (unsigned)(key >> shift) & dmask, e < n_here && (key >> hi) == want);
         }
         __syncthreads();
+        unsigned int *hb = cluster.map_shared_rank(hist_local[pass], 0);
         for (int i = t; i < (1 << bits); i += kThreads)
-            if (cs.lh[i]) atomicAdd(&cs0->hist[i], cs.lh[i]);
+            if (cs.lh[i]) atomicAdd(&hb[i], cs.lh[i]);
         cluster.sync();   // the cluster histogram of this pass is complete
         if (rank == 0) {
-            find_bucket<kThreads>([](int i) { return cs.hist[i]; }, 1 << bits, need, cs.s_tmp, &cs.bin,
+            unsigned int *h = hist_local[pass];
+            find_bucket<kThreads>([h](int i) { return h[i]; }, 1 << bits, need, cs.s_tmp, &cs.bin,
                                   &cs.bin_need);
             if (t == 0) {
-                cs.prefix = prefix | ((unsigned long long)cs.bin << shift);
-                cs.need = cs.bin_need;
+                const unsigned int in_bin = h[cs.bin];
+                cs.pub_prefix = prefix | ((unsigned long long)cs.bin << shift);
+                cs.pub_done = (cs.bin_need == in_bin) ? 1 : 0;
+                cs.pub_need = cs.bin_need;
             }
-            __syncthreads();
-            for (int i = t; i < kHistBins; i += kThreads) cs.hist[i] = 0u;   // for the next pass
         }
         cluster.sync();   // rank 0 published the bucket
-        prefix = cs0->prefix;
-        need = cs0->need;
+        prefix = cs0->pub_prefix;
+        need = cs0->pub_need;
+        done = cs0->pub_done != 0;
+        sh = shift;
     }
-    const unsigned long long T = prefix;
+    const unsigned long long Tsh = prefix >> sh;
     if (rank == 0 && t == 0) {
         SelState st;
-        st.prefix = T;
+        st.prefix = prefix;
         st.need = need;
-        st.pad = 0;
+        st.pad = (unsigned)sh;
         state[bh] = st;
     }
 
@@ -261,78 +285,105 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
         int g = 0, e = 0;
         if (r < rows_here)
             for (int c = lane; c < nbr; c += 32) {
-                const unsigned long long key = sk[r * nbr + c];
-                g += key > T;
-                e += key == T;
+                const unsigned long long kk = sk[r * nbr + c] >> sh;
+                g += kk > Tsh;
+                e += kk == Tsh;
             }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             g += __shfl_xor_sync(0xffffffffu, g, o);
             e += __shfl_xor_sync(0xffffffffu, e, o);
         }
-        if (lane == 0) {
-            cs.row_gt[r] = g;
-            cs.row_eq[r] = e;
+        if (lane == 0 && r < rows_here) {
+            cs0->all_gt[r0 + r] = g;
+            cs0->all_eq[r0 + r] = e;
+        }
+    }
+    cluster.sync();   // every row's counts are in rank 0
+    // every CTA scans all rows of the head (warp 0, four rows per lane) and
+    // keeps what concerns its own rows
+    if (warp == 0) {
+        constexpr int kPer = (kMaxCta * kRows) / 32;
+        int eqv[kPer], gtv[kPer];
+        int eq_local = 0;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int r = kPer * lane + j;
+            eqv[j] = r < nbr ? cs0->all_eq[r] : 0;
+            gtv[j] = r < nbr ? cs0->all_gt[r] : 0;
+            eq_local += eqv[j];
+        }
+        int x = eq_local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        int eq_before = x - eq_local;
+        int sel[kPer], itm[kPer], tk[kPer];
+        int sel_local = 0, it_local = 0;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int r = kPer * lane + j;
+            int take = (int)need - eq_before;
+            take = take < 0 ? 0 : (take > eqv[j] ? eqv[j] : take);
+            tk[j] = take;
+            sel[j] = r < nbr ? gtv[j] + take : 0;
+            itm[j] = r < nbr ? (sel[j] > 0 ? (sel[j] + chunk - 1) / chunk : 1) : 0;
+            eq_before += eqv[j];
+            sel_local += sel[j];
+            it_local += itm[j];
+        }
+        int xs = sel_local, xi = it_local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int ys = __shfl_up_sync(0xffffffffu, xs, o);
+            const int yi = __shfl_up_sync(0xffffffffu, xi, o);
+            if (lane >= o) {
+                xs += ys;
+                xi += yi;
+            }
+        }
+        int sb = xs - sel_local, ib = xi - it_local;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int r = kPer * lane + j;
+            if (r >= r0 && r < r0 + rows_here) {
+                cs.row_take[r - r0] = tk[j];
+                cs.row_sel[r - r0] = sel[j];
+                cs.row_start[r - r0] = sb;
+                cs.row_item[r - r0] = ib;
+            }
+            sb += sel[j];
+            ib += itm[j];
+        }
+        if (lane == 31) {
+            cs.total_sel = xs;
+            cs.total_items = xi;
         }
     }
     __syncthreads();
+    __shared__ int s_ok;
     if (t == 0) {
-        int te = 0;
-        for (int r = 0; r < kRows; ++r) te += cs.row_eq[r];
-        cs0->tot_eq[rank] = te;
-    }
-    cluster.sync();
-    if (t == 0) {
-        int eq_before = 0;
-        for (int i = 0; i < rank; ++i) eq_before += cs0->tot_eq[i];
-        int ts = 0, ti = 0;
-        for (int r = 0; r < rows_here; ++r) {
-            int take = (int)need - eq_before;
-            take = take < 0 ? 0 : (take > cs.row_eq[r] ? cs.row_eq[r] : take);
-            const int sel = cs.row_gt[r] + take;
-            cs.row_take[r] = take;
-            cs.row_sel[r] = sel;
-            cs.row_start[r] = ts;
-            cs.row_item[r] = ti;
-            ts += sel;
-            ti += sel > 0 ? (sel + kChunk - 1) / kChunk : 1;
-            eq_before += cs.row_eq[r];
-        }
-        cs0->tot_sel[rank] = ts;
-        cs0->tot_items[rank] = ti;
-    }
-    cluster.sync();
-    __shared__ int s_sel_before, s_item_before, s_ok;
-    if (t == 0) {
-        int sb = 0, ib = 0, st = 0, it = 0;
-        for (int i = 0; i < ncta; ++i) {
-            if (i < rank) {
-                sb += cs0->tot_sel[i];
-                ib += cs0->tot_items[i];
-            }
-            st += cs0->tot_sel[i];
-            it += cs0->tot_items[i];
-        }
-        s_sel_before = sb;
-        s_item_before = ib;
-        s_ok = (st == k && it <= cap);
+        s_ok = (cs.total_sel == k && cs.total_items <= cap);
         if (rank == 0) {
-            head_items[bh] = s_ok ? it : 0;
+            head_items[bh] = s_ok ? cs.total_items : 0;
             if (!s_ok) atomicOr(status, kDevCount);
         }
     }
     __syncthreads();
+    const int s_sel_before = 0, s_item_before = 0;
     if (s_ok) {
         // work items: one thread per local row
         for (int r = t; r < rows_here; r += kThreads) {
             const int sel = cs.row_sel[r];
-            const int nit = sel > 0 ? (sel + kChunk - 1) / kChunk : 1;
+            const int nit = sel > 0 ? (sel + chunk - 1) / chunk : 1;
             const int rs = bh * k + s_sel_before + cs.row_start[r];
             for (int j = 0; j < nit; ++j) {
                 WorkItem w;
                 w.row = bh * nbr + r0 + r;
-                w.col_start = rs + j * kChunk;
-                w.ncols = max(0, min(kChunk, sel - j * kChunk));
+                w.col_start = rs + j * chunk;
+                w.ncols = max(0, min(chunk, sel - j * chunk));
                 w.chunk_info = j | (nit << 16);
                 items[(size_t)bh * cap + s_item_before + cs.row_item[r] + j] = w;
             }
@@ -346,9 +397,9 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
             int eq_seen = 0, sel_seen = 0;
             for (int c0 = 0; c0 < nbr; c0 += 32) {
                 const int c = c0 + lane;
-                const unsigned long long key = c < nbr ? sk[r * nbr + c] : 0ull;
-                const bool is_gt = c < nbr && key > T;
-                const bool is_eq = c < nbr && key == T;
+                const unsigned long long kk = c < nbr ? (sk[r * nbr + c] >> sh) : 0ull;
+                const bool is_gt = c < nbr && kk > Tsh;
+                const bool is_eq = c < nbr && kk == Tsh;
                 const unsigned int eqb = __ballot_sync(0xffffffffu, is_eq);
                 const bool sel = is_gt || (is_eq && eq_seen + __popc(eqb & lt_mask) < take);
                 const unsigned int sb = __ballot_sync(0xffffffffu, sel);
@@ -370,7 +421,7 @@ template <int D>
 cudaError_t launch_typed(const Problem &p, const Workspace &w, float *logit_out, int32_t *sel_out,
                          cudaStream_t s) {
     const int ncta = (p.nbr + kRows - 1) / kRows;
-    const size_t smem = sizeof(float) * ((size_t)kRows * D + (size_t)D * kCT + (size_t)kRows * p.nbr) +
+    const size_t smem = sizeof(float) * ((size_t)kRows * D + (size_t)region_floats<D>() + (size_t)kRows * p.nbr) +
                         sizeof(unsigned long long) * (size_t)kRows * p.nbr + sizeof(int) * (size_t)p.nbr;
     auto kern = lowres_select_cluster_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -391,7 +442,7 @@ cudaError_t launch_typed(const Problem &p, const Workspace &w, float *logit_out,
     const float *qhat = w.pooled;
     const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;
     e = cudaLaunchKernelEx(&cfg, kern, qhat, khat, (const int *)w.cnt, p.H, p.nbr, scale, p.first_n,
-                           p.diag_n, p.k, p.cap, w.keys, w.mlo, logit_out, w.cols, sel_out,
+                           p.diag_n, p.k, p.cap, p.chunk, w.keys, w.mlo, logit_out, w.cols, sel_out,
                            p.mode == 0 ? w.bitmap : (unsigned int *)nullptr, w.words_per_row, w.items,
                            w.head_items, w.state, w.status);
     if (e != cudaSuccess) return e;

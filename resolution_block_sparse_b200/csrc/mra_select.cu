@@ -11,7 +11,7 @@
 // of the k-th key; after the third pass the threshold key T is exact and
 // `need` says how many keys equal to T are taken (the smallest indices).
 // Then, per block row, counts of keys above / equal to T, a per-head scan that
-// assigns CSR offsets and attention work items (chunks of at most kChunk
+// assigns CSR offsets and attention work items (chunks of at most `chunk`
 // columns), and the column lists in ascending column order.
 #include "mra_internal.cuh"
 #include "mra_select_common.cuh"
@@ -135,7 +135,7 @@ __device__ int block_exclusive_scan(int v, int *s_warp, int *total) {
 // One CTA per (batch, head): CSR row offsets and the attention work list.
 __global__ void __launch_bounds__(kScanThreads)
 row_scan_kernel(const int *__restrict__ gt, const int *__restrict__ eq,
-                const SelState *__restrict__ state, int nbr, int k, int cap,
+                const SelState *__restrict__ state, int nbr, int k, int cap, int chunk,
                 int *__restrict__ row_start, int *__restrict__ take_eq, WorkItem *__restrict__ items,
                 int *__restrict__ head_items, unsigned int *__restrict__ status) {
     __shared__ int s_warp[32];
@@ -165,7 +165,7 @@ row_scan_kernel(const int *__restrict__ gt, const int *__restrict__ eq,
     int sel_total;
     int sel_before = block_exclusive_scan(sel_local, s_warp, &sel_total);
     int it_local = 0;
-    for (int r = rbeg, i = 0; r < rend; ++r, ++i) it_local += sel[i] > 0 ? (sel[i] + kChunk - 1) / kChunk : 1;
+    for (int r = rbeg, i = 0; r < rend; ++r, ++i) it_local += sel[i] > 0 ? (sel[i] + chunk - 1) / chunk : 1;
     int it_total;
     int it_before = block_exclusive_scan(it_local, s_warp, &it_total);
 
@@ -173,12 +173,12 @@ row_scan_kernel(const int *__restrict__ gt, const int *__restrict__ eq,
         const int rs = bh * k + sel_before;
         row_start[base + r] = rs;
         take_eq[base + r] = tk[i];
-        const int n = sel[i] > 0 ? (sel[i] + kChunk - 1) / kChunk : 1;
+        const int n = sel[i] > 0 ? (sel[i] + chunk - 1) / chunk : 1;
         for (int j = 0; j < n && it_before + j < cap; ++j) {
             WorkItem w;
             w.row = base + r;
-            w.col_start = rs + j * kChunk;
-            w.ncols = min(kChunk, sel[i] - j * kChunk);
+            w.col_start = rs + j * chunk;
+            w.ncols = min(chunk, sel[i] - j * chunk);
             if (w.ncols < 0) w.ncols = 0;
             w.chunk_info = j | (n << 16);
             items[(size_t)bh * cap + it_before + j] = w;
@@ -242,7 +242,7 @@ constexpr int kSmallThreads = 1024;
 // list and the column lists.
 __global__ void __launch_bounds__(kSmallThreads)
 select_small_kernel(const unsigned long long *__restrict__ keys, SelState *__restrict__ state,
-                    int nbr, int k, int cap, int *__restrict__ cols, int32_t *__restrict__ sel_out,
+                    int nbr, int k, int cap, int chunk, int *__restrict__ cols, int32_t *__restrict__ sel_out,
                     unsigned int *__restrict__ bitmap, int wpr, WorkItem *__restrict__ items,
                     int *__restrict__ head_items, unsigned int *__restrict__ status) {
     extern __shared__ __align__(16) unsigned long long sk[];   // [nbr * nbr]
@@ -348,7 +348,7 @@ select_small_kernel(const unsigned long long *__restrict__ keys, SelState *__res
             int take = (int)need - eq_before;
             take = take < 0 ? 0 : (take > eqv[j] ? eqv[j] : take);
             sel[j] = r < nbr ? s_gt[r] + take : 0;
-            itm[j] = r < nbr ? (sel[j] > 0 ? (sel[j] + kChunk - 1) / kChunk : 1) : 0;
+            itm[j] = r < nbr ? (sel[j] > 0 ? (sel[j] + chunk - 1) / chunk : 1) : 0;
             if (r < nbr) s_take[r] = take;
             eq_before += eqv[j];
             sel_local += sel[j];
@@ -391,13 +391,13 @@ select_small_kernel(const unsigned long long *__restrict__ keys, SelState *__res
     // work items: one thread per row
     for (int r = t; r < nbr; r += kSmallThreads) {
         const int sel = s_sel[r];
-        const int nit = sel > 0 ? (sel + kChunk - 1) / kChunk : 1;
+        const int nit = sel > 0 ? (sel + chunk - 1) / chunk : 1;
         const int rs = bh * k + s_start[r];
         for (int j = 0; j < nit; ++j) {
             WorkItem w;
             w.row = bh * nbr + r;
-            w.col_start = rs + j * kChunk;
-            w.ncols = max(0, min(kChunk, sel - j * kChunk));
+            w.col_start = rs + j * chunk;
+            w.ncols = max(0, min(chunk, sel - j * chunk));
             w.chunk_info = j | (nit << 16);
             items[(size_t)bh * cap + s_item[r] + j] = w;
         }
@@ -448,7 +448,7 @@ cudaError_t launch_row_counts(const Problem &p, const Workspace &w, cudaStream_t
 }
 
 cudaError_t launch_row_scan(const Problem &p, const Workspace &w, cudaStream_t s) {
-    row_scan_kernel<<<p.BH, kScanThreads, 0, s>>>(w.gt, w.eq, w.state, p.nbr, p.k, p.cap,
+    row_scan_kernel<<<p.BH, kScanThreads, 0, s>>>(w.gt, w.eq, w.state, p.nbr, p.k, p.cap, p.chunk,
                                                   w.row_start, w.take_eq, w.items, w.head_items,
                                                   w.status);
     return cudaGetLastError();
@@ -461,7 +461,7 @@ cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *s
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     select_small_kernel<<<p.BH, kSmallThreads, smem, s>>>(
-        w.keys, w.state, p.nbr, p.k, p.cap, w.cols, sel_out, p.mode == 0 ? w.bitmap : nullptr,
+        w.keys, w.state, p.nbr, p.k, p.cap, p.chunk, w.cols, sel_out, p.mode == 0 ? w.bitmap : nullptr,
         w.words_per_row, w.items, w.head_items, w.status);
     return cudaGetLastError();
 }
