@@ -316,7 +316,8 @@ def main():
     esz = 2 if w.dtype == "bf16" else 4
     BH = w.B * w.H
     kernel_src = {"attention": "mra_attn.cu", "pool": "mra_pool.cu", "lowres_keys": "mra_lowres.cu",
-                  "lowres_pv": "mra_lowres.cu", "select": "mra_select.cu"}
+                  "lowres_pv": "mra_lowres.cu", "select": "mra_select.cu",
+                  "lowres_select": "mra_lowres_select.cu"}
     if dom == "attention":
         # compulsory Q, K, V read + O write of the attended heads; intensity
         # 16*block_per_row flop/B is below the bf16 ridge -> HBM bound
