@@ -89,6 +89,7 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     t.hist = (unsigned int *)take(sizeof(unsigned int) * BH * 3 * kHistBins);
     t.arrive = (unsigned int *)take(sizeof(unsigned int) * BH * 4);
     t.row_arrive = (int *)take(sizeof(int) * BH * nbr);
+    t.work_next = (int *)take(sizeof(int) * 4);
     t.zero_base = t.hist;
     t.zero_bytes = off;
     t.cnt = (int *)take(sizeof(int) * (size_t)p.B * nbr);

@@ -103,6 +103,7 @@ struct AttnArgs {
     const float *mlo, *olo, *llo;
     float *partial;
     int *row_arrive;
+    int *work_next;   // items handed out beyond the first wave (zeroed per call)
     void *out;
 };
 
@@ -120,6 +121,7 @@ struct Bf16Smem {
     float km[2][32];   // key mask per buffer
     int cols[kChunk];
     int last;
+    int next[2];   // next work index, alternating so a write never races a read
 };
 
 // One work item (block row, chunk of selected columns) on a 64-thread CTA.
@@ -348,18 +350,24 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
                                                 mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
 }
 
-// Persistent: each CTA walks the work items with a grid stride, in the order
-// (item index within its head) major, head minor.  The long rows of every
-// head (the first-n prior rows) come first in their head's list, so they
-// start in the first wave instead of forming the tail.
+// Persistent: the first wave takes items 0..gridDim.x-1, after that a CTA
+// takes the next index from a global counter as it finishes an item, so the
+// CTAs that drew short rows keep pulling work while the long ones run.  The
+// index order is (item index within its head) major, head minor: the long
+// rows of every head (the first-n prior rows) come first in their head's
+// list and start in the first wave.  The next index is fetched at the start
+// of an item, so the atomic's round trip hides behind the item's work.
 template <int D>
 __global__ void __launch_bounds__(kBf16Threads, 10)
 attn_bf16_kernel(const AttnArgs a, int total_slots, int heads) {
     __shared__ __align__(128) Bf16Smem<D> sh;
-    for (int i = blockIdx.x; i < total_slots; i += gridDim.x) {
+    int i = blockIdx.x;
+    for (int t = 0; i < total_slots; ++t) {
+        if (threadIdx.x == 0) sh.next[t & 1] = (int)gridDim.x + atomicAdd(a.work_next, 1);
         const int slot = (i % heads) * a.cap + i / heads;
         bf16_item<D>(a, slot, sh);
-        __syncthreads();   // shared buffers are free for the next item
+        __syncthreads();   // shared buffers are free for the next item; next[] is visible
+        i = sh.next[t & 1];
     }
 }
 
@@ -474,6 +482,7 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
     a.llo = w.llo;
     a.partial = w.partial;
     a.row_arrive = w.row_arrive;
+    a.work_next = w.work_next;
     a.out = out;
     const long long grid = (long long)p.BH * p.cap;
     // MRA_ATTN_IMPL=tc selects the tcgen05/TMA kernel (bf16, head size 64);

@@ -35,76 +35,138 @@ __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float x) { return
 template <>
 __device__ __forceinline__ float to_out<float>(float x) { return x; }
 
+// four consecutive outputs (8-byte store for bf16, 16-byte for fp32)
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<unsigned *>(&a);
+    u.y = *reinterpret_cast<unsigned *>(&b);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+__device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+
+template <bool G>
+__device__ __forceinline__ float4 ldp4(const float4 *p) {
+    if constexpr (G) return __ldcg(p);
+    else return *p;
+}
+
+constexpr int kMergeGroup = 16;   // partials whose (m, l) are staged at once
+
 struct MergeSmem {
-    float w[32][33];
-    float M[32], inv[32], beta[32];
+    float w[kMergeGroup][32];   // m of (chunk, row), then its weight
+    float l[kMergeGroup][32];
+    float M[32], den[32], resc[32];
 };
 
 // Merge nchunks partials (layout per slot: m[32], l[32], O[32][D]; m in log2
 // units, l and O relative to exp2(m)) with the low-resolution part of the row
 // (full mode) and write the 32 x D output block.
+//
+// The partials are taken in groups of kMergeGroup: all (m, l) pairs of a group
+// are loaded at once, the running per-row maximum and normaliser move to the
+// group's maximum (earlier groups rescaled), and the O tiles of four partials
+// are in flight together, so the merge costs a few memory round trips rather
+// than two per partial.
 template <int D, int NT, bool G, typename OutT, typename Sync>
 __device__ void merge_write(const float *src0, size_t slot_stride, int nchunks, int full,
                             float m_lo2, float l_lo, const float *olo_row, const float *qmask,
                             OutT *out_blk, MergeSmem &sm) {
+    static_assert((8 * D) % NT == 0, "a chunk's O tile must split evenly into float4 per thread");
+    constexpr int F = 8 * D / NT;   // float4 of one partial's O tile per thread
+    constexpr int kRowF4 = D / 4;
+    constexpr int kMergeUnroll = F >= 8 ? 1 : 8 / F;
     const int tid = threadIdx.x;
+    float4 acc[F];
+#pragma unroll
+    for (int i = 0; i < F; ++i) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (tid < 32) {
+        sm.M[tid] = -INFINITY;
+        sm.den[tid] = 0.0f;
+    }
+    for (int cg = 0; cg < nchunks; cg += kMergeGroup) {
+        const int nc = min(kMergeGroup, nchunks - cg);
+        for (int e = tid; e < nc * 32; e += NT) {
+            const int c = e >> 5, q = e & 31;
+            const float *P = src0 + (size_t)(cg + c) * slot_stride;
+            const float l = ldp<G>(P + 32 + q);
+            const float m = ldp<G>(P + q);
+            sm.w[c][q] = l > 0.0f ? m : -INFINITY;
+            sm.l[c][q] = l > 0.0f ? l : 0.0f;
+        }
+        Sync::sync();
+        if (tid < 32) {
+            const int q = tid;
+            const float m_old = sm.M[q];
+            float m_new = m_old;
+            for (int c = 0; c < nc; ++c) m_new = fmaxf(m_new, sm.w[c][q]);
+            const float resc = (m_old == -INFINITY) ? 0.0f : exp2f(m_old - m_new);
+            float den = sm.den[q] * resc;
+            for (int c = 0; c < nc; ++c) {
+                const float m = sm.w[c][q];
+                const float wgt = (m == -INFINITY) ? 0.0f : exp2f(m - m_new);
+                den = fmaf(wgt, sm.l[c][q], den);
+                sm.w[c][q] = wgt;
+            }
+            sm.M[q] = m_new;
+            sm.den[q] = den;
+            sm.resc[q] = resc;
+        }
+        Sync::sync();
+        if (cg > 0) {
+#pragma unroll
+            for (int i = 0; i < F; ++i) {
+                const float r = sm.resc[(tid + i * NT) / kRowF4];
+                acc[i].x *= r;
+                acc[i].y *= r;
+                acc[i].z *= r;
+                acc[i].w *= r;
+            }
+        }
+        // at most 8 float4 loads in flight per thread (register budget)
+#pragma unroll kMergeUnroll
+        for (int c = 0; c < nc; ++c) {
+            const float4 *O = reinterpret_cast<const float4 *>(src0 + (size_t)(cg + c) * slot_stride + 64);
+#pragma unroll
+            for (int i = 0; i < F; ++i) {
+                const int f = tid + i * NT;
+                const float wgt = sm.w[c][f / kRowF4];
+                const float4 v = ldp4<G>(O + f);
+                acc[i].x = fmaf(wgt, v.x, acc[i].x);
+                acc[i].y = fmaf(wgt, v.y, acc[i].y);
+                acc[i].z = fmaf(wgt, v.z, acc[i].z);
+                acc[i].w = fmaf(wgt, v.w, acc[i].w);
+            }
+        }
+        Sync::sync();
+    }
+    // low-resolution part at the shared maximum, normaliser, padded queries
     if (tid < 32) {
         const int q = tid;
-        float M = -INFINITY;
-        for (int c = 0; c < nchunks; ++c) {
-            const float *P = src0 + (size_t)c * slot_stride;
-            if (ldp<G>(P + 32 + q) > 0.0f) M = fmaxf(M, ldp<G>(P + q));
-        }
+        const float m_hi = sm.M[q];
         const bool lo = full && l_lo > 0.0f;
-        if (lo) M = fmaxf(M, m_lo2);
-        float inv = 0.0f, beta = 0.0f;
+        const float M = lo ? fmaxf(m_hi, m_lo2) : m_hi;
+        float a_hi = 0.0f, beta = 0.0f, inv = 0.0f;
         if (M != -INFINITY && (!qmask || qmask[q] > 0.0f)) {
-            float den = 0.0f;
-            for (int c = 0; c < nchunks; ++c) {
-                const float *P = src0 + (size_t)c * slot_stride;
-                const float l = ldp<G>(P + 32 + q);
-                if (l > 0.0f) den += exp2f(ldp<G>(P + q) - M) * l;
-            }
-            if (lo) {
-                beta = exp2f(m_lo2 - M);
-                den += beta * l_lo;
-            }
+            a_hi = (m_hi == -INFINITY) ? 0.0f : exp2f(m_hi - M);
+            beta = lo ? exp2f(m_lo2 - M) : 0.0f;
+            const float den = a_hi * sm.den[q] + beta * l_lo;
             inv = den > 0.0f ? 1.0f / den : 0.0f;
         }
-        sm.M[q] = (M == -INFINITY) ? 0.0f : M;
-        sm.inv[q] = inv;
-        sm.beta[q] = beta;
+        sm.resc[q] = a_hi * inv;   // factor of the merged high-resolution O
+        sm.den[q] = beta * inv;    // factor of the low-resolution output
     }
     Sync::sync();
-    constexpr int E = 32 * D / NT;
-    float acc[E];
 #pragma unroll
-    for (int i = 0; i < E; ++i) acc[i] = 0.0f;
-    for (int cg = 0; cg < nchunks; cg += 32) {
-        const int nc = min(32, nchunks - cg);
-        for (int e = tid; e < nc * 32; e += NT) {
-            const int c = e / 32, q = e % 32;
-            const float *P = src0 + (size_t)(cg + c) * slot_stride;
-            sm.w[c][q] = ldp<G>(P + 32 + q) > 0.0f ? exp2f(ldp<G>(P + q) - sm.M[q]) : 0.0f;
-        }
-        Sync::sync();
-        for (int c = 0; c < nc; ++c) {
-            const float *O = src0 + (size_t)(cg + c) * slot_stride + 64;
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                const int e = tid + i * NT;
-                acc[i] = fmaf(sm.w[c][e / D], ldp<G>(O + e), acc[i]);
-            }
-        }
-        Sync::sync();
-    }
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-        const int e = tid + i * NT;
-        const int q = e / D, d = e % D;
-        float val = acc[i];
-        if (full) val = fmaf(sm.beta[q], olo_row[d], val);
-        out_blk[e] = to_out<OutT>(val * sm.inv[q]);
+    for (int i = 0; i < F; ++i) {
+        const int f = tid + i * NT;
+        const int q = f / kRowF4, d = (f % kRowF4) * 4;
+        const float fa = sm.resc[q], fb = sm.den[q];
+        float4 ol = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (full) ol = *reinterpret_cast<const float4 *>(olo_row + d);
+        store4(out_blk + (size_t)q * D + d,
+               make_float4(fmaf(acc[i].x, fa, ol.x * fb), fmaf(acc[i].y, fa, ol.y * fb),
+                           fmaf(acc[i].z, fa, ol.z * fb), fmaf(acc[i].w, fa, ol.w * fb)));
     }
 }
 
@@ -123,8 +185,9 @@ __device__ void finish_item(float *stage, int slot, int chunk, int nchunks, int 
         merge_write<D, NT, false, OutT, Sync>(stage, stride, 1, full, m_lo2, l_lo, olo_row, qmask, out_blk, sm);
         return;
     }
-    float *dst = partial + (size_t)slot * stride;
-    for (int e = tid; e < (int)stride; e += NT) dst[e] = stage[e];
+    float4 *dst = reinterpret_cast<float4 *>(partial + (size_t)slot * stride);
+    const float4 *src = reinterpret_cast<const float4 *>(stage);
+    for (int e = tid; e < (int)stride / 4; e += NT) dst[e] = src[e];
     __threadfence();
     Sync::sync();
     if (tid == 0) *s_last = (atomicAdd(&row_arrive[row], 1) == nchunks - 1);

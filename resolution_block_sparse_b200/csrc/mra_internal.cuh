@@ -68,6 +68,7 @@ struct Workspace {
     unsigned int *hist;      // [BH][3][kHistBins]
     unsigned int *arrive;    // [BH][4]
     int *row_arrive;         // [BH*nbr]
+    int *work_next;          // [4]: attention work-item counter
     size_t zero_bytes;
     void *zero_base;
     // written before read every call

@@ -60,6 +60,9 @@ SMALL = [
     (1, 2, 1024, 64, torch.float32, 20, 0, 0, 0, None, 1.0),        # fp32 multi-chunk
     (1, 2, 512, 64, torch.bfloat16, 4, 0, 0, 0, None, 3.0),         # peaked scores
     (1, 2, 512, 64, torch.bfloat16, 4, 1, 1, 1, [17], 3.0),
+    (1, 1, 8192, 64, torch.bfloat16, 2, 0, 1, 0, None, 1.0),       # 32-item row: grouped merge
+    (1, 1, 8192, 64, torch.bfloat16, 2, 1, 1, 0, [300], 1.0),
+    (1, 1, 8192, 32, torch.float32, 2, 0, 1, 0, [300], 1.0),
 ]
 
 
