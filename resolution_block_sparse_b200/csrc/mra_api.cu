@@ -85,12 +85,14 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     };
     const size_t BH = (size_t)p.BH, nbr = (size_t)p.nbr, D = (size_t)p.D;
     Workspace t{};
-    // zeroed region
-    t.hist = (unsigned int *)take(sizeof(unsigned int) * BH * 3 * kHistBins);
+    // zeroed region (the radix histograms last: the fused selection does
+    // not use them, so its calls clear only the part before them)
     t.arrive = (unsigned int *)take(sizeof(unsigned int) * BH * 4);
     t.row_arrive = (int *)take(sizeof(int) * BH * nbr);
     t.work_next = (int *)take(sizeof(int) * 4);
-    t.zero_base = t.hist;
+    t.zero_bytes_no_hist = off;
+    t.hist = (unsigned int *)take(sizeof(unsigned int) * BH * 3 * kHistBins);
+    t.zero_base = t.arrive;
     t.zero_bytes = off;
     t.cnt = (int *)take(sizeof(int) * (size_t)p.B * nbr);
     t.pooled = (float *)take(sizeof(float) * 3 * BH * nbr * D);

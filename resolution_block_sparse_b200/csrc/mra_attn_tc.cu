@@ -29,6 +29,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include "mra_async.cuh"
 #include "mra_attn_common.cuh"
 #include "mra_internal.cuh"
 
@@ -36,6 +37,7 @@ namespace mra {
 namespace {
 
 using namespace attn;
+using namespace async;
 
 constexpr int kConsumers = 128;
 constexpr int kThreadsTC = kConsumers + 64;     // + producer warp + MMA warp
@@ -45,8 +47,6 @@ constexpr int kTile = 32 * 64 * 2;              // one 32 x 64 bf16 block (4 KB)
 constexpr int kStackBytes = kStack * kTile;     // 16 KB
 constexpr uint32_t kTmemCols = 128;             // S^T x2 at columns 0, 32; O^T at 64
 constexpr float kRescale = 8.0f;                // lazy-rescale threshold (log2 units)
-constexpr unsigned kSuspendHintNs = 20000;      // per try_wait
-constexpr unsigned kWaitLimit = 1u << 17;        // x hint: a few seconds at most
 
 constexpr int kOffQ = 0;                                  // 2 x 4 KB
 constexpr int kOffK = 2 * kTile;                          // kStages x 16 KB
@@ -60,44 +60,12 @@ constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((32u >> 3) <<
 constexpr uint32_t kIdescPV =
     (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((32u >> 3) << 17) | ((64u >> 4) << 24);
 
-__device__ __forceinline__ uint32_t saddr(const void *p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
 // Shared-memory matrix descriptor, 128-byte swizzle, Blackwell version bit.
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
     return (uint64_t)((addr >> 4) & 0x3fffu) | ((uint64_t)((lbo >> 4) & 0x3fffu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3fffu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
-// try_wait with a suspend-time hint: a waiting thread sleeps (up to the hint)
-// until the phase completes instead of spinning on issue slots
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait on one phase of an mbarrier; false when the limit expired.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (unsigned i = 0; i < kWaitLimit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
-}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint32_t bar) {
     asm volatile(

@@ -69,7 +69,8 @@ struct Workspace {
     unsigned int *arrive;    // [BH][4]
     int *row_arrive;         // [BH*nbr]
     int *work_next;          // [4]: attention work-item counter
-    size_t zero_bytes;
+    size_t zero_bytes;       // the whole region
+    size_t zero_bytes_no_hist;   // the region without the radix histograms
     void *zero_base;
     // written before read every call
     int *cnt;                // [B][nbr]

@@ -10,14 +10,15 @@
 // One thread-block cluster per (batch, head): each CTA computes 16 block rows
 // of the map (fp32 FFMA, 2x4 register tiles), keeps their 35-bit keys in
 // shared memory, and the cluster runs the three radix passes of the top-k
-// together: local histograms are added into the rank-0 CTA's histogram of
-// the pass through distributed shared memory, rank 0 locates the bucket of
-// the k-th key and publishes it, and a pass whose bucket is taken whole ends
-// the search.  Cluster barriers (hardware barriers, no spinning) separate the
-// steps.  The per-row counts, the scan that
-// assigns CSR offsets and attention work items across the cluster, and the
-// column lists follow in the same kernel.  The key encoding and the tie rule
-// are those of the multi-kernel path (mra_lowres.cu, mra_select.cu).
+// together: every CTA adds its histogram of a pass into every CTA's copy of
+// the cluster histogram through distributed shared memory, so after one
+// cluster barrier each CTA locates the bucket of the k-th key on its own; a
+// pass whose bucket is taken whole ends the search.  Cluster barriers
+// (hardware barriers, no spinning) separate the steps.  The per-row counts
+// (pushed to every CTA the same way), the scan that assigns CSR offsets and
+// attention work items across the cluster, and the column lists follow in
+// the same kernel.  The key encoding and the tie rule are those of the
+// multi-kernel path (mra_lowres.cu, mra_select.cu).
 #include <cooperative_groups.h>
 
 #include "mra_internal.cuh"
@@ -29,16 +30,34 @@ namespace mra {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 constexpr int kRows = 16;                 // block rows per CTA
-constexpr int kRG = 8, kCG = 32;          // row groups x column groups
+constexpr int kRG = 8, kCG = 32;          // row groups x column lanes of the GEMM
 constexpr int kMR = kRows / kRG;          // rows per thread tile (2)
-constexpr int kCT = 4 * kCG;              // columns per tile (128)
+constexpr int kCT = 128;                  // columns of the map (at most)
+constexpr int kCPT = kCT / kCG;           // columns per thread (4), strided by 32
 constexpr int kMaxCta = 8;                // portable cluster size
 
-// Floats of the region that holds the transposed K-hat tile during the GEMM
-// and the histograms of the first two radix passes afterwards.
+// Row stride of the K-hat tile in shared memory: D + 4 floats keeps rows
+// 16-byte aligned and puts the rows read by 8 consecutive lanes in distinct
+// bank groups.
 template <int D>
-constexpr int region_floats() { return D * kCT > 2 * kHistBins ? D * kCT : 2 * kHistBins; }
+constexpr int ks_stride() { return D + 4; }
+
+// Keys of the k-th key's first-digit bucket that rank 0 gathers to finish
+// the selection on its own.
+constexpr int kCand = 4096;
+
+// Words of the region that holds the K-hat tile during the GEMM and, after
+// it, the cluster histogram of the first digit (2048 words) followed by
+// either the gathered keys (kCand 64-bit keys) or the cluster histograms of
+// the two lower digits (2 x 4096 words).
+constexpr int kSelWords = (1 << kHist0Bits) + 2 * kHistBins;
+static_assert(2 * kCand <= 2 * kHistBins, "gathered keys share the lower-digit histograms' words");
+template <int D>
+__host__ __device__ constexpr int region_floats() {
+    return ks_stride<D>() * kCT > kSelWords ? ks_stride<D>() * kCT : kSelWords;
+}
 
 __device__ __forceinline__ int band_of(int r, int c, int g) {
     if (g <= 0) return 0;
@@ -48,16 +67,23 @@ __device__ __forceinline__ int band_of(int r, int c, int g) {
     return (off >= lo && off <= hi) ? 1 : 0;
 }
 
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
 struct ClusterShared {
-    unsigned int hist2[kHistBins];  // rank 0: cluster histogram of the third pass
-    unsigned int lh[kHistBins];     // this CTA's histogram
-    unsigned int s_tmp[kThreads];
+    unsigned int lh[kHistBins];     // this CTA's histogram of the current pass
+    unsigned int s_tot[kWarps];
     int bin;
     unsigned int bin_need;
-    unsigned long long pub_prefix;   // rank 0: result of the pass
+    int cand_n;                     // rank 0: keys gathered so far
+    unsigned long long pub_prefix;  // threshold published by rank 0
     unsigned int pub_need;
-    int pub_done;
-    int all_gt[kMaxCta * kRows], all_eq[kMaxCta * kRows];   // rank 0: per-row counts of the head
+    int pub_sh;
+    int all_gt[kMaxCta * kRows], all_eq[kMaxCta * kRows];   // per-row counts of the whole head
     int row_take[kRows], row_start[kRows], row_item[kRows], row_sel[kRows];
     int total_sel, total_items;
     int flag;
@@ -74,17 +100,18 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                              unsigned int *__restrict__ bitmap, int wpr, WorkItem *__restrict__ items,
                              int *__restrict__ head_items, SelState *__restrict__ state,
                              unsigned int *__restrict__ status) {
+    constexpr int KS = ks_stride<D>();
+    constexpr int kF4 = D / 4;   // float4 per row of Q-hat / K-hat
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
+    const int ncta = (int)cluster.num_blocks();
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *qs = reinterpret_cast<float *>(smem_raw);                     // [kRows][D]
-    float *kT = qs + kRows * D;                                           // [D][kCT]
-    float *lt = kT + region_floats<D>();                                  // [kRows][nbr]
+    float *ks = qs + kRows * D;                                           // [kCT][KS]
+    float *lt = ks + region_floats<D>();                                  // [kRows][nbr]
     unsigned long long *sk = reinterpret_cast<unsigned long long *>(lt + kRows * nbr);  // [kRows][nbr]
     int *cnts = reinterpret_cast<int *>(sk + kRows * nbr);                // [nbr]
     __shared__ ClusterShared cs;
-    __shared__ float rmax[kRows];
-    ClusterShared *cs0 = cluster.map_shared_rank(&cs, 0);
 
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int bh = blockIdx.y;
@@ -95,21 +122,31 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
     const float *qh = qhat + (size_t)bh * nbr * D;
     const float *kh = khat + (size_t)bh * nbr * D;
 
-    if (rank == 0)
-        for (int i = t; i < kHistBins; i += kThreads) cs.hist2[i] = 0u;
-    if (t == 0) cs.flag = 0;
+    for (int i = t; i < kHistBins; i += kThreads) cs.lh[i] = 0u;
+    if (t == 0) {
+        cs.flag = 0;
+        cs.cand_n = 0;
+    }
     // ------------------------------------------------------------ logits
     {
-        constexpr int kQ = (kRows * D / 4 + kThreads - 1) / kThreads;
-        float4 v[kQ];
-        int cv[(kMaxCta * kRows + kThreads - 1) / kThreads];
+        constexpr int kQ = (kRows * kF4 + kThreads - 1) / kThreads;
+        constexpr int kK = (kCT * kF4 + kThreads - 1) / kThreads;
+        float4 qv[kQ], kv[kK];
+        int cv[(kCT + kThreads - 1) / kThreads];
+        // all loads first (coalesced rows), then the shared-memory stores
 #pragma unroll
         for (int u = 0; u < kQ; ++u) {
             const int i = t + u * kThreads;
-            const int r = (4 * i) / D;
-            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < kRows * D / 4 && r < rows_here)
-                v[u] = reinterpret_cast<const float4 *>(qh + (size_t)(r0 + r) * D)[(4 * i) % D / 4];
+            const int r = i / kF4;
+            qv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < kRows * kF4 && r < rows_here)
+                qv[u] = reinterpret_cast<const float4 *>(qh + (size_t)(r0 + r) * D)[i % kF4];
+        }
+#pragma unroll
+        for (int u = 0; u < kK; ++u) {
+            const int i = t + u * kThreads;
+            kv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < nbr * kF4) kv[u] = reinterpret_cast<const float4 *>(kh)[i];
         }
 #pragma unroll
         for (int u = 0; u < (int)(sizeof(cv) / sizeof(int)); ++u) {
@@ -119,7 +156,12 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
 #pragma unroll
         for (int u = 0; u < kQ; ++u) {
             const int i = t + u * kThreads;
-            if (i < kRows * D / 4) reinterpret_cast<float4 *>(qs)[i] = v[u];
+            if (i < kRows * kF4) reinterpret_cast<float4 *>(qs)[i] = qv[u];
+        }
+#pragma unroll
+        for (int u = 0; u < kK; ++u) {
+            const int i = t + u * kThreads;
+            if (i < kCT * kF4) *reinterpret_cast<float4 *>(ks + (i / kF4) * KS + 4 * (i % kF4)) = kv[u];
         }
 #pragma unroll
         for (int u = 0; u < (int)(sizeof(cv) / sizeof(int)); ++u) {
@@ -127,149 +169,214 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
             if (c < nbr) cnts[c] = cv[u];
         }
     }
-    const int rg = t / kCG, cg_ = t % kCG;
-    for (int ct = 0; ct < nbr; ct += kCT) {
-        __syncthreads();
-        {
-            constexpr int kL = kCT * D / 4 / kThreads;
-            float4 v[kL];
-#pragma unroll
-            for (int u = 0; u < kL; ++u) {
-                const int e = t + u * kThreads;
-                const int c = e % kCT, d4 = e / kCT;
-                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (ct + c < nbr) v[u] = reinterpret_cast<const float4 *>(kh + (size_t)(ct + c) * D)[d4];
-            }
-#pragma unroll
-            for (int u = 0; u < kL; ++u) {
-                const int e = t + u * kThreads;
-                const int c = e % kCT, d4 = e / kCT;
-                kT[(4 * d4 + 0) * kCT + c] = v[u].x;
-                kT[(4 * d4 + 1) * kCT + c] = v[u].y;
-                kT[(4 * d4 + 2) * kCT + c] = v[u].z;
-                kT[(4 * d4 + 3) * kCT + c] = v[u].w;
-            }
-        }
-        __syncthreads();
-        float acc[kMR][4];
+    __syncthreads();
+    {
+        // thread tile: rows kMR*rg + i, columns cg_ + 32*j
+        const int rg = t / kCG, cg_ = t % kCG;
+        float acc[kMR][kCPT];
 #pragma unroll
         for (int i = 0; i < kMR; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+            for (int j = 0; j < kCPT; ++j) acc[i][j] = 0.0f;
 #pragma unroll 4
         for (int d = 0; d < D; d += 4) {
-            float4 qv[kMR];
+            float4 q4[kMR], k4[kCPT];
 #pragma unroll
-            for (int i = 0; i < kMR; ++i) qv[i] = *reinterpret_cast<const float4 *>(qs + (kMR * rg + i) * D + d);
+            for (int i = 0; i < kMR; ++i) q4[i] = *reinterpret_cast<const float4 *>(qs + (kMR * rg + i) * D + d);
 #pragma unroll
-            for (int dd = 0; dd < 4; ++dd) {
-                const float4 kv = *reinterpret_cast<const float4 *>(kT + (d + dd) * kCT + 4 * cg_);
+            for (int j = 0; j < kCPT; ++j) k4[j] = *reinterpret_cast<const float4 *>(ks + (cg_ + 32 * j) * KS + d);
 #pragma unroll
-                for (int i = 0; i < kMR; ++i) {
-                    const float qd = dd == 0 ? qv[i].x : dd == 1 ? qv[i].y : dd == 2 ? qv[i].z : qv[i].w;
-                    acc[i][0] = fmaf(qd, kv.x, acc[i][0]);
-                    acc[i][1] = fmaf(qd, kv.y, acc[i][1]);
-                    acc[i][2] = fmaf(qd, kv.z, acc[i][2]);
-                    acc[i][3] = fmaf(qd, kv.w, acc[i][3]);
+            for (int i = 0; i < kMR; ++i)
+#pragma unroll
+                for (int j = 0; j < kCPT; ++j) {
+                    acc[i][j] = fmaf(q4[i].x, k4[j].x, acc[i][j]);
+                    acc[i][j] = fmaf(q4[i].y, k4[j].y, acc[i][j]);
+                    acc[i][j] = fmaf(q4[i].z, k4[j].z, acc[i][j]);
+                    acc[i][j] = fmaf(q4[i].w, k4[j].w, acc[i][j]);
                 }
-            }
         }
-        const int c0 = ct + 4 * cg_;
 #pragma unroll
         for (int i = 0; i < kMR; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (c0 + j < nbr) lt[(kMR * rg + i) * nbr + c0 + j] = acc[i][j] * scale;
+            for (int j = 0; j < kCPT; ++j) {
+                const int c = cg_ + 32 * j;
+                if (c < nbr) lt[(kMR * rg + i) * nbr + c] = acc[i][j] * scale;
+            }
     }
     __syncthreads();
-    // row max over valid columns (0 when none)
-    for (int r = warp; r < kRows; r += kThreads / 32) {
-        float m = -INFINITY;
-        for (int c = lane; c < nbr; c += 32)
-            if (cnts[c] > 0) m = fmaxf(m, lt[r * nbr + c]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (m == -INFINITY) m = 0.0f;
-        if (lane == 0) {
-            rmax[r] = m;
-            if (r < rows_here) mlo[(size_t)bh * nbr + r0 + r] = m;
-        }
-    }
-    __syncthreads();
-    // keys (shared + global), exported logits
-    const int n_here = rows_here * nbr;
-    int flag = 0;
-    for (int e = t; e < n_here; e += kThreads) {
-        const int r = e / nbr, c = e - r * nbr;
-        const int gr = r0 + r;
-        const float l = lt[e];
-        float x = l - rmax[r];
-        if (x == 0.0f) x = 0.0f;   // canonical +0
-        if (!(fabsf(x) < 2500.0f)) flag = 1;
-        int tier = 0;
-        if (first_n > 0 && (gr < first_n || c < first_n)) ++tier;
-        tier += band_of(gr, c, diag_n);
-        if (cnts[gr] <= 0) tier -= 2;
-        if (cnts[c] <= 0) tier -= 2;
-        const unsigned long long key =
-            ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
-        sk[e] = key;
-        keys_out[(size_t)bh * nbr2 + (size_t)gr * nbr + c] = key;
-        if (logit_out) logit_out[(size_t)bh * nbr2 + (size_t)gr * nbr + c] = l;
-    }
-    if (flag) atomicOr(&cs.flag, 1);
-    // the histograms of the first two passes reuse the K-hat tile (rank 0's
-    // copy is cleared here, before any CTA adds into it)
-    unsigned int *hist01 = reinterpret_cast<unsigned int *>(kT);
-    if (rank == 0)
-        for (int i = t; i < 2 * kHistBins; i += kThreads) hist01[i] = 0u;
-    cluster.sync();   // histograms clear; every CTA of the cluster is running
-    if (t == 0 && cs.flag) atomicOr(status, kDevKeyRange);
+    // the K-hat tile is dead: it becomes the cluster histograms, cleared
+    // before this CTA's arrival at the cluster barrier that every CTA waits on
+    // before adding into another CTA's histograms
+    unsigned int *hist0 = reinterpret_cast<unsigned int *>(ks);
+    for (int i = t; i < kSelWords / 4; i += kThreads)
+        reinterpret_cast<uint4 *>(hist0)[i] = make_uint4(0u, 0u, 0u, 0u);
+    cluster_arrive();
 
-    // ------------------------------------------------------------ radix passes
-    // Every CTA adds its histogram into rank 0's buffer of the pass; rank 0
-    // locates the bucket of the k-th key in its own shared memory and
-    // publishes it.  A pass whose bucket is taken whole ends the search early:
-    // the threshold is then compared at that digit's bit.
-    unsigned int *hist_local[3] = {hist01, hist01 + kHistBins, cs.hist2};
-    unsigned long long prefix = 0ull;
-    unsigned int need = (unsigned)k;
-    int sh = 0;            // comparisons against the threshold use key >> sh
-    bool done = false;
-    for (int pass = 0; pass < 3 && !done; ++pass) {
-        const int shift = pass == 0 ? (kHist1Bits + kHist2Bits) : (pass == 1 ? kHist2Bits : 0);
-        const int bits = pass == 0 ? kHist0Bits : (pass == 1 ? kHist1Bits : kHist2Bits);
-        const int hi = shift + bits;
-        const unsigned long long want = prefix >> hi;
-        const unsigned int dmask = (1u << bits) - 1u;
-        for (int i = t; i < (1 << bits); i += kThreads) cs.lh[i] = 0u;
-        __syncthreads();
-        for (int e0 = (t & ~31); e0 < n_here; e0 += kThreads) {
-            const int e = e0 + lane;
-            const unsigned long long key = e < n_here ? sk[e] : ~0ull;
-            warp_hist_add(cs.lh, (unsigned)(key >> shift) & dmask, e < n_here && (key >> hi) == want);
-        }
-        __syncthreads();
-        unsigned int *hb = cluster.map_shared_rank(hist_local[pass], 0);
-        for (int i = t; i < (1 << bits); i += kThreads)
-            if (cs.lh[i]) atomicAdd(&hb[i], cs.lh[i]);
-        cluster.sync();   // the cluster histogram of this pass is complete
-        if (rank == 0) {
-            unsigned int *h = hist_local[pass];
-            find_bucket<kThreads>([h](int i) { return h[i]; }, 1 << bits, need, cs.s_tmp, &cs.bin,
-                                  &cs.bin_need);
-            if (t == 0) {
-                const unsigned int in_bin = h[cs.bin];
-                cs.pub_prefix = prefix | ((unsigned long long)cs.bin << shift);
-                cs.pub_done = (cs.bin_need == in_bin) ? 1 : 0;
-                cs.pub_need = cs.bin_need;
+    // ------------------------------------------------------------ row max, keys, pass-0 histogram
+    // one warp per row; lane owns columns lane + 32*j
+    {
+        int flag = 0;
+        for (int rr = warp; rr < kRows; rr += kWarps) {
+            const bool row_ok = rr < rows_here;   // warp-uniform
+            const int gr = r0 + rr;
+            float lv[kCPT];
+            float m = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kCPT; ++j) {
+                const int c = lane + 32 * j;
+                const bool ok = row_ok && c < nbr;
+                lv[j] = ok ? lt[rr * nbr + c] : 0.0f;
+                if (ok && cnts[c] > 0) m = fmaxf(m, lv[j]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (m == -INFINITY) m = 0.0f;
+            if (row_ok && lane == 0) mlo[(size_t)bh * nbr + gr] = m;
+            const int row_empty = row_ok && cnts[min(gr, nbr - 1)] <= 0;
+#pragma unroll
+            for (int j = 0; j < kCPT; ++j) {
+                const int c = lane + 32 * j;
+                const bool ok = row_ok && c < nbr;
+                unsigned long long key = 0ull;
+                if (ok) {
+                    float x = lv[j] - m;
+                    if (x == 0.0f) x = 0.0f;   // canonical +0
+                    if (!(fabsf(x) < 2500.0f)) flag = 1;
+                    int tier = 0;
+                    if (first_n > 0 && (gr < first_n || c < first_n)) ++tier;
+                    tier += band_of(gr, c, diag_n);
+                    if (row_empty) tier -= 2;
+                    if (cnts[c] <= 0) tier -= 2;
+                    key = ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
+                    sk[rr * nbr + c] = key;
+                    const size_t gi = (size_t)bh * nbr2 + (size_t)gr * nbr + c;
+                    if (keys_out) keys_out[gi] = key;
+                    if (logit_out) logit_out[gi] = lv[j];
+                }
+                warp_hist_add(cs.lh, (unsigned)(key >> (kHist1Bits + kHist2Bits)) & ((1u << kHist0Bits) - 1u), ok);
             }
         }
-        cluster.sync();   // rank 0 published the bucket
-        prefix = cs0->pub_prefix;
-        need = cs0->pub_need;
-        done = cs0->pub_done != 0;
-        sh = shift;
+        if (flag) atomicOr(&cs.flag, 1);
+    }
+    __syncthreads();
+    if (t == 0 && cs.flag) atomicOr(status, kDevKeyRange);
+    cluster_wait();   // every CTA's histograms are clear
+
+    // ------------------------------------------------------------ radix select
+    // First digit: every CTA adds its histogram into every CTA's copy of the
+    // cluster histogram, so after one cluster barrier each CTA locates the
+    // bucket of the k-th key on its own (same sums, same result everywhere).
+    // If the bucket is not taken whole, its keys (usually a few hundred) are
+    // gathered into rank 0, which resolves the two lower digits alone and
+    // publishes the threshold; a bucket too large to gather takes the lower
+    // digits through cluster histograms like the first.  A digit whose bucket
+    // is taken whole ends the search: the threshold is then compared at that
+    // digit's bit.
+    const int n_here = rows_here * nbr;
+    const unsigned int lt_mask = (1u << lane) - 1u;
+    auto push_hist = [&](unsigned int *hp, int nbins) {
+        for (int i = t; i < nbins; i += kThreads) {
+            const unsigned int v = cs.lh[i];
+            if (v) {
+                for (int j = 0; j < ncta; ++j) {
+                    int dst = rank + j;
+                    if (dst >= ncta) dst -= ncta;
+                    atomicAdd(cluster.map_shared_rank(hp, dst) + i, v);
+                }
+                cs.lh[i] = 0u;
+            }
+        }
+    };
+    constexpr int kShift0 = kHist1Bits + kHist2Bits;
+    push_hist(hist0, 1 << kHist0Bits);
+    cluster.sync();   // the first digit's cluster histogram is complete in every CTA
+    find_bucket_smem<kThreads>(hist0, 1 << kHist0Bits, (unsigned)k, cs.s_tot, &cs.bin, &cs.bin_need);
+    unsigned long long prefix = (unsigned long long)cs.bin << kShift0;
+    unsigned int need = cs.bin_need;
+    int sh = kShift0;
+    const unsigned int in_bin0 = hist0[cs.bin];
+    if (need != in_bin0) {
+        if (in_bin0 <= (unsigned)kCand) {
+            unsigned long long *cand = reinterpret_cast<unsigned long long *>(hist0 + (1 << kHist0Bits));
+            unsigned long long *cand0 = cluster.map_shared_rank(cand, 0);
+            int *cand_n0 = cluster.map_shared_rank(&cs.cand_n, 0);
+            const unsigned long long want0 = prefix >> kShift0;
+            for (int e0 = warp * 32; e0 < n_here; e0 += kThreads) {
+                const int e = e0 + lane;
+                const unsigned long long key = e < n_here ? sk[e] : 0ull;
+                const bool m = e < n_here && (key >> kShift0) == want0;
+                const unsigned int bal = __ballot_sync(0xffffffffu, m);
+                if (bal) {
+                    int base = 0;
+                    if (lane == 0) base = atomicAdd(cand_n0, __popc(bal));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (m) cand0[base + __popc(bal & lt_mask)] = key;
+                }
+            }
+            cluster.sync();   // rank 0 holds the bucket's keys
+            if (rank == 0) {
+                const int n = (int)in_bin0;
+                for (int pass = 1; pass < 3; ++pass) {
+                    const int shift = pass == 1 ? kHist2Bits : 0;
+                    const int bits = pass == 1 ? kHist1Bits : kHist2Bits;
+                    const int hi = shift + bits;
+                    const unsigned long long want = prefix >> hi;
+                    const unsigned int dmask = (1u << bits) - 1u;
+                    for (int e0 = warp * 32; e0 < n; e0 += kThreads) {
+                        const int e = e0 + lane;
+                        const unsigned long long key = e < n ? cand[e] : ~0ull;
+                        warp_hist_add(cs.lh, (unsigned)(key >> shift) & dmask, e < n && (key >> hi) == want);
+                    }
+                    __syncthreads();
+                    find_bucket_smem<kThreads>(cs.lh, 1 << bits, need, cs.s_tot, &cs.bin, &cs.bin_need);
+                    const int bin = cs.bin;
+                    const unsigned int bin_need = cs.bin_need;
+                    const bool whole = bin_need == cs.lh[bin];
+                    prefix |= (unsigned long long)bin << shift;
+                    need = bin_need;
+                    sh = shift;
+                    __syncthreads();   // lh[bin] read everywhere
+                    for (int i = t; i < (1 << bits); i += kThreads) cs.lh[i] = 0u;
+                    __syncthreads();
+                    if (whole) break;
+                }
+                if (t < ncta) {
+                    ClusterShared *dst = cluster.map_shared_rank(&cs, t);
+                    dst->pub_prefix = prefix;
+                    dst->pub_need = need;
+                    dst->pub_sh = sh;
+                }
+            }
+            cluster.sync();   // every CTA holds the threshold
+            prefix = cs.pub_prefix;
+            need = cs.pub_need;
+            sh = cs.pub_sh;
+        } else {
+            for (int pass = 1; pass < 3; ++pass) {
+                const int shift = pass == 1 ? kHist2Bits : 0;
+                const int bits = pass == 1 ? kHist1Bits : kHist2Bits;
+                const int hi = shift + bits;
+                const unsigned long long want = prefix >> hi;
+                const unsigned int dmask = (1u << bits) - 1u;
+                for (int e0 = warp * 32; e0 < n_here; e0 += kThreads) {
+                    const int e = e0 + lane;
+                    const unsigned long long key = e < n_here ? sk[e] : ~0ull;
+                    warp_hist_add(cs.lh, (unsigned)(key >> shift) & dmask, e < n_here && (key >> hi) == want);
+                }
+                __syncthreads();
+                unsigned int *hp = hist0 + (1 << kHist0Bits) + (pass - 1) * kHistBins;
+                push_hist(hp, 1 << bits);
+                cluster.sync();   // this digit's cluster histogram is complete in every CTA
+                find_bucket_smem<kThreads>(hp, 1 << bits, need, cs.s_tot, &cs.bin, &cs.bin_need);
+                const int bin = cs.bin;
+                const unsigned int bin_need = cs.bin_need;
+                const bool whole = bin_need == hp[bin];
+                prefix |= (unsigned long long)bin << shift;
+                need = bin_need;
+                sh = shift;
+                if (whole) break;
+            }
+        }
     }
     const unsigned long long Tsh = prefix >> sh;
     if (rank == 0 && t == 0) {
@@ -281,25 +388,27 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
     }
 
     // ------------------------------------------------------------ per-row counts and scans
-    for (int r = warp; r < kRows; r += kThreads / 32) {
+    // each row's (above, at) threshold counts go to every CTA of the cluster
+    for (int rr = warp; rr < kRows; rr += kWarps) {
         int g = 0, e = 0;
-        if (r < rows_here)
-            for (int c = lane; c < nbr; c += 32) {
-                const unsigned long long kk = sk[r * nbr + c] >> sh;
-                g += kk > Tsh;
-                e += kk == Tsh;
-            }
+        if (rr < rows_here)
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            g += __shfl_xor_sync(0xffffffffu, g, o);
-            e += __shfl_xor_sync(0xffffffffu, e, o);
-        }
-        if (lane == 0 && r < rows_here) {
-            cs0->all_gt[r0 + r] = g;
-            cs0->all_eq[r0 + r] = e;
+            for (int j = 0; j < kCPT; ++j) {
+                const int c = lane + 32 * j;
+                if (c < nbr) {
+                    const unsigned long long kk = sk[rr * nbr + c] >> sh;
+                    g += kk > Tsh;
+                    e += kk == Tsh;
+                }
+            }
+        g = __reduce_add_sync(0xffffffffu, g);
+        e = __reduce_add_sync(0xffffffffu, e);
+        if (rr < rows_here && lane < ncta) {
+            cluster.map_shared_rank(cs.all_gt, lane)[r0 + rr] = g;
+            cluster.map_shared_rank(cs.all_eq, lane)[r0 + rr] = e;
         }
     }
-    cluster.sync();   // every row's counts are in rank 0
+    cluster.sync();   // every row's counts are in every CTA; no remote access after this
     // every CTA scans all rows of the head (warp 0, four rows per lane) and
     // keeps what concerns its own rows
     if (warp == 0) {
@@ -309,8 +418,8 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
 #pragma unroll
         for (int j = 0; j < kPer; ++j) {
             const int r = kPer * lane + j;
-            eqv[j] = r < nbr ? cs0->all_eq[r] : 0;
-            gtv[j] = r < nbr ? cs0->all_gt[r] : 0;
+            eqv[j] = r < nbr ? cs.all_eq[r] : 0;
+            gtv[j] = r < nbr ? cs.all_gt[r] : 0;
             eq_local += eqv[j];
         }
         int x = eq_local;
@@ -363,58 +472,50 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
         }
     }
     __syncthreads();
-    __shared__ int s_ok;
-    if (t == 0) {
-        s_ok = (cs.total_sel == k && cs.total_items <= cap);
-        if (rank == 0) {
-            head_items[bh] = s_ok ? cs.total_items : 0;
-            if (!s_ok) atomicOr(status, kDevCount);
+    const bool ok = cs.total_sel == k && cs.total_items <= cap;
+    if (rank == 0 && t == 0) {
+        head_items[bh] = ok ? cs.total_items : 0;
+        if (!ok) atomicOr(status, kDevCount);
+    }
+    if (!ok) return;
+    // work items: one thread per local row
+    for (int r = t; r < rows_here; r += kThreads) {
+        const int sel = cs.row_sel[r];
+        const int nit = sel > 0 ? (sel + chunk - 1) / chunk : 1;
+        const int rs = bh * k + cs.row_start[r];
+        for (int j = 0; j < nit; ++j) {
+            WorkItem w;
+            w.row = bh * nbr + r0 + r;
+            w.col_start = rs + j * chunk;
+            w.ncols = max(0, min(chunk, sel - j * chunk));
+            w.chunk_info = j | (nit << 16);
+            items[(size_t)bh * cap + cs.row_item[r] + j] = w;
         }
     }
-    __syncthreads();
-    const int s_sel_before = 0, s_item_before = 0;
-    if (s_ok) {
-        // work items: one thread per local row
-        for (int r = t; r < rows_here; r += kThreads) {
-            const int sel = cs.row_sel[r];
-            const int nit = sel > 0 ? (sel + chunk - 1) / chunk : 1;
-            const int rs = bh * k + s_sel_before + cs.row_start[r];
-            for (int j = 0; j < nit; ++j) {
-                WorkItem w;
-                w.row = bh * nbr + r0 + r;
-                w.col_start = rs + j * chunk;
-                w.ncols = max(0, min(chunk, sel - j * chunk));
-                w.chunk_info = j | (nit << 16);
-                items[(size_t)bh * cap + s_item_before + cs.row_item[r] + j] = w;
+    // column lists: one warp per local row, ascending columns
+    for (int r = warp; r < rows_here; r += kWarps) {
+        const int rs = bh * k + cs.row_start[r];
+        const int take = cs.row_take[r];
+        const int gr = r0 + r;
+        int eq_seen = 0, sel_seen = 0;
+        for (int c0 = 0; c0 < nbr; c0 += 32) {
+            const int c = c0 + lane;
+            const unsigned long long kk = c < nbr ? (sk[r * nbr + c] >> sh) : 0ull;
+            const bool is_gt = c < nbr && kk > Tsh;
+            const bool is_eq = c < nbr && kk == Tsh;
+            const unsigned int eqb = __ballot_sync(0xffffffffu, is_eq);
+            const bool sel = is_gt || (is_eq && eq_seen + __popc(eqb & lt_mask) < take);
+            const unsigned int sb = __ballot_sync(0xffffffffu, sel);
+            if (sel) {
+                const int pos = rs + sel_seen + __popc(sb & lt_mask);
+                cols[pos] = c;
+                if (sel_out) sel_out[pos] = gr * nbr + c;
             }
-        }
-        // column lists: one warp per local row, ascending columns
-        const unsigned int lt_mask = (1u << lane) - 1u;
-        for (int r = warp; r < rows_here; r += kThreads / 32) {
-            const int rs = bh * k + s_sel_before + cs.row_start[r];
-            const int take = cs.row_take[r];
-            const int gr = r0 + r;
-            int eq_seen = 0, sel_seen = 0;
-            for (int c0 = 0; c0 < nbr; c0 += 32) {
-                const int c = c0 + lane;
-                const unsigned long long kk = c < nbr ? (sk[r * nbr + c] >> sh) : 0ull;
-                const bool is_gt = c < nbr && kk > Tsh;
-                const bool is_eq = c < nbr && kk == Tsh;
-                const unsigned int eqb = __ballot_sync(0xffffffffu, is_eq);
-                const bool sel = is_gt || (is_eq && eq_seen + __popc(eqb & lt_mask) < take);
-                const unsigned int sb = __ballot_sync(0xffffffffu, sel);
-                if (sel) {
-                    const int pos = rs + sel_seen + __popc(sb & lt_mask);
-                    cols[pos] = c;
-                    if (sel_out) sel_out[pos] = gr * nbr + c;
-                }
-                if (bitmap && lane == 0) bitmap[((size_t)bh * nbr + gr) * wpr + (c0 >> 5)] = sb;
-                eq_seen += __popc(eqb);
-                sel_seen += __popc(sb);
-            }
+            if (bitmap && lane == 0) bitmap[((size_t)bh * nbr + gr) * wpr + (c0 >> 5)] = sb;
+            eq_seen += __popc(eqb);
+            sel_seen += __popc(sb);
         }
     }
-    cluster.sync();   // no CTA leaves while another still reads its shared memory
 }
 
 template <int D>
@@ -442,7 +543,8 @@ cudaError_t launch_typed(const Problem &p, const Workspace &w, float *logit_out,
     const float *qhat = w.pooled;
     const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;
     e = cudaLaunchKernelEx(&cfg, kern, qhat, khat, (const int *)w.cnt, p.H, p.nbr, scale, p.first_n,
-                           p.diag_n, p.k, p.cap, p.chunk, w.keys, w.mlo, logit_out, w.cols, sel_out,
+                           p.diag_n, p.k, p.cap, p.chunk, p.mode == 0 ? w.keys : (unsigned long long *)nullptr,
+                           w.mlo, logit_out, w.cols, sel_out,
                            p.mode == 0 ? w.bitmap : (unsigned int *)nullptr, w.words_per_row, w.items,
                            w.head_items, w.state, w.status);
     if (e != cudaSuccess) return e;
@@ -452,7 +554,7 @@ cudaError_t launch_typed(const Problem &p, const Workspace &w, float *logit_out,
 }  // namespace
 
 bool lowres_select_fused_supported(const Problem &p) {
-    return p.nbr <= kMaxCta * kRows;
+    return p.nbr <= kMaxCta * kRows && p.nbr <= kCT;
 }
 
 cudaError_t launch_lowres_select_fused(const Problem &p, const Workspace &w, float *logit_out,

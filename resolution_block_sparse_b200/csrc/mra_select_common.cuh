@@ -62,6 +62,53 @@ static __device__ __forceinline__ void find_bucket(Load load, int nbins, unsigne
     __syncthreads();
 }
 
+// Same result as find_bucket for a histogram in shared memory, with two block
+// barriers: each warp sums a contiguous segment of the bins, the warp whose
+// segment holds the bucket walks it from the top 32 bins at a time with a
+// shuffle suffix sum.  nbins must be a multiple of 32 * (NT / 32).
+template <int NT>
+static __device__ __forceinline__ void find_bucket_smem(const unsigned int *h, int nbins,
+                                                        unsigned int need,
+                                                        unsigned int *s_tot /* >= NT / 32 */,
+                                                        int *out_bin, unsigned int *out_need) {
+    constexpr int W = NT / 32;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int seg = nbins / W;
+    const unsigned int *hw = h + warp * seg;
+    unsigned int sum = 0;
+    for (int j = lane; j < seg; j += 32) sum += hw[j];
+    sum = __reduce_add_sync(0xffffffffu, sum);
+    if (lane == 0) s_tot[warp] = sum;
+    if (t == 0) {
+        *out_bin = 0;
+        *out_need = 1;
+    }
+    __syncthreads();
+    unsigned int above = 0;
+    for (int w2 = warp + 1; w2 < W; ++w2) above += s_tot[w2];
+    if (above < need && need <= above + sum) {   // warp-uniform
+        for (int j0 = seg - 32; j0 >= 0; j0 -= 32) {
+            const unsigned int v = hw[j0 + lane];
+            unsigned int sfx = v;   // bins j0+lane .. j0+31
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned int y = __shfl_down_sync(0xffffffffu, sfx, o);
+                if (lane + o < 32) sfx += y;
+            }
+            const unsigned int chunk_total = __shfl_sync(0xffffffffu, sfx, 0);
+            if (above + chunk_total >= need) {
+                if (above + sfx >= need && above + sfx - v < need) {
+                    *out_bin = warp * seg + j0 + lane;
+                    *out_need = need - (above + sfx - v);
+                }
+                break;
+            }
+            above += chunk_total;
+        }
+    }
+    __syncthreads();
+}
+
 // The global-memory form used by the multi-CTA passes (histogram in L2).
 static __device__ __forceinline__ void find_bucket_256(const unsigned int *gh, int nbins,
                                                        unsigned int need, unsigned int *s_tmp,
