@@ -101,7 +101,7 @@ struct AttnArgs {
     int cap, H, N, nbr, full;
     float scale_log2;
     const float *mlo, *olo, *llo;
-    float *partial;
+    unsigned char *partial;   // split-row partial slots
     int *row_arrive;
     int *work_next;   // items handed out beyond the first wave (zeroed per call)
     void *out;
@@ -113,7 +113,7 @@ template <int D>
 struct Bf16Smem {
     static constexpr int kTile = 32 * D;
     static constexpr size_t kKvBytes = sizeof(__nv_bfloat16) * 4 * kTile;
-    static constexpr size_t kMergeBytes = sizeof(float) * 32 * (D + 2) + sizeof(MergeSmem);
+    static constexpr size_t kMergeBytes = partial_slot_bytes<D, __nv_bfloat16>() + sizeof(MergeSmem);
     __nv_bfloat16 q[kTile];
     // K/V double buffer; after the block loop the same bytes hold the output
     // staging or, for split rows, the partial and the merge scratch
@@ -327,7 +327,8 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
             reinterpret_cast<uint4 *>(out_blk)[e] = reinterpret_cast<const uint4 *>(ostage)[e];
         return;
     }
-    // row split across work items: (m, l, O) partial, merged by the last one
+    // row split across work items: (m, l) in fp32 and O in bf16 (the
+    // accumulators relative to the item's own maximum), merged by the last one
     float *stage = reinterpret_cast<float *>(&sKV[0][0][0]);
     if (tq == 0) {
         stage[ra] = m_a;
@@ -335,19 +336,19 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
         stage[32 + ra] = l_a;
         stage[32 + rb] = l_b;
     }
+    __nv_bfloat16 *ostage = reinterpret_cast<__nv_bfloat16 *>(stage + 64);
 #pragma unroll
     for (int nd = 0; nd < D / 8; ++nd) {
         const int d = nd * 8 + tq * 2;
-        stage[64 + ra * D + d] = o[nd][0];
-        stage[64 + ra * D + d + 1] = o[nd][1];
-        stage[64 + rb * D + d] = o[nd][2];
-        stage[64 + rb * D + d + 1] = o[nd][3];
+        *reinterpret_cast<__nv_bfloat162 *>(ostage + ra * D + d) = __floats2bfloat162_rn(o[nd][0], o[nd][1]);
+        *reinterpret_cast<__nv_bfloat162 *>(ostage + rb * D + d) = __floats2bfloat162_rn(o[nd][2], o[nd][3]);
     }
     __syncthreads();
-    MergeSmem &sm = *reinterpret_cast<MergeSmem *>(stage + 32 * (D + 2));
-    finish_item<D, kBf16Threads, __nv_bfloat16, SyncAll>(stage, slot, chunk, nchunks, it.row, a.full, a.mlo,
-                                                a.olo, a.llo, a.partial, a.row_arrive,
-                                                mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
+    MergeSmem &sm = *reinterpret_cast<MergeSmem *>(reinterpret_cast<unsigned char *>(stage) +
+                                                   partial_slot_bytes<D, __nv_bfloat16>());
+    finish_item<D, kBf16Threads, __nv_bfloat16, __nv_bfloat16, SyncAll>(
+        reinterpret_cast<const unsigned char *>(stage), slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
+        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
 }
 
 // Persistent: the first wave takes items 0..gridDim.x-1, after that a CTA
@@ -360,6 +361,7 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
 template <int D>
 __global__ void __launch_bounds__(kBf16Threads, 10)
 attn_bf16_kernel(const AttnArgs a, int total_slots, int heads) {
+    pdl_wait();
     __shared__ __align__(128) Bf16Smem<D> sh;
     int i = blockIdx.x;
     for (int t = 0; i < total_slots; ++t) {
@@ -377,6 +379,7 @@ constexpr int kF32Threads = 128;
 template <int D>
 __global__ void __launch_bounds__(kF32Threads)
 attn_f32_kernel(const AttnArgs a) {
+    pdl_wait();
     constexpr int kTile = 32 * D;
     constexpr int kDp = D / 4;
     __shared__ __align__(16) float sK[kTile];
@@ -454,9 +457,9 @@ attn_f32_kernel(const AttnArgs a) {
     for (int i = 0; i < kDp; ++i) stage[64 + qrow * D + d0 + i] = o[i];
     __syncthreads();
     float *out_blk = static_cast<float *>(a.out) + head_off + (size_t)r * kTile;
-    finish_item<D, kF32Threads, float, SyncAll>(stage, slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
-                                       a.llo, a.partial, a.row_arrive,
-                                       mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
+    finish_item<D, kF32Threads, float, float, SyncAll>(
+        reinterpret_cast<const unsigned char *>(stage), slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
+        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
 }
 
 }  // namespace
@@ -480,7 +483,7 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
     a.mlo = w.mlo;
     a.olo = w.olo;
     a.llo = w.llo;
-    a.partial = w.partial;
+    a.partial = reinterpret_cast<unsigned char *>(w.partial);
     a.row_arrive = w.row_arrive;
     a.work_next = w.work_next;
     a.out = out;
@@ -500,13 +503,14 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
             if (sms <= 0) sms = 148;
         }
         const long long pgrid = std::min<long long>(grid, 10LL * sms);
-        if (p.D == 64) attn_bf16_kernel<64><<<(unsigned)pgrid, kBf16Threads, 0, s>>>(a, (int)grid, p.BH);
-        else attn_bf16_kernel<32><<<(unsigned)pgrid, kBf16Threads, 0, s>>>(a, (int)grid, p.BH);
-    } else {
-        if (p.D == 64) attn_f32_kernel<64><<<(unsigned)grid, kF32Threads, 0, s>>>(a);
-        else attn_f32_kernel<32><<<(unsigned)grid, kF32Threads, 0, s>>>(a);
+        if (p.D == 64)
+            return launch_dependent(attn_bf16_kernel<64>, dim3((unsigned)pgrid), dim3(kBf16Threads), 0, s, a,
+                                    (int)grid, p.BH);
+        return launch_dependent(attn_bf16_kernel<32>, dim3((unsigned)pgrid), dim3(kBf16Threads), 0, s, a,
+                                (int)grid, p.BH);
     }
-    return cudaGetLastError();
+    if (p.D == 64) return launch_dependent(attn_f32_kernel<64>, dim3((unsigned)grid), dim3(kF32Threads), 0, s, a);
+    return launch_dependent(attn_f32_kernel<32>, dim3((unsigned)grid), dim3(kF32Threads), 0, s, a);
 }
 
 }  // namespace mra

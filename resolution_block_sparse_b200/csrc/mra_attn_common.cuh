@@ -45,10 +45,21 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v) {
 }
 __device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
 
+// four consecutive partial-output elements as fp32 (16-byte load for fp32
+// partials, 8-byte for bf16 ones); G: through L2 only (written by other CTAs)
 template <bool G>
-__device__ __forceinline__ float4 ldp4(const float4 *p) {
-    if constexpr (G) return __ldcg(p);
-    else return *p;
+__device__ __forceinline__ float4 ld_quad(const float *p) {
+    if constexpr (G) return __ldcg(reinterpret_cast<const float4 *>(p));
+    else return *reinterpret_cast<const float4 *>(p);
+}
+template <bool G>
+__device__ __forceinline__ float4 ld_quad(const __nv_bfloat16 *p) {
+    uint2 u;
+    if constexpr (G) u = __ldcg(reinterpret_cast<const uint2 *>(p));
+    else u = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
 }
 
 constexpr int kMergeGroup = 16;   // partials whose (m, l) are staged at once
@@ -59,23 +70,33 @@ struct MergeSmem {
     float M[32], den[32], resc[32];
 };
 
-// Merge nchunks partials (layout per slot: m[32], l[32], O[32][D]; m in log2
-// units, l and O relative to exp2(m)) with the low-resolution part of the row
-// (full mode) and write the 32 x D output block.
+// Bytes of one partial slot: m[32] and l[32] in fp32, then O[32][D] in PartT.
+template <int D, typename PartT>
+__host__ __device__ constexpr size_t partial_slot_bytes() {
+    return 64 * sizeof(float) + (size_t)32 * D * sizeof(PartT);
+}
+
+// Merge nchunks partials (slot layout above; m in log2 units, l and O
+// relative to exp2(m)) with the low-resolution part of the row (full mode)
+// and write the 32 x D output block.
 //
 // The partials are taken in groups of kMergeGroup: all (m, l) pairs of a group
 // are loaded at once, the running per-row maximum and normaliser move to the
-// group's maximum (earlier groups rescaled), and the O tiles of four partials
-// are in flight together, so the merge costs a few memory round trips rather
-// than two per partial.
-template <int D, int NT, bool G, typename OutT, typename Sync>
-__device__ void merge_write(const float *src0, size_t slot_stride, int nchunks, int full,
+// group's maximum (earlier groups rescaled), and the O tiles of several
+// partials are in flight together, so the merge costs a few memory round
+// trips rather than two per partial.
+template <int D, int NT, bool G, typename OutT, typename PartT, typename Sync>
+__device__ void merge_write(const unsigned char *src0, size_t slot_bytes, int nchunks, int full,
                             float m_lo2, float l_lo, const float *olo_row, const float *qmask,
                             OutT *out_blk, MergeSmem &sm) {
-    static_assert((8 * D) % NT == 0, "a chunk's O tile must split evenly into float4 per thread");
-    constexpr int F = 8 * D / NT;   // float4 of one partial's O tile per thread
-    constexpr int kRowF4 = D / 4;
-    constexpr int kMergeUnroll = F >= 8 ? 1 : 8 / F;
+    static_assert((8 * D) % NT == 0, "a chunk's O tile must split evenly into quads per thread");
+    constexpr int F = 8 * D / NT;   // quads (4 elements) of one partial's O tile per thread
+    constexpr int kRowQ = D / 4;
+    constexpr int kQuadBytes = 4 * (int)sizeof(PartT);
+    // partial tiles in flight per thread: at most 128 bytes of registers
+    constexpr int kMergeUnroll = F * kQuadBytes >= 128 ? 1 : 128 / (F * kQuadBytes);
+    constexpr int kML = kMergeGroup * 32 / NT;   // (m, l) pairs per thread per group
+    static_assert(kML >= 1 && (kMergeGroup * 32) % NT == 0, "merge group layout");
     const int tid = threadIdx.x;
     float4 acc[F];
 #pragma unroll
@@ -86,13 +107,29 @@ __device__ void merge_write(const float *src0, size_t slot_stride, int nchunks, 
     }
     for (int cg = 0; cg < nchunks; cg += kMergeGroup) {
         const int nc = min(kMergeGroup, nchunks - cg);
-        for (int e = tid; e < nc * 32; e += NT) {
-            const int c = e >> 5, q = e & 31;
-            const float *P = src0 + (size_t)(cg + c) * slot_stride;
-            const float l = ldp<G>(P + 32 + q);
-            const float m = ldp<G>(P + q);
-            sm.w[c][q] = l > 0.0f ? m : -INFINITY;
-            sm.l[c][q] = l > 0.0f ? l : 0.0f;
+        {
+            float mv[kML], lv[kML];
+#pragma unroll
+            for (int i = 0; i < kML; ++i) {
+                const int e = tid + i * NT;
+                const int c = e >> 5, q = e & 31;
+                mv[i] = -INFINITY;
+                lv[i] = 0.0f;
+                if (c < nc) {
+                    const float *P = reinterpret_cast<const float *>(src0 + (size_t)(cg + c) * slot_bytes);
+                    lv[i] = ldp<G>(P + 32 + q);
+                    mv[i] = ldp<G>(P + q);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kML; ++i) {
+                const int e = tid + i * NT;
+                const int c = e >> 5, q = e & 31;
+                if (c < nc) {
+                    sm.w[c][q] = lv[i] > 0.0f ? mv[i] : -INFINITY;
+                    sm.l[c][q] = lv[i] > 0.0f ? lv[i] : 0.0f;
+                }
+            }
         }
         Sync::sync();
         if (tid < 32) {
@@ -116,22 +153,22 @@ __device__ void merge_write(const float *src0, size_t slot_stride, int nchunks, 
         if (cg > 0) {
 #pragma unroll
             for (int i = 0; i < F; ++i) {
-                const float r = sm.resc[(tid + i * NT) / kRowF4];
+                const float r = sm.resc[(tid + i * NT) / kRowQ];
                 acc[i].x *= r;
                 acc[i].y *= r;
                 acc[i].z *= r;
                 acc[i].w *= r;
             }
         }
-        // at most 8 float4 loads in flight per thread (register budget)
 #pragma unroll kMergeUnroll
         for (int c = 0; c < nc; ++c) {
-            const float4 *O = reinterpret_cast<const float4 *>(src0 + (size_t)(cg + c) * slot_stride + 64);
+            const PartT *O = reinterpret_cast<const PartT *>(src0 + (size_t)(cg + c) * slot_bytes +
+                                                            64 * sizeof(float));
 #pragma unroll
             for (int i = 0; i < F; ++i) {
                 const int f = tid + i * NT;
-                const float wgt = sm.w[c][f / kRowF4];
-                const float4 v = ldp4<G>(O + f);
+                const float wgt = sm.w[c][f / kRowQ];
+                const float4 v = ld_quad<G>(O + 4 * f);
                 acc[i].x = fmaf(wgt, v.x, acc[i].x);
                 acc[i].y = fmaf(wgt, v.y, acc[i].y);
                 acc[i].z = fmaf(wgt, v.z, acc[i].z);
@@ -160,7 +197,7 @@ __device__ void merge_write(const float *src0, size_t slot_stride, int nchunks, 
 #pragma unroll
     for (int i = 0; i < F; ++i) {
         const int f = tid + i * NT;
-        const int q = f / kRowF4, d = (f % kRowF4) * 4;
+        const int q = f / kRowQ, d = (f % kRowQ) * 4;
         const float fa = sm.resc[q], fb = sm.den[q];
         float4 ol = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         if (full) ol = *reinterpret_cast<const float4 *>(olo_row + d);
@@ -170,32 +207,37 @@ __device__ void merge_write(const float *src0, size_t slot_stride, int nchunks, 
     }
 }
 
-// Shared epilogue: the item's (m, l, O) sit in `stage` (shared, slot layout).
-template <int D, int NT, typename OutT, typename Sync>
-__device__ void finish_item(float *stage, int slot, int chunk, int nchunks, int row, int full,
+// Shared epilogue: the item's (m, l, O) sit in `stage` (shared memory, slot
+// layout of partial_slot_bytes<D, PartT>).  A row that fits one item merges
+// and writes at once; otherwise the slot is copied to the partial buffer and
+// the last item of the row to arrive (counter, no waiting) merges them all.
+template <int D, int NT, typename OutT, typename PartT, typename Sync>
+__device__ void finish_item(const unsigned char *stage, int slot, int chunk, int nchunks, int row, int full,
                             const float *mlo, const float *olo, const float *llo,
-                            float *partial, int *row_arrive, const float *qmask, OutT *out_blk,
+                            unsigned char *partial, int *row_arrive, const float *qmask, OutT *out_blk,
                             MergeSmem &sm, int *s_last) {
+    constexpr size_t kSlot = partial_slot_bytes<D, PartT>();
+    static_assert(kSlot % 16 == 0, "partial slots stay 16-byte aligned");
     const int tid = threadIdx.x;
-    const size_t stride = (size_t)32 * (D + 2);
     const float m_lo2 = full ? mlo[row] * kLog2e : 0.0f;
     const float l_lo = full ? llo[row] : 0.0f;
     const float *olo_row = full ? olo + (size_t)row * D : nullptr;
     if (nchunks == 1) {
-        merge_write<D, NT, false, OutT, Sync>(stage, stride, 1, full, m_lo2, l_lo, olo_row, qmask, out_blk, sm);
+        merge_write<D, NT, false, OutT, PartT, Sync>(stage, kSlot, 1, full, m_lo2, l_lo, olo_row, qmask,
+                                                     out_blk, sm);
         return;
     }
-    float4 *dst = reinterpret_cast<float4 *>(partial + (size_t)slot * stride);
-    const float4 *src = reinterpret_cast<const float4 *>(stage);
-    for (int e = tid; e < (int)stride / 4; e += NT) dst[e] = src[e];
+    uint4 *dst = reinterpret_cast<uint4 *>(partial + (size_t)slot * kSlot);
+    const uint4 *src = reinterpret_cast<const uint4 *>(stage);
+    for (int e = tid; e < (int)(kSlot / 16); e += NT) dst[e] = src[e];
     __threadfence();
     Sync::sync();
     if (tid == 0) *s_last = (atomicAdd(&row_arrive[row], 1) == nchunks - 1);
     Sync::sync();
     if (!*s_last) return;
     __threadfence();
-    merge_write<D, NT, true, OutT, Sync>(partial + (size_t)(slot - chunk) * stride, stride, nchunks, full,
-                                   m_lo2, l_lo, olo_row, qmask, out_blk, sm);
+    merge_write<D, NT, true, OutT, PartT, Sync>(partial + (size_t)(slot - chunk) * kSlot, kSlot, nchunks, full,
+                                                m_lo2, l_lo, olo_row, qmask, out_blk, sm);
     if (tid == 0) row_arrive[row] = 0;
 }
 

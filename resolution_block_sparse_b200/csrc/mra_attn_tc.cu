@@ -150,7 +150,7 @@ struct TcArgs {
     int cap, H, N, nbr, total_slots, full;
     float scale_log2;
     const float *mlo, *olo, *llo;
-    float *partial;
+    unsigned char *partial;   // split-row partial slots
     int *row_arrive;
     __nv_bfloat16 *out;
     unsigned int *status;
@@ -181,6 +181,7 @@ struct ItemWalk {
 __global__ void __launch_bounds__(kThreadsTC, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, const TcArgs a) {
+    pdl_wait();
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) unsigned long long bar_qfull[2], bar_qempty[2], bar_kfull[kStages],
         bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages], bar_sfull[2], bar_sempty[2],
@@ -591,9 +592,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             } else {
                 // row split across work items: (max, sum, O) partial, the last
                 // item of the row merges (shared epilogue)
-                const size_t stride = (size_t)32 * (64 + 2);
+                constexpr size_t kSlot = partial_slot_bytes<64, float>();
                 const int slot = walk.slot;
-                float *dst = a.partial + (size_t)slot * stride;
+                float *dst = reinterpret_cast<float *>(a.partial + (size_t)slot * kSlot);
                 if (warp == 0) {
                     dst[lane] = m_hi;
                     dst[32 + lane] = l_hi;
@@ -612,8 +613,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     const float m_lo2 = a.full ? a.mlo[it.row] * kLog2e : 0.0f;
                     const float l_lo = a.full ? a.llo[it.row] : 0.0f;
                     const float *olo_row = a.full ? a.olo + (size_t)it.row * 64 : nullptr;
-                    merge_write<64, kConsumers, true, __nv_bfloat16, SyncNamed128>(
-                        a.partial + (size_t)(slot - chunk) * stride, stride, nchunks, a.full, m_lo2, l_lo,
+                    merge_write<64, kConsumers, true, __nv_bfloat16, float, SyncNamed128>(
+                        a.partial + (size_t)(slot - chunk) * kSlot, kSlot, nchunks, a.full, m_lo2, l_lo,
                         olo_row, qmask, out_blk, msm);
                     if (tid == 0) a.row_arrive[it.row] = 0;
                 }
@@ -710,13 +711,12 @@ cudaError_t launch_attention_tc(const Problem &p, const Workspace &w, const void
     a.mlo = w.mlo;
     a.olo = w.olo;
     a.llo = w.llo;
-    a.partial = w.partial;
+    a.partial = reinterpret_cast<unsigned char *>(w.partial);
     a.row_arrive = w.row_arrive;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.status = w.status;
     const int grid = (int)std::min<long long>((long long)a.total_slots, 2LL * g_num_sms);
-    attn_tc_kernel<<<grid, kThreadsTC, kSmemAlloc, s>>>(tq, tk, tv, a);
-    return cudaGetLastError();
+    return launch_dependent(attn_tc_kernel, dim3(grid), dim3(kThreadsTC), kSmemAlloc, s, tq, tk, tv, a);
 }
 
 }  // namespace mra

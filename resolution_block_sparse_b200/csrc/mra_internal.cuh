@@ -14,6 +14,8 @@
 //               online max/sum, merged with the low-resolution part
 #pragma once
 
+#include <utility>
+
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -106,6 +108,33 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
                     int *launch_count);
 
 // Launchers (each returns cudaGetLastError() of its launches).
+// ---------------------------------------------------------------- dependent launches
+// Every kernel after the first of a forward pass is launched with
+// programmatic stream serialization: it may be scheduled while the kernel
+// before it drains, and it calls pdl_wait() (which returns once every earlier
+// kernel of the stream has completed and its writes are visible) before it
+// touches their results.  Kernels call pdl_trigger() early so that the next
+// launch is not held back until they exit.  Without the launch attribute both
+// instructions are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_pool(const Problem &p, const Workspace &w, const void *q, const void *k,
                         const void *v, const float *mask, cudaStream_t s);
 cudaError_t launch_lowres_keys(const Problem &p, const Workspace &w, float *logit_out,

@@ -49,6 +49,7 @@ lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ kha
                    float *__restrict__ mlo, float *__restrict__ logit_out,
                    unsigned int *__restrict__ hist, unsigned int *__restrict__ arrive,
                    SelState *__restrict__ state, unsigned int *__restrict__ status) {
+    pdl_wait();
     constexpr int RG = R / 4;                  // row groups
     constexpr int CG = kLowresThreads / RG;    // column groups
     constexpr int CT = 4 * CG;                 // columns per tile
@@ -225,6 +226,7 @@ __global__ void __launch_bounds__(kLowresThreads)
 lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int *__restrict__ bitmap,
                  int wpr, const int *__restrict__ cnt, const float *__restrict__ vhat, int H,
                  int nbr, long long nbr2, float *__restrict__ olo, float *__restrict__ llo) {
+    pdl_wait();
     constexpr int R = 32;
     constexpr int kCt = 32;
     constexpr int kVL = kCt * D / 4 / kLowresThreads;      // float4 loads of the V-hat tile
@@ -332,10 +334,9 @@ cudaError_t launch_keys_rt(const Problem &p, const Workspace &w, float *logit_ou
     const float scale = 1.0f / sqrtf((float)p.D);
     const float *qhat = w.pooled;
     const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;
-    lowres_keys_kernel<D, R><<<grid, kLowresThreads, smem, s>>>(
+    return launch_dependent(lowres_keys_kernel<D, R>, dim3(grid), dim3(kLowresThreads), smem, s, 
         qhat, khat, w.cnt, p.H, p.nbr, p.nbr2, scale, p.first_n, p.diag_n, p.k, w.keys, w.mlo,
         logit_out, w.hist, w.arrive, w.state, w.status);
-    return cudaGetLastError();
 }
 
 template <int D>
@@ -358,14 +359,10 @@ cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t 
     dim3 grid((p.nbr + 31) / 32, p.BH);
     const float *vhat = w.pooled + (size_t)2 * p.BH * p.nbr * p.D;
     if (p.D == 64)
-        lowres_pv_kernel<64><<<grid, kLowresThreads, 0, s>>>(w.keys, w.bitmap, w.words_per_row,
-                                                             w.cnt, vhat, p.H, p.nbr, p.nbr2,
-                                                             w.olo, w.llo);
-    else
-        lowres_pv_kernel<32><<<grid, kLowresThreads, 0, s>>>(w.keys, w.bitmap, w.words_per_row,
-                                                             w.cnt, vhat, p.H, p.nbr, p.nbr2,
-                                                             w.olo, w.llo);
-    return cudaGetLastError();
+        return launch_dependent(lowres_pv_kernel<64>, grid, dim3(kLowresThreads), 0, s, w.keys, w.bitmap,
+                                w.words_per_row, w.cnt, vhat, p.H, p.nbr, p.nbr2, w.olo, w.llo);
+    return launch_dependent(lowres_pv_kernel<32>, grid, dim3(kLowresThreads), 0, s, w.keys, w.bitmap,
+                            w.words_per_row, w.cnt, vhat, p.H, p.nbr, p.nbr2, w.olo, w.llo);
 }
 
 }  // namespace mra

@@ -37,6 +37,9 @@ constexpr int kMR = kRows / kRG;          // rows per thread tile (2)
 constexpr int kCT = 128;                  // columns of the map (at most)
 constexpr int kCPT = kCT / kCG;           // columns per thread (4), strided by 32
 constexpr int kMaxCta = 8;                // portable cluster size
+constexpr int kHistBits12 = 12;           // the two lower digits
+constexpr unsigned int kMask12 = (1u << kHistBits12) - 1u;
+static_assert(kHist1Bits == kHistBits12 && kHist2Bits == kHistBits12, "lower digits are 12 bits");
 
 // Row stride of the K-hat tile in shared memory: D + 4 floats keeps rows
 // 16-byte aligned and puts the rows read by 8 consecutive lanes in distinct
@@ -80,6 +83,8 @@ struct ClusterShared {
     int bin;
     unsigned int bin_need;
     int cand_n;                     // rank 0: keys gathered so far
+    int small_n;                    // rank 0: keys of a bucket of at most 32
+    unsigned long long small[32];
     unsigned long long pub_prefix;  // threshold published by rank 0
     unsigned int pub_need;
     int pub_sh;
@@ -100,6 +105,7 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                              unsigned int *__restrict__ bitmap, int wpr, WorkItem *__restrict__ items,
                              int *__restrict__ head_items, SelState *__restrict__ state,
                              unsigned int *__restrict__ status) {
+    pdl_wait();
     constexpr int KS = ks_stride<D>();
     constexpr int kF4 = D / 4;   // float4 per row of Q-hat / K-hat
     cg::cluster_group cluster = cg::this_cluster();
@@ -290,7 +296,7 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
     constexpr int kShift0 = kHist1Bits + kHist2Bits;
     push_hist(hist0, 1 << kHist0Bits);
     cluster.sync();   // the first digit's cluster histogram is complete in every CTA
-    find_bucket_smem<kThreads>(hist0, 1 << kHist0Bits, (unsigned)k, cs.s_tot, &cs.bin, &cs.bin_need);
+    find_bucket_smem<kThreads, 1 << kHist0Bits>(hist0, (unsigned)k, cs.s_tot, &cs.bin, &cs.bin_need);
     unsigned long long prefix = (unsigned long long)cs.bin << kShift0;
     unsigned int need = cs.bin_need;
     int sh = kShift0;
@@ -301,16 +307,23 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
             unsigned long long *cand0 = cluster.map_shared_rank(cand, 0);
             int *cand_n0 = cluster.map_shared_rank(&cs.cand_n, 0);
             const unsigned long long want0 = prefix >> kShift0;
+            // one remote atomic per warp reserves the warp's slots
+            int nmine = 0;
             for (int e0 = warp * 32; e0 < n_here; e0 += kThreads) {
                 const int e = e0 + lane;
-                const unsigned long long key = e < n_here ? sk[e] : 0ull;
-                const bool m = e < n_here && (key >> kShift0) == want0;
-                const unsigned int bal = __ballot_sync(0xffffffffu, m);
-                if (bal) {
-                    int base = 0;
-                    if (lane == 0) base = atomicAdd(cand_n0, __popc(bal));
-                    base = __shfl_sync(0xffffffffu, base, 0);
+                nmine += __popc(__ballot_sync(0xffffffffu, e < n_here && (sk[min(e, n_here - 1)] >> kShift0) == want0));
+            }
+            if (nmine) {
+                int base = 0;
+                if (lane == 0) base = atomicAdd(cand_n0, nmine);
+                base = __shfl_sync(0xffffffffu, base, 0);
+                for (int e0 = warp * 32; e0 < n_here; e0 += kThreads) {
+                    const int e = e0 + lane;
+                    const unsigned long long key = e < n_here ? sk[e] : 0ull;
+                    const bool m = e < n_here && (key >> kShift0) == want0;
+                    const unsigned int bal = __ballot_sync(0xffffffffu, m);
                     if (m) cand0[base + __popc(bal & lt_mask)] = key;
+                    base += __popc(bal);
                 }
             }
             cluster.sync();   // rank 0 holds the bucket's keys
@@ -318,27 +331,62 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                 const int n = (int)in_bin0;
                 for (int pass = 1; pass < 3; ++pass) {
                     const int shift = pass == 1 ? kHist2Bits : 0;
-                    const int bits = pass == 1 ? kHist1Bits : kHist2Bits;
-                    const int hi = shift + bits;
+                    const int hi = shift + kHistBits12;
                     const unsigned long long want = prefix >> hi;
-                    const unsigned int dmask = (1u << bits) - 1u;
                     for (int e0 = warp * 32; e0 < n; e0 += kThreads) {
                         const int e = e0 + lane;
                         const unsigned long long key = e < n ? cand[e] : ~0ull;
-                        warp_hist_add(cs.lh, (unsigned)(key >> shift) & dmask, e < n && (key >> hi) == want);
+                        warp_hist_add(cs.lh, (unsigned)(key >> shift) & kMask12, e < n && (key >> hi) == want);
                     }
                     __syncthreads();
-                    find_bucket_smem<kThreads>(cs.lh, 1 << bits, need, cs.s_tot, &cs.bin, &cs.bin_need);
+                    find_bucket_smem<kThreads, kHistBins>(cs.lh, need, cs.s_tot, &cs.bin, &cs.bin_need);
                     const int bin = cs.bin;
                     const unsigned int bin_need = cs.bin_need;
-                    const bool whole = bin_need == cs.lh[bin];
+                    const unsigned int in_bin = cs.lh[bin];
                     prefix |= (unsigned long long)bin << shift;
                     need = bin_need;
                     sh = shift;
                     __syncthreads();   // lh[bin] read everywhere
-                    for (int i = t; i < (1 << bits); i += kThreads) cs.lh[i] = 0u;
-                    __syncthreads();
-                    if (whole) break;
+                    for (int i = t; i < kHistBins; i += kThreads) cs.lh[i] = 0u;
+                    if (bin_need == in_bin) break;   // bucket taken whole
+                    if (pass == 1 && in_bin <= 32u) {
+                        // at most 32 keys share the top 23 bits: warp 0 finds the
+                        // need-th largest of them by counting, at full precision
+                        if (t == 0) cs.small_n = 0;
+                        __syncthreads();
+                        const unsigned long long want1 = prefix >> kHist2Bits;
+                        for (int e0 = warp * 32; e0 < n; e0 += kThreads) {
+                            const int e = e0 + lane;
+                            const unsigned long long key = e < n ? cand[e] : 0ull;
+                            const bool m = e < n && (key >> kHist2Bits) == want1;
+                            const unsigned int bal = __ballot_sync(0xffffffffu, m);
+                            int base = 0;
+                            if (bal && lane == 0) base = atomicAdd(&cs.small_n, __popc(bal));
+                            base = __shfl_sync(0xffffffffu, base, 0);
+                            if (m) cs.small[base + __popc(bal & lt_mask)] = key;
+                        }
+                        __syncthreads();
+                        if (warp == 0) {
+                            const bool valid = lane < (int)in_bin;
+                            const unsigned long long mine = valid ? cs.small[lane] : 0ull;
+                            int gt = 0, ge = 0;
+                            for (int j = 0; j < (int)in_bin; ++j) {
+                                const unsigned long long kj = __shfl_sync(0xffffffffu, mine, j);
+                                gt += kj > mine;
+                                ge += kj >= mine;
+                            }
+                            if (valid && gt < (int)need && (int)need <= ge) {
+                                cs.pub_prefix = mine;   // equal keys write the same values
+                                cs.pub_need = need - (unsigned)gt;
+                            }
+                        }
+                        __syncthreads();
+                        prefix = cs.pub_prefix;
+                        need = cs.pub_need;
+                        sh = 0;
+                        break;
+                    }
+                    __syncthreads();   // lh cleared before the next pass adds
                 }
                 if (t < ncta) {
                     ClusterShared *dst = cluster.map_shared_rank(&cs, t);
@@ -367,7 +415,7 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                 unsigned int *hp = hist0 + (1 << kHist0Bits) + (pass - 1) * kHistBins;
                 push_hist(hp, 1 << bits);
                 cluster.sync();   // this digit's cluster histogram is complete in every CTA
-                find_bucket_smem<kThreads>(hp, 1 << bits, need, cs.s_tot, &cs.bin, &cs.bin_need);
+                find_bucket_smem<kThreads, kHistBins>(hp, need, cs.s_tot, &cs.bin, &cs.bin_need);
                 const int bin = cs.bin;
                 const unsigned int bin_need = cs.bin_need;
                 const bool whole = bin_need == hp[bin];
@@ -532,13 +580,15 @@ cudaError_t launch_typed(const Problem &p, const Workspace &w, float *logit_out,
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = ncta;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see launch_dependent
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const float scale = 1.0f / sqrtf((float)p.D);
     const float *qhat = w.pooled;
     const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;

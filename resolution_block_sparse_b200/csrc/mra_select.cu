@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(kThreads)
 radix_pass_kernel(const unsigned long long *__restrict__ keys, long long nbr2, long long chunk,
                   int pass, int shift, int bits, unsigned int *__restrict__ hist,
                   unsigned int *__restrict__ arrive, SelState *__restrict__ state) {
+    pdl_wait();
     __shared__ unsigned int h[kHistBins];
     __shared__ unsigned int s_tmp[256];
     __shared__ int s_last, s_bin;
@@ -79,6 +80,7 @@ radix_pass_kernel(const unsigned long long *__restrict__ keys, long long nbr2, l
 __global__ void __launch_bounds__(kThreads)
 row_counts_kernel(const unsigned long long *__restrict__ keys, const SelState *__restrict__ state,
                   int nbr, long long nbr2, int rows, int *__restrict__ gt, int *__restrict__ eq) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
     if (row >= rows) return;
@@ -138,6 +140,7 @@ row_scan_kernel(const int *__restrict__ gt, const int *__restrict__ eq,
                 const SelState *__restrict__ state, int nbr, int k, int cap, int chunk,
                 int *__restrict__ row_start, int *__restrict__ take_eq, WorkItem *__restrict__ items,
                 int *__restrict__ head_items, unsigned int *__restrict__ status) {
+    pdl_wait();
     __shared__ int s_warp[32];
     const int bh = blockIdx.x;
     const int t = threadIdx.x;
@@ -202,6 +205,7 @@ cols_kernel(const unsigned long long *__restrict__ keys, const SelState *__restr
             const int *__restrict__ row_start, const int *__restrict__ take_eq, int nbr,
             long long nbr2, int rows, int k, int *__restrict__ cols, int32_t *__restrict__ sel_out,
             unsigned int *__restrict__ bitmap, int wpr) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
     if (row >= rows) return;
@@ -245,6 +249,7 @@ select_small_kernel(const unsigned long long *__restrict__ keys, SelState *__res
                     int nbr, int k, int cap, int chunk, int *__restrict__ cols, int32_t *__restrict__ sel_out,
                     unsigned int *__restrict__ bitmap, int wpr, WorkItem *__restrict__ items,
                     int *__restrict__ head_items, unsigned int *__restrict__ status) {
+    pdl_wait();
     extern __shared__ __align__(16) unsigned long long sk[];   // [nbr * nbr]
     __shared__ unsigned int h[kHistBins];
     __shared__ unsigned int s_tmp[kSmallThreads];
@@ -435,23 +440,20 @@ cudaError_t launch_radix_pass(const Problem &p, const Workspace &w, int pass, cu
     const int shift = (pass == 1) ? kHist2Bits : 0;
     const int bits = (pass == 1) ? kHist1Bits : kHist2Bits;
     dim3 grid(p.radix_ctas, p.BH);
-    radix_pass_kernel<<<grid, kThreads, 0, s>>>(w.keys, p.nbr2, p.radix_chunk, pass, shift, bits,
+    return launch_dependent(radix_pass_kernel, dim3(grid), dim3(kThreads), 0, s, w.keys, p.nbr2, p.radix_chunk, pass, shift, bits,
                                                 w.hist, w.arrive, w.state);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_row_counts(const Problem &p, const Workspace &w, cudaStream_t s) {
     const int rows = p.BH * p.nbr;
     const int grid = (rows + kThreads / 32 - 1) / (kThreads / 32);
-    row_counts_kernel<<<grid, kThreads, 0, s>>>(w.keys, w.state, p.nbr, p.nbr2, rows, w.gt, w.eq);
-    return cudaGetLastError();
+    return launch_dependent(row_counts_kernel, dim3(grid), dim3(kThreads), 0, s, w.keys, w.state, p.nbr, p.nbr2, rows, w.gt, w.eq);
 }
 
 cudaError_t launch_row_scan(const Problem &p, const Workspace &w, cudaStream_t s) {
-    row_scan_kernel<<<p.BH, kScanThreads, 0, s>>>(w.gt, w.eq, w.state, p.nbr, p.k, p.cap, p.chunk,
+    return launch_dependent(row_scan_kernel, dim3(p.BH), dim3(kScanThreads), 0, s, w.gt, w.eq, w.state, p.nbr, p.k, p.cap, p.chunk,
                                                   w.row_start, w.take_eq, w.items, w.head_items,
                                                   w.status);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *sel_out,
@@ -460,19 +462,17 @@ cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *s
     cudaError_t e = cudaFuncSetAttribute(select_small_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    select_small_kernel<<<p.BH, kSmallThreads, smem, s>>>(
+    return launch_dependent(select_small_kernel, dim3(p.BH), dim3(kSmallThreads), smem, s,
         w.keys, w.state, p.nbr, p.k, p.cap, p.chunk, w.cols, sel_out, p.mode == 0 ? w.bitmap : nullptr,
         w.words_per_row, w.items, w.head_items, w.status);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_cols(const Problem &p, const Workspace &w, int32_t *sel_out, cudaStream_t s) {
     const int rows = p.BH * p.nbr;
     const int grid = (rows + kThreads / 32 - 1) / (kThreads / 32);
-    cols_kernel<<<grid, kThreads, 0, s>>>(w.keys, w.state, w.row_start, w.take_eq, p.nbr, p.nbr2,
+    return launch_dependent(cols_kernel, dim3(grid), dim3(kThreads), 0, s, w.keys, w.state, w.row_start, w.take_eq, p.nbr, p.nbr2,
                                           rows, p.k, w.cols, sel_out, p.mode == 0 ? w.bitmap : nullptr,
                                           w.words_per_row);
-    return cudaGetLastError();
 }
 
 }  // namespace mra

@@ -63,21 +63,32 @@ static __device__ __forceinline__ void find_bucket(Load load, int nbins, unsigne
 }
 
 // Same result as find_bucket for a histogram in shared memory, with two block
-// barriers: each warp sums a contiguous segment of the bins, the warp whose
-// segment holds the bucket walks it from the top 32 bins at a time with a
-// shuffle suffix sum.  nbins must be a multiple of 32 * (NT / 32).
-template <int NT>
-static __device__ __forceinline__ void find_bucket_smem(const unsigned int *h, int nbins,
-                                                        unsigned int need,
+// barriers: each warp sums a contiguous segment of the bins; in the warp whose
+// segment holds the bucket every lane sums its own run of NBINS / NT bins, a
+// shuffle suffix sum over the lanes finds the run, and that lane walks it.
+template <int NT, int NBINS>
+static __device__ __forceinline__ void find_bucket_smem(const unsigned int *h, unsigned int need,
                                                         unsigned int *s_tot /* >= NT / 32 */,
                                                         int *out_bin, unsigned int *out_need) {
     constexpr int W = NT / 32;
+    constexpr int kSeg = NBINS / W;   // bins per warp
+    constexpr int kPer = kSeg / 32;   // bins per lane
+    static_assert(kPer >= 4 && kPer % 4 == 0 && kPer <= 16, "bins per lane");
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int seg = nbins / W;
-    const unsigned int *hw = h + warp * seg;
-    unsigned int sum = 0;
-    for (int j = lane; j < seg; j += 32) sum += hw[j];
-    sum = __reduce_add_sync(0xffffffffu, sum);
+    const unsigned int *hl = h + warp * kSeg + lane * kPer;
+    unsigned int v[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; i += 4) {
+        const uint4 x = *reinterpret_cast<const uint4 *>(hl + i);
+        v[i] = x.x;
+        v[i + 1] = x.y;
+        v[i + 2] = x.z;
+        v[i + 3] = x.w;
+    }
+    unsigned int mine = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) mine += v[i];
+    const unsigned int sum = __reduce_add_sync(0xffffffffu, mine);
     if (lane == 0) s_tot[warp] = sum;
     if (t == 0) {
         *out_bin = 0;
@@ -87,23 +98,23 @@ static __device__ __forceinline__ void find_bucket_smem(const unsigned int *h, i
     unsigned int above = 0;
     for (int w2 = warp + 1; w2 < W; ++w2) above += s_tot[w2];
     if (above < need && need <= above + sum) {   // warp-uniform
-        for (int j0 = seg - 32; j0 >= 0; j0 -= 32) {
-            const unsigned int v = hw[j0 + lane];
-            unsigned int sfx = v;   // bins j0+lane .. j0+31
+        unsigned int sfx = mine;   // runs of lanes lane..31
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned int y = __shfl_down_sync(0xffffffffu, sfx, o);
-                if (lane + o < 32) sfx += y;
-            }
-            const unsigned int chunk_total = __shfl_sync(0xffffffffu, sfx, 0);
-            if (above + chunk_total >= need) {
-                if (above + sfx >= need && above + sfx - v < need) {
-                    *out_bin = warp * seg + j0 + lane;
-                    *out_need = need - (above + sfx - v);
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned int y = __shfl_down_sync(0xffffffffu, sfx, o);
+            if (lane + o < 32) sfx += y;
+        }
+        unsigned int cum = above + sfx - mine;   // bins above this lane's run
+        if (cum < need && need <= cum + mine) {
+#pragma unroll
+            for (int i = kPer - 1; i >= 0; --i) {
+                if (cum + v[i] >= need) {
+                    *out_bin = warp * kSeg + lane * kPer + i;
+                    *out_need = need - cum;
+                    break;
                 }
-                break;
+                cum += v[i];
             }
-            above += chunk_total;
         }
     }
     __syncthreads();
