@@ -78,7 +78,8 @@ __host__ __device__ constexpr size_t partial_slot_bytes() {
 
 // Merge nchunks partials (slot layout above; m in log2 units, l and O
 // relative to exp2(m)) with the low-resolution part of the row (full mode)
-// and write the 32 x D output block.
+// and write the 32 x D output block.  Run by NT threads, tid = 0..NT-1 their
+// index, that Sync synchronises.
 //
 // The partials are taken in groups of kMergeGroup: all (m, l) pairs of a group
 // are loaded at once, the running per-row maximum and normaliser move to the
@@ -88,7 +89,7 @@ __host__ __device__ constexpr size_t partial_slot_bytes() {
 template <int D, int NT, bool G, typename OutT, typename PartT, typename Sync>
 __device__ void merge_write(const unsigned char *src0, size_t slot_bytes, int nchunks, int full,
                             float m_lo2, float l_lo, const float *olo_row, const float *qmask,
-                            OutT *out_blk, MergeSmem &sm) {
+                            OutT *out_blk, MergeSmem &sm, int tid) {
     static_assert((8 * D) % NT == 0, "a chunk's O tile must split evenly into quads per thread");
     constexpr int F = 8 * D / NT;   // quads (4 elements) of one partial's O tile per thread
     constexpr int kRowQ = D / 4;
@@ -97,7 +98,6 @@ __device__ void merge_write(const unsigned char *src0, size_t slot_bytes, int nc
     constexpr int kMergeUnroll = F * kQuadBytes >= 128 ? 1 : 128 / (F * kQuadBytes);
     constexpr int kML = kMergeGroup * 32 / NT;   // (m, l) pairs per thread per group
     static_assert(kML >= 1 && (kMergeGroup * 32) % NT == 0, "merge group layout");
-    const int tid = threadIdx.x;
     float4 acc[F];
 #pragma unroll
     for (int i = 0; i < F; ++i) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -224,7 +224,7 @@ __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int
     const float *olo_row = full ? olo + (size_t)row * D : nullptr;
     if (nchunks == 1) {
         merge_write<D, NT, false, OutT, PartT, Sync>(stage, kSlot, 1, full, m_lo2, l_lo, olo_row, qmask,
-                                                     out_blk, sm);
+                                                     out_blk, sm, tid);
         return;
     }
     uint4 *dst = reinterpret_cast<uint4 *>(partial + (size_t)slot * kSlot);
@@ -237,7 +237,7 @@ __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int
     if (!*s_last) return;
     __threadfence();
     merge_write<D, NT, true, OutT, PartT, Sync>(partial + (size_t)(slot - chunk) * kSlot, kSlot, nchunks, full,
-                                                m_lo2, l_lo, olo_row, qmask, out_blk, sm);
+                                                m_lo2, l_lo, olo_row, qmask, out_blk, sm, tid);
     if (tid == 0) row_arrive[row] = 0;
 }
 

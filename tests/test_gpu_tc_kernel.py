@@ -1,8 +1,10 @@
-"""Parity of the tcgen05/TMA attention kernel (selected with MRA_ATTN_IMPL=tc).
+"""Parity of the tcgen05/TMA attention kernel (transposed scores over stacks
+of key blocks), selected with MRA_ATTN_IMPL=tc.
 
 The kernel choice is read once per process, so each case runs in a child
 process with the variable set; the child compares the CUDA output with the
-oracle on the same seeded inputs and reports the error.
+oracle on the same seeded inputs and reports the error, and checks that the
+device status word stayed clear.
 """
 import json
 import os
@@ -32,6 +34,8 @@ else:
 gpu = tl.run_gpu(inputs, **kw)
 ora = tl.run_oracle(inputs, **kw)
 stats = tl.compare(inputs, gpu, ora)
+from resolution_block_sparse_b200 import mra_get_device_status
+assert mra_get_device_status() == 0, mra_get_device_status()
 print("RESULT " + json.dumps(stats))
 '''
 
@@ -39,14 +43,19 @@ CASES = [
     {"workload": 4},
     {"workload": 2},
     {"workload": 5},
+    {"workload": 3},
     {"B": 1, "H": 2, "N": 1024, "bpr": 4, "mode": 0, "f": 1, "g": 1, "seed": 3, "pad": [100]},
     {"B": 1, "H": 2, "N": 2048, "bpr": 40, "mode": 1, "f": 1, "g": 1, "seed": 4},
+    {"B": 2, "H": 3, "N": 288, "bpr": 2, "mode": 0, "f": 1, "g": 1, "seed": 5, "pad": [0, 70]},
+    {"B": 1, "H": 1, "N": 8192, "bpr": 2, "mode": 0, "f": 1, "g": 0, "seed": 6},
+    {"B": 2, "H": 1, "N": 256, "bpr": 2, "mode": 1, "f": 0, "g": 0, "seed": 7, "pad": [256, 0]},
 ]
 
 
+@pytest.mark.parametrize("impl", ["tc"])
 @pytest.mark.parametrize("case", CASES, ids=[json.dumps(c, sort_keys=True) for c in CASES])
-def test_tc_kernel_parity(case):
-    env = dict(os.environ, MRA_ATTN_IMPL="tc")
+def test_tc_kernel_parity(case, impl):
+    env = dict(os.environ, MRA_ATTN_IMPL=impl)
     r = subprocess.run([sys.executable, "-c", CHILD, ROOT, json.dumps(case)], env=env,
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-3000:]
