@@ -229,34 +229,46 @@ def run_cuda(args, w, world, rank, local):
             "d2h": oh.numel() * oh.element_size()}
 
 
-def oracle_sample(w, target_s: float = 15.0):
-    """Time the CPU oracle on a bounded sample of the workload: the first S
-    (batch, head) slices, S grown until the run takes a few seconds; return
-    (tokens/s of the whole workload at that rate, sample text, cores)."""
+def oracle_sampler(w, target_s: float = 15.0):
+    """A bounded sample of the workload for the CPU oracle: the first S
+    (batch, head) slices, S grown (once) until one run takes about target_s
+    / 4 to target_s seconds.  Returns (run, sample text, cores); run() times
+    one oracle pass over the sample and returns tokens/s of the whole
+    workload at that rate."""
     import oracle
 
     inputs = make_inputs(w)
     cores = os.cpu_count() or 1
     BH = w.B * w.H
-    S = 1
-    while True:
+
+    def slices(S):
         q = inputs["q"].reshape(BH, 1, w.N, w.D)[:S].double().numpy()
         k = inputs["k"].reshape(BH, 1, w.N, w.D)[:S].double().numpy()
         v = inputs["v"].reshape(BH, 1, w.N, w.D)[:S].double().numpy()
         m = None
         if inputs["mask"] is not None:
             m = inputs["mask"].repeat_interleave(w.H, dim=0)[:S].double().numpy()
+        return q, k, v, m
+
+    def timed(args):
         t0 = time.perf_counter()
-        oracle.forward(q, k, v, m, block_per_row=w.block_per_row, approx_mode=w.approx_mode,
-                       first_n=w.first_n, diag_n=w.diag_n, nthreads=cores,
-                       want_intermediates=False)
-        dt = time.perf_counter() - t0
+        oracle.forward(*args, block_per_row=w.block_per_row, approx_mode=w.approx_mode,
+                       first_n=w.first_n, diag_n=w.diag_n, nthreads=cores, want_intermediates=False)
+        return time.perf_counter() - t0
+
+    S = 1
+    while True:
+        dt = timed(slices(S))
         if dt >= target_s / 4 or S >= BH:
             break
         S = min(BH, S * 2)
-    full_s = dt * BH / S
+    sample = slices(S)
     tokens = w.B * w.N
-    return tokens / full_s, f"{S} of {BH} (batch, head) slices, fp64, scaled to the full step", cores, dt
+
+    def run():
+        return tokens / (timed(sample) * BH / S)
+
+    return run, f"{S} of {BH} (batch, head) slices, fp64, scaled to the full step", cores
 
 
 def main():
@@ -283,14 +295,17 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        steps_s = []
-        val, sample, cores, _ = oracle_sample(w, target_s=4.0)
-        for _ in range(max(1, min(args.steps, 3))):
-            v2, _, _, dt = oracle_sample(w, target_s=4.0)
-            steps_s.append(v2)
+        # W warm-up and K timed steps, each a bounded sample (about 2 s of
+        # oracle work) of the workload, scaled to the full step
+        run, sample, cores = oracle_sampler(w, target_s=2.0)
+        for _ in range(args.warmup):
+            run()
+        steps_s = [run() for _ in range(max(1, args.steps))]
         value = statistics.mean(steps_s)
+        config = dict(config, timing="oracle on the host cores, wall clock per bounded sample, "
+                                     "scaled to the full step")
         line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-                "n_gpus": 1, "steps": len(steps_s), "warmup": 1,
+                "n_gpus": 1, "steps": len(steps_s), "warmup": args.warmup,
                 "ms_per_step": 1000.0 * tokens / value, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": config,
@@ -347,7 +362,8 @@ def main():
             "gpu_launches": res["launches_per_step"] * args.steps,
             "device_status": res["status"], "clocks": res["clocks"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, sample, cores, _ = oracle_sample(w)
+        run, sample, cores = oracle_sampler(w)
+        val = run()
         line["cpu_baseline"] = {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     if world > 1:
