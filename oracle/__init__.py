@@ -1,4 +1,5 @@
-"""CPU oracle of the MRA-2 forward pass (fp64, plain C, OpenMP over heads).
+"""CPU oracle of the MRA-2 forward pass and its gradient (fp64, plain C,
+OpenMP over heads).
 
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline / reference legs of ``bench.py`` may import this package.  The
@@ -27,6 +28,14 @@ What pins each function (tests marked ``not gpu``):
 * ``forward`` (low-res part) - block-constant Q and K make full mode equal
                              dense attention for any budget; probes with
                              one-hot V measure the count weighting.
+* ``backward``             - torch autograd (fp64) of a dense restatement of
+                             the forward (exact scores on selected blocks,
+                             block logits of differentiable block means on
+                             unselected ones in full mode, -inf in sparse
+                             mode); autograd of SDPA where the budget selects
+                             every block; central finite differences of
+                             ``forward`` with the selection unchanged
+                             (``tests/test_oracle_backward_pins.py``).
 * padded-query outputs (0), the empty-row output (0), the prior band offsets
   and the exact bias arithmetic are readings of the page, not fixed by it:
   **parity unpinned** beyond internal consistency.
@@ -81,6 +90,8 @@ def _bind(path: str):
     lib.mra_oracle_select.argtypes = [dp, c_int, c_int, c_long, ip]
     lib.mra_oracle_forward.restype = c_int
     lib.mra_oracle_forward.argtypes = [dp, dp, dp, dp] + [c_int] * 8 + [dp, ip, dp, dp, dp, dp, c_int]
+    lib.mra_oracle_backward.restype = c_int
+    lib.mra_oracle_backward.argtypes = [dp, dp, dp, dp, dp] + [c_int] * 8 + [dp, dp, dp, c_int]
     lib.mra_oracle_attend_with_selection.restype = c_int
     lib.mra_oracle_attend_with_selection.argtypes = [dp, dp, dp, dp] + [c_int] * 5 + [ip, c_long, dp, c_int]
     return lib
@@ -259,3 +270,23 @@ def attend_with_selection(q, k, v, mask, sel, *, approx_mode: int = 0, nthreads:
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out
+
+
+def backward(q, k, v, mask, dout, *, block_per_row: int, approx_mode: int = 0, first_n: int = 0,
+             diag_n: int = 0, nthreads: int = 0):
+    """Gradients (dq, dk, dv) [B,H,N,D] fp64 of the forward output with the
+    selection held fixed, for the incoming gradient dout [B,H,N,D]."""
+    B, H, N, D = q.shape
+    qa, qp = _d(q)
+    ka, kp = _d(k)
+    va, vp = _d(v)
+    ma, mp = _d(mask)
+    ga, gp = _d(dout)
+    dq, dqp = _out((B, H, N, D))
+    dk, dkp = _out((B, H, N, D))
+    dv, dvp = _out((B, H, N, D))
+    rc = _load().mra_oracle_backward(qp, kp, vp, mp, gp, B, H, N, D, block_per_row, approx_mode,
+                                     first_n, diag_n, dqp, dkp, dvp, nthreads)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return dq, dk, dv

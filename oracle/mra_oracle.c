@@ -1,6 +1,6 @@
 /*
  * mra_oracle.c - plain, slow fp64 CPU oracle of the MRA-2 approximate
- * self-attention forward pass.
+ * self-attention forward pass and of its gradient.
  *
  * TEST INFRASTRUCTURE ONLY.  This file is compiled into a separate shared
  * library that only the test-suite, the smoke check and the benchmark's
@@ -447,4 +447,185 @@ int mra_oracle_attend_with_selection(const double *q, const double *k, const dou
     }
     free(cnt);
     return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------ backward
+ * Gradient of the forward output with respect to q, k and v, with the
+ * selected set held fixed (the top-k indices are not differentiated).
+ * [MRA page, step three: the sampled-dense products are autograd functions
+ * whose backward passes reuse the same kernels through transposed indices, so
+ * the model trains end to end; step four: in "sparse" mode the
+ * low-resolution branch only chooses blocks, under no_grad, so no gradient
+ * flows through it; in "full" mode the low-resolution output is part of the
+ * result and its gradient flows through the pooled Q, K and V.]
+ *
+ * For query i (m_i = 1) with included terms t (as in attend_head), weights
+ * p_t = w_t / sum(w), output out_i = sum_t p_t value_t and incoming dout_i,
+ * with Dlt_i = dout_i . out_i:
+ *   hi term (key j of a selected block):  ds_ij = p_ij (dout_i . v_j - Dlt_i)
+ *       dv_j += p_ij dout_i,   dq_i += ds_ij k_j / sqrt(D),   dk_j += ds_ij q_i / sqrt(D)
+ *   lo term (unselected block c, full mode):  dl_rc += p_ic (dout_i . vhat_c - Dlt_i)
+ *       dvhat_c += p_ic dout_i
+ * then dqhat_r += dl_rc khat_c / sqrt(D), dkhat_c += dl_rc qhat_r / sqrt(D), and
+ * the block means hand their gradients to their valid tokens:
+ *   dx_t += dxhat_b / cnt_b  for m_t = 1, t in block b.
+ * A padded query and a row without terms output the constant 0: no gradient. */
+static void backward_head(const double *q, const double *k, const double *v,
+                          const double *mask_row, const double *cnt_row, const double *qh,
+                          const double *kh, const double *vh, const double *logit,
+                          const unsigned char *selected, const double *dout, int N, int D,
+                          int full_mode, double *dq, double *dk, double *dv)
+{
+    int nbr = N / MRA_ORACLE_BLOCK;
+    double scale = 1.0 / sqrt((double)D);
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    double *o = (double *)malloc(sizeof(double) * (size_t)D);
+    double *dl = (double *)calloc((size_t)nbr * nbr, sizeof(double));
+    double *dqh = (double *)calloc((size_t)nbr * D, sizeof(double));
+    double *dkh = (double *)calloc((size_t)nbr * D, sizeof(double));
+    double *dvh = (double *)calloc((size_t)nbr * D, sizeof(double));
+    for (size_t e = 0; e < (size_t)N * D; ++e) dq[e] = dk[e] = dv[e] = 0.0;
+
+    for (int i = 0; i < N; ++i) {
+        int r = i / MRA_ORACLE_BLOCK;
+        if (mask_row && !(mask_row[i] > 0.0)) continue;
+        const double *qi = q + (size_t)i * D;
+        const double *gi = dout + (size_t)i * D;
+        /* the forward terms of query i: exponents, maximum, normaliser, output */
+        int any = 0;
+        double mx = 0.0;
+        for (int c = 0; c < nbr; ++c) {
+            if (selected[(size_t)r * nbr + c]) {
+                for (int j = c * MRA_ORACLE_BLOCK; j < (c + 1) * MRA_ORACLE_BLOCK; ++j) {
+                    if (mask_row && !(mask_row[j] > 0.0)) continue;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += qi[d] * k[(size_t)j * D + d];
+                    s[j] = dot * scale;
+                    if (!any || s[j] > mx) mx = s[j];
+                    any = 1;
+                }
+            } else if (full_mode && cnt_row[c] > 0.0) {
+                double l = logit[(size_t)r * nbr + c];
+                if (!any || l > mx) mx = l;
+                any = 1;
+            }
+        }
+        if (!any) continue;
+        double den = 0.0;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        for (int c = 0; c < nbr; ++c) {
+            if (selected[(size_t)r * nbr + c]) {
+                for (int j = c * MRA_ORACLE_BLOCK; j < (c + 1) * MRA_ORACLE_BLOCK; ++j) {
+                    if (mask_row && !(mask_row[j] > 0.0)) continue;
+                    double w = exp(s[j] - mx);
+                    den += w;
+                    for (int d = 0; d < D; ++d) o[d] += w * v[(size_t)j * D + d];
+                }
+            } else if (full_mode && cnt_row[c] > 0.0) {
+                double w = cnt_row[c] * exp(logit[(size_t)r * nbr + c] - mx);
+                den += w;
+                for (int d = 0; d < D; ++d) o[d] += w * vh[(size_t)c * D + d];
+            }
+        }
+        double delta = 0.0;
+        for (int d = 0; d < D; ++d) {
+            o[d] /= den;
+            delta += gi[d] * o[d];
+        }
+        /* the gradients of every term */
+        for (int c = 0; c < nbr; ++c) {
+            if (selected[(size_t)r * nbr + c]) {
+                for (int j = c * MRA_ORACLE_BLOCK; j < (c + 1) * MRA_ORACLE_BLOCK; ++j) {
+                    if (mask_row && !(mask_row[j] > 0.0)) continue;
+                    double p = exp(s[j] - mx) / den;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += gi[d] * v[(size_t)j * D + d];
+                    double ds = p * (dot - delta);
+                    for (int d = 0; d < D; ++d) {
+                        dv[(size_t)j * D + d] += p * gi[d];
+                        dq[(size_t)i * D + d] += ds * scale * k[(size_t)j * D + d];
+                        dk[(size_t)j * D + d] += ds * scale * qi[d];
+                    }
+                }
+            } else if (full_mode && cnt_row[c] > 0.0) {
+                double p = cnt_row[c] * exp(logit[(size_t)r * nbr + c] - mx) / den;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d) dot += gi[d] * vh[(size_t)c * D + d];
+                dl[(size_t)r * nbr + c] += p * (dot - delta);
+                for (int d = 0; d < D; ++d) dvh[(size_t)c * D + d] += p * gi[d];
+            }
+        }
+    }
+    /* low-resolution logits -> block means -> tokens */
+    for (int r = 0; r < nbr; ++r)
+        for (int c = 0; c < nbr; ++c) {
+            double g = dl[(size_t)r * nbr + c];
+            if (g == 0.0) continue;
+            for (int d = 0; d < D; ++d) {
+                dqh[(size_t)r * D + d] += g * scale * kh[(size_t)c * D + d];
+                dkh[(size_t)c * D + d] += g * scale * qh[(size_t)r * D + d];
+            }
+        }
+    for (int t = 0; t < N; ++t) {
+        int b = t / MRA_ORACLE_BLOCK;
+        if (mask_row && !(mask_row[t] > 0.0)) continue;
+        if (!(cnt_row[b] > 0.0)) continue;
+        for (int d = 0; d < D; ++d) {
+            dq[(size_t)t * D + d] += dqh[(size_t)b * D + d] / cnt_row[b];
+            dk[(size_t)t * D + d] += dkh[(size_t)b * D + d] / cnt_row[b];
+            dv[(size_t)t * D + d] += dvh[(size_t)b * D + d] / cnt_row[b];
+        }
+    }
+    free(s); free(o); free(dl); free(dqh); free(dkh); free(dvh);
+}
+
+/* The backward pass: the forward's selection (recomputed exactly as in
+ * mra_oracle_forward), then backward_head per (batch, head).
+ * q, k, v, dout, dq, dk, dv: [B][H][N][D]; mask: [B][N] of 0/1 or NULL.
+ * Returns 0, or -1 on the forward's invalid arguments. */
+int mra_oracle_backward(const double *q, const double *k, const double *v, const double *mask,
+                        const double *dout, int B, int H, int N, int D, int block_per_row, int mode,
+                        int first_n, int diag_n, double *dq, double *dk, double *dv, int nthreads)
+{
+    if (B < 1 || H < 1 || N < MRA_ORACLE_BLOCK || N % MRA_ORACLE_BLOCK != 0 || D < 1) return -1;
+    if (block_per_row < 1 || (mode != 0 && mode != 1)) return -1;
+    int nbr = N / MRA_ORACLE_BLOCK;
+    if (first_n < 0 || first_n > nbr || diag_n < 0 || diag_n > nbr) return -1;
+    long kk = mra_oracle_num_block(N, block_per_row);
+    int BH = B * H;
+    double *cnt = (double *)malloc(sizeof(double) * (size_t)B * nbr);
+    mra_oracle_block_counts(mask, B, N, cnt);
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; ++bh) {
+        int b = bh / H;
+        size_t xoff = (size_t)bh * N * D;
+        const double *mrow = mask ? mask + (size_t)b * N : NULL;
+        const double *crow = cnt + (size_t)b * nbr;
+        double *qh = (double *)malloc(sizeof(double) * (size_t)nbr * D);
+        double *kh = (double *)malloc(sizeof(double) * (size_t)nbr * D);
+        double *vh = (double *)malloc(sizeof(double) * (size_t)nbr * D);
+        double *lg = (double *)malloc(sizeof(double) * (size_t)nbr * nbr);
+        double *ml = (double *)malloc(sizeof(double) * (size_t)nbr);
+        double *ky = (double *)malloc(sizeof(double) * (size_t)nbr * nbr);
+        int32_t *sl = (int32_t *)malloc(sizeof(int32_t) * (size_t)kk);
+        unsigned char *is_sel = (unsigned char *)calloc((size_t)nbr * nbr, 1);
+        pool_head(q + xoff, mrow, N, D, qh);
+        pool_head(k + xoff, mrow, N, D, kh);
+        pool_head(v + xoff, mrow, N, D, vh);
+        lowres_logits_head(qh, kh, nbr, D, lg);
+        row_max_head(lg, crow, nbr, ml);
+        selection_keys_head(lg, ml, crow, nbr, first_n, diag_n, ky);
+        select_head(ky, nbr, kk, sl);
+        for (long i = 0; i < kk; ++i) is_sel[sl[i]] = 1;
+        backward_head(q + xoff, k + xoff, v + xoff, mrow, crow, qh, kh, vh, lg, is_sel, dout + xoff, N,
+                      D, mode == 0, dq + xoff, dk + xoff, dv + xoff);
+        free(qh); free(kh); free(vh); free(lg); free(ml); free(ky); free(sl); free(is_sel);
+    }
+    free(cnt);
+    return 0;
 }

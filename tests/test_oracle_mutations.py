@@ -8,6 +8,7 @@ expects at least one of them to fail.  Nothing here touches a GPU.
 import pytest
 
 import oracle
+import test_oracle_backward_pins as bwd
 import test_oracle_pins as pins
 
 # (name, text to replace, replacement, pins expected to catch it)
@@ -52,6 +53,19 @@ MUTATIONS = [
     ("num_block without the cap at the full block count",
      "return budget < all ? budget : all;", "return budget;",
      ["num_block"]),
+    ("backward: score gradient without the output term",
+     "double ds = p * (dot - delta);", "double ds = p * dot;",
+     ["bwd_dense", "bwd_fd"]),
+    ("backward: low-resolution logit gradient dropped",
+     "dl[(size_t)r * nbr + c] += p * (dot - delta);", "",
+     ["bwd_dense_full"]),
+    ("backward: block-mean gradient not divided by the count",
+     "dq[(size_t)t * D + d] += dqh[(size_t)b * D + d] / cnt_row[b];",
+     "dq[(size_t)t * D + d] += dqh[(size_t)b * D + d];",
+     ["bwd_dense_full"]),
+    ("backward: key gradient without 1/sqrt(D)",
+     "dk[(size_t)j * D + d] += ds * scale * qi[d];", "dk[(size_t)j * D + d] += ds * qi[d];",
+     ["bwd_dense", "bwd_saturated"]),
 ]
 
 PINS = {
@@ -67,6 +81,10 @@ PINS = {
     "block_constant": lambda: pins.test_block_constant_qk_full_mode_equals_dense(1, 0, 0, [0, 45]),
     "sum_to_one": lambda: pins.test_rows_sum_to_one(1),
     "probe": lambda: pins.test_one_hot_value_probe_measures_block_mass(),
+    "bwd_dense": lambda: bwd.test_backward_equals_autograd_of_dense_restatement(1, [20, 0], 2, 1, 1),
+    "bwd_dense_full": lambda: bwd.test_backward_equals_autograd_of_dense_restatement(0, [64, 40], 3, 2, 3),
+    "bwd_saturated": lambda: bwd.test_saturated_budget_backward_equals_dense_attention_autograd([0, 45]),
+    "bwd_fd": lambda: bwd.test_backward_matches_finite_differences(0),
 }
 
 
