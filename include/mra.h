@@ -119,6 +119,33 @@ MRA_API int mra_attention_fwd_host(const void *q_host, const void *k_host, const
                            int D, int block_per_row, int approx_mode, int first_n, int diag_n,
                            int dtype, cudaStream_t stream);
 
+/* Backward pass: gradients of the forward output (same arguments, same
+ * selection) with respect to q, k and v, for the incoming gradient dout.
+ *
+ * Page "深入解析 Transformers 中的 MRA 模型", section "源码级原理", steps three
+ * and four: the block-sparse products are differentiated through transposed
+ * block indices; the selected set (the top-k) is held fixed; in "sparse" mode
+ * the low-resolution branch only chooses blocks and takes no gradient; in
+ * "full" mode its output is part of the result, so the gradient also flows
+ * through the masked block means of q, k and v.  Padded queries (output 0)
+ * pass no gradient.
+ *
+ * q, k, v, dout: device, [B][H][N][D] row-major, 16-byte aligned; bf16 for
+ * mra_attention_bwd, fp32 for mra_attention_bwd_f32.  key_mask as in the
+ * forward pass.  dq, dk, dv: device fp32 [B][H][N][D], 16-byte aligned,
+ * written (not accumulated); dq is also the scratch of the internal forward
+ * pass.  The call re-runs the forward pass (the selection is deterministic,
+ * so it is the one the forward call made) and needs no saved state.
+ * Asynchronous on `stream`; errors as for mra_attention_fwd. */
+MRA_API int mra_attention_bwd(const void *q, const void *k, const void *v, const float *key_mask,
+                              const void *dout, float *dq, float *dk, float *dv, int B, int H, int N,
+                              int D, int block_per_row, int approx_mode, int first_n, int diag_n,
+                              cudaStream_t stream);
+MRA_API int mra_attention_bwd_f32(const float *q, const float *k, const float *v,
+                                  const float *key_mask, const float *dout, float *dq, float *dk,
+                                  float *dv, int B, int H, int N, int D, int block_per_row,
+                                  int approx_mode, int first_n, int diag_n, cudaStream_t stream);
+
 /* Size of the static device array behind mra_attention_fwd_noalloc. */
 #define MRA_NOALLOC_SCRATCH_BYTES (16u << 20)
 

@@ -1,4 +1,4 @@
-"""B200-native MRA-2 approximate self-attention (forward pass).
+"""B200-native MRA-2 approximate self-attention (forward and backward passes).
 
 The compute path lives in the CUDA library ``libmra_b200.so`` behind the C-ABI
 declared in ``include/mra.h``; this package is a thin ctypes binding to it
@@ -15,6 +15,7 @@ from ._binding import (  # noqa: F401
     MraError,
     load_library,
     mra2_attention,
+    mra_attention_bwd,
     mra_attention_fwd,
     mra_attention_fwd_ex,
     mra_attention_fwd_f32,

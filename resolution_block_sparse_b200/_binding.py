@@ -25,7 +25,8 @@ MRA_DEV_KEY_RANGE, MRA_DEV_COUNT = 1, 2
 EXPORTED = (
     "mra_attention_fwd", "mra_attention_fwd_f32", "mra_attention_fwd_ex", "mra_attention_fwd_host",
     "mra_num_block", "mra_status_string", "mra_get_device_status", "mra_profile_enable",
-    "mra_profile_read", "mra_last_launch_count", "mra_attention_fwd_noalloc",
+    "mra_profile_read", "mra_last_launch_count", "mra_attention_fwd_noalloc", "mra_attention_bwd",
+    "mra_attention_bwd_f32",
 )
 
 _lock = threading.Lock()
@@ -61,6 +62,10 @@ def load_library(path: str = LIB_PATH):
         lib.mra_attention_fwd_ex.restype = c_int
         lib.mra_attention_fwd_host.argtypes = [vp, vp, vp, vp, vp] + [c_int] * 9 + [vp]
         lib.mra_attention_fwd_host.restype = c_int
+        for name in ("mra_attention_bwd", "mra_attention_bwd_f32"):
+            fn = getattr(lib, name)
+            fn.argtypes = [vp] * 8 + [c_int] * 8 + [vp]
+            fn.restype = c_int
         lib.mra_num_block.argtypes = [c_int, c_int]
         lib.mra_num_block.restype = ctypes.c_size_t
         lib.mra_status_string.argtypes = [c_int]
@@ -141,6 +146,19 @@ def mra_attention_fwd_noalloc(q, k, v, key_mask, out, block_per_row, approx_mode
                                                   _stream(stream))
     _check(st, "mra_attention_fwd_noalloc")
     return out
+
+
+def mra_attention_bwd(q, k, v, key_mask, dout, dq, dk, dv, block_per_row, approx_mode, first_n, diag_n,
+                      stream=None):
+    """Backward on device tensors: q, k, v, dout [B,H,N,D] (bf16 or fp32);
+    dq, dk, dv fp32 [B,H,N,D] are written."""
+    B, H, N, D = _shape(q)
+    lib = load_library()
+    fn = lib.mra_attention_bwd if q.dtype == torch.bfloat16 else lib.mra_attention_bwd_f32
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(key_mask), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, D,
+            block_per_row, _mode(approx_mode), first_n, diag_n, _stream(stream))
+    _check(st, "mra_attention_bwd")
+    return dq, dk, dv
 
 
 def mra_attention_fwd_ex(q, k, v, key_mask, out, block_per_row, approx_mode, first_n, diag_n,

@@ -43,6 +43,7 @@ int validate(const void *q, const void *k, const void *v, const void *out, int B
 Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n,
                      int dtype) {
     Problem p;
+    p.bwd = 0;
     p.B = B;
     p.H = H;
     p.N = N;
@@ -111,6 +112,12 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     t.olo = (float *)take(sizeof(float) * BH * nbr * D);
     t.llo = (float *)take(sizeof(float) * BH * nbr);
     t.partial = (float *)take(sizeof(float) * BH * (size_t)p.cap * 32 * (D + 2));
+    if (p.bwd) {
+        t.lse2 = (float *)take(sizeof(float) * BH * (size_t)p.N);
+        t.delta = (float *)take(sizeof(float) * BH * (size_t)p.N);
+        t.lo_ab = (float *)take(sizeof(float) * BH * nbr * (D + 4));
+        t.lo_dxh = (float *)take(sizeof(float) * 3 * BH * nbr * D);
+    }
     if (w) *w = t;
     return off;
 }
@@ -232,7 +239,7 @@ namespace mra {
 int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const void *k,
                     const void *v, const float *mask, void *out, int32_t *sel_out,
                     float *logit_out, float *pooled_out, cudaStream_t s, bool profile,
-                    int *launch_count) {
+                    int *launch_count, const GradStats *gs) {
     const bool prof = profile && g_prof;
     int launches = 0;
     {
@@ -271,7 +278,7 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
     }
     {
         PhaseScope ps("attention", s, prof);
-        MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s));
+        MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s, gs));
         ++launches;
     }
     if (pooled_out) {
@@ -314,9 +321,61 @@ int forward_locked(const void *q, const void *k, const void *v, const float *mas
     return MRA_OK;
 }
 
+// The backward pass: the forward pass (same selection, the attention kernel
+// exporting each query's log-sum-exp and dout . out, its output written to
+// dq as scratch), then the gradient kernels.  The caller holds g_mutex.
+int backward_locked(const void *q, const void *k, const void *v, const float *mask, const void *dout,
+                    float *dq, float *dk, float *dv, int B, int H, int N, int D, int bpr, int mode,
+                    int first_n, int diag_n, int dtype, cudaStream_t s) {
+    int rc = validate(q, k, v, dq, B, H, N, D, bpr, mode, first_n, diag_n);
+    if (rc != MRA_OK) return rc;
+    if (!dout || !dk || !dv) return MRA_ERR_INVALID_ARG;
+    if ((((uintptr_t)dout) | ((uintptr_t)dk) | ((uintptr_t)dv)) & 15u) return MRA_ERR_INVALID_ARG;
+    if (mask && (((uintptr_t)mask) & 3u)) return MRA_ERR_INVALID_ARG;
+    int dev;
+    rc = current_device(&dev);
+    if (rc != MRA_OK) return rc;
+    Problem p = make_problem(B, H, N, D, bpr, mode, first_n, diag_n, dtype);
+    p.bwd = 1;
+    Workspace w;
+    rc = ensure_workspace(dev, p, &w);
+    if (rc != MRA_OK) return rc;
+    GradStats gs{};
+    gs.dout = dout;
+    gs.dout_f32 = dtype == MRA_DTYPE_F32 ? 1 : 0;
+    gs.lse2 = w.lse2;
+    gs.delta = w.delta;
+    int launches = 0;
+    rc = enqueue_forward(p, w, q, k, v, mask, dq, nullptr, nullptr, nullptr, s, true, &launches, &gs);
+    if (rc != MRA_OK) return rc;
+    const size_t bytes = sizeof(float) * (size_t)B * H * N * D;
+    MRA_TRY(cudaMemsetAsync(dq, 0, bytes, s));
+    MRA_TRY(cudaMemsetAsync(dk, 0, bytes, s));
+    MRA_TRY(cudaMemsetAsync(dv, 0, bytes, s));
+    MRA_TRY(launch_backward(p, w, q, k, v, mask, dout, dq, dk, dv, s));
+    g_last_launches = launches + (mode == MRA_FULL ? 5 : 1);
+    return MRA_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int mra_attention_bwd(const void *q, const void *k, const void *v, const float *key_mask,
+                      const void *dout, float *dq, float *dk, float *dv, int B, int H, int N, int D,
+                      int block_per_row, int approx_mode, int first_n, int diag_n, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    return backward_locked(q, k, v, key_mask, dout, dq, dk, dv, B, H, N, D, block_per_row, approx_mode,
+                           first_n, diag_n, MRA_DTYPE_BF16, stream);
+}
+
+int mra_attention_bwd_f32(const float *q, const float *k, const float *v, const float *key_mask,
+                          const float *dout, float *dq, float *dk, float *dv, int B, int H, int N, int D,
+                          int block_per_row, int approx_mode, int first_n, int diag_n, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    return backward_locked(q, k, v, key_mask, dout, dq, dk, dv, B, H, N, D, block_per_row, approx_mode,
+                           first_n, diag_n, MRA_DTYPE_F32, stream);
+}
 
 int mra_attention_fwd(const void *q, const void *k, const void *v, const float *key_mask,
                       void *out, int B, int H, int N, int D, int block_per_row, int approx_mode,

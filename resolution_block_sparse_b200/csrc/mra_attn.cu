@@ -105,6 +105,7 @@ struct AttnArgs {
     int *row_arrive;
     int *work_next;   // items handed out beyond the first wave (zeroed per call)
     void *out;
+    GradStats gs;     // backward-pass statistics (gs.lse2 == nullptr: forward only)
 };
 
 constexpr int kBf16Threads = 64;
@@ -292,9 +293,11 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
         const float l_lo = a.full ? a.llo[it.row] : 0.0f;
         const bool lo = a.full && l_lo > 0.0f;
         float fa_a, fb_a, fa_b, fb_b;   // output = O * fa + O_lo * fb, per row
+        float lse_a, lse_b;             // base-2 log-sum-exp of the row (backward statistics)
         {
-            auto factors = [&](float m, float l, int row, float &fa, float &fb) {
+            auto factors = [&](float m, float l, int row, float &fa, float &fb, float &lse) {
                 fa = fb = 0.0f;
+                lse = INFINITY;
                 const bool hi = l > 0.0f;
                 float M = hi ? m : -INFINITY;
                 if (lo) M = fmaxf(M, m_lo2);
@@ -305,21 +308,42 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
                 if (den > 0.0f) {
                     fa = al / den;
                     fb = be / den;
+                    lse = M + log2f(den);
                 }
             };
-            factors(m_a, l_a, ra, fa_a, fb_a);
-            factors(m_b, l_b, rb, fa_b, fb_b);
+            factors(m_a, l_a, ra, fa_a, fb_a, lse_a);
+            factors(m_b, l_b, rb, fa_b, fb_b, lse_b);
         }
+        float dsum_a = 0.0f, dsum_b = 0.0f;   // dout . out of rows ra, rb (this thread's dims)
         __nv_bfloat16 *ostage = &sKV[0][0][0];   // [32][D] bf16 staging
+        const size_t qbase = (size_t)bh * a.N + (size_t)r * 32;
 #pragma unroll
         for (int nd = 0; nd < D / 8; ++nd) {
             const int d = nd * 8 + tq * 2;
             float2 ol = make_float2(0.0f, 0.0f);
             if (lo) ol = *reinterpret_cast<const float2 *>(a.olo + (size_t)it.row * D + d);
-            *reinterpret_cast<__nv_bfloat162 *>(ostage + ra * D + d) =
-                __floats2bfloat162_rn(fmaf(o[nd][0], fa_a, ol.x * fb_a), fmaf(o[nd][1], fa_a, ol.y * fb_a));
-            *reinterpret_cast<__nv_bfloat162 *>(ostage + rb * D + d) =
-                __floats2bfloat162_rn(fmaf(o[nd][2], fa_b, ol.x * fb_b), fmaf(o[nd][3], fa_b, ol.y * fb_b));
+            const float x0 = fmaf(o[nd][0], fa_a, ol.x * fb_a), x1 = fmaf(o[nd][1], fa_a, ol.y * fb_a);
+            const float y0 = fmaf(o[nd][2], fa_b, ol.x * fb_b), y1 = fmaf(o[nd][3], fa_b, ol.y * fb_b);
+            *reinterpret_cast<__nv_bfloat162 *>(ostage + ra * D + d) = __floats2bfloat162_rn(x0, x1);
+            *reinterpret_cast<__nv_bfloat162 *>(ostage + rb * D + d) = __floats2bfloat162_rn(y0, y1);
+            if (a.gs.lse2) {
+                const size_t ia = (qbase + ra) * D + d, ib = (qbase + rb) * D + d;
+                dsum_a += x0 * a.gs.dout_at(ia) + x1 * a.gs.dout_at(ia + 1);
+                dsum_b += y0 * a.gs.dout_at(ib) + y1 * a.gs.dout_at(ib + 1);
+            }
+        }
+        if (a.gs.lse2) {
+#pragma unroll
+            for (int off = 1; off < 4; off <<= 1) {
+                dsum_a += __shfl_xor_sync(0xffffffffu, dsum_a, off);
+                dsum_b += __shfl_xor_sync(0xffffffffu, dsum_b, off);
+            }
+            if (tq == 0) {
+                a.gs.lse2[qbase + ra] = lse_a;
+                a.gs.lse2[qbase + rb] = lse_b;
+                a.gs.delta[qbase + ra] = dsum_a;
+                a.gs.delta[qbase + rb] = dsum_b;
+            }
         }
         __syncthreads();
 #pragma unroll
@@ -346,9 +370,11 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
     __syncthreads();
     MergeSmem &sm = *reinterpret_cast<MergeSmem *>(reinterpret_cast<unsigned char *>(stage) +
                                                    partial_slot_bytes<D, __nv_bfloat16>());
+    GradStats gs = a.gs;
+    gs.qbase = (size_t)bh * a.N + (size_t)r * 32;
     finish_item<D, kBf16Threads, __nv_bfloat16, __nv_bfloat16, SyncAll>(
         reinterpret_cast<const unsigned char *>(stage), slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
-        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
+        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last, gs);
 }
 
 // Persistent: the first wave takes items 0..gridDim.x-1, after that a CTA
@@ -457,16 +483,20 @@ attn_f32_kernel(const AttnArgs a) {
     for (int i = 0; i < kDp; ++i) stage[64 + qrow * D + d0 + i] = o[i];
     __syncthreads();
     float *out_blk = static_cast<float *>(a.out) + head_off + (size_t)r * kTile;
+    GradStats gs = a.gs;
+    gs.qbase = (size_t)bh * a.N + (size_t)r * 32;
     finish_item<D, kF32Threads, float, float, SyncAll>(
         reinterpret_cast<const unsigned char *>(stage), slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
-        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last);
+        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last, gs);
 }
 
 }  // namespace
 
 cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
-                             const void *v, const float *mask, void *out, cudaStream_t s) {
+                             const void *v, const float *mask, void *out, cudaStream_t s,
+                             const GradStats *gs) {
     AttnArgs a;
+    a.gs = gs ? *gs : GradStats{};
     a.q = q;
     a.k = k;
     a.v = v;
@@ -493,7 +523,8 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
     // the sparse workloads (a few 32x32 blocks per block row)
     static const char *impl = getenv("MRA_ATTN_IMPL");
     const bool want_tc = impl && impl[0] == 't';
-    if (want_tc && attention_tc_supported(p)) return launch_attention_tc(p, w, q, k, v, mask, out, s);
+    // the backward pass's statistics come from the kernels below
+    if (want_tc && !gs && attention_tc_supported(p)) return launch_attention_tc(p, w, q, k, v, mask, out, s);
     if (p.dtype == 0) {
         static int sms = 0;
         if (sms == 0) {

@@ -68,6 +68,7 @@ struct MergeSmem {
     float w[kMergeGroup][32];   // m of (chunk, row), then its weight
     float l[kMergeGroup][32];
     float M[32], den[32], resc[32];
+    float lse2[32], dsum[32];   // per-row statistics for the backward pass
 };
 
 // Bytes of one partial slot: m[32] and l[32] in fp32, then O[32][D] in PartT.
@@ -89,7 +90,7 @@ __host__ __device__ constexpr size_t partial_slot_bytes() {
 template <int D, int NT, bool G, typename OutT, typename PartT, typename Sync>
 __device__ void merge_write(const unsigned char *src0, size_t slot_bytes, int nchunks, int full,
                             float m_lo2, float l_lo, const float *olo_row, const float *qmask,
-                            OutT *out_blk, MergeSmem &sm, int tid) {
+                            OutT *out_blk, MergeSmem &sm, int tid, const GradStats &gs) {
     static_assert((8 * D) % NT == 0, "a chunk's O tile must split evenly into quads per thread");
     constexpr int F = 8 * D / NT;   // quads (4 elements) of one partial's O tile per thread
     constexpr int kRowQ = D / 4;
@@ -183,15 +184,18 @@ __device__ void merge_write(const unsigned char *src0, size_t slot_bytes, int nc
         const float m_hi = sm.M[q];
         const bool lo = full && l_lo > 0.0f;
         const float M = lo ? fmaxf(m_hi, m_lo2) : m_hi;
-        float a_hi = 0.0f, beta = 0.0f, inv = 0.0f;
+        float a_hi = 0.0f, beta = 0.0f, inv = 0.0f, lse2 = INFINITY;
         if (M != -INFINITY && (!qmask || qmask[q] > 0.0f)) {
             a_hi = (m_hi == -INFINITY) ? 0.0f : exp2f(m_hi - M);
             beta = lo ? exp2f(m_lo2 - M) : 0.0f;
             const float den = a_hi * sm.den[q] + beta * l_lo;
             inv = den > 0.0f ? 1.0f / den : 0.0f;
+            if (den > 0.0f) lse2 = M + log2f(den);
         }
         sm.resc[q] = a_hi * inv;   // factor of the merged high-resolution O
         sm.den[q] = beta * inv;    // factor of the low-resolution output
+        sm.lse2[q] = lse2;
+        sm.dsum[q] = 0.0f;
     }
     Sync::sync();
 #pragma unroll
@@ -201,9 +205,21 @@ __device__ void merge_write(const unsigned char *src0, size_t slot_bytes, int nc
         const float fa = sm.resc[q], fb = sm.den[q];
         float4 ol = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         if (full) ol = *reinterpret_cast<const float4 *>(olo_row + d);
-        store4(out_blk + (size_t)q * D + d,
-               make_float4(fmaf(acc[i].x, fa, ol.x * fb), fmaf(acc[i].y, fa, ol.y * fb),
-                           fmaf(acc[i].z, fa, ol.z * fb), fmaf(acc[i].w, fa, ol.w * fb)));
+        const float4 ov = make_float4(fmaf(acc[i].x, fa, ol.x * fb), fmaf(acc[i].y, fa, ol.y * fb),
+                                      fmaf(acc[i].z, fa, ol.z * fb), fmaf(acc[i].w, fa, ol.w * fb));
+        store4(out_blk + (size_t)q * D + d, ov);
+        if (gs.lse2) {
+            const size_t gi = (gs.qbase + q) * D + d;
+            atomicAdd(&sm.dsum[q], ov.x * gs.dout_at(gi) + ov.y * gs.dout_at(gi + 1) +
+                                       ov.z * gs.dout_at(gi + 2) + ov.w * gs.dout_at(gi + 3));
+        }
+    }
+    if (gs.lse2) {
+        Sync::sync();
+        if (tid < 32) {
+            gs.lse2[gs.qbase + tid] = sm.lse2[tid];
+            gs.delta[gs.qbase + tid] = sm.dsum[tid];
+        }
     }
 }
 
@@ -215,7 +231,7 @@ template <int D, int NT, typename OutT, typename PartT, typename Sync>
 __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int nchunks, int row, int full,
                             const float *mlo, const float *olo, const float *llo,
                             unsigned char *partial, int *row_arrive, const float *qmask, OutT *out_blk,
-                            MergeSmem &sm, int *s_last) {
+                            MergeSmem &sm, int *s_last, const GradStats &gs) {
     constexpr size_t kSlot = partial_slot_bytes<D, PartT>();
     static_assert(kSlot % 16 == 0, "partial slots stay 16-byte aligned");
     const int tid = threadIdx.x;
@@ -224,7 +240,7 @@ __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int
     const float *olo_row = full ? olo + (size_t)row * D : nullptr;
     if (nchunks == 1) {
         merge_write<D, NT, false, OutT, PartT, Sync>(stage, kSlot, 1, full, m_lo2, l_lo, olo_row, qmask,
-                                                     out_blk, sm, tid);
+                                                     out_blk, sm, tid, gs);
         return;
     }
     uint4 *dst = reinterpret_cast<uint4 *>(partial + (size_t)slot * kSlot);
@@ -237,7 +253,7 @@ __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int
     if (!*s_last) return;
     __threadfence();
     merge_write<D, NT, true, OutT, PartT, Sync>(partial + (size_t)(slot - chunk) * kSlot, kSlot, nchunks, full,
-                                                m_lo2, l_lo, olo_row, qmask, out_blk, sm, tid);
+                                                m_lo2, l_lo, olo_row, qmask, out_blk, sm, tid, gs);
     if (tid == 0) row_arrive[row] = 0;
 }
 

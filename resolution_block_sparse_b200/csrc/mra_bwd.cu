@@ -1,0 +1,414 @@
+// mra_bwd.cu - backward pass: gradients of the forward output with respect to
+// Q, K and V, with the selected blocks held fixed.
+//
+// Page "深入解析 Transformers 中的 MRA 模型", section "源码级原理":
+//   step three - the sampled-dense products are autograd functions whose
+//                backward reuses the forward's kernels through transposed
+//                block indices, so the model trains end to end;
+//   step four  - in sparse mode the low-resolution branch only picks blocks
+//                (no gradient); in full mode its output is part of the result
+//                and the gradient flows through the block means of Q, K, V.
+//
+// With p the softmax weights of a query row i (high- and low-resolution terms
+// under one normaliser), lse2_i the base-2 log-sum-exp and delta_i = dO_i.O_i,
+// both exported by the forward kernels:
+//   high resolution, selected block (r, c), query i in r, key j in c:
+//     p_ij = 2^(s_ij log2e - lse2_i),  ds_ij = p_ij (dO_i.v_j - delta_i)
+//     dQ_i += ds_ij k_j / sqrt(D),  dK_j += ds_ij q_i / sqrt(D),  dV_j += p_ij dO_i
+//   low resolution (full mode), unselected block c with cnt_c > 0, row block b:
+//     W_bc = cnt_c 2^(l_bc log2e - R_b),  A_b = sum_i 2^(R_b - lse2_i) dO_i,
+//     B_b = sum_i 2^(R_b - lse2_i) delta_i  (R_b: the smallest lse2 of b)
+//     dl_bc = W_bc (vhat_c.A_b - B_b),  dvhat_c += W_bc A_b,
+//     dqhat_b += dl_bc khat_c / sqrt(D),  dkhat_c += dl_bc qhat_b / sqrt(D)
+//   and every valid token of a block takes its block mean's gradient / cnt.
+//
+// Kernels: bwd_item (one CTA per forward work item: dQ of its rows in
+// registers, dK and dV of its key blocks added with vector fp32 atomics, the
+// transposed index traversal being the atomics' addresses), and in full mode
+// lowres_bwd_prep (A, B, R per row block), lowres_bwd_rows (dqhat),
+// lowres_bwd_cols (dkhat, dvhat, a traversal of the map by key block) and
+// lowres_bwd_scatter (block means to tokens).  All arithmetic is fp32 (FFMA).
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "mra_internal.cuh"
+
+namespace mra {
+namespace {
+
+constexpr float kLog2eB = 1.4426950408889634f;
+constexpr int kBwdThreads = 128;   // four threads per query row
+
+template <typename T>
+__device__ __forceinline__ float ldf(const T *p, size_t i);
+template <>
+__device__ __forceinline__ float ldf<float>(const float *p, size_t i) { return p[i]; }
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+
+__device__ __forceinline__ void atomic_add4(float *p, float4 v) {
+    atomicAdd(reinterpret_cast<float4 *>(p), v);
+}
+
+struct BwdArgs {
+    const void *q, *k, *v, *dout;
+    const float *mask;
+    const WorkItem *items;
+    const int *head_items;
+    const int *cols;
+    int cap, H, N, nbr;
+    float scale, scale_log2;
+    const float *lse2, *delta;
+    float *dq, *dk, *dv;
+};
+
+// One work item (block row r, up to `chunk` selected key blocks).
+template <typename T, int D>
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_item_kernel(const BwdArgs a) {
+    pdl_wait();
+    constexpr int kDp = D / 4;
+    __shared__ __align__(16) float sQ[32][D];
+    __shared__ __align__(16) float sG[32][D];   // dO of the row block
+    __shared__ __align__(16) float sK[32][D];
+    __shared__ __align__(16) float sV[32][D];
+    __shared__ float sP[32][33], sS[32][33];     // p and ds, [query][key]
+    __shared__ float sKm[32];
+
+    const int slot = blockIdx.x;
+    const int bh = slot / a.cap, local = slot % a.cap;
+    if (local >= a.head_items[bh]) return;
+    const WorkItem it = a.items[slot];
+    if (it.ncols <= 0) return;
+    const int r = it.row % a.nbr;
+    const int b = bh / a.H;
+    const size_t head = (size_t)bh * a.N;
+    const T *qg = static_cast<const T *>(a.q) + head * D;
+    const T *kg = static_cast<const T *>(a.k) + head * D;
+    const T *vg = static_cast<const T *>(a.v) + head * D;
+    const T *gg = static_cast<const T *>(a.dout) + head * D;
+    const float *mrow = a.mask ? a.mask + (size_t)b * a.N : nullptr;
+    const int tid = threadIdx.x, qrow = tid >> 2, part = tid & 3, d0 = part * kDp;
+    const size_t qi = (size_t)r * 32 + qrow;
+
+    for (int e = tid; e < 32 * D; e += kBwdThreads) {
+        sQ[e / D][e % D] = ldf(qg, (size_t)r * 32 * D + e);
+        sG[e / D][e % D] = ldf(gg, (size_t)r * 32 * D + e);
+    }
+    const float lse2 = a.lse2[head + qi];   // +inf: the row's output is a constant
+    const float dlt = a.delta[head + qi];
+    float dq[kDp];
+#pragma unroll
+    for (int i = 0; i < kDp; ++i) dq[i] = 0.0f;
+
+    for (int j = 0; j < it.ncols; ++j) {
+        const int c = a.cols[it.col_start + j];
+        __syncthreads();   // previous tile consumed (and sQ / sG written)
+        for (int e = tid; e < 32 * D; e += kBwdThreads) {
+            sK[e / D][e % D] = ldf(kg, (size_t)c * 32 * D + e);
+            sV[e / D][e % D] = ldf(vg, (size_t)c * 32 * D + e);
+        }
+        if (tid < 32) sKm[tid] = mrow ? mrow[c * 32 + tid] : 1.0f;
+        __syncthreads();
+        for (int kj = 0; kj < 32; ++kj) {
+            float s = 0.0f, dp = 0.0f;
+#pragma unroll
+            for (int i = 0; i < kDp; ++i) {
+                s = fmaf(sQ[qrow][d0 + i], sK[kj][d0 + i], s);
+                dp = fmaf(sG[qrow][d0 + i], sV[kj][d0 + i], dp);
+            }
+            s += __shfl_xor_sync(0xffffffffu, s, 1);
+            s += __shfl_xor_sync(0xffffffffu, s, 2);
+            dp += __shfl_xor_sync(0xffffffffu, dp, 1);
+            dp += __shfl_xor_sync(0xffffffffu, dp, 2);
+            const float p = (sKm[kj] > 0.0f) ? exp2f(fmaf(s, a.scale_log2, -lse2)) : 0.0f;
+            const float ds = p * (dp - dlt);
+            if (part == 0) {
+                sP[qrow][kj] = p;
+                sS[qrow][kj] = ds;
+            }
+            const float w = ds * a.scale;
+#pragma unroll
+            for (int i = 0; i < kDp; ++i) dq[i] = fmaf(w, sK[kj][d0 + i], dq[i]);
+        }
+        __syncthreads();
+        // key kj = tid / 4 of block c: dK and dV over the 32 query rows
+        {
+            const int kj = tid >> 2;
+            float dk[kDp], dv[kDp];
+#pragma unroll
+            for (int i = 0; i < kDp; ++i) dk[i] = dv[i] = 0.0f;
+            for (int qr = 0; qr < 32; ++qr) {
+                const float ds = sS[qr][kj] * a.scale, p = sP[qr][kj];
+#pragma unroll
+                for (int i = 0; i < kDp; ++i) {
+                    dk[i] = fmaf(ds, sQ[qr][d0 + i], dk[i]);
+                    dv[i] = fmaf(p, sG[qr][d0 + i], dv[i]);
+                }
+            }
+            float *dkr = a.dk + (head + (size_t)c * 32 + kj) * D + d0;
+            float *dvr = a.dv + (head + (size_t)c * 32 + kj) * D + d0;
+#pragma unroll
+            for (int i = 0; i < kDp; i += 4) {
+                atomic_add4(dkr + i, make_float4(dk[i], dk[i + 1], dk[i + 2], dk[i + 3]));
+                atomic_add4(dvr + i, make_float4(dv[i], dv[i + 1], dv[i + 2], dv[i + 3]));
+            }
+        }
+    }
+    float *dqr = a.dq + (head + qi) * D + d0;
+#pragma unroll
+    for (int i = 0; i < kDp; i += 4) atomic_add4(dqr + i, make_float4(dq[i], dq[i + 1], dq[i + 2], dq[i + 3]));
+}
+
+// ------------------------------------------------------------------ low resolution (full mode)
+
+struct LoArgs {
+    const void *dout;
+    const float *lse2, *delta;
+    const float *qhat, *khat, *vhat;   // [BH][nbr][D]
+    const int *cnt;                    // [B][nbr]
+    const unsigned int *bitmap;        // selected blocks, [BH*nbr][wpr]
+    int wpr, H, N, nbr;
+    float scale;
+    float *ab;                         // [BH*nbr][D + 4]: A (D), B, R, valid
+    float *dxh;                        // [3][BH][nbr][D]: dqhat, dkhat, dvhat
+};
+
+// A_b, B_b, R_b of one row block (one CTA of D threads).
+template <typename T, int D>
+__global__ void __launch_bounds__(D)
+lowres_bwd_prep_kernel(const LoArgs a) {
+    pdl_wait();
+    __shared__ float w[32];
+    __shared__ float s_r;
+    const int rb = blockIdx.x;   // bh * nbr + b
+    const int bh = rb / a.nbr, b = rb % a.nbr;
+    const size_t q0 = (size_t)bh * a.N + (size_t)b * 32;
+    const int t = threadIdx.x;
+    if (t < 32) {
+        const float l = a.lse2[q0 + t];
+        float m = l;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fminf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        w[t] = (l == INFINITY) ? 0.0f : exp2f(m - l);
+        if (t == 0) s_r = m;
+    }
+    __syncthreads();
+    const T *g = static_cast<const T *>(a.dout) + q0 * D;
+    float acc = 0.0f;
+    for (int i = 0; i < 32; ++i) acc = fmaf(w[i], ldf(g, (size_t)i * D + t), acc);
+    float *out = a.ab + (size_t)rb * (D + 4);
+    out[t] = acc;
+    if (t == 0) {
+        float bsum = 0.0f;
+        for (int i = 0; i < 32; ++i) bsum = fmaf(w[i], a.delta[q0 + i], bsum);
+        out[D] = bsum;
+        out[D + 1] = s_r;
+        out[D + 2] = (s_r == INFINITY) ? 0.0f : 1.0f;   // the row block has a query with terms
+    }
+}
+
+// dl_bc and W_bc of one (row block b, key block c) pair, or 0 when the pair
+// takes no low-resolution weight (selected, empty column, or no query).
+// One warp: lane holds dims lane and lane + 32 (D = 64) or lane (D = 32).
+template <int D>
+__device__ __forceinline__ void lo_pair(const LoArgs &a, int bh, int b, int c, const float *qb,
+                                        const float *ab, int lane, float &W, float &dl) {
+    W = dl = 0.0f;
+    const int cntc = a.cnt[(size_t)(bh / a.H) * a.nbr + c];
+    const bool sel = (a.bitmap[((size_t)bh * a.nbr + b) * a.wpr + (c >> 5)] >> (c & 31)) & 1u;
+    if (cntc <= 0 || sel || ab[D + 2] == 0.0f) return;
+    const float *kc = a.khat + ((size_t)bh * a.nbr + c) * D;
+    const float *vc = a.vhat + ((size_t)bh * a.nbr + c) * D;
+    float lg = 0.0f, va = 0.0f;
+#pragma unroll
+    for (int d = lane; d < D; d += 32) {
+        lg = fmaf(qb[d], kc[d], lg);
+        va = fmaf(vc[d], ab[d], va);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lg += __shfl_xor_sync(0xffffffffu, lg, o);
+        va += __shfl_xor_sync(0xffffffffu, va, o);
+    }
+    W = (float)cntc * exp2f(fmaf(lg * a.scale, kLog2eB, -ab[D + 1]));
+    dl = W * (va - ab[D]);
+}
+
+// dqhat_b = sum_c dl_bc khat_c / sqrt(D): one CTA of 4 warps per row block.
+template <int D>
+__global__ void __launch_bounds__(128)
+lowres_bwd_rows_kernel(const LoArgs a) {
+    pdl_wait();
+    __shared__ float qb[D], abs_[D + 4], red[4][D];
+    const int rb = blockIdx.x;
+    const int bh = rb / a.nbr, b = rb % a.nbr;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    for (int d = t; d < D; d += 128) qb[d] = a.qhat[(size_t)rb * D + d];
+    for (int d = t; d < D + 4; d += 128) abs_[d] = a.ab[(size_t)rb * (D + 4) + d];
+    __syncthreads();
+    float acc[D / 32];
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) acc[i] = 0.0f;
+    for (int c = warp; c < a.nbr; c += 4) {
+        float W, dl;
+        lo_pair<D>(a, bh, b, c, qb, abs_, lane, W, dl);
+        if (dl != 0.0f) {
+            const float *kc = a.khat + ((size_t)bh * a.nbr + c) * D;
+#pragma unroll
+            for (int i = 0; i < D / 32; ++i) acc[i] = fmaf(dl * a.scale, kc[lane + 32 * i], acc[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) red[warp][lane + 32 * i] = acc[i];
+    __syncthreads();
+    for (int d = t; d < D; d += 128)
+        a.dxh[(size_t)rb * D + d] = red[0][d] + red[1][d] + red[2][d] + red[3][d];
+}
+
+// dkhat_c = sum_b dl_bc qhat_b / sqrt(D) and dvhat_c = sum_b W_bc A_b: one CTA
+// of 4 warps per key block.
+template <int D>
+__global__ void __launch_bounds__(128)
+lowres_bwd_cols_kernel(const LoArgs a, int BH) {
+    pdl_wait();
+    __shared__ float rk[4][D], rv[4][D];
+    const int cb = blockIdx.x;   // bh * nbr + c
+    const int bh = cb / a.nbr, c = cb % a.nbr;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    float ak[D / 32], av[D / 32];
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) ak[i] = av[i] = 0.0f;
+    for (int b = warp; b < a.nbr; b += 4) {
+        const size_t rb = (size_t)bh * a.nbr + b;
+        const float *qb = a.qhat + rb * D;
+        const float *ab = a.ab + rb * (D + 4);
+        float W, dl;
+        lo_pair<D>(a, bh, b, c, qb, ab, lane, W, dl);
+        if (W != 0.0f) {
+#pragma unroll
+            for (int i = 0; i < D / 32; ++i) {
+                ak[i] = fmaf(dl * a.scale, qb[lane + 32 * i], ak[i]);
+                av[i] = fmaf(W, ab[lane + 32 * i], av[i]);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+        rk[warp][lane + 32 * i] = ak[i];
+        rv[warp][lane + 32 * i] = av[i];
+    }
+    __syncthreads();
+    const size_t plane = (size_t)BH * a.nbr * D;
+    for (int d = t; d < D; d += 128) {
+        a.dxh[plane + (size_t)cb * D + d] = rk[0][d] + rk[1][d] + rk[2][d] + rk[3][d];
+        a.dxh[2 * plane + (size_t)cb * D + d] = rv[0][d] + rv[1][d] + rv[2][d] + rv[3][d];
+    }
+}
+
+// Every valid token takes its block mean's gradient divided by the count.
+template <int D>
+__global__ void __launch_bounds__(256)
+lowres_bwd_scatter_kernel(const float *__restrict__ dxh, const int *__restrict__ cnt,
+                          const float *__restrict__ mask, int H, int N, int nbr, int BH, float *dq, float *dk,
+                          float *dv) {
+    pdl_wait();
+    const size_t n4 = (size_t)BH * N * D / 4;
+    const size_t plane = (size_t)BH * nbr * D;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (size_t)gridDim.x * blockDim.x) {
+        const size_t i = 4 * e;
+        const size_t tok = i / D;                   // bh * N + t
+        const int d = (int)(i % D);
+        const int bh = (int)(tok / N), t = (int)(tok % N);
+        const int b = t / 32;
+        const int cb = cnt[(size_t)(bh / H) * nbr + b];
+        if (cb <= 0) continue;
+        if (mask && !(mask[(size_t)(bh / H) * N + t] > 0.0f)) continue;
+        const float inv = 1.0f / (float)cb;
+        const size_t src = ((size_t)bh * nbr + b) * D + d;
+        float4 x;
+        x = *reinterpret_cast<float4 *>(dq + i);
+        x.x = fmaf(dxh[src], inv, x.x); x.y = fmaf(dxh[src + 1], inv, x.y);
+        x.z = fmaf(dxh[src + 2], inv, x.z); x.w = fmaf(dxh[src + 3], inv, x.w);
+        *reinterpret_cast<float4 *>(dq + i) = x;
+        x = *reinterpret_cast<float4 *>(dk + i);
+        x.x = fmaf(dxh[plane + src], inv, x.x); x.y = fmaf(dxh[plane + src + 1], inv, x.y);
+        x.z = fmaf(dxh[plane + src + 2], inv, x.z); x.w = fmaf(dxh[plane + src + 3], inv, x.w);
+        *reinterpret_cast<float4 *>(dk + i) = x;
+        x = *reinterpret_cast<float4 *>(dv + i);
+        x.x = fmaf(dxh[2 * plane + src], inv, x.x); x.y = fmaf(dxh[2 * plane + src + 1], inv, x.y);
+        x.z = fmaf(dxh[2 * plane + src + 2], inv, x.z); x.w = fmaf(dxh[2 * plane + src + 3], inv, x.w);
+        *reinterpret_cast<float4 *>(dv + i) = x;
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_typed(const Problem &p, const Workspace &w, const void *q, const void *k, const void *v,
+                         const float *mask, const void *dout, float *dq, float *dk, float *dv, cudaStream_t s) {
+    BwdArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.dout = dout;
+    a.mask = mask;
+    a.items = w.items;
+    a.head_items = w.head_items;
+    a.cols = w.cols;
+    a.cap = p.cap;
+    a.H = p.H;
+    a.N = p.N;
+    a.nbr = p.nbr;
+    a.scale = 1.0f / sqrtf((float)D);
+    a.scale_log2 = a.scale * kLog2eB;
+    a.lse2 = w.lse2;
+    a.delta = w.delta;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    cudaError_t e = launch_dependent(bwd_item_kernel<T, D>, dim3((unsigned)(p.BH * p.cap)), dim3(kBwdThreads), 0, s, a);
+    if (e != cudaSuccess) return e;
+    if (p.mode != 0) return cudaSuccess;
+    LoArgs l;
+    l.dout = dout;
+    l.lse2 = w.lse2;
+    l.delta = w.delta;
+    l.qhat = w.pooled;
+    l.khat = w.pooled + (size_t)p.BH * p.nbr * D;
+    l.vhat = w.pooled + (size_t)2 * p.BH * p.nbr * D;
+    l.cnt = w.cnt;
+    l.bitmap = w.bitmap;
+    l.wpr = w.words_per_row;
+    l.H = p.H;
+    l.N = p.N;
+    l.nbr = p.nbr;
+    l.scale = a.scale;
+    l.ab = w.lo_ab;
+    l.dxh = w.lo_dxh;
+    const unsigned blocks = (unsigned)(p.BH * p.nbr);
+    e = launch_dependent(lowres_bwd_prep_kernel<T, D>, dim3(blocks), dim3(D), 0, s, l);
+    if (e != cudaSuccess) return e;
+    e = launch_dependent(lowres_bwd_rows_kernel<D>, dim3(blocks), dim3(128), 0, s, l);
+    if (e != cudaSuccess) return e;
+    e = launch_dependent(lowres_bwd_cols_kernel<D>, dim3(blocks), dim3(128), 0, s, l, p.BH);
+    if (e != cudaSuccess) return e;
+    const size_t n4 = (size_t)p.BH * p.N * D / 4;
+    const unsigned grid = (unsigned)std::min<size_t>((n4 + 255) / 256, 148 * 16);
+    return launch_dependent(lowres_bwd_scatter_kernel<D>, dim3(grid), dim3(256), 0, s, w.lo_dxh, w.cnt, mask, p.H,
+                            p.N, p.nbr, p.BH, dq, dk, dv);
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const Problem &p, const Workspace &w, const void *q, const void *k, const void *v,
+                            const float *mask, const void *dout, float *dq, float *dk, float *dv, cudaStream_t s) {
+    if (p.dtype == 0)
+        return p.D == 64 ? launch_typed<__nv_bfloat16, 64>(p, w, q, k, v, mask, dout, dq, dk, dv, s)
+                         : launch_typed<__nv_bfloat16, 32>(p, w, q, k, v, mask, dout, dq, dk, dv, s);
+    return p.D == 64 ? launch_typed<float, 64>(p, w, q, k, v, mask, dout, dq, dk, dv, s)
+                     : launch_typed<float, 32>(p, w, q, k, v, mask, dout, dq, dk, dv, s);
+}
+
+}  // namespace mra

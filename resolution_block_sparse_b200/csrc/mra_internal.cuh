@@ -14,6 +14,8 @@
 //               online max/sum, merged with the low-resolution part
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include <utility>
 
 #include <cuda_runtime.h>
@@ -63,6 +65,7 @@ struct Problem {
     int lowres_ctas;  // CTAs per head of the low-res key kernel
     int radix_ctas;   // CTAs per head of a radix pass
     long long radix_chunk;  // keys per radix CTA
+    int bwd;          // the workspace also holds the backward pass's buffers
 };
 
 struct Workspace {
@@ -92,6 +95,10 @@ struct Workspace {
     float *llo;              // [BH*nbr]
     float *partial;          // [BH*cap][32*(D+2)]
     unsigned int *status;    // 1 word, persistent across calls
+    // backward pass only (Problem::bwd)
+    float *lse2, *delta;     // [BH*N]: base-2 log-sum-exp and dout . out per query
+    float *lo_ab;            // [BH*nbr][D+4]: A, B, R, valid of each row block
+    float *lo_dxh;           // [3][BH][nbr][D]: gradients of the block means
 };
 
 // Planning and the launch sequence shared by the entry points (mra_api.cu).
@@ -105,9 +112,24 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w);
 int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const void *k,
                     const void *v, const float *mask, void *out, int32_t *sel_out,
                     float *logit_out, float *pooled_out, cudaStream_t s, bool profile,
-                    int *launch_count);
+                    int *launch_count, const struct GradStats *gs = nullptr);
 
 // Launchers (each returns cudaGetLastError() of its launches).
+// What the backward pass takes from a forward run, per query row: the base-2
+// log-sum-exp of the row's terms (high and low resolution, under the true
+// maximum; +inf where the output is the constant 0) and delta = dout . out
+// from the fp32 output before rounding.  lse2 == nullptr: not wanted.
+struct GradStats {
+    const void *dout;   // [rows][D] in the input dtype
+    int dout_f32;
+    float *lse2, *delta;
+    size_t qbase;       // global query row of the block's first row
+    __device__ __forceinline__ float dout_at(size_t i) const {
+        return dout_f32 ? static_cast<const float *>(dout)[i]
+                        : __bfloat162float(static_cast<const __nv_bfloat16 *>(dout)[i]);
+    }
+};
+
 // ---------------------------------------------------------------- dependent launches
 // Every kernel after the first of a forward pass is launched with
 // programmatic stream serialization: it may be scheduled while the kernel
@@ -154,7 +176,10 @@ cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *s
                                 cudaStream_t s);
 cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t s);
 cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
-                             const void *v, const float *mask, void *out, cudaStream_t s);
+                             const void *v, const float *mask, void *out, cudaStream_t s,
+                             const GradStats *gs = nullptr);
+cudaError_t launch_backward(const Problem &p, const Workspace &w, const void *q, const void *k, const void *v,
+                            const float *mask, const void *dout, float *dq, float *dk, float *dv, cudaStream_t s);
 // tcgen05 / TMA attention (bf16, D = 64); used by launch_attention when supported.
 bool attention_tc_supported(const Problem &p);
 cudaError_t launch_attention_tc(const Problem &p, const Workspace &w, const void *q, const void *k,
