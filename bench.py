@@ -229,6 +229,102 @@ def run_cuda(args, w, world, rank, local):
             "d2h": oh.numel() * oh.element_size()}
 
 
+def run_cuda_backward(args, w, world, rank, local):
+    """The backward pass (mra_attention_bwd) on the same workload: seeded
+    incoming gradient, CUDA-graph replays timed with events, per-phase
+    events (forward re-run, clearing, per-item kernel, low-resolution part)."""
+    import resolution_block_sparse_b200 as mra
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    mra.load_library()
+    inputs = make_inputs(w, seed=None if rank == 0 else weak_scaling_seed(1000 + w.index, rank))
+    q, k, v = (inputs[x].to(dev) for x in ("q", "k", "v"))
+    mask = None if inputs["mask"] is None else inputs["mask"].to(dev)
+    gen = torch.Generator("cpu").manual_seed(2000 + w.index + 7919 * rank)
+    dout = torch.randn(q.shape, generator=gen).to(q.dtype).to(dev)
+    dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3))
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(st=None):
+        mra.mra_attention_bwd(q, k, v, mask, dout, dq, dk, dv, w.block_per_row, w.approx_mode, w.first_n,
+                              w.diag_n, st if st is not None else torch.cuda.current_stream(dev))
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    status = mra.mra_get_device_status()
+    launches_per_step = mra.mra_last_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    mra.mra_profile_enable(True)
+    mra.mra_profile_read()
+    for _ in range(args.steps):
+        flush.zero_()
+        torch.cuda._sleep(2_000_000)
+        step(stream)
+    torch.cuda.synchronize()
+    phases = mra.mra_profile_read()
+    mra.mra_profile_enable(False)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        graph.replay()
+        stops[i].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in zip(starts, stops))
+    ms = max_over_ranks([ms], device=dev)[0]
+    del graph
+    return {"ms": ms, "phases": phases, "status": status, "launches_per_step": launches_per_step,
+            "clocks": clocks}
+
+
+def oracle_backward_sampler(w, target_s: float = 15.0):
+    """The oracle's backward on a bounded sample of the workload, like
+    oracle_sampler."""
+    import oracle
+
+    inputs = make_inputs(w)
+    gen = torch.Generator("cpu").manual_seed(2000 + w.index)
+    dout = torch.randn(inputs["q"].shape, generator=gen).to(inputs["q"].dtype)
+    cores = os.cpu_count() or 1
+    BH = w.B * w.H
+
+    def slices(S):
+        xs = [inputs[x].reshape(BH, 1, w.N, w.D)[:S].double().numpy() for x in ("q", "k", "v")]
+        g = dout.reshape(BH, 1, w.N, w.D)[:S].double().numpy()
+        m = None
+        if inputs["mask"] is not None:
+            m = inputs["mask"].repeat_interleave(w.H, dim=0)[:S].double().numpy()
+        return xs[0], xs[1], xs[2], m, g
+
+    def timed(a):
+        t0 = time.perf_counter()
+        oracle.backward(*a, block_per_row=w.block_per_row, approx_mode=w.approx_mode, first_n=w.first_n,
+                        diag_n=w.diag_n, nthreads=cores)
+        return time.perf_counter() - t0
+
+    S = 1
+    while True:
+        dt = timed(slices(S))
+        if dt >= target_s / 4 or S >= BH:
+            break
+        S = min(BH, S * 2)
+    return w.B * w.N / (dt * BH / S), f"{S} of {BH} (batch, head) slices, fp64, scaled to the full step", cores
+
+
 def oracle_sampler(w, target_s: float = 15.0):
     """A bounded sample of the workload for the CPU oracle: the first S
     (batch, head) slices, S grown (once) until one run takes about target_s
@@ -279,6 +375,8 @@ def main():
     ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                    help="backward: time mra_attention_bwd on the workload instead (own JSON line)")
     args = ap.parse_args()
     world, rank, local = dist_env()
     w = WORKLOADS[args.workload]
@@ -318,6 +416,40 @@ def main():
 
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    if args.which == "backward":
+        res = run_cuda_backward(args, w, world, rank, local)
+        ms = res["ms"]
+        sel_blocks = w.B * w.H * w.num_block
+        flops = 10 * 32 * 32 * w.D * sel_blocks   # S, dP, dQ, dK, dV per selected block
+        item_us = res["phases"].get("bwd_items", (1, 0.0))
+        item_s = item_us[1] / max(1, item_us[0]) / 1e3
+        clk = res["clocks"].get("sm_max_mhz") or 1965.0
+        peak = 148 * 128 * 2 * clk * 1e6 / 1e12   # fp32 FFMA TFLOP/s
+        achieved = flops / item_s / 1e12 if item_s > 0 else None
+        line = {"metric": f"MRA-2 attention bwd tokens/s (selected blocks) at N={w.N}", "pass": "backward",
+                "value": world * tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32 (" + w.dtype + " inputs)", "data": "synthetic",
+                "config": dict(config, timing="CUDA-graph replay of one mra_attention_bwd call per step "
+                                              "(forward re-run included), CUDA events"),
+                "phases_us": {k_: {"launches": v_[0], "avg_us": 1e3 * v_[1] / max(1, v_[0])}
+                              for k_, v_ in res["phases"].items()},
+                "roofline": {"kernel": "bwd_items", "bound": "alu", "achieved": achieved, "peak": peak,
+                             "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None, "traffic": None,
+                             "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x max SM clock",
+                             "algorithmic_flops_per_launch": flops},
+                "gpu_launches": res["launches_per_step"] * args.steps, "device_status": res["status"],
+                "clocks": res["clocks"]}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            val, sample, cores = oracle_backward_sampler(w)
+            line["cpu_baseline"] = {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                    "sample": sample}
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line))
+        return
     res = run_cuda(args, w, world, rank, local)
     peaks, peak_src = load_peaks()
 

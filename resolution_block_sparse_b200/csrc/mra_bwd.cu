@@ -368,9 +368,12 @@ cudaError_t launch_typed(const Problem &p, const Workspace &w, const void *q, co
     a.dq = dq;
     a.dk = dk;
     a.dv = dv;
-    cudaError_t e = launch_dependent(bwd_item_kernel<T, D>, dim3((unsigned)(p.BH * p.cap)), dim3(kBwdThreads), 0, s, a);
-    if (e != cudaSuccess) return e;
-    if (p.mode != 0) return cudaSuccess;
+    return launch_dependent(bwd_item_kernel<T, D>, dim3((unsigned)(p.BH * p.cap)), dim3(kBwdThreads), 0, s, a);
+}
+
+template <typename T, int D>
+cudaError_t launch_lowres_typed(const Problem &p, const Workspace &w, const float *mask, const void *dout,
+                                float *dq, float *dk, float *dv, cudaStream_t s) {
     LoArgs l;
     l.dout = dout;
     l.lse2 = w.lse2;
@@ -384,11 +387,11 @@ cudaError_t launch_typed(const Problem &p, const Workspace &w, const void *q, co
     l.H = p.H;
     l.N = p.N;
     l.nbr = p.nbr;
-    l.scale = a.scale;
+    l.scale = 1.0f / sqrtf((float)D);
     l.ab = w.lo_ab;
     l.dxh = w.lo_dxh;
     const unsigned blocks = (unsigned)(p.BH * p.nbr);
-    e = launch_dependent(lowres_bwd_prep_kernel<T, D>, dim3(blocks), dim3(D), 0, s, l);
+    cudaError_t e = launch_dependent(lowres_bwd_prep_kernel<T, D>, dim3(blocks), dim3(D), 0, s, l);
     if (e != cudaSuccess) return e;
     e = launch_dependent(lowres_bwd_rows_kernel<D>, dim3(blocks), dim3(128), 0, s, l);
     if (e != cudaSuccess) return e;
@@ -402,13 +405,23 @@ cudaError_t launch_typed(const Problem &p, const Workspace &w, const void *q, co
 
 }  // namespace
 
-cudaError_t launch_backward(const Problem &p, const Workspace &w, const void *q, const void *k, const void *v,
-                            const float *mask, const void *dout, float *dq, float *dk, float *dv, cudaStream_t s) {
+cudaError_t launch_backward_items(const Problem &p, const Workspace &w, const void *q, const void *k,
+                                  const void *v, const float *mask, const void *dout, float *dq, float *dk,
+                                  float *dv, cudaStream_t s) {
     if (p.dtype == 0)
         return p.D == 64 ? launch_typed<__nv_bfloat16, 64>(p, w, q, k, v, mask, dout, dq, dk, dv, s)
                          : launch_typed<__nv_bfloat16, 32>(p, w, q, k, v, mask, dout, dq, dk, dv, s);
     return p.D == 64 ? launch_typed<float, 64>(p, w, q, k, v, mask, dout, dq, dk, dv, s)
                      : launch_typed<float, 32>(p, w, q, k, v, mask, dout, dq, dk, dv, s);
+}
+
+cudaError_t launch_backward_lowres(const Problem &p, const Workspace &w, const float *mask, const void *dout,
+                                   float *dq, float *dk, float *dv, cudaStream_t s) {
+    if (p.dtype == 0)
+        return p.D == 64 ? launch_lowres_typed<__nv_bfloat16, 64>(p, w, mask, dout, dq, dk, dv, s)
+                         : launch_lowres_typed<__nv_bfloat16, 32>(p, w, mask, dout, dq, dk, dv, s);
+    return p.D == 64 ? launch_lowres_typed<float, 64>(p, w, mask, dout, dq, dk, dv, s)
+                     : launch_lowres_typed<float, 32>(p, w, mask, dout, dq, dk, dv, s);
 }
 
 }  // namespace mra

@@ -178,8 +178,11 @@ cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t 
 cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
                              const void *v, const float *mask, void *out, cudaStream_t s,
                              const GradStats *gs = nullptr);
-cudaError_t launch_backward(const Problem &p, const Workspace &w, const void *q, const void *k, const void *v,
-                            const float *mask, const void *dout, float *dq, float *dk, float *dv, cudaStream_t s);
+cudaError_t launch_backward_items(const Problem &p, const Workspace &w, const void *q, const void *k,
+                                  const void *v, const float *mask, const void *dout, float *dq, float *dk,
+                                  float *dv, cudaStream_t s);
+cudaError_t launch_backward_lowres(const Problem &p, const Workspace &w, const float *mask, const void *dout,
+                                   float *dq, float *dk, float *dv, cudaStream_t s);
 // tcgen05 / TMA attention (bf16, D = 64); used by launch_attention when supported.
 bool attention_tc_supported(const Problem &p);
 cudaError_t launch_attention_tc(const Problem &p, const Workspace &w, const void *q, const void *k,
