@@ -424,8 +424,14 @@ def main():
         item_us = res["phases"].get("bwd_items", (1, 0.0))
         item_s = item_us[1] / max(1, item_us[0]) / 1e3
         clk = res["clocks"].get("sm_max_mhz") or 1965.0
-        peak = 148 * 128 * 2 * clk * 1e6 / 1e12   # fp32 FFMA TFLOP/s
         achieved = flops / item_s / 1e12 if item_s > 0 else None
+        if w.dtype == "bf16":   # the per-item kernel runs its products on the tensor cores
+            peaks, src = load_peaks()
+            bound, peak = "tensor", peaks["bf16_tflops"]
+            peak_source = f"{src} (burst) bf16 tensor"
+        else:                   # fp32 inputs: FFMA
+            bound, peak = "alu", 148 * 128 * 2 * clk * 1e6 / 1e12
+            peak_source = "derived: 148 SMs x 128 fp32 lanes x 2 flop x max SM clock"
         line = {"metric": f"MRA-2 attention bwd tokens/s (selected blocks) at N={w.N}", "pass": "backward",
                 "value": world * tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -434,10 +440,9 @@ def main():
                                               "(forward re-run included), CUDA events"),
                 "phases_us": {k_: {"launches": v_[0], "avg_us": 1e3 * v_[1] / max(1, v_[0])}
                               for k_, v_ in res["phases"].items()},
-                "roofline": {"kernel": "bwd_items", "bound": "alu", "achieved": achieved, "peak": peak,
+                "roofline": {"kernel": "bwd_items", "bound": bound, "achieved": achieved, "peak": peak,
                              "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None, "traffic": None,
-                             "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x max SM clock",
-                             "algorithmic_flops_per_launch": flops},
+                             "peak_source": peak_source, "algorithmic_flops_per_launch": flops},
                 "gpu_launches": res["launches_per_step"] * args.steps, "device_status": res["status"],
                 "clocks": res["clocks"]}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -33,6 +33,7 @@
 #include <algorithm>
 
 #include "mra_internal.cuh"
+#include "mra_mma.cuh"
 
 namespace mra {
 namespace {
@@ -161,6 +162,216 @@ bwd_item_kernel(const BwdArgs a) {
     float *dqr = a.dq + (head + qi) * D + d0;
 #pragma unroll
     for (int i = 0; i < kDp; i += 4) atomic_add4(dqr + i, make_float4(dq[i], dq[i + 1], dq[i + 2], dq[i + 3]));
+}
+
+// The same work item on the tensor cores (bf16 inputs, warp-level
+// mma.sync m16n8k16, fp32 accumulation), two warps of 16 query rows:
+//   S = Q K^T and dP = dO V^T from ldmatrix fragments (as in the forward),
+//   P and dS in fp32 registers, dQ += dS K with dS packed to bf16 in
+//   registers, then (from bf16 copies of P and dS in shared memory, read
+//   transposed by ldmatrix.trans) dK = dS^T Q and dV = P^T dO with each warp
+//   owning 16 of the block's keys.  dK, dV and finally dQ are staged in
+//   shared memory and added to global memory with float4 atomics.
+constexpr int kMmaThreads = 64;
+constexpr int kPS = 40;   // row stride (bf16) of the P and dS tiles: 80 bytes, conflict-free ldmatrix
+
+template <int D>
+struct BwdMmaSmem {
+    static constexpr int kTile = 32 * D;
+    __nv_bfloat16 q[kTile], g[kTile];     // Q and dO of the row block, swizzled
+    __nv_bfloat16 kv[2][2][kTile];        // K/V double buffer, swizzled
+    __nv_bfloat16 p[32 * kPS], ds[32 * kPS];   // [query][key]
+    float stage[32][D + 4];               // fp32 staging of a 32 x D gradient tile
+    float km[2][32];
+    int cols[kChunk];
+};
+
+template <int D>
+__device__ __forceinline__ void add_stage_atomic(float (*stage)[D + 4], float *gbase, int tid) {
+    // gbase: row 0 of the 32 x D gradient tile in global memory
+    for (int e = tid; e < 32 * D / 4; e += kMmaThreads) {
+        const int row = e / (D / 4), c4 = (e % (D / 4)) * 4;
+        atomic_add4(gbase + (size_t)row * D + c4, *reinterpret_cast<const float4 *>(&stage[row][c4]));
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kMmaThreads)
+bwd_item_mma_kernel(const BwdArgs a) {
+    using namespace mma;
+    pdl_wait();
+    constexpr int kTile = 32 * D;
+    __shared__ __align__(128) BwdMmaSmem<D> sh;
+    const int slot = blockIdx.x;
+    const int bh = slot / a.cap, local = slot % a.cap;
+    if (local >= a.head_items[bh]) return;
+    const WorkItem it = a.items[slot];
+    if (it.ncols <= 0) return;
+    const int r = it.row % a.nbr;
+    const int b = bh / a.H;
+    const size_t head = (size_t)bh * a.N;
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q) + head * D;
+    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k) + head * D;
+    const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(a.v) + head * D;
+    const __nv_bfloat16 *gg = static_cast<const __nv_bfloat16 *>(a.dout) + head * D;
+    const float *mrow = a.mask ? a.mask + (size_t)b * a.N : nullptr;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, tq = lane & 3;
+    const int ra = warp * 16 + g, rb = ra + 8;   // this thread's query rows (C fragments)
+
+    load_tile_async<D, kMmaThreads>(sh.q, qg + (size_t)r * kTile, tid);
+    load_tile_async<D, kMmaThreads>(sh.g, gg + (size_t)r * kTile, tid);
+    const int ncols = it.ncols;
+    for (int j = tid; j < ncols; j += kMmaThreads) sh.cols[j] = a.cols[it.col_start + j];
+    __syncthreads();
+    {
+        const int c0 = sh.cols[0];
+        load_tile_async<D, kMmaThreads>(sh.kv[0][0], kg + (size_t)c0 * kTile, tid);
+        load_tile_async<D, kMmaThreads>(sh.kv[0][1], vg + (size_t)c0 * kTile, tid);
+        if (tid < 32) sh.km[0][tid] = mrow ? mrow[c0 * 32 + tid] : 1.0f;
+    }
+    cp_async_commit();
+    const float lse_a = a.lse2[head + (size_t)r * 32 + ra], lse_b = a.lse2[head + (size_t)r * 32 + rb];
+    const float dl_a = a.delta[head + (size_t)r * 32 + ra], dl_b = a.delta[head + (size_t)r * 32 + rb];
+
+    float dq[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.0f;
+    unsigned qf[D / 16][4], gf[D / 16][4];
+
+    for (int j = 0; j < ncols; ++j) {
+        const int buf = j & 1;
+        if (j + 1 < ncols) {
+            const int c1 = sh.cols[j + 1];
+            load_tile_async<D, kMmaThreads>(sh.kv[buf ^ 1][0], kg + (size_t)c1 * kTile, tid);
+            load_tile_async<D, kMmaThreads>(sh.kv[buf ^ 1][1], vg + (size_t)c1 * kTile, tid);
+            if (tid < 32) sh.km[buf ^ 1][tid] = mrow ? mrow[c1 * 32 + tid] : 1.0f;
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        if (j == 0) {
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int row = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int ch = 2 * ks + (lane >> 4);
+                ldsm_x4(qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], smem_u32(sh.q + swz<D>(row, ch)));
+                ldsm_x4(gf[ks][0], gf[ks][1], gf[ks][2], gf[ks][3], smem_u32(sh.g + swz<D>(row, ch)));
+            }
+        }
+        const int c = sh.cols[j];
+        const __nv_bfloat16 *sK = sh.kv[buf][0];
+        const __nv_bfloat16 *sV = sh.kv[buf][1];
+        // S = Q K^T and dP = dO V^T for this warp's 16 rows x 32 keys
+        float sc[4][4], dp[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[nt][e] = dp[nt][e] = 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ks += 2) {
+                const int key = nt * 8 + (lane & 7);
+                const int ch = 2 * ks + (lane >> 3);
+                unsigned b0, b1, b2, b3;
+                ldsm_x4(b0, b1, b2, b3, smem_u32(sK + swz<D>(key, ch)));
+                mma16816(sc[nt], qf[ks], b0, b1);
+                mma16816(sc[nt], qf[ks + 1], b2, b3);
+                ldsm_x4(b0, b1, b2, b3, smem_u32(sV + swz<D>(key, ch)));
+                mma16816(dp[nt], gf[ks], b0, b1);
+                mma16816(dp[nt], gf[ks + 1], b2, b3);
+            }
+        }
+        // P = 2^(s scale log2e - lse2), dS = P (dP - delta); both to shared memory (bf16)
+        unsigned pk[4][2], dk_[4][2];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const int kc = nt * 8 + tq * 2;
+            const bool v0 = sh.km[buf][kc] > 0.0f, v1 = sh.km[buf][kc + 1] > 0.0f;
+            const float p0 = v0 ? fast_exp2(fmaf(sc[nt][0], a.scale_log2, -lse_a)) : 0.0f;
+            const float p1 = v1 ? fast_exp2(fmaf(sc[nt][1], a.scale_log2, -lse_a)) : 0.0f;
+            const float p2 = v0 ? fast_exp2(fmaf(sc[nt][2], a.scale_log2, -lse_b)) : 0.0f;
+            const float p3 = v1 ? fast_exp2(fmaf(sc[nt][3], a.scale_log2, -lse_b)) : 0.0f;
+            const float d0v = p0 * (dp[nt][0] - dl_a), d1v = p1 * (dp[nt][1] - dl_a);
+            const float d2v = p2 * (dp[nt][2] - dl_b), d3v = p3 * (dp[nt][3] - dl_b);
+            pk[nt][0] = pack_bf16(p0, p1);
+            pk[nt][1] = pack_bf16(p2, p3);
+            dk_[nt][0] = pack_bf16(d0v, d1v);
+            dk_[nt][1] = pack_bf16(d2v, d3v);
+            *reinterpret_cast<unsigned *>(&sh.p[ra * kPS + kc]) = pk[nt][0];
+            *reinterpret_cast<unsigned *>(&sh.p[rb * kPS + kc]) = pk[nt][1];
+            *reinterpret_cast<unsigned *>(&sh.ds[ra * kPS + kc]) = dk_[nt][0];
+            *reinterpret_cast<unsigned *>(&sh.ds[rb * kPS + kc]) = dk_[nt][1];
+        }
+        // dQ += dS K  (A = dS from registers, B = K read transposed, k = key)
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            unsigned af[4] = {dk_[2 * kk][0], dk_[2 * kk][1], dk_[2 * kk + 1][0], dk_[2 * kk + 1][1]};
+#pragma unroll
+            for (int nd2 = 0; nd2 < D / 16; ++nd2) {
+                const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int ch = 2 * nd2 + (lane >> 4);
+                unsigned b0, b1, b2, b3;
+                ldsm_x4_t(b0, b1, b2, b3, smem_u32(sK + swz<D>(key, ch)));
+                mma16816(dq[2 * nd2], af, b0, b1);
+                mma16816(dq[2 * nd2 + 1], af, b2, b3);
+            }
+        }
+        __syncthreads();   // P and dS of both warps in shared memory
+        // dK = dS^T Q, then dV = P^T dO: this warp's keys 16 warp .. +15
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+            const __nv_bfloat16 *src = which == 0 ? sh.ds : sh.p;
+            const __nv_bfloat16 *rhs = which == 0 ? sh.q : sh.g;
+            float acc[D / 8][4];
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+#pragma unroll
+            for (int kq = 0; kq < 2; ++kq) {
+                // A (16 keys x 16 queries) = src^T: matrix i of the x4 load
+                // takes rows q = 16 kq + (i / 2) 8 + lane % 8 at key offset (i % 2) 8
+                unsigned af[4];
+                {
+                    const int i = lane >> 3;
+                    const int qr = 16 * kq + (i >> 1) * 8 + (lane & 7);
+                    const int key = warp * 16 + (i & 1) * 8;
+                    ldsm_x4_t(af[0], af[1], af[2], af[3], smem_u32(src + qr * kPS + key));
+                }
+#pragma unroll
+                for (int nd2 = 0; nd2 < D / 16; ++nd2) {
+                    const int qrow = kq * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int ch = 2 * nd2 + (lane >> 4);
+                    unsigned b0, b1, b2, b3;
+                    ldsm_x4_t(b0, b1, b2, b3, smem_u32(rhs + swz<D>(qrow, ch)));
+                    mma16816(acc[2 * nd2], af, b0, b1);
+                    mma16816(acc[2 * nd2 + 1], af, b2, b3);
+                }
+            }
+            const float f = which == 0 ? a.scale : 1.0f;
+            const int ka = warp * 16 + g, kb = ka + 8;
+#pragma unroll
+            for (int nd = 0; nd < D / 8; ++nd) {
+                const int d = nd * 8 + tq * 2;
+                *reinterpret_cast<float2 *>(&sh.stage[ka][d]) = make_float2(acc[nd][0] * f, acc[nd][1] * f);
+                *reinterpret_cast<float2 *>(&sh.stage[kb][d]) = make_float2(acc[nd][2] * f, acc[nd][3] * f);
+            }
+            __syncthreads();
+            add_stage_atomic<D>(sh.stage, (which == 0 ? a.dk : a.dv) + (head + (size_t)c * 32) * D, tid);
+            __syncthreads();
+        }
+    }
+    // dQ of the item's rows
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd) {
+        const int d = nd * 8 + tq * 2;
+        *reinterpret_cast<float2 *>(&sh.stage[ra][d]) = make_float2(dq[nd][0] * a.scale, dq[nd][1] * a.scale);
+        *reinterpret_cast<float2 *>(&sh.stage[rb][d]) = make_float2(dq[nd][2] * a.scale, dq[nd][3] * a.scale);
+    }
+    __syncthreads();
+    add_stage_atomic<D>(sh.stage, a.dq + (head + (size_t)r * 32) * D, tid);
 }
 
 // ------------------------------------------------------------------ low resolution (full mode)
@@ -368,7 +579,10 @@ cudaError_t launch_typed(const Problem &p, const Workspace &w, const void *q, co
     a.dq = dq;
     a.dk = dk;
     a.dv = dv;
-    return launch_dependent(bwd_item_kernel<T, D>, dim3((unsigned)(p.BH * p.cap)), dim3(kBwdThreads), 0, s, a);
+    if constexpr (sizeof(T) == 2)
+        return launch_dependent(bwd_item_mma_kernel<D>, dim3((unsigned)(p.BH * p.cap)), dim3(kMmaThreads), 0, s, a);
+    else
+        return launch_dependent(bwd_item_kernel<T, D>, dim3((unsigned)(p.BH * p.cap)), dim3(kBwdThreads), 0, s, a);
 }
 
 template <typename T, int D>
