@@ -36,6 +36,13 @@ What pins each function (tests marked ``not gpu``):
                              every block; central finite differences of
                              ``forward`` with the selection unchanged
                              (``tests/test_oracle_backward_pins.py``).
+* ``bigbird_blocks``       - the BigBird page's pattern rules checked row by
+                             row by counting; attention on the pattern
+                             (``attend_with_selection``, sparse mode) against
+                             SDPA with the same token mask in fp64
+                             (``tests/test_oracle_bigbird_pins.py``).  Which
+                             two blocks are global, the clipped window and
+                             the union of repeated blocks are readings.
 * padded-query outputs (0), the empty-row output (0), the prior band offsets
   and the exact bias arithmetic are readings of the page, not fixed by it:
   **parity unpinned** beyond internal consistency.
@@ -290,3 +297,45 @@ def backward(q, k, v, mask, dout, *, block_per_row: int, approx_mode: int = 0, f
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return dq, dk, dv
+
+
+def bigbird_blocks(N: int, block_size: int, rand_blocks):
+    """Selected 32-token blocks (sorted flat indices r * nbr + c, nbr = N / 32)
+    of one head under the BigBird block-sparse pattern.
+
+    Page "Transformers 中的 BigBird：面向超长序列的稀疏注意力模型完全指南",
+    sections on the attention mechanism and the usage notes: three kinds of
+    attention combined - a window of 3 blocks, 2 global blocks that attend to
+    every block and that every block attends to, and num_random_blocks random
+    blocks per query block (at least one); the sequence length a multiple of
+    the block size; sequences of at most (5 + 2 * num_random_blocks) blocks
+    use full attention.  Readings (the page does not fix them): the global
+    blocks are the first and the last block; the window of block i is
+    {i - 1, i, i + 1} inside the sequence; attention runs over the union of
+    the blocks (a block chosen twice counts once); the random blocks are an
+    input (rand_blocks [nb][r] of block indices, drawn by the caller).
+    Each block_size block (a multiple of 32) maps to the 32-token blocks it
+    covers."""
+    import numpy as np
+
+    if block_size % BLOCK != 0 or N % block_size != 0:
+        raise ValueError("block_size must be a multiple of 32 and divide N")
+    rand_blocks = np.asarray(rand_blocks, dtype=np.int64)
+    nb = N // block_size
+    r = rand_blocks.shape[1] if rand_blocks.ndim == 2 else 0
+    if r < 1 or rand_blocks.shape[0] != nb:
+        raise ValueError("rand_blocks must be [nb][r] with r >= 1")
+    if rand_blocks.min() < 0 or rand_blocks.max() >= nb:
+        raise ValueError("random block out of range")
+    full = nb <= 5 + 2 * r
+    sel = np.zeros((nb, nb), dtype=bool)
+    for i in range(nb):
+        if full or i == 0 or i == nb - 1:
+            sel[i, :] = True
+            continue
+        sel[i, [0, nb - 1]] = True
+        sel[i, max(0, i - 1):min(nb, i + 2)] = True
+        sel[i, rand_blocks[i]] = True
+    f = block_size // BLOCK
+    fine = np.kron(sel, np.ones((f, f), dtype=bool))
+    return np.flatnonzero(fine.ravel()).astype(np.int32)
