@@ -291,6 +291,137 @@ def run_cuda_backward(args, w, world, rank, local):
             "clocks": clocks}
 
 
+def bigbird_lists(bw, rank=0):
+    """Per-(batch, head) BigBird block lists of the workload from the
+    library's host generator, -1 padded to the longest: int32 [BH, cap]."""
+    import numpy as np
+
+    import resolution_block_sparse_b200 as mra
+    from resolution_block_sparse_b200.workloads import bigbird_random_blocks
+
+    BH = bw.B * bw.H
+    rb = bigbird_random_blocks(BH, bw.N // bw.block_size, bw.num_random, bw.seed + 7919 * rank)
+    lists = [mra.mra_bigbird_block_list(bw.N, bw.block_size, rb[h]) for h in range(BH)]
+    cap = max(len(x) for x in lists)
+    arr = np.full((BH, cap), -1, dtype=np.int32)
+    for h, x in enumerate(lists):
+        arr[h, :len(x)] = x
+    return arr, rb
+
+
+def run_cuda_bigbird(args, bw, world, rank, local):
+    """Block-sparse attention on the BigBird pattern (mra_blocksparse_attention_fwd):
+    the lists are built once on the host (the layer's fixed pattern, like a
+    weight) and stay on the device; CUDA-graph replays timed with events;
+    end to end: pinned-host Q, K, V in, output back, through the same call."""
+    import resolution_block_sparse_b200 as mra
+    from resolution_block_sparse_b200.workloads import random_inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    mra.load_library()
+    inputs = random_inputs(bw.B, bw.H, bw.N, bw.D, dtype=torch.bfloat16, seed=bw.seed + 7919 * rank)
+    q, k, v = (inputs[x].to(dev) for x in ("q", "k", "v"))
+    lists, _ = bigbird_lists(bw, rank)
+    idx = torch.from_numpy(lists).to(dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(st=None):
+        mra.mra_blocksparse_attention_fwd(q, k, v, None, out, idx, st if st is not None else stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    status = mra.mra_get_device_status()
+    launches_per_step = mra.mra_last_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    mra.mra_profile_enable(True)
+    mra.mra_profile_read()
+    for _ in range(args.steps):
+        flush.zero_()
+        torch.cuda._sleep(2_000_000)
+        step(stream)
+    torch.cuda.synchronize()
+    phases = mra.mra_profile_read()
+    mra.mra_profile_enable(False)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        graph.replay()
+        stops[i].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in zip(starts, stops))
+    # end to end: host Q, K, V (pinned) to the device, the call, the output back
+    qh, kh, vh = (inputs[x].pin_memory() for x in ("q", "k", "v"))
+    oh = torch.empty_like(qh).pin_memory()
+    e2e_ms = []
+    for i in range(max(args.warmup, 3) + args.steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        step(stream)
+        oh.copy_(out, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i >= max(args.warmup, 3):
+            e2e_ms.append(a.elapsed_time(b))
+    clocks = sampler.stop()
+    e2e = statistics.mean(e2e_ms)
+    ms, e2e = max_over_ranks([ms, e2e], device=dev)
+    del graph
+    return {"ms": ms, "e2e_ms": e2e, "phases": phases, "status": status, "launches_per_step": launches_per_step,
+            "clocks": clocks, "sel_blocks": int((lists >= 0).sum()),
+            "h2d": 3 * q.numel() * q.element_size(), "d2h": out.numel() * out.element_size()}
+
+
+def oracle_bigbird_sampler(bw, target_s: float = 15.0):
+    """The oracle's sparse-mode attention on the BigBird lists (the oracle's
+    own pattern generator), the first S (batch, head) slices, scaled."""
+    import numpy as np
+
+    import oracle
+    from resolution_block_sparse_b200.workloads import bigbird_random_blocks, random_inputs
+
+    inputs = random_inputs(bw.B, bw.H, bw.N, bw.D, dtype=torch.bfloat16, seed=bw.seed)
+    BH = bw.B * bw.H
+    rb = bigbird_random_blocks(BH, bw.N // bw.block_size, bw.num_random, bw.seed)
+    cores = os.cpu_count() or 1
+
+    def timed(S):
+        xs = [inputs[x].reshape(BH, 1, bw.N, bw.D)[:S].double().numpy() for x in ("q", "k", "v")]
+        lists = [oracle.bigbird_blocks(bw.N, bw.block_size, rb[h]) for h in range(S)]
+        cap = max(len(x) for x in lists)
+        sel = np.stack([np.concatenate([x, np.full(cap - len(x), x[0], np.int32)]) for x in lists])
+        t0 = time.perf_counter()
+        oracle.attend_with_selection(xs[0], xs[1], xs[2], None, sel, approx_mode=1, nthreads=cores)
+        return time.perf_counter() - t0
+
+    S = 1
+    while True:
+        dt = timed(S)
+        if dt >= target_s / 4 or S >= BH:
+            break
+        S = min(BH, S * 2)
+    return bw.B * bw.N / (dt * BH / S), f"{S} of {BH} (batch, head) slices, fp64, scaled to the full step", cores
+
+
 def oracle_backward_sampler(w, target_s: float = 15.0):
     """The oracle's backward on a bounded sample of the workload, like
     oracle_sampler."""
@@ -375,8 +506,9 @@ def main():
     ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
-                    help="backward: time mra_attention_bwd on the workload instead (own JSON line)")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward", "bigbird"],
+                    help="backward: time mra_attention_bwd on the workload instead; bigbird: block-sparse "
+                         "attention on the BigBird pattern (own JSON lines)")
     args = ap.parse_args()
     world, rank, local = dist_env()
     w = WORKLOADS[args.workload]
@@ -416,6 +548,55 @@ def main():
 
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    if args.which == "bigbird":
+        from resolution_block_sparse_b200.workloads import BIGBIRD as bw
+
+        res = run_cuda_bigbird(args, bw, world, rank, local)
+        ms = res["ms"]
+        bb_tokens = bw.B * bw.N
+        flops = 4 * 32 * 32 * bw.D * res["sel_blocks"]
+        bytes_ = 4 * bw.B * bw.H * bw.N * bw.D * 2          # Q, K, V read + O write (bf16)
+        att = res["phases"].get("attention", (1, 0.0))
+        att_s = att[1] / max(1, att[0]) / 1e3
+        peaks, src = load_peaks()
+        t_hbm = bytes_ / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+        if t_tc >= t_hbm:
+            bound, unit, achieved, peak = "tensor", "TFLOP/s", flops / att_s / 1e12, peaks["bf16_tflops"]
+        else:
+            bound, unit, achieved, peak = "hbm", "GB/s", bytes_ / att_s / 1e9, peaks["hbm_gbs"]
+        bconfig = {"workload": bw.name, "B": bw.B, "H": bw.H, "N": bw.N, "D": bw.D,
+                   "block_size": bw.block_size, "num_random_blocks": bw.num_random,
+                   "selected_32x32_blocks": res["sel_blocks"],
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "timing": "CUDA-graph replay of one mra_blocksparse_attention_fwd call per step, CUDA events",
+                   "parallelism": f"replicas x{world} (independent (batch, head) shards)"}
+        line = {"metric": f"BigBird block-sparse attention fwd tokens/s at N={bw.N}", "pass": "bigbird",
+                "value": world * bb_tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": bconfig,
+                "tflops_selected_blocks": world * flops / (ms / 1e3) / 1e12,
+                "phases_us": {k_: {"launches": v_[0], "avg_us": 1e3 * v_[1] / max(1, v_[0])}
+                              for k_, v_ in res["phases"].items()},
+                "roofline": {"kernel": "attention", "bound": bound, "achieved": achieved, "peak": peak,
+                             "unit": unit, "frac": achieved / peak, "traffic": None,
+                             "peak_source": f"{src} (burst)", "algorithmic_bytes_per_launch": bytes_,
+                             "algorithmic_flops_per_launch": flops},
+                "e2e": {"value": world * bb_tokens / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+                "gpu_launches": res["launches_per_step"] * args.steps, "device_status": res["status"],
+                "clocks": res["clocks"]}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            val, sample, cores = oracle_bigbird_sampler(bw)
+            line["cpu_baseline"] = {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                    "sample": sample}
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line))
+        return
     if args.which == "backward":
         res = run_cuda_backward(args, w, world, rank, local)
         ms = res["ms"]

@@ -179,6 +179,46 @@ MRA_API int mra_attention_fwd_noalloc(const void *q, const void *k, const void *
                                       int D, int block_per_row, int approx_mode, int first_n,
                                       int diag_n, cudaStream_t stream);
 
+/* Block-sparse attention on a given set of 32x32 blocks per (batch, head):
+ * the attention of step three with the softmax over the union of the given
+ * blocks only (the sparse mode of step four), for any block pattern - the
+ * BigBird pattern of mra_bigbird_block_list among them.  ([MRA page] steps
+ * three and four; page "Transformers 中的 BigBird：面向超长序列的稀疏注意力
+ * 模型完全指南", section on the attention mechanism, for the pattern.)
+ *   q, k, v, out, key_mask: as in the forward pass; dtype MRA_DTYPE_BF16 or
+ *     MRA_DTYPE_F32 selects the element type of q, k, v and out.
+ *   block_idx: DEVICE int32 [B*H][cap_sel], 4-byte aligned; row bh lists the
+ *     head's blocks as flat indices r * (N/32) + c (query block row r, key
+ *     block c) in strictly ascending order, followed by -1 padding.  Heads
+ *     may hold different counts; 1 <= cap_sel <= (N/32)^2.
+ *   Query rows whose block row holds no block, and padded queries, get 0.
+ *   A head whose list is not ascending, holds an index outside
+ *   [0, (N/32)^2) or has an entry >= 0 after a -1 gets no output (out is not
+ *   written for it) and sets MRA_DEV_COUNT in the device status word; the
+ *   other heads are unaffected.
+ * Two kernels; asynchronous on `stream`.  Returns an mra_status value. */
+MRA_API int mra_blocksparse_attention_fwd(const void *q, const void *k, const void *v,
+                                          const float *key_mask, void *out, int B, int H, int N,
+                                          int D, const int32_t *block_idx, int cap_sel, int dtype,
+                                          cudaStream_t stream);
+
+/* The BigBird block pattern of one head as ascending flat 32-token block
+ * indices, host code (page "Transformers 中的 BigBird：面向超长序列的稀疏注意力
+ * 模型完全指南", sections on the attention mechanism and the usage notes):
+ * with nb = N / block_size blocks, block i attends to the window
+ * {i-1, i, i+1} (clipped at the ends), to the first and the last block (the
+ * two global blocks, which also attend to every block) and to its
+ * num_random random blocks rand_blocks[i][0..num_random) (HOST int32
+ * [nb][num_random], each in [0, nb), drawn by the caller); a block chosen
+ * twice counts once; when nb <= 5 + 2 * num_random every block attends to
+ * every block.  block_size is a multiple of 32 that divides N; each
+ * block_size block maps to the (block_size/32)^2 32-token blocks it covers.
+ * out: HOST int32 [capacity]; *count gets the number written.  Returns
+ * MRA_ERR_INVALID_ARG for bad sizes or random blocks, MRA_ERR_TOO_LARGE when
+ * capacity is short, MRA_ERR_UNSUPPORTED for N > 65536. */
+MRA_API int mra_bigbird_block_list(int N, int block_size, int num_random, const int32_t *rand_blocks,
+                                   int32_t *out, int capacity, int *count);
+
 /* num_block = min((N/32) * block_per_row, (N/32)^2); 0 for invalid input. */
 MRA_API size_t mra_num_block(int N, int block_per_row);
 

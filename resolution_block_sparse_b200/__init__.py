@@ -1,4 +1,5 @@
-"""B200-native MRA-2 approximate self-attention (forward and backward passes).
+"""B200-native MRA-2 approximate self-attention (forward and backward passes),
+and block-sparse attention on given block patterns (BigBird among them).
 
 The compute path lives in the CUDA library ``libmra_b200.so`` behind the C-ABI
 declared in ``include/mra.h``; this package is a thin ctypes binding to it
@@ -21,6 +22,8 @@ from ._binding import (  # noqa: F401
     mra_attention_fwd_f32,
     mra_attention_fwd_host,
     mra_attention_fwd_noalloc,
+    mra_bigbird_block_list,
+    mra_blocksparse_attention_fwd,
     mra_get_device_status,
     mra_last_launch_count,
     mra_num_block,

@@ -26,7 +26,7 @@ EXPORTED = (
     "mra_attention_fwd", "mra_attention_fwd_f32", "mra_attention_fwd_ex", "mra_attention_fwd_host",
     "mra_num_block", "mra_status_string", "mra_get_device_status", "mra_profile_enable",
     "mra_profile_read", "mra_last_launch_count", "mra_attention_fwd_noalloc", "mra_attention_bwd",
-    "mra_attention_bwd_f32",
+    "mra_attention_bwd_f32", "mra_blocksparse_attention_fwd", "mra_bigbird_block_list",
 )
 
 _lock = threading.Lock()
@@ -66,6 +66,10 @@ def load_library(path: str = LIB_PATH):
             fn = getattr(lib, name)
             fn.argtypes = [vp] * 8 + [c_int] * 8 + [vp]
             fn.restype = c_int
+        lib.mra_blocksparse_attention_fwd.argtypes = [vp] * 5 + [c_int] * 4 + [vp, c_int, c_int, vp]
+        lib.mra_blocksparse_attention_fwd.restype = c_int
+        lib.mra_bigbird_block_list.argtypes = [c_int, c_int, c_int, vp, vp, c_int, ctypes.POINTER(c_int)]
+        lib.mra_bigbird_block_list.restype = c_int
         lib.mra_num_block.argtypes = [c_int, c_int]
         lib.mra_num_block.restype = ctypes.c_size_t
         lib.mra_status_string.argtypes = [c_int]
@@ -184,6 +188,39 @@ def mra_attention_fwd_host(q, k, v, key_mask, out, block_per_row, approx_mode, f
                                                first_n, diag_n, dtype, _stream(stream))
     _check(st, "mra_attention_fwd_host")
     return out
+
+
+def mra_blocksparse_attention_fwd(q, k, v, key_mask, out, block_idx, stream=None):
+    """Attention on given 32x32 blocks: block_idx int32 [B*H, cap_sel] on the
+    device, ascending flat indices r * (N/32) + c per head, -1 padded."""
+    B, H, N, D = _shape(q)
+    if block_idx.dtype != torch.int32 or block_idx.dim() != 2 or block_idx.shape[0] != B * H:
+        raise ValueError("block_idx must be int32 [B*H, cap_sel]")
+    if not block_idx.is_contiguous():
+        raise ValueError("block_idx must be contiguous")
+    dtype = MRA_DTYPE_BF16 if q.dtype == torch.bfloat16 else MRA_DTYPE_F32
+    st = load_library().mra_blocksparse_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(key_mask), _ptr(out),
+                                                      B, H, N, D, _ptr(block_idx), int(block_idx.shape[1]),
+                                                      dtype, _stream(stream))
+    _check(st, "mra_blocksparse_attention_fwd")
+    return out
+
+
+def mra_bigbird_block_list(N: int, block_size: int, rand_blocks):
+    """The BigBird pattern of one head (host): rand_blocks int [nb, r] ->
+    int32 numpy array of ascending flat 32-token block indices."""
+    import numpy as np
+
+    rb = np.ascontiguousarray(np.asarray(rand_blocks), dtype=np.int32)
+    if rb.ndim != 2:
+        raise ValueError("rand_blocks must be [nb, r]")
+    nbr = N // 32 if N > 0 else 0
+    out = np.empty(max(1, nbr * nbr), dtype=np.int32)
+    count = ctypes.c_int(0)
+    st = load_library().mra_bigbird_block_list(N, block_size, int(rb.shape[1]), rb.ctypes.data_as(ctypes.c_void_p),
+                                               out.ctypes.data_as(ctypes.c_void_p), int(out.size), ctypes.byref(count))
+    _check(st, "mra_bigbird_block_list")
+    return out[:count.value].copy()
 
 
 def mra_num_block(N: int, block_per_row: int) -> int:

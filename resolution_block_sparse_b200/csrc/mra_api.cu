@@ -51,17 +51,11 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
     p.nbr = N / kBlock;
     p.BH = B * H;
     p.nbr2 = (long long)p.nbr * p.nbr;
-    p.k = (int)std::min<long long>((long long)p.nbr * bpr, p.nbr2);
     p.mode = mode;
     p.first_n = first_n;
     p.diag_n = diag_n;
     p.dtype = dtype;
-    // work items of at most `chunk` blocks: short items keep the critical path
-    // of the long (prior) rows short when rows hold few blocks on average;
-    // longer items amortise the split-row merge when rows are dense
-    const int per_row = (p.k + p.nbr - 1) / p.nbr;
-    p.chunk = per_row <= 4 ? 8 : (per_row <= 16 ? 16 : kChunk);
-    p.cap = p.nbr + p.k / p.chunk;
+    set_budget(p, (int)std::min<long long>((long long)p.nbr * bpr, p.nbr2));
     // low-res rows per CTA: at most 64 KB of logits per CTA, and enough CTAs
     // to cover the SMs twice when the problem allows
     // low-res rows per CTA: the logits of a CTA's rows stay in shared memory
@@ -74,6 +68,16 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
     p.radix_ctas = (int)ctas;
     p.radix_chunk = (p.nbr2 + ctas - 1) / ctas;
     return p;
+}
+
+void set_budget(Problem &p, int k) {
+    p.k = k;
+    // work items of at most `chunk` blocks: short items keep the critical path
+    // of the long (prior) rows short when rows hold few blocks on average;
+    // longer items amortise the split-row merge when rows are dense
+    const int per_row = (p.k + p.nbr - 1) / p.nbr;
+    p.chunk = per_row <= 4 ? 8 : (per_row <= 16 ? 16 : kChunk);
+    p.cap = p.nbr + p.k / p.chunk;
 }
 
 // Carves the workspace; with base == nullptr only computes the size.
@@ -368,9 +372,54 @@ int backward_locked(const void *q, const void *k, const void *v, const float *ma
     return MRA_OK;
 }
 
+// Block-sparse attention on given block lists: the list kernel (work items,
+// column lists, per-call counters), then the attention kernel in sparse
+// mode.  The caller holds g_mutex.
+int blocksparse_locked(const void *q, const void *k, const void *v, const float *mask, void *out, int B, int H,
+                       int N, int D, const int32_t *lists, int cap_sel, int dtype, cudaStream_t s) {
+    if (N < kBlock || (N % kBlock) != 0) return MRA_ERR_INVALID_ARG;
+    const long long nbr = N / kBlock;
+    if (cap_sel < 1 || cap_sel > nbr * nbr || !lists || (((uintptr_t)lists) & 3u)) return MRA_ERR_INVALID_ARG;
+    const int bpr = (int)((cap_sel + nbr - 1) / nbr);
+    int rc = validate(q, k, v, out, B, H, N, D, bpr, MRA_SPARSE, 0, 0);
+    if (rc != MRA_OK) return rc;
+    if (dtype != MRA_DTYPE_BF16 && dtype != MRA_DTYPE_F32) return MRA_ERR_INVALID_ARG;
+    if (mask && (((uintptr_t)mask) & 3u)) return MRA_ERR_INVALID_ARG;
+    int dev;
+    rc = current_device(&dev);
+    if (rc != MRA_OK) return rc;
+    Problem p = make_problem(B, H, N, D, bpr, MRA_SPARSE, 0, 0, dtype);
+    set_budget(p, cap_sel);
+    Workspace w;
+    rc = ensure_workspace(dev, p, &w);
+    if (rc != MRA_OK) return rc;
+    {
+        PhaseScope ps("blocklist_items", s, g_prof);
+        MRA_TRY(launch_blocklist_items(p, w, lists, cap_sel, s));
+    }
+    {
+        PhaseScope ps("attention", s, g_prof);
+        MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s));
+    }
+    g_last_launches = 2;
+    return MRA_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int mra_blocksparse_attention_fwd(const void *q, const void *k, const void *v, const float *key_mask, void *out,
+                                  int B, int H, int N, int D, const int32_t *block_idx, int cap_sel, int dtype,
+                                  cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    return blocksparse_locked(q, k, v, key_mask, out, B, H, N, D, block_idx, cap_sel, dtype, stream);
+}
+
+int mra_bigbird_block_list(int N, int block_size, int num_random, const int32_t *rand_blocks, int32_t *out,
+                           int capacity, int *count) {
+    return bigbird_block_list(N, block_size, num_random, rand_blocks, out, capacity, count);
+}
 
 int mra_attention_bwd(const void *q, const void *k, const void *v, const float *key_mask,
                       const void *dout, float *dq, float *dk, float *dv, int B, int H, int N, int D,

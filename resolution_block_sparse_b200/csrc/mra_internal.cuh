@@ -107,6 +107,8 @@ int validate(const void *q, const void *k, const void *v, const void *out, int B
              int D, int bpr, int mode, int first_n, int diag_n);
 Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n,
                      int dtype);
+// Sets the per-head block budget k and the work-item plan that follows from it.
+void set_budget(Problem &p, int k);
 // Carves the workspace out of base (size only when base is null); returns bytes.
 size_t carve_workspace(const Problem &p, char *base, Workspace *w);
 int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const void *k,
@@ -187,6 +189,15 @@ cudaError_t launch_backward_lowres(const Problem &p, const Workspace &w, const f
 bool attention_tc_supported(const Problem &p);
 cudaError_t launch_attention_tc(const Problem &p, const Workspace &w, const void *q, const void *k,
                                 const void *v, const float *mask, void *out, cudaStream_t s);
+// Block-sparse attention on caller-given block lists (mra_blocklist.cu): the
+// work items, column lists and per-call counters from lists [BH][cap_sel]
+// of ascending flat block indices padded with -1 (p.k == cap_sel).
+cudaError_t launch_blocklist_items(const Problem &p, const Workspace &w, const int32_t *lists, int cap_sel,
+                                   cudaStream_t s);
+// The BigBird pattern of one head as ascending flat 32-token block indices
+// (host code); returns an mra_status value.
+int bigbird_block_list(int N, int block_size, int num_random, const int32_t *rand_blocks, int32_t *out,
+                       int capacity, int *count);
 
 // ---------------------------------------------------------------- device helpers
 #ifdef __CUDACC__

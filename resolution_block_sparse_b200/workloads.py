@@ -128,3 +128,30 @@ def random_inputs(B: int, H: int, N: int, D: int, dtype=torch.float32, seed: int
             if p > 0:
                 mask[b, N - p:] = 0.0
     return {"q": q, "k": k, "v": v, "mask": mask}
+
+
+# BigBird block-sparse workload (page "Transformers 中的 BigBird：面向超长序列的
+# 稀疏注意力模型完全指南": block size 64 and 3 random blocks per query block by
+# default, sequences up to 4096 tokens), run through the block-list attention
+# entry point.  Q, K, V are N(0, 1) bf16 from random_inputs(seed=2000).
+@dataclasses.dataclass(frozen=True)
+class BigBirdWorkload:
+    name: str
+    B: int
+    H: int
+    N: int
+    D: int
+    block_size: int
+    num_random: int
+    seed: int
+
+
+BIGBIRD = BigBirdWorkload("bigbird_b2_h12_n4096_d64_bs64_r3", 2, 12, 4096, 64, 64, 3, 2000)
+
+
+def bigbird_random_blocks(BH: int, nb: int, r: int, seed: int):
+    """Random blocks of the BigBird pattern, drawn per (batch*head, block row):
+    int32 [BH, nb, r], uniform on [0, nb) (a draw may repeat a window or global
+    block; the pattern counts it once)."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    return torch.randint(0, nb, (BH, nb, r), generator=gen, dtype=torch.int64).to(torch.int32).numpy()
