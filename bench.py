@@ -329,7 +329,9 @@ def run_cuda_bigbird(args, bw, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     def step(st=None):
-        mra.mra_blocksparse_attention_fwd(q, k, v, None, out, idx, st if st is not None else stream)
+        # the current stream at call time: the capture stream inside torch.cuda.graph
+        mra.mra_blocksparse_attention_fwd(q, k, v, None, out, idx,
+                                          st if st is not None else torch.cuda.current_stream(dev))
 
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
