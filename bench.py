@@ -424,6 +424,118 @@ def oracle_bigbird_sampler(bw, target_s: float = 15.0):
     return bw.B * bw.N / (dt * BH / S), f"{S} of {BH} (batch, head) slices, fp64, scaled to the full step", cores
 
 
+def run_cuda_layer(args, lw, world, rank, local):
+    """The MraSelfAttention layer (mra_self_attention_fwd): CUDA-graph replays
+    timed with events, per-phase events, and end to end with pinned-host x in
+    and the output back."""
+    import resolution_block_sparse_b200 as mra
+    from resolution_block_sparse_b200.workloads import layer_inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    mra.load_library()
+    xh, wq, bq = layer_inputs(lw, seed=None if rank == 0 else lw.seed + 7919 * rank)
+    x, w, b = xh.to(dev), wq.to(dev), bq.to(dev)
+    out = torch.empty_like(x)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(st=None):
+        mra.mra_self_attention_fwd(x, w, b, None, out, lw.H, lw.block_per_row, lw.approx_mode, lw.first_n,
+                                   lw.diag_n, st if st is not None else torch.cuda.current_stream(dev))
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    status = mra.mra_get_device_status()
+    launches_per_step = mra.mra_last_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    mra.mra_profile_enable(True)
+    mra.mra_profile_read()
+    for _ in range(args.steps):
+        flush.zero_()
+        torch.cuda._sleep(2_000_000)
+        step(stream)
+    torch.cuda.synchronize()
+    phases = mra.mra_profile_read()
+    mra.mra_profile_enable(False)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        graph.replay()
+        stops[i].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in zip(starts, stops))
+    xp = xh.pin_memory()
+    oh = torch.empty_like(xp).pin_memory()
+    e2e_ms = []
+    for i in range(max(args.warmup, 3) + args.steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x.copy_(xp, non_blocking=True)
+        step(stream)
+        oh.copy_(out, non_blocking=True)
+        e.record(stream)
+        e.synchronize()
+        if i >= max(args.warmup, 3):
+            e2e_ms.append(a.elapsed_time(e))
+    clocks = sampler.stop()
+    e2e = statistics.mean(e2e_ms)
+    ms, e2e = max_over_ranks([ms, e2e], device=dev)
+    del graph
+    return {"ms": ms, "e2e_ms": e2e, "phases": phases, "status": status, "launches_per_step": launches_per_step,
+            "clocks": clocks, "h2d": x.numel() * x.element_size(), "d2h": out.numel() * out.element_size()}
+
+
+def oracle_layer_sampler(lw, target_s: float = 15.0):
+    """The oracle's layer on a sample of the work: the first S heads of the
+    first batch entry (their slice of the projection and their attention),
+    scaled to the full step by the number of (batch, head) slices."""
+    import oracle
+    from resolution_block_sparse_b200.workloads import layer_inputs
+
+    x, w, b = layer_inputs(lw)
+    cores = os.cpu_count() or 1
+    d = lw.hidden // lw.H
+    xd = x[:1].double().numpy()
+
+    def timed(S):
+        rows = [j * lw.hidden + i for j in range(3) for i in range(S * d)]
+        ws = w.double().numpy()[rows][:, :]
+        bs = b.double().numpy()[rows]
+        t0 = time.perf_counter()
+        # S heads of one batch entry: hidden_out = S * d, input width unchanged
+        proj = xd @ ws.T + bs
+        q, k, v = (proj[:, :, j * S * d:(j + 1) * S * d].reshape(1, lw.N, S, d).transpose(0, 2, 1, 3)
+                   for j in range(3))
+        oracle.forward(q, k, v, None, block_per_row=lw.block_per_row, approx_mode=lw.approx_mode,
+                       first_n=lw.first_n, diag_n=lw.diag_n, nthreads=cores, want_intermediates=False)
+        return time.perf_counter() - t0
+
+    S = 1
+    while True:
+        dt = timed(S)
+        if dt >= target_s / 4 or S >= lw.H:
+            break
+        S = min(lw.H, S * 2)
+    heads_total = lw.B * lw.H
+    return (lw.B * lw.N / (dt * heads_total / S),
+            f"{S} of {heads_total} (batch, head) slices (their projection and attention), fp64, scaled", cores)
+
+
 def oracle_backward_sampler(w, target_s: float = 15.0):
     """The oracle's backward on a bounded sample of the workload, like
     oracle_sampler."""
@@ -508,9 +620,9 @@ def main():
     ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward", "bigbird"],
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward", "bigbird", "layer"],
                     help="backward: time mra_attention_bwd on the workload instead; bigbird: block-sparse "
-                         "attention on the BigBird pattern (own JSON lines)")
+                         "attention on the BigBird pattern; layer: the MraSelfAttention layer (own JSON lines)")
     args = ap.parse_args()
     world, rank, local = dist_env()
     w = WORKLOADS[args.workload]
@@ -550,6 +662,46 @@ def main():
 
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    if args.which == "layer":
+        from resolution_block_sparse_b200.workloads import LAYER as lw
+
+        res = run_cuda_layer(args, lw, world, rank, local)
+        ms = res["ms"]
+        lt = lw.B * lw.N
+        phases = {k_: {"launches": v_[0], "avg_us": 1e3 * v_[1] / max(1, v_[0])} for k_, v_ in res["phases"].items()}
+        proj_flops = 2 * lw.B * lw.N * 3 * lw.hidden * lw.hidden
+        prj = phases.get("qkv_proj", {"avg_us": 0.0})
+        peaks, src = load_peaks()
+        achieved = proj_flops / (prj["avg_us"] * 1e-6) / 1e12 if prj["avg_us"] > 0 else None
+        lconfig = {"workload": lw.name, "B": lw.B, "N": lw.N, "hidden": lw.hidden, "H": lw.H,
+                   "block_per_row": lw.block_per_row, "approx_mode": "full" if lw.approx_mode == 0 else "sparse",
+                   "first_n": lw.first_n, "diag_n": lw.diag_n,
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "timing": "CUDA-graph replay of one mra_self_attention_fwd call per step, CUDA events",
+                   "parallelism": f"replicas x{world} (independent batch shards)"}
+        line = {"metric": f"MraSelfAttention layer fwd tokens/s at N={lw.N}", "pass": "layer",
+                "value": world * lt / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": lconfig,
+                "phases_us": phases,
+                "roofline": {"kernel": "qkv_proj", "bound": "tensor", "achieved": achieved,
+                             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": (achieved / peaks["bf16_tflops"]) if achieved else None, "traffic": None,
+                             "peak_source": f"{src} (burst)", "algorithmic_flops_per_launch": proj_flops},
+                "e2e": {"value": world * lt / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+                "gpu_launches": res["launches_per_step"] * args.steps, "device_status": res["status"],
+                "clocks": res["clocks"]}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            val, sample, cores = oracle_layer_sampler(lw)
+            line["cpu_baseline"] = {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                    "sample": sample}
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line))
+        return
     if args.which == "bigbird":
         from resolution_block_sparse_b200.workloads import BIGBIRD as bw
 

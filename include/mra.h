@@ -219,6 +219,39 @@ MRA_API int mra_blocksparse_attention_fwd(const void *q, const void *k, const vo
 MRA_API int mra_bigbird_block_list(int N, int block_size, int num_random, const int32_t *rand_blocks,
                                    int32_t *out, int capacity, int *count);
 
+/* The MraSelfAttention layer ([MRA page]: a BERT-style self-attention whose
+ * attention is mra2_attention; heads of size d = hidden / H, zero-padded to
+ * 32 when d < 32, section "源码级原理", notes after step four):
+ *   q, k, v = x W_q^T + b_q, x W_k^T + b_k, x W_v^T + b_v, split into H heads
+ *   (feature h*d + e of a projection is element e of head h), the MRA-2
+ *   forward pass per head with scores scaled by 1/sqrt(d), and the heads
+ *   merged back: out[b][n][h*d + e].
+ *   x:     DEVICE bf16 [B][N][hidden], 16-byte aligned (the hidden states).
+ *   w_qkv: DEVICE bf16 [3*hidden][hidden], 16-byte aligned: the query, key
+ *          and value weights stacked in that order, each [hidden out][hidden
+ *          in] (a linear layer's weight layout).
+ *   b_qkv: DEVICE fp32 [3*hidden] or NULL (no bias).
+ *   key_mask, block_per_row, approx_mode, first_n, diag_n: as in the forward
+ *          pass; out: DEVICE bf16 [B][N][hidden], 16-byte aligned.
+ *   hidden must be a multiple of H and of 8, d = hidden / H <= 64; heads
+ *   with d < 32 are padded to 32 and 32 < d < 64 to 64 (Q is scaled by
+ *   sqrt(padded / d) so that the scores keep 1/sqrt(d)).  The projected
+ *   Q, K, V live in bf16, as the kernels' inputs do.
+ * The projection runs on the tcgen05 tensor cores; the library's workspace
+ * holds the projected heads.  Asynchronous on `stream`; returns an
+ * mra_status value. */
+MRA_API int mra_self_attention_fwd(const void *x, const void *w_qkv, const float *b_qkv,
+                                   const float *key_mask, void *out, int B, int N, int hidden, int H,
+                                   int block_per_row, int approx_mode, int first_n, int diag_n,
+                                   cudaStream_t stream);
+
+/* The layer's projection alone: qkv (DEVICE bf16 [3][B][H][N][Dp], 16-byte
+ * aligned, Dp = 32 when d <= 32 else 64) gets the projected, head-split,
+ * zero-padded Q (scaled by sqrt(Dp / d)), K and V of mra_self_attention_fwd.
+ * Arguments as there.  Returns an mra_status value. */
+MRA_API int mra_qkv_projection(const void *x, const void *w_qkv, const float *b_qkv, void *qkv,
+                               int B, int N, int hidden, int H, cudaStream_t stream);
+
 /* num_block = min((N/32) * block_per_row, (N/32)^2); 0 for invalid input. */
 MRA_API size_t mra_num_block(int N, int block_per_row);
 

@@ -43,6 +43,12 @@ What pins each function (tests marked ``not gpu``):
                              (``tests/test_oracle_bigbird_pins.py``).  Which
                              two blocks are global, the clipped window and
                              the union of repeated blocks are readings.
+* ``self_attention``       - a budget that selects every block equals torch's
+                             multi-head attention (fp64, identity output
+                             projection) on the same weights; permuting the
+                             heads of the weights permutes the output's head
+                             slices; one head with identity weights is the
+                             forward pass itself (``tests/test_oracle_layer_pins.py``).
 * padded-query outputs (0), the empty-row output (0), the prior band offsets
   and the exact bias arithmetic are readings of the page, not fixed by it:
   **parity unpinned** beyond internal consistency.
@@ -339,3 +345,33 @@ def bigbird_blocks(N: int, block_size: int, rand_blocks):
     f = block_size // BLOCK
     fine = np.kron(sel, np.ones((f, f), dtype=bool))
     return np.flatnonzero(fine.ravel()).astype(np.int32)
+
+
+def self_attention(x, w_qkv, b_qkv, mask, H: int, *, block_per_row: int, approx_mode: int = 0,
+                   first_n: int = 0, diag_n: int = 0, nthreads: int = 0):
+    """The MraSelfAttention layer in fp64: x [B,N,hidden], w_qkv
+    [3*hidden, hidden] (query, key, value weights stacked, each [out][in]),
+    b_qkv [3*hidden] or None, mask [B,N] or None.  Returns [B,N,hidden].
+
+    Page "深入解析 Transformers 中的 MRA 模型", the architecture paragraph
+    (BERT-style self-attention: linear query, key and value maps of the
+    hidden states, H heads of size hidden/H) and the engineering notes after
+    step four (heads below 32 are zero-padded for the kernels and cut back:
+    read as leaving the result unchanged, so here the heads keep their own
+    size d and the scores their 1/sqrt(d)).  Feature h*d + e of a projection
+    is element e of head h; the merged output puts head h's output at
+    features h*d .. h*d + d - 1."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_qkv, dtype=np.float64)
+    B, N, hidden = x.shape
+    if hidden % H != 0 or w.shape != (3 * hidden, hidden):
+        raise ValueError("hidden must divide by H and w_qkv be [3*hidden, hidden]")
+    d = hidden // H
+    proj = x @ w.T                                            # [B, N, 3*hidden]
+    if b_qkv is not None:
+        proj = proj + np.asarray(b_qkv, dtype=np.float64)
+    heads = [proj[:, :, j * hidden:(j + 1) * hidden].reshape(B, N, H, d).transpose(0, 2, 1, 3)
+             for j in range(3)]                               # [B, H, N, d] each
+    out = forward(heads[0], heads[1], heads[2], mask, block_per_row=block_per_row, approx_mode=approx_mode,
+                  first_n=first_n, diag_n=diag_n, nthreads=nthreads, want_intermediates=False)["out"]
+    return np.ascontiguousarray(out.transpose(0, 2, 1, 3).reshape(B, N, hidden))

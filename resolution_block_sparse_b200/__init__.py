@@ -29,5 +29,7 @@ from ._binding import (  # noqa: F401
     mra_num_block,
     mra_profile_enable,
     mra_profile_read,
+    mra_qkv_projection,
+    mra_self_attention_fwd,
     mra_status_string,
 )

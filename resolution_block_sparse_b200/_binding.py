@@ -27,6 +27,7 @@ EXPORTED = (
     "mra_num_block", "mra_status_string", "mra_get_device_status", "mra_profile_enable",
     "mra_profile_read", "mra_last_launch_count", "mra_attention_fwd_noalloc", "mra_attention_bwd",
     "mra_attention_bwd_f32", "mra_blocksparse_attention_fwd", "mra_bigbird_block_list",
+    "mra_self_attention_fwd", "mra_qkv_projection",
 )
 
 _lock = threading.Lock()
@@ -70,6 +71,10 @@ def load_library(path: str = LIB_PATH):
         lib.mra_blocksparse_attention_fwd.restype = c_int
         lib.mra_bigbird_block_list.argtypes = [c_int, c_int, c_int, vp, vp, c_int, ctypes.POINTER(c_int)]
         lib.mra_bigbird_block_list.restype = c_int
+        lib.mra_self_attention_fwd.argtypes = [vp] * 5 + [c_int] * 8 + [vp]
+        lib.mra_self_attention_fwd.restype = c_int
+        lib.mra_qkv_projection.argtypes = [vp] * 4 + [c_int] * 4 + [vp]
+        lib.mra_qkv_projection.restype = c_int
         lib.mra_num_block.argtypes = [c_int, c_int]
         lib.mra_num_block.restype = ctypes.c_size_t
         lib.mra_status_string.argtypes = [c_int]
@@ -221,6 +226,39 @@ def mra_bigbird_block_list(N: int, block_size: int, rand_blocks):
                                                out.ctypes.data_as(ctypes.c_void_p), int(out.size), ctypes.byref(count))
     _check(st, "mra_bigbird_block_list")
     return out[:count.value].copy()
+
+
+def _layer_shape(x, w_qkv, H):
+    if x.dim() != 3 or x.dtype != torch.bfloat16 or w_qkv.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16 [B, N, hidden] and w_qkv bf16 [3*hidden, hidden]")
+    B, N, hidden = (int(s) for s in x.shape)
+    if tuple(w_qkv.shape) != (3 * hidden, hidden):
+        raise ValueError("w_qkv must be [3*hidden, hidden]")
+    return B, N, hidden
+
+
+def mra_self_attention_fwd(x, w_qkv, b_qkv, key_mask, out, H, block_per_row, approx_mode, first_n, diag_n,
+                           stream=None):
+    """The MraSelfAttention layer on device tensors: x bf16 [B, N, hidden],
+    w_qkv bf16 [3*hidden, hidden], b_qkv fp32 [3*hidden] or None, key_mask
+    fp32 [B, N] or None; out bf16 [B, N, hidden] is written."""
+    B, N, hidden = _layer_shape(x, w_qkv, H)
+    st = load_library().mra_self_attention_fwd(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(key_mask), _ptr(out), B,
+                                               N, hidden, H, block_per_row, _mode(approx_mode), first_n, diag_n,
+                                               _stream(stream))
+    _check(st, "mra_self_attention_fwd")
+    return out
+
+
+def mra_qkv_projection(x, w_qkv, b_qkv, qkv, H, stream=None):
+    """The layer's projection alone: qkv bf16 [3, B, H, N, Dp] (Dp = 32 if
+    hidden/H <= 32 else 64) gets the head-split, zero-padded Q (scaled by
+    sqrt(Dp/d)), K and V."""
+    B, N, hidden = _layer_shape(x, w_qkv, H)
+    st = load_library().mra_qkv_projection(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(qkv), B, N, hidden, H,
+                                           _stream(stream))
+    _check(st, "mra_qkv_projection")
+    return qkv
 
 
 def mra_num_block(N: int, block_per_row: int) -> int:

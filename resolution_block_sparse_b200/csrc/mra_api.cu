@@ -44,6 +44,7 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
                      int dtype) {
     Problem p;
     p.bwd = 0;
+    p.layer = 0;
     p.B = B;
     p.H = H;
     p.N = N;
@@ -121,6 +122,10 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
         t.delta = (float *)take(sizeof(float) * BH * (size_t)p.N);
         t.lo_ab = (float *)take(sizeof(float) * BH * nbr * (D + 4));
         t.lo_dxh = (float *)take(sizeof(float) * 3 * BH * nbr * D);
+    }
+    if (p.layer) {
+        t.lqkv = take(2 * 3 * BH * (size_t)p.N * D);
+        t.lout = take(2 * BH * (size_t)p.N * D);
     }
     if (w) *w = t;
     return off;
@@ -405,6 +410,56 @@ int blocksparse_locked(const void *q, const void *k, const void *v, const float 
     return MRA_OK;
 }
 
+// Checks of the layer's arguments; d gets the head size.
+int validate_layer(const void *x, const void *w_qkv, const float *b_qkv, const void *out, int B, int N, int hidden,
+                   int H, int *d) {
+    if (!x || !w_qkv || !out) return MRA_ERR_INVALID_ARG;
+    if ((((uintptr_t)x) | ((uintptr_t)w_qkv) | ((uintptr_t)out)) & 15u) return MRA_ERR_INVALID_ARG;
+    if (b_qkv && (((uintptr_t)b_qkv) & 3u)) return MRA_ERR_INVALID_ARG;
+    if (B < 1 || N < kBlock || (N % kBlock) != 0 || H < 1 || hidden < H || hidden % H != 0) return MRA_ERR_INVALID_ARG;
+    *d = hidden / H;
+    if (*d > 64 || (hidden % 8) != 0) return MRA_ERR_UNSUPPORTED;
+    if ((long long)B * N * 3 * hidden > 0x7fffffffLL) return MRA_ERR_UNSUPPORTED;
+    return MRA_OK;
+}
+
+// The layer: projection, the forward pass on the projected heads, head merge.
+// The caller holds g_mutex.
+int layer_locked(const void *x, const void *w_qkv, const float *b_qkv, const float *mask, void *out, int B, int N,
+                 int hidden, int H, int bpr, int mode, int first_n, int diag_n, cudaStream_t s) {
+    int d = 0;
+    int rc = validate_layer(x, w_qkv, b_qkv, out, B, N, hidden, H, &d);
+    if (rc != MRA_OK) return rc;
+    const int Dp = head_padded_size(d);
+    rc = validate_sizes(B, H, N, Dp, bpr, mode, first_n, diag_n);
+    if (rc != MRA_OK) return rc;
+    if (mask && (((uintptr_t)mask) & 3u)) return MRA_ERR_INVALID_ARG;
+    int dev;
+    rc = current_device(&dev);
+    if (rc != MRA_OK) return rc;
+    Problem p = make_problem(B, H, N, Dp, bpr, mode, first_n, diag_n, MRA_DTYPE_BF16);
+    p.layer = 1;
+    Workspace w;
+    rc = ensure_workspace(dev, p, &w);
+    if (rc != MRA_OK) return rc;
+    const size_t plane = 2 * (size_t)B * H * N * Dp;
+    char *qkv = static_cast<char *>(w.lqkv);
+    {
+        PhaseScope ps("qkv_proj", s, g_prof);
+        MRA_TRY(launch_qkv_projection(x, w_qkv, b_qkv, qkv, B, N, hidden, H, w.status, s));
+    }
+    int launches = 0;
+    rc = enqueue_forward(p, w, qkv, qkv + plane, qkv + 2 * plane, mask, w.lout, nullptr, nullptr, nullptr, s, true,
+                         &launches);
+    if (rc != MRA_OK) return rc;
+    {
+        PhaseScope ps("merge_heads", s, g_prof);
+        MRA_TRY(launch_merge_heads(w.lout, out, B, N, H, d, s));
+    }
+    g_last_launches = launches + 2;
+    return MRA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -414,6 +469,33 @@ int mra_blocksparse_attention_fwd(const void *q, const void *k, const void *v, c
                                   cudaStream_t stream) {
     std::lock_guard<std::mutex> lock(g_mutex);
     return blocksparse_locked(q, k, v, key_mask, out, B, H, N, D, block_idx, cap_sel, dtype, stream);
+}
+
+int mra_qkv_projection(const void *x, const void *w_qkv, const float *b_qkv, void *qkv, int B, int N, int hidden,
+                       int H, cudaStream_t stream) {
+    int d = 0;
+    int rc = validate_layer(x, w_qkv, b_qkv, qkv, B, N, hidden, H, &d);
+    if (rc != MRA_OK) return rc;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int dev;
+    rc = current_device(&dev);
+    if (rc != MRA_OK) return rc;
+    DeviceCtx &ctx = g_dev[dev];
+    if (!ctx.status) {
+        if (cudaMalloc(&ctx.status, 256) != cudaSuccess) return MRA_ERR_ALLOC;
+        if (cudaMemset(ctx.status, 0, 256) != cudaSuccess) return MRA_ERR_CUDA;
+    }
+    MRA_TRY(launch_qkv_projection(x, w_qkv, b_qkv, qkv, B, N, hidden, H, ctx.status, stream));
+    g_last_launches = 1;
+    return MRA_OK;
+}
+
+int mra_self_attention_fwd(const void *x, const void *w_qkv, const float *b_qkv, const float *key_mask, void *out,
+                           int B, int N, int hidden, int H, int block_per_row, int approx_mode, int first_n,
+                           int diag_n, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    return layer_locked(x, w_qkv, b_qkv, key_mask, out, B, N, hidden, H, block_per_row, approx_mode, first_n,
+                        diag_n, stream);
 }
 
 int mra_bigbird_block_list(int N, int block_size, int num_random, const int32_t *rand_blocks, int32_t *out,

@@ -66,6 +66,7 @@ struct Problem {
     int radix_ctas;   // CTAs per head of a radix pass
     long long radix_chunk;  // keys per radix CTA
     int bwd;          // the workspace also holds the backward pass's buffers
+    int layer;        // the workspace also holds the layer's Q/K/V and output (bf16 [B][H][N][D] each)
 };
 
 struct Workspace {
@@ -99,6 +100,9 @@ struct Workspace {
     float *lse2, *delta;     // [BH*N]: base-2 log-sum-exp and dout . out per query
     float *lo_ab;            // [BH*nbr][D+4]: A, B, R, valid of each row block
     float *lo_dxh;           // [3][BH][nbr][D]: gradients of the block means
+    // layer only (Problem::layer)
+    void *lqkv;              // [3][B][H][N][D] bf16: projected, head-split Q, K, V
+    void *lout;              // [B][H][N][D] bf16: attention output before the head merge
 };
 
 // Planning and the launch sequence shared by the entry points (mra_api.cu).
@@ -194,6 +198,12 @@ cudaError_t launch_attention_tc(const Problem &p, const Workspace &w, const void
 // of ascending flat block indices padded with -1 (p.k == cap_sel).
 cudaError_t launch_blocklist_items(const Problem &p, const Workspace &w, const int32_t *lists, int cap_sel,
                                    cudaStream_t s);
+// The MraSelfAttention layer (mra_layer.cu): head size d padded to 32 or 64;
+// the Q/K/V projection (tcgen05 GEMM, head-split epilogue) and the head merge.
+int head_padded_size(int d);
+cudaError_t launch_qkv_projection(const void *x, const void *w, const float *bias, void *qkv, int B, int N,
+                                  int hidden, int H, unsigned int *status, cudaStream_t s);
+cudaError_t launch_merge_heads(const void *o, void *out, int B, int N, int H, int d, cudaStream_t s);
 // The BigBird pattern of one head as ascending flat 32-token block indices
 // (host code); returns an mra_status value.
 int bigbird_block_list(int N, int block_size, int num_random, const int32_t *rand_blocks, int32_t *out,

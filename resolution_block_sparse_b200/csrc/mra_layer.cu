@@ -1,0 +1,328 @@
+// mra_layer.cu - the MraSelfAttention layer around the MRA-2 forward pass:
+// the Q/K/V projection as one tcgen05 GEMM whose epilogue adds the bias,
+// splits the heads, zero-pads a head size below the kernel's 32 or 64 and
+// writes bf16 Q, K, V in [B][H][N][Dp]; and the merge of the attention output
+// back into [B][N][H*d].
+//
+// Page "深入解析 Transformers 中的 MRA 模型" (blog.gitcode.com): the layer
+// follows BERT's self-attention (query, key and value linear maps of the
+// hidden states, heads of size hidden/H); when the head size is below 32 the
+// layer pads Q, K and V with zeros to 32 before the attention and cuts the
+// result back (section "源码级原理", the engineering notes after step four).
+// Reading: the padding is meant to leave the result unchanged, so the scores
+// keep the 1/sqrt(d) of the true head size d: Q is scaled by sqrt(Dp/d) in
+// the epilogue, which turns the kernel's 1/sqrt(Dp) into 1/sqrt(d).
+#include <cuda_bf16.h>
+
+#include "mra.h"
+#include "mra_async.cuh"
+#include "mra_internal.cuh"
+#include "mra_tcgen05.cuh"
+
+namespace mra {
+namespace {
+
+using namespace async;
+using namespace tc;
+
+// CTA tile 128 x 256 (rows x output columns), K step 64 (one 128-byte
+// swizzled row of bf16), four stages of 48 KB, two TMEM accumulators of 256
+// columns so that the epilogue of one tile overlaps the MMAs of the next.
+constexpr int kGM = 128, kGN = 256, kGK = 64, kGStages = 4;
+constexpr uint32_t kABytes = kGM * kGK * 2;
+constexpr uint32_t kBBytes = kGN * kGK * 2;
+constexpr uint32_t kGStageBytes = kABytes + kBBytes;
+constexpr int kGThreads = 192;   // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr uint32_t kGTmemCols = 2 * kGN;
+constexpr size_t kGemmSmem = (size_t)kGStages * kGStageBytes + 1024;
+// kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
+// K-major, N = 256, M = 128
+constexpr uint32_t kIdescG =
+    (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kGN >> 3) << 17) | ((uint32_t)(kGM >> 4) << 24);
+
+struct ProjArgs {
+    int M, NC, ktiles;      // rows B*N, output columns 3*hidden, K steps
+    int mtiles, ntiles;
+    int B, N, H, d, Dp, hidden;
+    float qscale;           // sqrt(Dp / d), applied to Q
+    const float *bias;      // [3*hidden] or null
+    __nv_bfloat16 *qkv;     // [3][B][H][N][Dp]
+    unsigned int *status;
+};
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Writes the 32 accumulator columns c0 .. c0+31 of row m.
+__device__ __forceinline__ void store_chunk(const ProjArgs &a, int m, int c0, const uint32_t (&r)[32]) {
+    const int b = m / a.N, n = m - b * a.N;
+    if (a.d == a.Dp && (a.d & 31) == 0) {
+        // the chunk is 32 consecutive elements of one head
+        const int which = c0 / a.hidden, within = c0 - which * a.hidden;
+        const int h = within / a.d, e0 = within - h * a.d;
+        const float *bias = a.bias ? a.bias + c0 : nullptr;
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float x0 = __uint_as_float(r[2 * i]), x1 = __uint_as_float(r[2 * i + 1]);
+            if (bias) {
+                x0 += __ldg(bias + 2 * i);
+                x1 += __ldg(bias + 2 * i + 1);
+            }
+            w[i] = pack2(x0, x1);
+        }
+        __nv_bfloat16 *dst = a.qkv + ((((size_t)which * a.B + b) * a.H + h) * a.N + n) * a.Dp + e0;
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        return;
+    }
+    // general head size: element by element; the column that ends a head
+    // also writes the head's zero padding
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int c = c0 + i;
+        if (c >= a.NC) continue;
+        const int which = c / a.hidden, within = c - which * a.hidden;
+        const int h = within / a.d, e = within - h * a.d;
+        float x = __uint_as_float(r[i]) + (a.bias ? __ldg(a.bias + c) : 0.0f);
+        if (which == 0) x *= a.qscale;
+        __nv_bfloat16 *row = a.qkv + ((((size_t)which * a.B + b) * a.H + h) * a.N + n) * a.Dp;
+        row[e] = __float2bfloat16_rn(x);
+        if (e == a.d - 1)
+            for (int z = a.d; z < a.Dp; ++z) row[z] = __float2bfloat16_rn(0.0f);
+    }
+}
+
+__global__ void __launch_bounds__(kGThreads, 1)
+qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw, ProjArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ __align__(8) unsigned long long bar_full[kGStages], bar_empty[kGStages];
+    __shared__ __align__(8) unsigned long long bar_tfull[2], bar_tempty[2], bar_fin;
+    __shared__ uint32_t s_tmem;
+    unsigned char *base = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = saddr(base);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntotal = a.mtiles * a.ntiles;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kGStages; ++i) {
+            mbar_init(saddr(&bar_full[i]), 1);
+            mbar_init(saddr(&bar_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(saddr(&bar_tfull[i]), 1);
+            mbar_init(saddr(&bar_tempty[i]), 4);
+        }
+        mbar_init(saddr(&bar_fin), 1);
+        mbar_init_fence();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(saddr(&s_tmem)),
+                     "r"(kGTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    pdl_wait();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            int it = 0;
+            for (int t = blockIdx.x; t < ntotal && ok; t += gridDim.x) {
+                const int mt = t % a.mtiles, nt = t / a.mtiles;
+                for (int kt = 0; kt < a.ktiles; ++kt, ++it) {
+                    const int s = it % kGStages, use = it / kGStages;
+                    if (use > 0 && !mbar_wait(saddr(&bar_empty[s]), (use - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = sbase + s * kGStageBytes;
+                    mbar_expect_tx(saddr(&bar_full[s]), kGStageBytes);
+                    tma_load_2d(sa, &tx, kt * kGK, mt * kGM, saddr(&bar_full[s]));
+                    tma_load_2d(sa + kABytes, &tw, kt * kGK, nt * kGN, saddr(&bar_full[s]));
+                }
+            }
+            if (!ok) atomicOr(a.status, kDevTimeout);
+            // the loads issued last into each stage have landed before the CTA
+            // leaves (they have, unless a wait above gave up)
+            for (int s = 0; s < kGStages && s < it; ++s) {
+                const int last = it - 1 - ((it - 1 - s) % kGStages);
+                mbar_wait(saddr(&bar_full[s]), (last / kGStages) & 1);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            int it = 0, tl = 0;
+            for (int t = blockIdx.x; t < ntotal && ok; t += gridDim.x, ++tl) {
+                const int buf = tl & 1, ub = tl >> 1;
+                if (ub > 0 && !mbar_wait(saddr(&bar_tempty[buf]), (ub - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t acc = tmem + buf * kGN;
+                for (int kt = 0; kt < a.ktiles; ++kt, ++it) {
+                    const int s = it % kGStages, use = it / kGStages;
+                    if (!mbar_wait(saddr(&bar_full[s]), use & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = sbase + s * kGStageBytes;
+#pragma unroll
+                    for (int ks = 0; ks < kGK / 16; ++ks)
+                        mma_f16(acc, sdesc(sa + ks * 32, 16, 1024), sdesc(sa + kABytes + ks * 32, 16, 1024),
+                                kIdescG, (kt | ks) != 0);
+                    mma_commit(saddr(&bar_empty[s]));
+                }
+                if (ok) mma_commit(saddr(&bar_tfull[buf]));
+            }
+            if (!ok) atomicOr(a.status, kDevTimeout);
+            // every MMA issued by this thread has completed before TMEM is freed
+            mma_commit(saddr(&bar_fin));
+            mbar_wait(saddr(&bar_fin), 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;   // the TMEM lanes this warp may read
+        int tl = 0;
+        for (int t = blockIdx.x; t < ntotal; t += gridDim.x, ++tl) {
+            const int mt = t % a.mtiles, nt = t / a.mtiles;
+            const int buf = tl & 1, ub = tl >> 1;
+            if (!mbar_wait(saddr(&bar_tfull[buf]), ub & 1)) {
+                atomicOr(a.status, kDevTimeout);
+                break;
+            }
+            tc_fence_after();
+            const int m = mt * kGM + quarter * 32 + lane;
+            const uint32_t row_addr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * kGN;
+#pragma unroll 1
+            for (int j = 0; j < kGN / 32; ++j) {
+                uint32_t r[32];
+                tmem_ld32(row_addr + j * 32, r);
+                tmem_wait_ld();
+                const int c0 = nt * kGN + j * 32;
+                if (m < a.M && c0 < a.NC) store_chunk(a, m, c0, r);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(saddr(&bar_tempty[buf]));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kGTmemCols)
+                     : "memory");
+}
+
+// Attention output [B][H][N][Dp] -> context [B][N][H*d] (the padding cut).
+__global__ void merge_heads_vec_kernel(const __nv_bfloat16 *__restrict__ o, __nv_bfloat16 *__restrict__ out,
+                                       int B, int N, int H, int d, int Dp) {
+    pdl_wait();
+    const int chunks = d >> 3;   // 16-byte chunks per head row
+    const long long total = (long long)B * N * H * chunks;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int c = (int)(i % chunks);
+        long long r = i / chunks;
+        const int h = (int)(r % H);
+        r /= H;
+        const int n = (int)(r % N);
+        const int b = (int)(r / N);
+        const uint4 v = *reinterpret_cast<const uint4 *>(o + (((size_t)b * H + h) * N + n) * Dp + c * 8);
+        *reinterpret_cast<uint4 *>(out + ((size_t)b * N + n) * H * d + h * d + c * 8) = v;
+    }
+}
+
+__global__ void merge_heads_kernel(const __nv_bfloat16 *__restrict__ o, __nv_bfloat16 *__restrict__ out, int B,
+                                   int N, int H, int d, int Dp) {
+    pdl_wait();
+    const long long total = (long long)B * N * H * d;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int e = (int)(i % d);
+        long long r = i / d;
+        const int h = (int)(r % H);
+        r /= H;
+        const int n = (int)(r % N);
+        const int b = (int)(r / N);
+        out[i] = o[(((size_t)b * H + h) * N + n) * Dp + e];
+    }
+}
+
+int sm_count() {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
+}  // namespace
+
+int head_padded_size(int d) { return d <= 32 ? 32 : 64; }
+
+cudaError_t launch_qkv_projection(const void *x, const void *w, const float *bias, void *qkv, int B, int N,
+                                  int hidden, int H, unsigned int *status, cudaStream_t s) {
+    const int d = hidden / H, Dp = head_padded_size(d);
+    CUtensorMap tx, tw;
+    const unsigned long long M = (unsigned long long)B * N, NC = 3ull * hidden;
+    if (!make_map_2d(&tx, x, hidden, M, kGK, kGM) || !make_map_2d(&tw, w, hidden, NC, kGK, kGN))
+        return cudaErrorInvalidValue;
+    ProjArgs a;
+    a.M = (int)M;
+    a.NC = (int)NC;
+    a.ktiles = (hidden + kGK - 1) / kGK;
+    a.mtiles = (int)((M + kGM - 1) / kGM);
+    a.ntiles = (int)((NC + kGN - 1) / kGN);
+    a.B = B;
+    a.N = N;
+    a.H = H;
+    a.d = d;
+    a.Dp = Dp;
+    a.hidden = hidden;
+    a.qscale = sqrtf((float)Dp / (float)d);
+    a.bias = bias;
+    a.qkv = static_cast<__nv_bfloat16 *>(qkv);
+    a.status = status;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kGemmSmem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const int tiles = a.mtiles * a.ntiles;
+    const int grid = tiles < sm_count() ? tiles : sm_count();
+    qkv_proj_kernel<<<grid, kGThreads, kGemmSmem, s>>>(tx, tw, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_merge_heads(const void *o, void *out, int B, int N, int H, int d, cudaStream_t s) {
+    const int Dp = head_padded_size(d);
+    const auto *src = static_cast<const __nv_bfloat16 *>(o);
+    auto *dst = static_cast<__nv_bfloat16 *>(out);
+    const int grid = 4 * sm_count();
+    if ((d & 7) == 0) return launch_dependent(merge_heads_vec_kernel, dim3(grid), dim3(256), 0, s, src, dst, B, N, H, d, Dp);
+    return launch_dependent(merge_heads_kernel, dim3(grid), dim3(256), 0, s, src, dst, B, N, H, d, Dp);
+}
+
+}  // namespace mra

@@ -100,5 +100,21 @@ inline bool make_map(CUtensorMap *m, const void *base, unsigned long long rows) 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major [outer][inner] bf16 matrix, (box_inner x box_outer) boxes,
+// 128-byte swizzle (box_inner * 2 must be 128); reads past either edge fill
+// zeros.  inner * 2 must be a multiple of 16 bytes.
+inline bool make_map_2d(CUtensorMap *m, const void *base, unsigned long long inner, unsigned long long outer,
+                        unsigned box_inner, unsigned box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tc
 }  // namespace mra

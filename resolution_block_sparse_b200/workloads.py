@@ -155,3 +155,34 @@ def bigbird_random_blocks(BH: int, nb: int, r: int, seed: int):
     block; the pattern counts it once)."""
     gen = torch.Generator("cpu").manual_seed(seed)
     return torch.randint(0, nb, (BH, nb, r), generator=gen, dtype=torch.int64).to(torch.int32).numpy()
+
+
+# MraSelfAttention layer workload: the metric's attention (B=2, N=4096, 12
+# heads of 64, sparse, 4 blocks per row, priors 2 and 3) behind its Q/K/V
+# projection from hidden 768 (the page's MraConfig defaults).  x ~ N(0, 1),
+# weights N(0, 1/hidden), bias N(0, 0.01), bf16 x and weights.
+@dataclasses.dataclass(frozen=True)
+class LayerWorkload:
+    name: str
+    B: int
+    N: int
+    hidden: int
+    H: int
+    block_per_row: int
+    approx_mode: int
+    first_n: int
+    diag_n: int
+    seed: int
+
+
+LAYER = LayerWorkload("mra_self_attention_b2_n4096_hidden768_h12_sparse_bpr4_f2_g3", 2, 4096, 768, 12, 4, 1, 2, 3,
+                      3000)
+
+
+def layer_inputs(lw: LayerWorkload, seed: Optional[int] = None):
+    """x bf16 [B, N, hidden], w_qkv bf16 [3*hidden, hidden], b_qkv fp32 [3*hidden]."""
+    gen = torch.Generator("cpu").manual_seed(lw.seed if seed is None else seed)
+    x = torch.randn(lw.B, lw.N, lw.hidden, generator=gen).to(torch.bfloat16)
+    w = (torch.randn(3 * lw.hidden, lw.hidden, generator=gen) * lw.hidden ** -0.5).to(torch.bfloat16)
+    b = torch.randn(3 * lw.hidden, generator=gen) * 0.1
+    return x, w, b

@@ -81,3 +81,26 @@ def test_blocksparse_rejects_bad_arguments(N, D, cap, dtype, lst, expected):
                                              None) == expected
     odd = ctypes.c_void_p(4096 + 8)
     assert lib.mra_blocksparse_attention_fwd(odd, FAKE, FAKE, None, FAKE, 1, 1, 64, 64, FAKE, 4, 0, None) == 1
+
+
+@pytest.mark.parametrize("B,N,hidden,H,expected", [
+    (1, 64, 64, 3, 1),       # hidden not a multiple of H
+    (1, 48, 64, 2, 1),       # N not a multiple of 32
+    (0, 64, 64, 2, 1),       # empty batch
+    (1, 64, 256, 2, 2),      # head size 128 > 64
+    (1, 64, 36, 3, 2),       # hidden not a multiple of 8
+])
+def test_layer_rejects_bad_sizes(B, N, hidden, H, expected):
+    lib = mra.load_library()
+    assert lib.mra_self_attention_fwd(FAKE, FAKE, None, None, FAKE, B, N, hidden, H, 2, 1, 0, 0, None) == expected
+    assert lib.mra_qkv_projection(FAKE, FAKE, None, FAKE, B, N, hidden, H, None) == expected
+
+
+def test_layer_rejects_bad_pointers():
+    lib = mra.load_library()
+    odd = ctypes.c_void_p(4096 + 8)
+    assert lib.mra_self_attention_fwd(odd, FAKE, None, None, FAKE, 1, 64, 64, 2, 2, 1, 0, 0, None) == 1
+    assert lib.mra_self_attention_fwd(FAKE, FAKE, ctypes.c_void_p(4098), None, FAKE, 1, 64, 64, 2, 2, 1, 0, 0,
+                                      None) == 1
+    assert lib.mra_self_attention_fwd(FAKE, FAKE, None, None, FAKE, 1, 64, 64, 2, 2, 5, 0, 0, None) == 1  # mode
+    assert lib.mra_qkv_projection(FAKE, None, None, FAKE, 1, 64, 64, 2, None) == 1

@@ -1,0 +1,156 @@
+"""GPU parity of the MraSelfAttention layer (through the C ABI) with the
+oracle's layer, and of its tcgen05 projection with an fp64 projection.
+
+The projection's bf16 output is compared with the fp64 projection of the same
+bf16 inputs within bf16 rounding (2^-8 relative, plus a small absolute term
+for the fp32 accumulation).  The layer's Q, K, V are bf16 on the GPU and
+fp64 in the oracle, so the two selections may differ on blocks whose oracle
+key lies within the logit perturbation of bf16 rounding of the k-th key:
+layer outputs are compared on every query row whose block row holds no such
+block (and everywhere when the budget selects every block), with the forward
+pass's bf16 tolerance of 2e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import resolution_block_sparse_b200 as mra
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 2e-2
+KEY_MARGIN = 0.05
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    mra.load_library()
+    mra.mra_get_device_status()
+    yield
+
+
+def _layer_inputs(B, N, hidden, seed, bias=True, pad=None, blocky=False):
+    """blocky: every 32-token block of x is its own N(0, 1) centre plus
+    0.5 N(0, 1) per token, so that block means, and with them the
+    low-resolution logits, spread over O(1) instead of sitting near 0."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    x = torch.randn(B, N, hidden, generator=g)
+    if blocky:
+        centres = torch.randn(B, N // 32, 1, hidden, generator=g)
+        x = (centres + 0.5 * x.reshape(B, N // 32, 32, hidden)).reshape(B, N, hidden)
+    x = x.to(torch.bfloat16)
+    w = (torch.randn(3 * hidden, hidden, generator=g) * hidden ** -0.5).to(torch.bfloat16)
+    b = (torch.randn(3 * hidden, generator=g) * 0.1) if bias else None
+    mask = None
+    if pad is not None:
+        mask = torch.ones(B, N)
+        for i, p in enumerate(pad):
+            if p:
+                mask[i, N - p:] = 0.0
+    return x, w, b, mask
+
+
+def _ref_projection(x, w, b, H):
+    B, N, hidden = x.shape
+    d = hidden // H
+    Dp = 32 if d <= 32 else 64
+    proj = x.double().numpy() @ w.double().numpy().T
+    if b is not None:
+        proj = proj + b.double().numpy()
+    out = np.zeros((3, B, H, N, Dp))
+    for j in range(3):
+        out[j, :, :, :, :d] = proj[:, :, j * hidden:(j + 1) * hidden].reshape(B, N, H, d).transpose(0, 2, 1, 3)
+    out[0] *= np.sqrt(Dp / d)
+    return out, Dp
+
+
+@pytest.mark.parametrize("B,N,hidden,H,bias", [
+    (2, 4096, 768, 12, True),    # the layer workload: d = 64, 64 x 9 tiles, 12 K steps
+    (1, 96, 128, 8, True),       # d = 16 (padded to 32), a partial row tile
+    (3, 160, 200, 5, True),      # d = 40 (padded to 64), a K tail and a partial column tile
+    (1, 64, 64, 2, False),       # d = 32, no bias
+    (2, 1024, 1024, 16, True),   # 16 K steps, 192 tiles: CTAs run two tiles (both accumulators)
+])
+def test_projection_parity(B, N, hidden, H, bias):
+    x, w, b, _ = _layer_inputs(B, N, hidden, seed=hidden + N, bias=bias)
+    ref, Dp = _ref_projection(x, w, b, H)
+    dev = torch.device("cuda:0")
+    qkv = torch.full((3, B, H, N, Dp), float("nan"), dtype=torch.bfloat16, device=dev)
+    mra.mra_qkv_projection(x.to(dev), w.to(dev), None if b is None else b.to(dev), qkv, H)
+    torch.cuda.synchronize()
+    assert mra.mra_get_device_status() == 0
+    got = qkv.float().cpu().numpy()
+    assert np.all(np.isfinite(got))                  # every element, padding included, was written
+    err = np.abs(got - ref)
+    bound = 2.0 ** -8 * np.abs(ref) + 1e-4
+    assert np.all(err <= bound), float(np.max(err - bound))
+
+
+def _compare_layer(x, w, b, mask, H, *, bpr, mode, f=0, g=0, min_rows=0.5):
+    B, N, hidden = x.shape
+    dev = torch.device("cuda:0")
+    out = torch.full((B, N, hidden), float("nan"), dtype=torch.bfloat16, device=dev)
+    mra.mra_self_attention_fwd(x.to(dev), w.to(dev), None if b is None else b.to(dev),
+                               None if mask is None else mask.to(dev), out, H, bpr, mode, f, g)
+    torch.cuda.synchronize()
+    assert mra.mra_get_device_status() == 0
+    got = out.float().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    kw = dict(block_per_row=bpr, approx_mode=mode, first_n=f, diag_n=g)
+    m = None if mask is None else mask.double().numpy()
+    want = oracle.self_attention(x.double().numpy(), w.double().numpy(), None if b is None else b.double().numpy(),
+                                 m, H, **kw)
+    # rows whose selection cannot differ: no block of the row within the margin of the k-th key
+    d = hidden // H
+    nbr = N // 32
+    proj = x.double().numpy() @ w.double().numpy().T + (0 if b is None else b.double().numpy())
+    heads = [proj[:, :, j * hidden:(j + 1) * hidden].reshape(B, N, H, d).transpose(0, 2, 1, 3) for j in range(2)]
+    res = oracle.forward(heads[0], heads[1], heads[0], m, **kw)
+    kk = res["k"]
+    keep = np.ones((B, H, nbr), dtype=bool)
+    if kk < nbr * nbr:
+        key = res["key"].reshape(B * H, nbr, nbr)
+        for bh in range(B * H):
+            kth = np.sort(key[bh].ravel())[::-1][kk - 1]
+            near = np.abs(key[bh] - kth) <= KEY_MARGIN
+            keep[bh // H, bh % H] = ~near.any(axis=1)
+    frac = float(keep.mean())
+    assert frac >= min_rows, frac
+    got_h = got.reshape(B, N, H, d).transpose(0, 2, 1, 3).reshape(B, H, nbr, 32, d)
+    want_h = want.reshape(B, N, H, d).transpose(0, 2, 1, 3).reshape(B, H, nbr, 32, d)
+    err = float(np.max(np.abs(got_h[keep] - want_h[keep])))
+    assert err <= OUT_TOL, err
+    return err, frac
+
+
+@pytest.mark.parametrize("B,N,hidden,H,mode,pad", [
+    (2, 256, 64, 4, 0, [0, 45]),     # d = 16: zero padding and the Q scale of the padded heads
+    (2, 256, 64, 4, 1, [70, 0]),
+    (1, 512, 768, 12, 0, None),      # d = 64
+    (1, 192, 200, 5, 1, [33]),       # d = 40
+])
+def test_layer_saturated_budget(B, N, hidden, H, mode, pad):
+    x, w, b, mask = _layer_inputs(B, N, hidden, seed=31 + N, pad=pad)
+    err, frac = _compare_layer(x, w, b, mask, H, bpr=N // 32, mode=mode)
+    assert frac == 1.0
+
+
+@pytest.mark.parametrize("B,N,hidden,H,bpr,mode,f,g,pad", [
+    (1, 1024, 256, 4, 4, 1, 2, 3, None),     # the metric's pattern on a smaller layer
+    (1, 1024, 256, 4, 4, 0, 2, 3, [100]),
+    (2, 512, 128, 8, 2, 0, 1, 1, [0, 64]),   # d = 16
+])
+def test_layer_sparse_budget(B, N, hidden, H, bpr, mode, f, g, pad):
+    x, w, b, mask = _layer_inputs(B, N, hidden, seed=41 + N + hidden, pad=pad, blocky=True)
+    err, frac = _compare_layer(x, w, b, mask, H, bpr=bpr, mode=mode, f=f, g=g)
+    print(f"layer N={N} hidden={hidden}: max-abs {err:.3e} on {frac:.0%} of the rows")
+
+
+def test_layer_workload():
+    """B=2, N=4096, hidden=768, H=12, sparse, 4 blocks per row, priors 2 and 3."""
+    x, w, b, mask = _layer_inputs(2, 4096, 768, seed=4096, blocky=True)
+    err, frac = _compare_layer(x, w, b, mask, 12, bpr=4, mode=1, f=2, g=3, min_rows=0.6)
+    print(f"layer workload: max-abs {err:.3e} on {frac:.0%} of the rows")
