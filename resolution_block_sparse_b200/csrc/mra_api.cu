@@ -248,7 +248,7 @@ namespace mra {
 int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const void *k,
                     const void *v, const float *mask, void *out, int32_t *sel_out,
                     float *logit_out, float *pooled_out, cudaStream_t s, bool profile,
-                    int *launch_count, const GradStats *gs) {
+                    int *launch_count, const GradStats *gs, const OutLayout *ol) {
     const bool prof = profile && g_prof;
     int launches = 0;
     {
@@ -287,7 +287,7 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
     }
     {
         PhaseScope ps("attention", s, prof);
-        MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s, gs));
+        MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s, gs, ol));
         ++launches;
     }
     if (pooled_out) {
@@ -449,6 +449,16 @@ int layer_locked(const void *x, const void *w_qkv, const float *b_qkv, const flo
         MRA_TRY(launch_qkv_projection(x, w_qkv, b_qkv, qkv, B, N, hidden, H, w.status, s));
     }
     int launches = 0;
+    if (d == Dp) {
+        // the attention writes the merged heads itself: element (b, h, n, e)
+        // of the result is out[b][n][h*d + e]
+        const OutLayout ol{(long long)N * hidden, d, hidden};
+        rc = enqueue_forward(p, w, qkv, qkv + plane, qkv + 2 * plane, mask, out, nullptr, nullptr, nullptr, s,
+                             true, &launches, nullptr, &ol);
+        if (rc != MRA_OK) return rc;
+        g_last_launches = launches + 1;
+        return MRA_OK;
+    }
     rc = enqueue_forward(p, w, qkv, qkv + plane, qkv + 2 * plane, mask, w.lout, nullptr, nullptr, nullptr, s, true,
                          &launches);
     if (rc != MRA_OK) return rc;

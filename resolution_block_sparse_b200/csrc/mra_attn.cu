@@ -46,6 +46,9 @@ struct AttnArgs {
     int *row_arrive;
     int *work_next;   // items handed out beyond the first wave (zeroed per call)
     void *out;
+    // output layout: element (b, h, n, e) at b * ob + h * oh + n * orow + e
+    long long ob;
+    int oh, orow;
     GradStats gs;     // backward-pass statistics (gs.lse2 == nullptr: forward only)
 };
 
@@ -224,7 +227,8 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
         l_a += __shfl_xor_sync(0xffffffffu, l_a, off);
         l_b += __shfl_xor_sync(0xffffffffu, l_b, off);
     }
-    __nv_bfloat16 *out_blk = static_cast<__nv_bfloat16 *>(a.out) + head_off + (size_t)r * kTile;
+    __nv_bfloat16 *out_blk = static_cast<__nv_bfloat16 *>(a.out) + (size_t)b * a.ob + (size_t)(bh - b * a.H) * a.oh +
+                             (size_t)r * 32 * a.orow;
     const int ra = warp * 16 + g, rb = ra + 8;
     __syncthreads();   // every warp is done with the K/V buffers
     if (nchunks == 1) {
@@ -288,8 +292,11 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
         }
         __syncthreads();
 #pragma unroll
-        for (int e = tid; e < kTile / 8; e += kBf16Threads)
-            reinterpret_cast<uint4 *>(out_blk)[e] = reinterpret_cast<const uint4 *>(ostage)[e];
+        for (int e = tid; e < kTile / 8; e += kBf16Threads) {
+            const int row = e / (D / 8), c = e - row * (D / 8);
+            *reinterpret_cast<uint4 *>(out_blk + (size_t)row * a.orow + c * 8) =
+                reinterpret_cast<const uint4 *>(ostage)[e];
+        }
         return;
     }
     // row split across work items: (m, l) in fp32 and O in bf16 (the
@@ -315,7 +322,7 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
     gs.qbase = (size_t)bh * a.N + (size_t)r * 32;
     finish_item<D, kBf16Threads, __nv_bfloat16, __nv_bfloat16, SyncAll>(
         reinterpret_cast<const unsigned char *>(stage), slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
-        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last, gs);
+        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, a.orow, sm, &s_last, gs);
 }
 
 // Persistent: the first wave takes items 0..gridDim.x-1, after that a CTA
@@ -423,20 +430,30 @@ attn_f32_kernel(const AttnArgs a) {
 #pragma unroll
     for (int i = 0; i < kDp; ++i) stage[64 + qrow * D + d0 + i] = o[i];
     __syncthreads();
-    float *out_blk = static_cast<float *>(a.out) + head_off + (size_t)r * kTile;
+    float *out_blk = static_cast<float *>(a.out) + (size_t)b * a.ob + (size_t)(bh - b * a.H) * a.oh +
+                     (size_t)r * 32 * a.orow;
     GradStats gs = a.gs;
     gs.qbase = (size_t)bh * a.N + (size_t)r * 32;
     finish_item<D, kF32Threads, float, float, SyncAll>(
         reinterpret_cast<const unsigned char *>(stage), slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
-        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, sm, &s_last, gs);
+        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, a.orow, sm, &s_last, gs);
 }
 
 }  // namespace
 
 cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
                              const void *v, const float *mask, void *out, cudaStream_t s,
-                             const GradStats *gs) {
+                             const GradStats *gs, const OutLayout *ol) {
     AttnArgs a;
+    if (ol) {
+        a.ob = ol->ob;
+        a.oh = ol->oh;
+        a.orow = ol->orow;
+    } else {
+        a.ob = (long long)p.H * p.N * p.D;
+        a.oh = p.N * p.D;
+        a.orow = p.D;
+    }
     a.gs = gs ? *gs : GradStats{};
     a.q = q;
     a.k = k;
@@ -465,7 +482,7 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
     static const char *impl = getenv("MRA_ATTN_IMPL");
     const bool want_tc = impl && impl[0] == 't';
     // the backward pass's statistics come from the kernels below
-    if (want_tc && !gs && attention_tc_supported(p)) return launch_attention_tc(p, w, q, k, v, mask, out, s);
+    if (want_tc && !gs && !ol && attention_tc_supported(p)) return launch_attention_tc(p, w, q, k, v, mask, out, s);
     if (p.dtype == 0) {
         static int sms = 0;
         if (sms == 0) {

@@ -90,7 +90,7 @@ __host__ __device__ constexpr size_t partial_slot_bytes() {
 template <int D, int NT, bool G, typename OutT, typename PartT, typename Sync>
 __device__ void merge_write(const unsigned char *src0, size_t slot_bytes, int nchunks, int full,
                             float m_lo2, float l_lo, const float *olo_row, const float *qmask,
-                            OutT *out_blk, MergeSmem &sm, int tid, const GradStats &gs) {
+                            OutT *out_blk, int orow, MergeSmem &sm, int tid, const GradStats &gs) {
     static_assert((8 * D) % NT == 0, "a chunk's O tile must split evenly into quads per thread");
     constexpr int F = 8 * D / NT;   // quads (4 elements) of one partial's O tile per thread
     constexpr int kRowQ = D / 4;
@@ -207,7 +207,7 @@ __device__ void merge_write(const unsigned char *src0, size_t slot_bytes, int nc
         if (full) ol = *reinterpret_cast<const float4 *>(olo_row + d);
         const float4 ov = make_float4(fmaf(acc[i].x, fa, ol.x * fb), fmaf(acc[i].y, fa, ol.y * fb),
                                       fmaf(acc[i].z, fa, ol.z * fb), fmaf(acc[i].w, fa, ol.w * fb));
-        store4(out_blk + (size_t)q * D + d, ov);
+        store4(out_blk + (size_t)q * orow + d, ov);
         if (gs.lse2) {
             const size_t gi = (gs.qbase + q) * D + d;
             atomicAdd(&sm.dsum[q], ov.x * gs.dout_at(gi) + ov.y * gs.dout_at(gi + 1) +
@@ -231,7 +231,7 @@ template <int D, int NT, typename OutT, typename PartT, typename Sync>
 __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int nchunks, int row, int full,
                             const float *mlo, const float *olo, const float *llo,
                             unsigned char *partial, int *row_arrive, const float *qmask, OutT *out_blk,
-                            MergeSmem &sm, int *s_last, const GradStats &gs) {
+                            int orow, MergeSmem &sm, int *s_last, const GradStats &gs) {
     constexpr size_t kSlot = partial_slot_bytes<D, PartT>();
     static_assert(kSlot % 16 == 0, "partial slots stay 16-byte aligned");
     const int tid = threadIdx.x;
@@ -240,7 +240,7 @@ __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int
     const float *olo_row = full ? olo + (size_t)row * D : nullptr;
     if (nchunks == 1) {
         merge_write<D, NT, false, OutT, PartT, Sync>(stage, kSlot, 1, full, m_lo2, l_lo, olo_row, qmask,
-                                                     out_blk, sm, tid, gs);
+                                                     out_blk, orow, sm, tid, gs);
         return;
     }
     uint4 *dst = reinterpret_cast<uint4 *>(partial + (size_t)slot * kSlot);
@@ -253,7 +253,7 @@ __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int
     if (!*s_last) return;
     __threadfence();
     merge_write<D, NT, true, OutT, PartT, Sync>(partial + (size_t)(slot - chunk) * kSlot, kSlot, nchunks, full,
-                                                m_lo2, l_lo, olo_row, qmask, out_blk, sm, tid, gs);
+                                                m_lo2, l_lo, olo_row, qmask, out_blk, orow, sm, tid, gs);
     if (tid == 0) row_arrive[row] = 0;
 }
 

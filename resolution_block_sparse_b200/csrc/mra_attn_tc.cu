@@ -566,7 +566,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     const float *olo_row = a.full ? a.olo + (size_t)it.row * 64 : nullptr;
                     merge_write<64, kConsumers, true, __nv_bfloat16, float, SyncNamed128>(
                         a.partial + (size_t)(slot - chunk) * kSlot, kSlot, nchunks, a.full, m_lo2, l_lo,
-                        olo_row, qmask, out_blk, msm, tid, GradStats{});
+                        olo_row, qmask, out_blk, 64, msm, tid, GradStats{});
                     if (tid == 0) a.row_arrive[it.row] = 0;
                 }
             }

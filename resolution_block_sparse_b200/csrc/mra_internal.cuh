@@ -118,7 +118,8 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w);
 int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const void *k,
                     const void *v, const float *mask, void *out, int32_t *sel_out,
                     float *logit_out, float *pooled_out, cudaStream_t s, bool profile,
-                    int *launch_count, const struct GradStats *gs = nullptr);
+                    int *launch_count, const struct GradStats *gs = nullptr,
+                    const struct OutLayout *ol = nullptr);
 
 // Launchers (each returns cudaGetLastError() of its launches).
 // What the backward pass takes from a forward run, per query row: the base-2
@@ -181,9 +182,16 @@ cudaError_t launch_lowres_select_fused(const Problem &p, const Workspace &w, flo
 cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *sel_out,
                                 cudaStream_t s);
 cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t s);
+// Output layout of the attention kernels: element (b, h, n, e) of the
+// [B][H][N][D] result at out[b * ob + h * oh + n * orow + e] (null: the
+// contiguous [B][H][N][D] layout).
+struct OutLayout {
+    long long ob;
+    int oh, orow;
+};
 cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
                              const void *v, const float *mask, void *out, cudaStream_t s,
-                             const GradStats *gs = nullptr);
+                             const GradStats *gs = nullptr, const OutLayout *ol = nullptr);
 cudaError_t launch_backward_items(const Problem &p, const Workspace &w, const void *q, const void *k,
                                   const void *v, const float *mask, const void *dout, float *dq, float *dk,
                                   float *dv, cudaStream_t s);

@@ -34,7 +34,11 @@ constexpr uint32_t kBBytes = kGN * kGK * 2;
 constexpr uint32_t kGStageBytes = kABytes + kBBytes;
 constexpr int kGThreads = 192;   // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
 constexpr uint32_t kGTmemCols = 2 * kGN;
-constexpr size_t kGemmSmem = (size_t)kGStages * kGStageBytes + 1024;
+// epilogue staging for the TMA stores of 64-wide heads: two 32 x 64 bf16
+// boxes (4 KB, 128-byte swizzle) per epilogue warp
+constexpr uint32_t kStgBytes = 32 * 64 * 2;
+constexpr uint32_t kStgOffset = kGStages * kGStageBytes;
+constexpr size_t kGemmSmem = (size_t)kStgOffset + 4 * 2 * kStgBytes + 1024;
 // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
 // K-major, N = 256, M = 128
 constexpr uint32_t kIdescG =
@@ -48,7 +52,19 @@ struct ProjArgs {
     const float *bias;      // [3*hidden] or null
     __nv_bfloat16 *qkv;     // [3][B][H][N][Dp]
     unsigned int *status;
+    int tma_out;            // d == Dp == 64: heads leave through TMA stores
 };
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// the shared-memory sources of all but the newest group have been read
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -97,7 +113,8 @@ __device__ __forceinline__ void store_chunk(const ProjArgs &a, int m, int c0, co
 }
 
 __global__ void __launch_bounds__(kGThreads, 1)
-qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw, ProjArgs a) {
+qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
+                const __grid_constant__ CUtensorMap ty, ProjArgs a) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) unsigned long long bar_full[kGStages], bar_empty[kGStages];
     __shared__ __align__(8) unsigned long long bar_tfull[2], bar_tempty[2], bar_fin;
@@ -198,6 +215,8 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
     } else {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;   // the TMEM lanes this warp may read
+        const uint32_t stg = sbase + kStgOffset + (warp - 2) * 2 * kStgBytes;
+        int n_stores = 0;
         int tl = 0;
         for (int t = blockIdx.x; t < ntotal; t += gridDim.x, ++tl) {
             const int mt = t % a.mtiles, nt = t / a.mtiles;
@@ -207,20 +226,69 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
                 break;
             }
             tc_fence_after();
-            const int m = mt * kGM + quarter * 32 + lane;
+            const int m0 = mt * kGM + quarter * 32;
             const uint32_t row_addr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * kGN;
+            if (a.tma_out) {
+                // each 64-column group is one head: the warp's 32 rows of it
+                // go through a swizzled staging box and one TMA store
 #pragma unroll 1
-            for (int j = 0; j < kGN / 32; ++j) {
-                uint32_t r[32];
-                tmem_ld32(row_addr + j * 32, r);
-                tmem_wait_ld();
-                const int c0 = nt * kGN + j * 32;
-                if (m < a.M && c0 < a.NC) store_chunk(a, m, c0, r);
+                for (int g = 0; g < kGN / 64; ++g) {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(row_addr + g * 64, r0);
+                    tmem_ld32(row_addr + g * 64 + 32, r1);
+                    tmem_wait_ld();
+                    const int c0 = nt * kGN + g * 64;
+                    if (m0 >= a.M || c0 >= a.NC) continue;   // warp-uniform
+                    const float b0 = a.bias ? __ldg(a.bias + c0 + lane) : 0.0f;
+                    const float b1 = a.bias ? __ldg(a.bias + c0 + 32 + lane) : 0.0f;
+                    if (n_stores >= 2 && lane == 0) bulk_wait_read1();
+                    __syncwarp();
+                    const uint32_t box = stg + (n_stores & 1) * kStgBytes;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int col = 8 * c + 2 * i;   // 0..63
+                            const float x0 = __uint_as_float(col < 32 ? r0[col] : r1[col - 32]) +
+                                             __shfl_sync(0xffffffffu, col < 32 ? b0 : b1, col & 31);
+                            const float x1 = __uint_as_float(col < 32 ? r0[col + 1] : r1[col - 31]) +
+                                             __shfl_sync(0xffffffffu, col < 32 ? b0 : b1, (col + 1) & 31);
+                            w[i] = pack2(x0, x1);
+                        }
+                        const uint32_t dst = box + lane * 128 + ((c ^ (lane & 7)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(dst), "r"(w[0]), "r"(w[1]),
+                                     "r"(w[2]), "r"(w[3])
+                                     : "memory");
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int which = c0 / a.hidden, h = (c0 - which * a.hidden) >> 6;
+                        const int b = m0 / a.N, n0 = m0 - b * a.N;
+                        tma_store_2d(&ty, box, 0, ((which * a.B + b) * a.H + h) * a.N + n0);
+                        bulk_commit();
+                    }
+                    ++n_stores;
+                }
+            } else {
+                const int m = m0 + lane;
+#pragma unroll 1
+                for (int j = 0; j < kGN / 32; ++j) {
+                    uint32_t r[32];
+                    tmem_ld32(row_addr + j * 32, r);
+                    tmem_wait_ld();
+                    const int c0 = nt * kGN + j * 32;
+                    if (m < a.M && c0 < a.NC) store_chunk(a, m, c0, r);
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(saddr(&bar_tempty[buf]));
         }
+        // the TMA stores have finished before the CTA (and its shared memory) goes
+        if (lane == 0 && n_stores > 0) bulk_wait_all();
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
@@ -230,37 +298,33 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
                      : "memory");
 }
 
-// Attention output [B][H][N][Dp] -> context [B][N][H*d] (the padding cut).
+// Attention output [B][H][N][Dp] -> context [B][N][H*d] (the padding cut),
+// for head sizes other than 32 and 64 (those are written merged by the
+// attention kernel itself).  One thread per 16-byte chunk (d % 8 == 0) or
+// per element; the host keeps B*N*hidden below 2^31, so 32-bit indices hold.
 __global__ void merge_heads_vec_kernel(const __nv_bfloat16 *__restrict__ o, __nv_bfloat16 *__restrict__ out,
                                        int B, int N, int H, int d, int Dp) {
     pdl_wait();
-    const int chunks = d >> 3;   // 16-byte chunks per head row
-    const long long total = (long long)B * N * H * chunks;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const int c = (int)(i % chunks);
-        long long r = i / chunks;
-        const int h = (int)(r % H);
-        r /= H;
-        const int n = (int)(r % N);
-        const int b = (int)(r / N);
+    const unsigned chunks = (unsigned)d >> 3, per_row = (unsigned)H * chunks;
+    const unsigned total = (unsigned)B * N * per_row;
+    for (unsigned i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+        const unsigned tok = i / per_row, within = i - tok * per_row;
+        const unsigned h = within / chunks, c = within - h * chunks;
+        const unsigned b = tok / N, n = tok - b * N;
         const uint4 v = *reinterpret_cast<const uint4 *>(o + (((size_t)b * H + h) * N + n) * Dp + c * 8);
-        *reinterpret_cast<uint4 *>(out + ((size_t)b * N + n) * H * d + h * d + c * 8) = v;
+        *reinterpret_cast<uint4 *>(out + (size_t)i * 8) = v;
     }
 }
 
 __global__ void merge_heads_kernel(const __nv_bfloat16 *__restrict__ o, __nv_bfloat16 *__restrict__ out, int B,
                                    int N, int H, int d, int Dp) {
     pdl_wait();
-    const long long total = (long long)B * N * H * d;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const int e = (int)(i % d);
-        long long r = i / d;
-        const int h = (int)(r % H);
-        r /= H;
-        const int n = (int)(r % N);
-        const int b = (int)(r / N);
+    const unsigned per_row = (unsigned)H * d;
+    const unsigned total = (unsigned)B * N * per_row;
+    for (unsigned i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+        const unsigned tok = i / per_row, within = i - tok * per_row;
+        const unsigned h = within / d, e = within - h * d;
+        const unsigned b = tok / N, n = tok - b * N;
         out[i] = o[(((size_t)b * H + h) * N + n) * Dp + e];
     }
 }
@@ -283,10 +347,14 @@ int head_padded_size(int d) { return d <= 32 ? 32 : 64; }
 cudaError_t launch_qkv_projection(const void *x, const void *w, const float *bias, void *qkv, int B, int N,
                                   int hidden, int H, unsigned int *status, cudaStream_t s) {
     const int d = hidden / H, Dp = head_padded_size(d);
-    CUtensorMap tx, tw;
+    CUtensorMap tx, tw, ty;
     const unsigned long long M = (unsigned long long)B * N, NC = 3ull * hidden;
     if (!make_map_2d(&tx, x, hidden, M, kGK, kGM) || !make_map_2d(&tw, w, hidden, NC, kGK, kGN))
         return cudaErrorInvalidValue;
+    const int tma_out = (d == 64) ? 1 : 0;
+    // [3*B*H*N][64] view of Q, K, V; 32 x 64 boxes
+    if (tma_out && !make_map_2d(&ty, qkv, 64, 3ull * B * H * N, 64, 32)) return cudaErrorInvalidValue;
+    if (!tma_out) ty = tx;   // unused
     ProjArgs a;
     a.M = (int)M;
     a.NC = (int)NC;
@@ -303,6 +371,7 @@ cudaError_t launch_qkv_projection(const void *x, const void *w, const float *bia
     a.bias = bias;
     a.qkv = static_cast<__nv_bfloat16 *>(qkv);
     a.status = status;
+    a.tma_out = tma_out;
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -312,7 +381,7 @@ cudaError_t launch_qkv_projection(const void *x, const void *w, const float *bia
     }
     const int tiles = a.mtiles * a.ntiles;
     const int grid = tiles < sm_count() ? tiles : sm_count();
-    qkv_proj_kernel<<<grid, kGThreads, kGemmSmem, s>>>(tx, tw, a);
+    qkv_proj_kernel<<<grid, kGThreads, kGemmSmem, s>>>(tx, tw, ty, a);
     return cudaGetLastError();
 }
 

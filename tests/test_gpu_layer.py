@@ -131,6 +131,7 @@ def _compare_layer(x, w, b, mask, H, *, bpr, mode, f=0, g=0, min_rows=0.5):
     (2, 256, 64, 4, 1, [70, 0]),
     (1, 512, 768, 12, 0, None),      # d = 64
     (1, 192, 200, 5, 1, [33]),       # d = 40
+    (2, 320, 128, 4, 0, [0, 20]),    # d = 32
 ])
 def test_layer_saturated_budget(B, N, hidden, H, mode, pad):
     x, w, b, mask = _layer_inputs(B, N, hidden, seed=31 + N, pad=pad)
