@@ -5,7 +5,9 @@
 One step = one whole forward pass (pool, low-resolution logits and keys,
 top-k selection, CSR build, [low-resolution PV], block-sparse attention and
 combine) over one batch of the seeded synthetic workload, inputs resident in
-HBM.  L2 is flushed (a 256 MiB write) before every timed step; each step is
+HBM.  L2 is flushed before every timed step (a 256 MiB write, then a 256 MiB
+read, so that the step starts with its inputs out of L2 and no dirty lines
+left to write back); each step is
 timed with CUDA events on the launching stream.  Under torchrun every rank
 runs its own copy of the workload (independent (batch, head) shards: weak
 scaling, no data-path collective); the reported time is the max over ranks.
@@ -35,6 +37,21 @@ from resolution_block_sparse_b200.workloads import WORKLOADS, make_inputs  # noq
 METRIC = "MRA-2 attention fwd tokens/s and TFLOP/s (selected blocks) at N=4096; % of roofline"
 L2_FLUSH_BYTES = 256 << 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+class L2Flush:
+    """Evicts everything from L2: writes a 256 MiB buffer, then reads another
+    one, so that L2 ends up holding clean lines of the second buffer (the
+    write-back of the first happens here, not in the next timed kernel)."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.acc = torch.zeros((), dtype=torch.float32, device=dev)
+
+    def zero_(self):
+        self.w.zero_()
+        torch.sum(self.r, dim=0, out=self.acc)
 
 
 def load_peaks():
@@ -141,7 +158,7 @@ def run_cuda(args, w, world, rank, local):
     q, k, v = (inputs[x].to(dev) for x in ("q", "k", "v"))
     mask = None if inputs["mask"] is None else inputs["mask"].to(dev)
     out = torch.empty_like(q)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     fwd = mra.mra_attention_fwd if w.dtype == "bf16" else mra.mra_attention_fwd_f32
 
@@ -244,7 +261,7 @@ def run_cuda_backward(args, w, world, rank, local):
     gen = torch.Generator("cpu").manual_seed(2000 + w.index + 7919 * rank)
     dout = torch.randn(q.shape, generator=gen).to(q.dtype).to(dev)
     dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3))
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(st=None):
@@ -325,7 +342,7 @@ def run_cuda_bigbird(args, bw, world, rank, local):
     lists, _ = bigbird_lists(bw, rank)
     idx = torch.from_numpy(lists).to(dev)
     out = torch.empty_like(q)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(st=None):
@@ -437,7 +454,7 @@ def run_cuda_layer(args, lw, world, rank, local):
     xh, wq, bq = layer_inputs(lw, seed=None if rank == 0 else lw.seed + 7919 * rank)
     x, w, b = xh.to(dev), wq.to(dev), bq.to(dev)
     out = torch.empty_like(x)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(st=None):
@@ -632,7 +649,7 @@ def main():
               "block_per_row": w.block_per_row, "num_block": w.num_block,
               "approx_mode": "full" if w.approx_mode == 0 else "sparse",
               "first_n": w.first_n, "diag_n": w.diag_n,
-              "l2": "flushed before every timed step (256 MiB write)",
+              "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)",
               "timing": "CUDA-graph replay of one mra_attention_fwd call per step, CUDA events",
               "parallelism": f"replicas x{world} (independent (batch, head) shards)"}
 
@@ -676,7 +693,7 @@ def main():
         lconfig = {"workload": lw.name, "B": lw.B, "N": lw.N, "hidden": lw.hidden, "H": lw.H,
                    "block_per_row": lw.block_per_row, "approx_mode": "full" if lw.approx_mode == 0 else "sparse",
                    "first_n": lw.first_n, "diag_n": lw.diag_n,
-                   "l2": "flushed before every timed step (256 MiB write)",
+                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)",
                    "timing": "CUDA-graph replay of one mra_self_attention_fwd call per step, CUDA events",
                    "parallelism": f"replicas x{world} (independent batch shards)"}
         line = {"metric": f"MraSelfAttention layer fwd tokens/s at N={lw.N}", "pass": "layer",
@@ -722,7 +739,7 @@ def main():
         bconfig = {"workload": bw.name, "B": bw.B, "H": bw.H, "N": bw.N, "D": bw.D,
                    "block_size": bw.block_size, "num_random_blocks": bw.num_random,
                    "selected_32x32_blocks": res["sel_blocks"],
-                   "l2": "flushed before every timed step (256 MiB write)",
+                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)",
                    "timing": "CUDA-graph replay of one mra_blocksparse_attention_fwd call per step, CUDA events",
                    "parallelism": f"replicas x{world} (independent (batch, head) shards)"}
         line = {"metric": f"BigBird block-sparse attention fwd tokens/s at N={bw.N}", "pass": "bigbird",
