@@ -58,9 +58,11 @@ __device__ int cta_exclusive_scan(int v, int *warp_sums, int *total) {
 // One CTA per (batch, head): clears the attention kernel's per-call counters
 // (the head's row arrival counts; CTA 0 the work counter), validates the
 // head's list (entries in [0, nbr^2), strictly increasing, -1 padding only at
-// the end), then writes the CSR column list, the work items and the head's
-// item count.  An invalid list flags MRA_DEV_COUNT and leaves the head with no
-// work items.
+// the end) while counting its entries per block row and writing the column
+// list, then builds the work items (row starts = exclusive scan of the row
+// counts, which is where each row's run begins in the sorted list) and the
+// head's item count.  An invalid list flags MRA_DEV_COUNT and leaves the head
+// with no work items.
 __global__ void __launch_bounds__(kListThreads)
 blocklist_items_kernel(const int32_t *__restrict__ lists, int cap_sel, int nbr, int k, int cap, int chunk,
                        int *__restrict__ cols, WorkItem *__restrict__ items, int *__restrict__ head_items,
@@ -68,12 +70,16 @@ blocklist_items_kernel(const int32_t *__restrict__ lists, int cap_sel, int nbr, 
                        unsigned int *__restrict__ status) {
     pdl_wait();
     __shared__ int warp_sums[33];
+    __shared__ int s_cnt[kMaxN / kBlock];
     __shared__ int s_len, s_bad;
     const int bh = blockIdx.x, t = threadIdx.x;
-    for (int r = t; r < nbr; r += kListThreads) row_arrive[(size_t)bh * nbr + r] = 0;
-    if (bh == 0 && t < 4) work_next[t] = 0;
     const int32_t *lst = lists + (size_t)bh * cap_sel;
     const long long nbr2 = (long long)nbr * nbr;
+    for (int r = t; r < nbr; r += kListThreads) {
+        row_arrive[(size_t)bh * nbr + r] = 0;
+        s_cnt[r] = 0;
+    }
+    if (bh == 0 && t < 4) work_next[t] = 0;
     if (t == 0) {
         s_len = cap_sel;
         s_bad = 0;
@@ -85,8 +91,17 @@ blocklist_items_kernel(const int32_t *__restrict__ lists, int cap_sel, int nbr, 
     const int n = s_len;
     for (int i = t; i < cap_sel; i += kListThreads) {
         const int32_t x = lst[i];
-        const bool ok = (i < n) ? (x < nbr2 && (i + 1 >= n || x < lst[i + 1])) : (x < 0);
-        if (!ok) s_bad = 1;
+        if (i < n) {
+            if (x < nbr2 && (i + 1 >= n || x < lst[i + 1])) {
+                const int r = x / nbr;
+                atomicAdd(&s_cnt[r], 1);
+                cols[(size_t)bh * k + i] = x - r * nbr;
+            } else {
+                s_bad = 1;
+            }
+        } else if (x >= 0) {
+            s_bad = 1;
+        }
     }
     __syncthreads();
     if (s_bad || n > k) {
@@ -96,31 +111,20 @@ blocklist_items_kernel(const int32_t *__restrict__ lists, int cap_sel, int nbr, 
         }
         return;
     }
-    for (int i = t; i < n; i += kListThreads) cols[(size_t)bh * k + i] = lst[i] % nbr;
-    // rows: start = first entry >= r * nbr (the list is row-major sorted)
+    // rows t*kRowsPer .. : counts, their exclusive scan (row starts), items
     constexpr int kRowsPer = (kMaxN / kBlock + kListThreads - 1) / kListThreads;   // 2
-    int start[kRowsPer], cnt[kRowsPer], nit[kRowsPer];
-    int it_local = 0;
+    int cnt[kRowsPer], nit[kRowsPer];
+    int sel_local = 0, it_local = 0;
 #pragma unroll
     for (int u = 0; u < kRowsPer; ++u) {
         const int r = t * kRowsPer + u;
-        start[u] = cnt[u] = nit[u] = 0;
-        if (r >= nbr) continue;
-        auto lower = [&](long long key) {
-            int lo = 0, hi = n;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if ((long long)lst[mid] < key) lo = mid + 1;
-                else hi = mid;
-            }
-            return lo;
-        };
-        start[u] = lower((long long)r * nbr);
-        cnt[u] = lower((long long)(r + 1) * nbr) - start[u];
-        nit[u] = cnt[u] > 0 ? (cnt[u] + chunk - 1) / chunk : 1;
+        cnt[u] = r < nbr ? s_cnt[r] : 0;
+        nit[u] = r < nbr ? (cnt[u] > 0 ? (cnt[u] + chunk - 1) / chunk : 1) : 0;
+        sel_local += cnt[u];
         it_local += nit[u];
     }
-    int total;
+    int sel_total, total;
+    int sel_before = cta_exclusive_scan(sel_local, warp_sums, &sel_total);
     int it_before = cta_exclusive_scan(it_local, warp_sums, &total);
     if (total > cap) {
         if (t == 0) {
@@ -136,11 +140,12 @@ blocklist_items_kernel(const int32_t *__restrict__ lists, int cap_sel, int nbr, 
         for (int j = 0; j < nit[u]; ++j) {
             WorkItem w;
             w.row = bh * nbr + r;
-            w.col_start = bh * k + start[u] + j * chunk;
+            w.col_start = bh * k + sel_before + j * chunk;
             w.ncols = max(0, min(chunk, cnt[u] - j * chunk));
             w.chunk_info = j | (nit[u] << 16);
             items[(size_t)bh * cap + it_before + j] = w;
         }
+        sel_before += cnt[u];
         it_before += nit[u];
     }
     if (t == 0) head_items[bh] = total;

@@ -1,5 +1,6 @@
 // mra_layer.cu - the MraSelfAttention layer around the MRA-2 forward pass:
-// the Q/K/V projection as one tcgen05 GEMM whose epilogue adds the bias,
+// the Q/K/V projection as one tcgen05 GEMM (CTA pairs, cta_group::2) whose
+// epilogue adds the bias,
 // splits the heads, zero-pads a head size below the kernel's 32 or 64 and
 // writes bf16 Q, K, V in [B][H][N][Dp]; and the merge of the attention output
 // back into [B][N][H*d].
@@ -25,14 +26,21 @@ namespace {
 using namespace async;
 using namespace tc;
 
-// CTA tile 128 x 256 (rows x output columns), K step 64 (one 128-byte
-// swizzled row of bf16), four stages of 48 KB, two TMEM accumulators of 256
-// columns so that the epilogue of one tile overlaps the MMAs of the next.
-constexpr int kGM = 128, kGN = 256, kGK = 64, kGStages = 4;
-constexpr uint32_t kABytes = kGM * kGK * 2;
-constexpr uint32_t kBBytes = kGN * kGK * 2;
+// A pair of CTAs (a cluster of two) computes one 256 x 256 tile with
+// tcgen05.mma.cta_group::2: each CTA holds 128 rows of x and 128 rows of W
+// (half of the tile's output columns) per 64-deep K step, the even CTA issues
+// the MMAs for both, and each CTA's tensor memory holds its own 128 rows of
+// the 256 columns.  Per CTA and K step that is 32 KB of operands for a
+// 128 x 256 x 64 product, two thirds of what a one-CTA 128 x 256 tile reads,
+// and six 32 KB stages keep five K steps of loads in flight.  Two TMEM
+// accumulators of 256 columns let the epilogue of one tile overlap the MMAs
+// of the next.
+constexpr int kGM = 256, kGN = 256, kGK = 64, kGStages = 6;
+constexpr int kHalf = 128;                     // rows of x and of W per CTA
+constexpr uint32_t kABytes = kHalf * kGK * 2;
+constexpr uint32_t kBBytes = kHalf * kGK * 2;
 constexpr uint32_t kGStageBytes = kABytes + kBBytes;
-constexpr int kGThreads = 192;   // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr int kGThreads = 192;   // warp 0: TMA, warp 1: MMA (even CTA), warps 2-5: epilogue
 constexpr uint32_t kGTmemCols = 2 * kGN;
 // epilogue staging for the TMA stores of 64-wide heads: two 32 x 64 bf16
 // boxes (4 KB, 128-byte swizzle) per epilogue warp
@@ -40,7 +48,7 @@ constexpr uint32_t kStgBytes = 32 * 64 * 2;
 constexpr uint32_t kStgOffset = kGStages * kGStageBytes;
 constexpr size_t kGemmSmem = (size_t)kStgOffset + 4 * 2 * kStgBytes + 1024;
 // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
-// K-major, N = 256, M = 128
+// K-major, N = 256, M = 256 (the pair)
 constexpr uint32_t kIdescG =
     (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kGN >> 3) << 17) | ((uint32_t)(kGM >> 4) << 24);
 
@@ -65,6 +73,55 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;\n" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+// --- the CTA pair (cluster of two)
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank`
+__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void pair_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on an
+// mbarrier of the pair (here: the even CTA's)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                                 uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.cta_group::2 [%0], [%1, {%2, %3}], [%4];\n"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// arrives on the mbarrier at the same offset in both CTAs once the MMAs
+// issued so far have completed
+__device__ __forceinline__ void commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n"
+        ::"r"(bar), "h"((unsigned short)3)
+        : "memory");
+}
+__device__ __forceinline__ void commit_pair_local(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(bar_cluster) : "memory");
+}
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -112,7 +169,7 @@ __device__ __forceinline__ void store_chunk(const ProjArgs &a, int m, int c0, co
     }
 }
 
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
 qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
                 const __grid_constant__ CUtensorMap ty, ProjArgs a) {
     extern __shared__ unsigned char smem_raw[];
@@ -123,6 +180,8 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = saddr(base);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();   // 0: issues the MMAs of the pair
+    const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
     const int ntotal = a.mtiles * a.ntiles;
 
     if (threadIdx.x == 0) {
@@ -132,29 +191,31 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(saddr(&bar_tfull[i]), 1);
-            mbar_init(saddr(&bar_tempty[i]), 4);
+            mbar_init(saddr(&bar_tempty[i]), 8);   // the epilogue warps of both CTAs
         }
         mbar_init(saddr(&bar_fin), 1);
         mbar_init_fence();
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(saddr(&s_tmem)),
+        // one warp of each CTA allocates the pair's accumulators together
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(saddr(&s_tmem)),
                      "r"(kGTmemCols)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
+    pair_sync();   // both CTAs' barriers are initialised before either signals the other
     tc_fence_after();
     const uint32_t tmem = s_tmem;
     pdl_wait();
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             bool ok = true;
             int it = 0;
-            for (int t = blockIdx.x; t < ntotal && ok; t += gridDim.x) {
+            for (int t = pair; t < ntotal && ok; t += npairs) {
                 const int mt = t % a.mtiles, nt = t / a.mtiles;
                 for (int kt = 0; kt < a.ktiles; ++kt, ++it) {
                     const int s = it % kGStages, use = it / kGStages;
@@ -163,26 +224,29 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
                         break;
                     }
                     const uint32_t sa = sbase + s * kGStageBytes;
-                    mbar_expect_tx(saddr(&bar_full[s]), kGStageBytes);
-                    tma_load_2d(sa, &tx, kt * kGK, mt * kGM, saddr(&bar_full[s]));
-                    tma_load_2d(sa + kABytes, &tw, kt * kGK, nt * kGN, saddr(&bar_full[s]));
+                    const uint32_t full0 = map_rank(saddr(&bar_full[s]), 0);
+                    if (rank == 0) mbar_expect_tx(saddr(&bar_full[s]), 2 * kGStageBytes);
+                    tma_load_2d_pair(sa, &tx, kt * kGK, mt * kGM + (int)rank * kHalf, full0);
+                    tma_load_2d_pair(sa + kABytes, &tw, kt * kGK, nt * kGN + (int)rank * kHalf, full0);
                 }
             }
             if (!ok) atomicOr(a.status, kDevTimeout);
-            // the loads issued last into each stage have landed before the CTA
-            // leaves (they have, unless a wait above gave up)
-            for (int s = 0; s < kGStages && s < it; ++s) {
-                const int last = it - 1 - ((it - 1 - s) % kGStages);
-                mbar_wait(saddr(&bar_full[s]), (last / kGStages) & 1);
-            }
+            // the even CTA's full barriers count the bytes of both CTAs: once
+            // the last phase of each stage is complete no load of the pair is
+            // still writing shared memory (the pair waits for each other below)
+            if (rank == 0)
+                for (int s = 0; s < kGStages && s < it; ++s) {
+                    const int last = it - 1 - ((it - 1 - s) % kGStages);
+                    mbar_wait(saddr(&bar_full[s]), (last / kGStages) & 1);
+                }
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (lane == 0 && rank == 0) {
             bool ok = true;
             int it = 0, tl = 0;
-            for (int t = blockIdx.x; t < ntotal && ok; t += gridDim.x, ++tl) {
+            for (int t = pair; t < ntotal && ok; t += npairs, ++tl) {
                 const int buf = tl & 1, ub = tl >> 1;
                 if (ub > 0 && !mbar_wait(saddr(&bar_tempty[buf]), (ub - 1) & 1)) {
                     ok = false;
@@ -200,25 +264,26 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
                     const uint32_t sa = sbase + s * kGStageBytes;
 #pragma unroll
                     for (int ks = 0; ks < kGK / 16; ++ks)
-                        mma_f16(acc, sdesc(sa + ks * 32, 16, 1024), sdesc(sa + kABytes + ks * 32, 16, 1024),
-                                kIdescG, (kt | ks) != 0);
-                    mma_commit(saddr(&bar_empty[s]));
+                        mma_pair(acc, sdesc(sa + ks * 32, 16, 1024), sdesc(sa + kABytes + ks * 32, 16, 1024),
+                                 kIdescG, (kt | ks) != 0);
+                    commit_pair(saddr(&bar_empty[s]));   // the stage is free in both CTAs
                 }
-                if (ok) mma_commit(saddr(&bar_tfull[buf]));
+                if (ok) commit_pair(saddr(&bar_tfull[buf]));
             }
             if (!ok) atomicOr(a.status, kDevTimeout);
-            // every MMA issued by this thread has completed before TMEM is freed
-            mma_commit(saddr(&bar_fin));
+            // every MMA issued here has completed before the pair frees TMEM
+            commit_pair_local(saddr(&bar_fin));
             mbar_wait(saddr(&bar_fin), 0);
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ epilogue
+        // ------------------------------------------------------------ epilogue (both CTAs)
         const int quarter = warp & 3;   // the TMEM lanes this warp may read
         const uint32_t stg = sbase + kStgOffset + (warp - 2) * 2 * kStgBytes;
+        const uint32_t tempty_a = map_rank(saddr(&bar_tempty[0]), 0), tempty_b = map_rank(saddr(&bar_tempty[1]), 0);
         int n_stores = 0;
         int tl = 0;
-        for (int t = blockIdx.x; t < ntotal; t += gridDim.x, ++tl) {
+        for (int t = pair; t < ntotal; t += npairs, ++tl) {
             const int mt = t % a.mtiles, nt = t / a.mtiles;
             const int buf = tl & 1, ub = tl >> 1;
             if (!mbar_wait(saddr(&bar_tfull[buf]), ub & 1)) {
@@ -226,7 +291,7 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
                 break;
             }
             tc_fence_after();
-            const int m0 = mt * kGM + quarter * 32;
+            const int m0 = mt * kGM + (int)rank * kHalf + quarter * 32;
             const uint32_t row_addr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * kGN;
             if (a.tma_out) {
                 // each 64-column group is one head: the warp's 32 rows of it
@@ -284,7 +349,7 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(saddr(&bar_tempty[buf]));
+            if (lane == 0) mbar_arrive_remote(buf ? tempty_b : tempty_a);   // the even CTA's barrier
         }
         // the TMA stores have finished before the CTA (and its shared memory) goes
         if (lane == 0 && n_stores > 0) bulk_wait_all();
@@ -292,9 +357,12 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ 
     }
     tc_fence_before();
     __syncthreads();
+    // neither CTA leaves (or frees the pair's TMEM) while the other may still
+    // read its shared memory through the MMAs or signal its barriers
+    pair_sync();
     tc_fence_after();
     if (warp == 1)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kGTmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kGTmemCols)
                      : "memory");
 }
 
@@ -349,7 +417,7 @@ cudaError_t launch_qkv_projection(const void *x, const void *w, const float *bia
     const int d = hidden / H, Dp = head_padded_size(d);
     CUtensorMap tx, tw, ty;
     const unsigned long long M = (unsigned long long)B * N, NC = 3ull * hidden;
-    if (!make_map_2d(&tx, x, hidden, M, kGK, kGM) || !make_map_2d(&tw, w, hidden, NC, kGK, kGN))
+    if (!make_map_2d(&tx, x, hidden, M, kGK, kHalf) || !make_map_2d(&tw, w, hidden, NC, kGK, kHalf))
         return cudaErrorInvalidValue;
     const int tma_out = (d == 64) ? 1 : 0;
     // [3*B*H*N][64] view of Q, K, V; 32 x 64 boxes
@@ -380,8 +448,8 @@ cudaError_t launch_qkv_projection(const void *x, const void *w, const float *bia
         attr = true;
     }
     const int tiles = a.mtiles * a.ntiles;
-    const int grid = tiles < sm_count() ? tiles : sm_count();
-    qkv_proj_kernel<<<grid, kGThreads, kGemmSmem, s>>>(tx, tw, ty, a);
+    const int pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;
+    qkv_proj_kernel<<<2 * pairs, kGThreads, kGemmSmem, s>>>(tx, tw, ty, a);
     return cudaGetLastError();
 }
 
