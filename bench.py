@@ -494,6 +494,25 @@ def run_cuda_layer(args, lw, world, rank, local):
         stops[i].record(stream)
     torch.cuda.synchronize()
     ms = statistics.mean(s_.elapsed_time(e_) for s_, e_ in zip(starts, stops))
+    # the projection alone against the library GEMM on the same shape
+    # (cuBLAS through torch: x W^T + b with a row-major output), back to back
+    qkv = torch.empty((3, lw.B, lw.H, lw.N, 32 if lw.hidden // lw.H <= 32 else 64), dtype=torch.bfloat16,
+                      device=dev)
+    x2 = x.reshape(-1, lw.hidden)
+    b16 = b.to(torch.bfloat16)
+    lib_out = torch.empty(x2.shape[0], 3 * lw.hidden, dtype=torch.bfloat16, device=dev)
+    cmp_us = {}
+    for name, fn in (("mra_qkv_projection", lambda: mra.mra_qkv_projection(x, w, b, qkv, lw.H)),
+                     ("torch_addmm_cublas", lambda: torch.addmm(b16, x2, w.t(), out=lib_out))):
+        for _ in range(10):
+            fn()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(200):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        cmp_us[name] = ev0.elapsed_time(ev1) / 200 * 1e3
     xp = xh.pin_memory()
     oh = torch.empty_like(xp).pin_memory()
     e2e_ms = []
@@ -514,7 +533,8 @@ def run_cuda_layer(args, lw, world, rank, local):
     ms, e2e = max_over_ranks([ms, e2e], device=dev)
     del graph
     return {"ms": ms, "e2e_ms": e2e, "phases": phases, "status": status, "launches_per_step": launches_per_step,
-            "clocks": clocks, "h2d": x.numel() * x.element_size(), "d2h": out.numel() * out.element_size()}
+            "clocks": clocks, "h2d": x.numel() * x.element_size(), "d2h": out.numel() * out.element_size(),
+            "projection_vs_library_us": cmp_us}
 
 
 def oracle_layer_sampler(lw, target_s: float = 15.0):
@@ -707,6 +727,7 @@ def main():
                              "peak_source": f"{src} (burst)", "algorithmic_flops_per_launch": proj_flops},
                 "e2e": {"value": world * lt / (res["e2e_ms"] / 1e3), "unit": "tokens/s",
                         "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+                "projection_vs_library_us": res["projection_vs_library_us"],
                 "gpu_launches": res["launches_per_step"] * args.steps, "device_status": res["status"],
                 "clocks": res["clocks"]}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -110,10 +110,15 @@ MRA_API int mra_attention_fwd_ex(const void *q, const void *k, const void *v, co
                          float *lowres_logit, float *pooled, cudaStream_t stream);
 
 /* End-to-end convenience call on HOST buffers: copies q, k, v (and the mask)
- * from host memory to a library-owned device staging area on `stream`, runs
- * the forward pass and copies `out` back, then synchronises `stream`.  Pinned
- * host memory gives asynchronous copies; pageable memory works but is
- * slower.  Same arguments as mra_attention_fwd_ex without intermediates. */
+ * from host memory to a library-owned device staging area, runs the forward
+ * pass and copies `out` back, then synchronises.  The work is cut into about
+ * eight chunks of heads (within one batch entry each): inputs go in on a
+ * library copy stream, each chunk's forward pass runs on `stream` once its
+ * inputs have landed, and its output goes back on a second library copy
+ * stream, so transfers in both directions overlap the computation.  The
+ * copies start after the work already queued on `stream`.  Pinned host
+ * memory gives asynchronous copies; pageable memory works but is slower.
+ * Same arguments as mra_attention_fwd_ex without intermediates. */
 MRA_API int mra_attention_fwd_host(const void *q_host, const void *k_host, const void *v_host,
                            const float *key_mask_host, void *out_host, int B, int H, int N,
                            int D, int block_per_row, int approx_mode, int first_n, int diag_n,

@@ -2,6 +2,7 @@
 // workspace, and the stream-ordered launch sequence of the forward pass.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -143,6 +144,9 @@ struct DeviceCtx {
     unsigned int *status = nullptr;  // persistent status word
     void *stage = nullptr;           // host-entry staging buffers
     size_t stage_bytes = 0;
+    // host entry: copy streams (inputs in, outputs out) and per-chunk events
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    std::vector<cudaEvent_t> events;
 };
 
 std::mutex g_mutex;
@@ -584,20 +588,60 @@ int mra_attention_fwd_host(const void *q_host, const void *k_host, const void *v
         }
         ctx.stage_bytes = need;
     }
+    if (!ctx.s_in) {
+        MRA_TRY(cudaStreamCreateWithFlags(&ctx.s_in, cudaStreamNonBlocking));
+        MRA_TRY(cudaStreamCreateWithFlags(&ctx.s_out, cudaStreamNonBlocking));
+    }
+    // Chunks of heads within one batch entry (about eight in all): the
+    // inputs of chunk c + 1 cross PCIe while chunk c is computed, and chunk
+    // c's output goes back on a second copy stream while later inputs still
+    // arrive.  Every (batch, head) is independent, so a chunk is a forward
+    // pass of its own with B = 1.
+    const int hc = std::max(1, std::min(H, (B * H + 7) / 8));
+    const int per_b = (H + hc - 1) / hc;
+    const int nchunks = B * per_b;
+    while ((int)ctx.events.size() < 2 * nchunks + 1) {
+        cudaEvent_t e = nullptr;
+        MRA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+        ctx.events.push_back(e);
+    }
     char *base = static_cast<char *>(ctx.stage);
     char *qd = base, *kd = base + tensor, *vd = base + 2 * tensor, *od = base + 3 * tensor;
     float *md = key_mask_host ? reinterpret_cast<float *>(base + 4 * tensor) : nullptr;
-    const size_t tb = esz * (size_t)B * H * N * D;
-    MRA_TRY(cudaMemcpyAsync(qd, q_host, tb, cudaMemcpyHostToDevice, stream));
-    MRA_TRY(cudaMemcpyAsync(kd, k_host, tb, cudaMemcpyHostToDevice, stream));
-    MRA_TRY(cudaMemcpyAsync(vd, v_host, tb, cudaMemcpyHostToDevice, stream));
+    // the copies follow the work already queued on `stream`
+    MRA_TRY(cudaEventRecord(ctx.events[2 * nchunks], stream));
+    MRA_TRY(cudaStreamWaitEvent(ctx.s_in, ctx.events[2 * nchunks], 0));
     if (md)
-        MRA_TRY(cudaMemcpyAsync(md, key_mask_host, sizeof(float) * (size_t)B * N,
-                                cudaMemcpyHostToDevice, stream));
-    rc = forward_locked(qd, kd, vd, md, od, B, H, N, D, block_per_row, approx_mode, first_n, diag_n,
-                        dtype, nullptr, nullptr, nullptr, stream);
-    if (rc != MRA_OK) return rc;
-    MRA_TRY(cudaMemcpyAsync(out_host, od, tb, cudaMemcpyDeviceToHost, stream));
+        MRA_TRY(cudaMemcpyAsync(md, key_mask_host, sizeof(float) * (size_t)B * N, cudaMemcpyHostToDevice,
+                                ctx.s_in));
+    const size_t head_bytes = esz * (size_t)N * D;
+    for (int c = 0; c < nchunks; ++c) {
+        const int b = c / per_b, h0 = (c % per_b) * hc, nh = std::min(hc, H - h0);
+        const size_t off = ((size_t)b * H + h0) * head_bytes, bytes = (size_t)nh * head_bytes;
+        MRA_TRY(cudaMemcpyAsync(qd + off, static_cast<const char *>(q_host) + off, bytes, cudaMemcpyHostToDevice,
+                                ctx.s_in));
+        MRA_TRY(cudaMemcpyAsync(kd + off, static_cast<const char *>(k_host) + off, bytes, cudaMemcpyHostToDevice,
+                                ctx.s_in));
+        MRA_TRY(cudaMemcpyAsync(vd + off, static_cast<const char *>(v_host) + off, bytes, cudaMemcpyHostToDevice,
+                                ctx.s_in));
+        MRA_TRY(cudaEventRecord(ctx.events[2 * c], ctx.s_in));
+    }
+    int launches = 0;
+    for (int c = 0; c < nchunks; ++c) {
+        const int b = c / per_b, h0 = (c % per_b) * hc, nh = std::min(hc, H - h0);
+        const size_t off = ((size_t)b * H + h0) * head_bytes, bytes = (size_t)nh * head_bytes;
+        MRA_TRY(cudaStreamWaitEvent(stream, ctx.events[2 * c], 0));
+        rc = forward_locked(qd + off, kd + off, vd + off, md ? md + (size_t)b * N : nullptr, od + off, 1, nh, N, D,
+                            block_per_row, approx_mode, first_n, diag_n, dtype, nullptr, nullptr, nullptr, stream);
+        if (rc != MRA_OK) return rc;
+        launches += g_last_launches;
+        MRA_TRY(cudaEventRecord(ctx.events[2 * c + 1], stream));
+        MRA_TRY(cudaStreamWaitEvent(ctx.s_out, ctx.events[2 * c + 1], 0));
+        MRA_TRY(cudaMemcpyAsync(static_cast<char *>(out_host) + off, od + off, bytes, cudaMemcpyDeviceToHost,
+                                ctx.s_out));
+    }
+    g_last_launches = launches;
+    MRA_TRY(cudaStreamSynchronize(ctx.s_out));
     MRA_TRY(cudaStreamSynchronize(stream));
     return MRA_OK;
 }

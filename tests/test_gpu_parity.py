@@ -96,17 +96,35 @@ def test_plain_entry_points_match_ex():
     np.testing.assert_array_equal(a["out"], b["out"])   # deterministic, bit-identical
 
 
-def test_host_entry_matches_device_entry():
-    w = WORKLOADS[4]
+@pytest.mark.parametrize("index", [2, 4])
+def test_host_entry_matches_device_entry(index):
+    """The host entry computes in chunks of heads; every (batch, head) is
+    independent, so its output is bit-identical to the device entry's."""
+    w = WORKLOADS[index]
     inputs = make_inputs(w)
     kw = dict(block_per_row=w.block_per_row, approx_mode=w.approx_mode, first_n=w.first_n,
               diag_n=w.diag_n)
     dev = tl.run_gpu(inputs, want_intermediates=False, **kw)
     q, k, v = (inputs[x].pin_memory() for x in ("q", "k", "v"))
+    m = None if inputs["mask"] is None else inputs["mask"].pin_memory()
     out = torch.empty_like(q).pin_memory()
-    mra.mra_attention_fwd_host(q, k, v, None, out, w.block_per_row, w.approx_mode, w.first_n,
-                               w.diag_n)
+    mra.mra_attention_fwd_host(q, k, v, m, out, w.block_per_row, w.approx_mode, w.first_n, w.diag_n)
     np.testing.assert_array_equal(out.float().numpy(), dev["out"])
+
+
+@pytest.mark.parametrize("B,H,dtype", [(3, 5, torch.bfloat16), (1, 5, torch.float32), (1, 1, torch.bfloat16)])
+def test_host_entry_ragged_chunks(B, H, dtype):
+    """Head counts that do not divide into equal chunks (3 x 5 heads: chunks
+    of 2, 2, 1 per batch entry; 1 x 5: five chunks of 1)."""
+    N, D = 640, 64
+    inputs = random_inputs(B, H, N, D, dtype=dtype, seed=B * 10 + H, pad_tokens=[37] * B)
+    kw = dict(block_per_row=3, approx_mode=0, first_n=1, diag_n=1)
+    dev = tl.run_gpu(inputs, want_intermediates=False, **kw)
+    q, k, v = (inputs[x].pin_memory() for x in ("q", "k", "v"))
+    out = torch.empty_like(q).pin_memory()
+    mra.mra_attention_fwd_host(q, k, v, inputs["mask"].pin_memory(), out, 3, 0, 1, 1)
+    np.testing.assert_array_equal(out.float().numpy(), dev["out"])
+    tl.compare(inputs, dev, tl.run_oracle(inputs, **kw), check_intermediates=False)
 
 
 def test_workspace_regrows_across_sizes():
