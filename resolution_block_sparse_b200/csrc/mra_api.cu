@@ -46,6 +46,7 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
     Problem p;
     p.bwd = 0;
     p.layer = 0;
+    p.fused = -1;
     p.B = B;
     p.H = H;
     p.N = N;
@@ -255,6 +256,19 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
                     int *launch_count, const GradStats *gs, const OutLayout *ol) {
     const bool prof = profile && g_prof;
     int launches = 0;
+    // small maps: the whole pass of a head in one CTA, one launch, where that
+    // is faster (MRA_FUSED=1 takes it wherever it fits, MRA_FUSED=0 never)
+    const char *fused_env = getenv("MRA_FUSED");
+    const bool fused = fused_env && fused_env[0] == '0'   ? false
+                       : fused_env && fused_env[0] == '1' ? true
+                       : p.fused >= 0                     ? p.fused == 1
+                                                          : fused_small_preferred(p);
+    if (!gs && fused && fused_small_supported(p)) {
+        PhaseScope ps("fused", s, prof);
+        MRA_TRY(launch_fused_small(p, w, q, k, v, mask, out, sel_out, logit_out, pooled_out, ol, s));
+        *launch_count = 1;
+        return MRA_OK;
+    }
     {
         // the pool kernel also clears the per-call counters and histograms
         PhaseScope ps("pool", s, prof);
@@ -313,7 +327,7 @@ namespace {
 int forward_locked(const void *q, const void *k, const void *v, const float *mask, void *out,
                    int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n,
                    int dtype, int32_t *sel_out, float *logit_out, float *pooled_out,
-                   cudaStream_t s) {
+                   cudaStream_t s, int fused = -1) {
     int rc = validate(q, k, v, out, B, H, N, D, bpr, mode, first_n, diag_n);
     if (rc != MRA_OK) return rc;
     if (dtype != MRA_DTYPE_BF16 && dtype != MRA_DTYPE_F32) return MRA_ERR_INVALID_ARG;
@@ -321,7 +335,8 @@ int forward_locked(const void *q, const void *k, const void *v, const float *mas
     int dev;
     rc = current_device(&dev);
     if (rc != MRA_OK) return rc;
-    const Problem p = make_problem(B, H, N, D, bpr, mode, first_n, diag_n, dtype);
+    Problem p = make_problem(B, H, N, D, bpr, mode, first_n, diag_n, dtype);
+    p.fused = fused;
     Workspace w;
     rc = ensure_workspace(dev, p, &w);
     if (rc != MRA_OK) return rc;
@@ -626,13 +641,18 @@ int mra_attention_fwd_host(const void *q_host, const void *k_host, const void *v
                                 ctx.s_in));
         MRA_TRY(cudaEventRecord(ctx.events[2 * c], ctx.s_in));
     }
+    // the chunks take the path the whole problem would take, so that the
+    // result is the device entry's, bit for bit
+    const int fused = fused_small_preferred(make_problem(B, H, N, D, block_per_row, approx_mode, first_n, diag_n,
+                                                         dtype)) ? 1 : 0;
     int launches = 0;
     for (int c = 0; c < nchunks; ++c) {
         const int b = c / per_b, h0 = (c % per_b) * hc, nh = std::min(hc, H - h0);
         const size_t off = ((size_t)b * H + h0) * head_bytes, bytes = (size_t)nh * head_bytes;
         MRA_TRY(cudaStreamWaitEvent(stream, ctx.events[2 * c], 0));
         rc = forward_locked(qd + off, kd + off, vd + off, md ? md + (size_t)b * N : nullptr, od + off, 1, nh, N, D,
-                            block_per_row, approx_mode, first_n, diag_n, dtype, nullptr, nullptr, nullptr, stream);
+                            block_per_row, approx_mode, first_n, diag_n, dtype, nullptr, nullptr, nullptr, stream,
+                            fused);
         if (rc != MRA_OK) return rc;
         launches += g_last_launches;
         MRA_TRY(cudaEventRecord(ctx.events[2 * c + 1], stream));

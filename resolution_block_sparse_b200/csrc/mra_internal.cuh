@@ -67,6 +67,7 @@ struct Problem {
     long long radix_chunk;  // keys per radix CTA
     int bwd;          // the workspace also holds the backward pass's buffers
     int layer;        // the workspace also holds the layer's Q/K/V and output (bf16 [B][H][N][D] each)
+    int fused;        // single-launch pass for small maps: -1 by preference, 0 never, 1 wherever it fits
 };
 
 struct Workspace {
@@ -212,6 +213,14 @@ int head_padded_size(int d);
 cudaError_t launch_qkv_projection(const void *x, const void *w, const float *bias, void *qkv, int B, int N,
                                   int hidden, int H, unsigned int *status, cudaStream_t s);
 cudaError_t launch_merge_heads(const void *o, void *out, int B, int N, int H, int d, cudaStream_t s);
+// The whole forward pass of one (batch, head) per CTA for maps of at most
+// 16 x 16 blocks whose head fits in shared memory (mra_fused.cu); writes the
+// same intermediates as the multi-kernel path when asked.
+bool fused_small_supported(const Problem &p);
+bool fused_small_preferred(const Problem &p);
+cudaError_t launch_fused_small(const Problem &p, const Workspace &w, const void *q, const void *k, const void *v,
+                               const float *mask, void *out, int32_t *sel_out, float *logit_out, float *pooled_out,
+                               const OutLayout *ol, cudaStream_t s);
 // The BigBird pattern of one head as ascending flat 32-token block indices
 // (host code); returns an mra_status value.
 int bigbird_block_list(int N, int block_size, int num_random, const int32_t *rand_blocks, int32_t *out,
