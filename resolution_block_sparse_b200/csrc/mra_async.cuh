@@ -1,5 +1,6 @@
-// mra_async.cuh - mbarrier and bulk-copy helpers (PTX) shared by the kernels
-// that stage global memory into shared memory with the copy engine.
+// mra_async.cuh - mbarrier helpers (PTX) shared by the kernels whose copies
+// or tensor-core work complete on mbarriers (the tcgen05 attention and the
+// layer's projection GEMM).
 //
 // Every wait is bounded: a waiting thread sleeps up to kSuspendHintNs per
 // try_wait and gives up after kWaitLimit tries (a few seconds), so a copy that
@@ -48,14 +49,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     for (unsigned i = 0; i < kWaitLimit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
-}
-// Contiguous global -> shared copy by the copy engine; completion is counted
-// in bytes on the mbarrier.  dst, src and bytes must be multiples of 16.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
 }
 
 }  // namespace async
