@@ -107,17 +107,17 @@ __device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t a, uint64_t b
         ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-// arrives on the mbarrier at the same offset in both CTAs once the MMAs
-// issued so far have completed
-__device__ __forceinline__ void commit_pair(uint32_t bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n"
-        ::"r"(bar), "h"((unsigned short)3)
-        : "memory");
-}
+// arrives on one mbarrier (a shared::cluster address: this CTA's or the odd
+// CTA's) once the MMAs issued so far have completed
 __device__ __forceinline__ void commit_pair_local(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
                  : "memory");
+}
+// arrives on the mbarrier at the same offset in both CTAs of the pair (two
+// commits, one per CTA)
+__device__ __forceinline__ void commit_pair(uint32_t bar) {
+    commit_pair_local(bar);
+    commit_pair_local(map_rank(bar, 1));
 }
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(bar_cluster) : "memory");
