@@ -104,3 +104,27 @@ def test_layer_rejects_bad_pointers():
                                       None) == 1
     assert lib.mra_self_attention_fwd(FAKE, FAKE, None, None, FAKE, 1, 64, 64, 2, 2, 5, 0, 0, None) == 1  # mode
     assert lib.mra_qkv_projection(FAKE, None, None, FAKE, 1, 64, 64, 2, None) == 1
+
+
+def test_bindings_check_shapes_before_calling_the_library():
+    """The Python wrappers reject tensors of the wrong dtype or shape before
+    any pointer reaches the library (CPU tensors, nothing launched)."""
+    import torch
+
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mra.mra_blocksparse_attention_fwd(q, q, q, None, q, torch.zeros(2, 4, dtype=torch.int64))
+    with pytest.raises(ValueError):
+        mra.mra_blocksparse_attention_fwd(q, q, q, None, q, torch.zeros(3, 4, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        mra.mra_blocksparse_attention_fwd(q, q, q, None, q, torch.zeros(4, 2, dtype=torch.int32).t())
+    x = torch.zeros(1, 64, 128, dtype=torch.bfloat16)
+    w = torch.zeros(3 * 128, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mra.mra_self_attention_fwd(x.float(), w, None, None, x, 2, 2, 1, 0, 0)
+    with pytest.raises(ValueError):
+        mra.mra_self_attention_fwd(x, w[:128], None, None, x, 2, 2, 1, 0, 0)
+    with pytest.raises(ValueError):
+        mra.mra_qkv_projection(x[0], w, None, x, 2)
+    with pytest.raises(ValueError):
+        mra.mra_bigbird_block_list(256, 64, np.zeros(4, dtype=np.int32))
