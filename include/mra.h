@@ -40,6 +40,13 @@
  *     the GPU and then race on the workspace: issue them on one stream.
  *   - Errors are returned synchronously, before any launch, as mra_status
  *     values; nothing aborts or prints.
+ *   - Two environment switches choose between equivalent kernels (results
+ *     agree within the stated tolerances; the defaults are the faster ones):
+ *     MRA_FUSED=1 runs maps of at most 16x16 blocks as one launch per call
+ *     wherever the head fits in shared memory, MRA_FUSED=0 never (by default
+ *     only bf16 problems with at least 64 heads take it); MRA_ATTN_IMPL=tc
+ *     (read once per process) selects the tcgen05 attention kernel for bf16,
+ *     D = 64 forward passes instead of the warp-level one.
  */
 #ifndef MRA_B200_H
 #define MRA_B200_H
