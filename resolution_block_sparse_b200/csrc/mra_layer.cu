@@ -440,13 +440,10 @@ cudaError_t launch_qkv_projection(const void *x, const void *w, const float *bia
     a.qkv = static_cast<__nv_bfloat16 *>(qkv);
     a.status = status;
     a.tma_out = tma_out;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kGemmSmem);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    // per call: the attribute belongs to the current device's context
+    cudaError_t e = cudaFuncSetAttribute(qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kGemmSmem);
+    if (e != cudaSuccess) return e;
     const int tiles = a.mtiles * a.ntiles;
     const int pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;
     qkv_proj_kernel<<<2 * pairs, kGThreads, kGemmSmem, s>>>(tx, tw, ty, a);
