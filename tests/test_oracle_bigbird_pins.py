@@ -87,3 +87,36 @@ def test_attention_on_pattern_equals_masked_dense(pad):
         if d["mask"] is not None:
             ref = ref * (d["mask"][b] > 0)[:, None]
         np.testing.assert_allclose(out[b, h], ref.numpy(), rtol=0, atol=1e-12)
+
+
+def _golden_counts():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "bigbird_keys_per_query.txt")
+    rows = []
+    for line in open(path):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            rows.append(tuple(int(x) for x in line.split()))
+    return rows
+
+
+@pytest.mark.parametrize("N,bs,r,g_keys,w_keys,r_keys,total", _golden_counts())
+def test_keys_per_query_match_the_pages_count(N, bs, r, g_keys, w_keys, r_keys, total):
+    """A middle block whose random blocks avoid its window and the global
+    blocks attends to exactly the page's global + window + random keys."""
+    nb = N // bs
+    i = nb // 2
+    rb = _rand(nb, r, 5)
+    avoid = {0, nb - 1, i - 1, i, i + 1}
+    free = [j for j in range(nb) if j not in avoid]
+    rb[i] = free[:r]                      # distinct, outside window and globals
+    flat = oracle.bigbird_blocks(N, bs, rb)
+    nbr = N // 32
+    f = bs // 32
+    row = (i * f) * nbr                   # first 32-token row of block i
+    cols = flat[(flat >= row) & (flat < row + nbr)] % nbr
+    assert g_keys + w_keys + r_keys == total
+    assert len(cols) * 32 == total
+    # and a global row attends to the whole sequence
+    cols0 = flat[flat < nbr] % nbr
+    assert len(cols0) * 32 == N
