@@ -155,3 +155,22 @@ def test_layer_workload():
     x, w, b, mask = _layer_inputs(2, 4096, 768, seed=4096, blocky=True)
     err, frac = _compare_layer(x, w, b, mask, 12, bpr=4, mode=1, f=2, g=3, min_rows=0.6)
     print(f"layer workload: max-abs {err:.3e} on {frac:.0%} of the rows")
+
+
+@pytest.mark.parametrize("B,N,hidden,H,mode,pad,launches", [
+    (2, 256, 64, 4, 0, [0, 45], 3),    # d = 16: projection, single-launch pass, head merge
+    (1, 512, 768, 12, 1, None, 2),     # d = 64: the pass writes the merged layout itself
+])
+def test_layer_on_the_single_launch_pass(B, N, hidden, H, mode, pad, launches):
+    """MRA_FUSED=1 puts the layer's attention on the single-launch pass for
+    small maps, which then writes through the layer's output strides."""
+    import os
+
+    x, w, b, mask = _layer_inputs(B, N, hidden, seed=77 + N, pad=pad)
+    os.environ["MRA_FUSED"] = "1"
+    try:
+        err, frac = _compare_layer(x, w, b, mask, H, bpr=N // 32, mode=mode)
+        assert mra.mra_last_launch_count() == launches
+    finally:
+        del os.environ["MRA_FUSED"]
+    assert frac == 1.0
