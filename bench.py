@@ -840,9 +840,11 @@ def main():
     dom_s = phases[dom]["avg_us"] * 1e-6
     esz = 2 if w.dtype == "bf16" else 4
     BH = w.B * w.H
-    kernel_src = {"attention": "mra_attn.cu", "pool": "mra_pool.cu", "lowres_keys": "mra_lowres.cu",
-                  "lowres_pv": "mra_lowres.cu", "select": "mra_select.cu",
-                  "lowres_select": "mra_lowres_select.cu"}
+    # bf16 head size 64 runs the tcgen05 kernel unless MRA_ATTN_IMPL=mma
+    tc_attn = w.dtype == "bf16" and w.D == 64 and not os.environ.get("MRA_ATTN_IMPL", "").startswith("m")
+    kernel_src = {"attention": "mra_attn_tc.cu" if tc_attn else "mra_attn.cu", "pool": "mra_pool.cu",
+                  "lowres_keys": "mra_lowres.cu", "lowres_pv": "mra_lowres.cu", "select": "mra_select.cu",
+                  "lowres_select": "mra_lowres_select.cu", "group_plan": "mra_group_plan.cu"}
     if dom == "attention":
         # compulsory Q, K, V read + O write of the attended heads; intensity
         # 16*block_per_row flop/B is below the bf16 ridge -> HBM bound

@@ -44,9 +44,11 @@
  *     agree within the stated tolerances; the defaults are the faster ones):
  *     MRA_FUSED=1 runs maps of at most 16x16 blocks as one launch per call
  *     wherever the head fits in shared memory, MRA_FUSED=0 never (by default
- *     only bf16 problems with at least 64 heads take it); MRA_ATTN_IMPL=tc
- *     (read once per process) selects the tcgen05 attention kernel for bf16,
- *     D = 64 forward passes instead of the warp-level one.
+ *     only bf16 problems with at least 64 heads take it).  bf16 forward
+ *     passes with D = 64 run the exact attention on the tcgen05 tensor cores
+ *     (groups of four block rows over the union of their selected blocks);
+ *     MRA_ATTN_IMPL=mma (read once per process) keeps them on the warp-level
+ *     kernel that fp32, D = 32 and the backward pass use.
  */
 #ifndef MRA_B200_H
 #define MRA_B200_H
@@ -75,7 +77,8 @@ typedef enum {
     MRA_ERR_UNSUPPORTED = 2,     /* D not in {32, 64}, or N above the maximum       */
     MRA_ERR_CUDA = 3,            /* a CUDA call or launch failed                    */
     MRA_ERR_ALLOC = 4,           /* workspace allocation failed                     */
-    MRA_ERR_DEVICE_TIMEOUT = 5,  /* reserved: a bounded device wait gave up         */
+    MRA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device wait gave up (the MRA_DEV_TIMEOUT
+                                    bit of a status word, see mra_status_from_device) */
     MRA_ERR_TOO_LARGE = 6        /* the problem needs more scratch than the static
                                     array of mra_attention_fwd_noalloc holds         */
 } mra_status;
@@ -183,13 +186,21 @@ MRA_API int mra_attention_bwd_f32(const float *q, const float *k, const float *v
  *     call clears what must start at zero.  Calls whose kernels overlap on the
  *     GPU (different streams, or several host threads with different streams)
  *     race on the array and give wrong results: issue them on one stream.
- *   - Device status flags of these calls are not reported by
+ *   - Device status flags of these calls (MRA_DEV_*) are kept in a word of
+ *     the static array and reported by mra_get_noalloc_status, not by
  *     mra_get_device_status.
  * Returns mra_status values like mra_attention_fwd. */
 MRA_API int mra_attention_fwd_noalloc(const void *q, const void *k, const void *v,
                                       const float *key_mask, void *out, int B, int H, int N,
                                       int D, int block_per_row, int approx_mode, int first_n,
                                       int diag_n, cudaStream_t stream);
+
+/* Status word of the mra_attention_fwd_noalloc calls on the current device:
+ * copied to the host on `stream` after the work queued there (the call waits
+ * for it), then cleared on `stream`; allocates nothing.  Returns the bitwise
+ * OR of the MRA_DEV_* flags raised since the previous read (0 before the
+ * first no-allocation call on the device), or -MRA_ERR_CUDA. */
+MRA_API int mra_get_noalloc_status(cudaStream_t stream);
 
 /* Block-sparse attention on a given set of 32x32 blocks per (batch, head):
  * the attention of step three with the softmax over the union of the given
@@ -274,6 +285,16 @@ MRA_API const char *mra_status_string(int status);
  * the current device (a bitwise OR of MRA_DEV_* flags set by kernels since the
  * previous read), or -MRA_ERR_CUDA on a CUDA error. */
 MRA_API int mra_get_device_status(cudaStream_t stream);
+
+/* Maps a status word returned by mra_get_device_status or
+ * mra_get_noalloc_status to an mra_status: a negative word is the negated
+ * error of the read itself; MRA_DEV_TIMEOUT gives MRA_ERR_DEVICE_TIMEOUT (a
+ * kernel stopped early, its output is incomplete); MRA_DEV_COUNT gives
+ * MRA_ERR_INVALID_ARG (a selection or block list the kernels refused: those
+ * heads have no output); MRA_DEV_KEY_RANGE alone (the selection order may
+ * differ from exact additive biases, the output is still computed) and 0
+ * give MRA_OK.  Host code, no CUDA call. */
+MRA_API int mra_status_from_device(int word);
 
 /* Kernel timing for benchmarks.  When enabled, the library records CUDA events
  * on `stream` around each kernel phase of every call; mra_profile_read

@@ -25,11 +25,13 @@ from ._binding import (  # noqa: F401
     mra_bigbird_block_list,
     mra_blocksparse_attention_fwd,
     mra_get_device_status,
+    mra_get_noalloc_status,
     mra_last_launch_count,
     mra_num_block,
     mra_profile_enable,
     mra_profile_read,
     mra_qkv_projection,
     mra_self_attention_fwd,
+    mra_status_from_device,
     mra_status_string,
 )

@@ -27,7 +27,7 @@ EXPORTED = (
     "mra_num_block", "mra_status_string", "mra_get_device_status", "mra_profile_enable",
     "mra_profile_read", "mra_last_launch_count", "mra_attention_fwd_noalloc", "mra_attention_bwd",
     "mra_attention_bwd_f32", "mra_blocksparse_attention_fwd", "mra_bigbird_block_list",
-    "mra_self_attention_fwd", "mra_qkv_projection",
+    "mra_self_attention_fwd", "mra_qkv_projection", "mra_get_noalloc_status", "mra_status_from_device",
 )
 
 _lock = threading.Lock()
@@ -80,6 +80,10 @@ def load_library(path: str = LIB_PATH):
         lib.mra_status_string.argtypes = [c_int]
         lib.mra_status_string.restype = ctypes.c_char_p
         lib.mra_get_device_status.argtypes = [vp]
+        lib.mra_get_noalloc_status.argtypes = [vp]
+        lib.mra_get_noalloc_status.restype = c_int
+        lib.mra_status_from_device.argtypes = [c_int]
+        lib.mra_status_from_device.restype = c_int
         lib.mra_get_device_status.restype = c_int
         lib.mra_profile_enable.argtypes = [c_int]
         lib.mra_profile_enable.restype = None
@@ -277,6 +281,16 @@ mra_status_string = status_string
 
 def mra_get_device_status(stream=None) -> int:
     return int(load_library().mra_get_device_status(_stream(stream)))
+
+
+def mra_get_noalloc_status(stream=None) -> int:
+    """Reads and clears the status word of the no-allocation entry point."""
+    return int(load_library().mra_get_noalloc_status(_stream(stream)))
+
+
+def mra_status_from_device(word: int) -> int:
+    """mra_status for a device status word (host-side mapping)."""
+    return int(load_library().mra_status_from_device(int(word)))
 
 
 def mra_profile_enable(enable: bool) -> None:

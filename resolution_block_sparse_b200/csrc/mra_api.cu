@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -17,6 +18,17 @@ namespace mra {
 
 // ---------------------------------------------------------------- planning
 size_t align_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int device_sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
 
 int validate_sizes(int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n) {
     if (B < 1 || H < 1 || N < kBlock || (N % kBlock) != 0 || bpr < 1) return MRA_ERR_INVALID_ARG;
@@ -81,6 +93,12 @@ void set_budget(Problem &p, int k) {
     const int per_row = (p.k + p.nbr - 1) / p.nbr;
     p.chunk = per_row <= 4 ? 8 : (per_row <= 16 ? 16 : kChunk);
     p.cap = p.nbr + p.k / p.chunk;
+    // tcgen05 kernel: items of at most gchunk union key blocks per group of
+    // four block rows; sparse maps take short items so that the long prior
+    // rows split over many CTAs, dense maps long ones (fewer merges)
+    p.ngroups = (p.nbr + kGroupRows - 1) / kGroupRows;
+    p.gchunk = per_row <= 4 ? 16 : (per_row <= 16 ? 32 : 64);
+    p.gcap = p.ngroups + p.k / p.gchunk;
 }
 
 // Carves the workspace; with base == nullptr only computes the size.
@@ -98,6 +116,7 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     t.arrive = (unsigned int *)take(sizeof(unsigned int) * BH * 4);
     t.row_arrive = (int *)take(sizeof(int) * BH * nbr);
     t.work_next = (int *)take(sizeof(int) * 4);
+    t.group_arrive = (int *)take(sizeof(int) * BH * (size_t)p.ngroups);
     t.zero_bytes_no_hist = off;
     t.hist = (unsigned int *)take(sizeof(unsigned int) * BH * 3 * kHistBins);
     t.zero_base = t.arrive;
@@ -118,7 +137,11 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     t.head_items = (int *)take(sizeof(int) * BH);
     t.olo = (float *)take(sizeof(float) * BH * nbr * D);
     t.llo = (float *)take(sizeof(float) * BH * nbr);
-    t.partial = (float *)take(sizeof(float) * BH * (size_t)p.cap * 32 * (D + 2));
+    t.partial = (float *)take(sizeof(float) * BH * (D + 2) *
+                              std::max((size_t)p.cap * 32, (size_t)p.gcap * 32 * kGroupRows));
+    t.ucols = (int *)take(sizeof(int) * BH * (size_t)p.k);
+    t.gitems = (GroupItem *)take(sizeof(GroupItem) * BH * (size_t)p.gcap);
+    t.head_gitems = (int *)take(sizeof(int) * BH);
     if (p.bwd) {
         t.lse2 = (float *)take(sizeof(float) * BH * (size_t)p.N);
         t.delta = (float *)take(sizeof(float) * BH * (size_t)p.N);
@@ -303,6 +326,11 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
         MRA_TRY(launch_lowres_pv(p, w, s));
         ++launches;
     }
+    if (attention_uses_tc(p, gs)) {
+        PhaseScope ps("group_plan", s, prof);
+        MRA_TRY(launch_group_plan(p, w, mask, true, s));
+        ++launches;
+    }
     {
         PhaseScope ps("attention", s, prof);
         MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s, gs, ol));
@@ -421,11 +449,16 @@ int blocksparse_locked(const void *q, const void *k, const void *v, const float 
         PhaseScope ps("blocklist_items", s, g_prof);
         MRA_TRY(launch_blocklist_items(p, w, lists, cap_sel, s));
     }
+    const bool tc = attention_uses_tc(p, nullptr);
+    if (tc) {
+        PhaseScope ps("group_plan", s, g_prof);
+        MRA_TRY(launch_group_plan(p, w, mask, false, s));
+    }
     {
         PhaseScope ps("attention", s, g_prof);
         MRA_TRY(launch_attention(p, w, q, k, v, mask, out, s));
     }
-    g_last_launches = 2;
+    g_last_launches = tc ? 3 : 2;
     return MRA_OK;
 }
 
@@ -698,6 +731,13 @@ int mra_get_device_status(cudaStream_t stream) {
         return -MRA_ERR_CUDA;
     if (cudaMemset(ctx.status, 0, sizeof(word)) != cudaSuccess) return -MRA_ERR_CUDA;
     return (int)word;
+}
+
+int mra_status_from_device(int word) {
+    if (word < 0) return -word;
+    if (word & MRA_DEV_TIMEOUT) return MRA_ERR_DEVICE_TIMEOUT;
+    if (word & MRA_DEV_COUNT) return MRA_ERR_INVALID_ARG;
+    return MRA_OK;
 }
 
 void mra_profile_enable(int enable) {

@@ -441,6 +441,16 @@ attn_f32_kernel(const AttnArgs a) {
 
 }  // namespace
 
+// bf16 forward passes with head size 64 run on the tcgen05 kernel; fp32,
+// head size 32 and the backward pass's forward re-run (which exports per-row
+// statistics) on the warp-level kernels above.  MRA_ATTN_IMPL=mma (read once
+// per process) keeps every call on the warp-level kernels.
+bool attention_uses_tc(const Problem &p, const GradStats *gs) {
+    static const char *impl = getenv("MRA_ATTN_IMPL");
+    const bool force_mma = impl && impl[0] == 'm';
+    return !force_mma && !gs && attention_tc_supported(p);
+}
+
 cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
                              const void *v, const float *mask, void *out, cudaStream_t s,
                              const GradStats *gs, const OutLayout *ol) {
@@ -476,22 +486,9 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
     a.work_next = w.work_next;
     a.out = out;
     const long long grid = (long long)p.BH * p.cap;
-    // MRA_ATTN_IMPL=tc selects the tcgen05/TMA kernel (bf16, head size 64);
-    // the default is the warp-level kernel below, which measures faster on
-    // the sparse workloads (a few 32x32 blocks per block row)
-    static const char *impl = getenv("MRA_ATTN_IMPL");
-    const bool want_tc = impl && impl[0] == 't';
-    // the backward pass's statistics come from the kernels below
-    if (want_tc && !gs && !ol && attention_tc_supported(p)) return launch_attention_tc(p, w, q, k, v, mask, out, s);
+    if (attention_uses_tc(p, gs)) return launch_attention_tc(p, w, q, k, v, mask, out, ol, s);
     if (p.dtype == 0) {
-        static int sms = 0;
-        if (sms == 0) {
-            int dev = 0;
-            cudaGetDevice(&dev);
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-            if (sms <= 0) sms = 148;
-        }
-        const long long pgrid = std::min<long long>(grid, 10LL * sms);
+        const long long pgrid = std::min<long long>(grid, 10LL * device_sm_count());
         if (p.D == 64)
             return launch_dependent(attn_bf16_kernel<64>, dim3((unsigned)pgrid), dim3(kBf16Threads), 0, s, a,
                                     (int)grid, p.BH);

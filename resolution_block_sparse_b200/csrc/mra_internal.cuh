@@ -52,6 +52,21 @@ struct WorkItem {
     int chunk_info;  // chunk | (nchunks << 16)
 };
 
+// Work item of the tcgen05 attention kernel: a group of kGroupRows adjacent
+// block rows of one head (M = 128 query rows) and a chunk of the union of
+// their selected key blocks.
+constexpr int kGroupRows = 4;
+struct GroupItem {
+    int group;       // bh * ngroups + g (block rows kGroupRows*g ..)
+    int ustart;      // index into ucols[] of the chunk's first union entry
+    int ucount;      // union entries in this chunk (0..gchunk)
+    int chunk_info;  // chunk | (nchunks << 16)
+};
+// Union entry: key block c | (rows of the group that selected it, 4 bits) << 16
+// | (the key block is partly padded) << 20.
+constexpr int kUnionRowShift = 16;
+constexpr int kUnionPartial = 1 << 20;
+
 struct Problem {
     int B, H, N, D, nbr, BH;
     long long nbr2;
@@ -68,6 +83,9 @@ struct Problem {
     int bwd;          // the workspace also holds the backward pass's buffers
     int layer;        // the workspace also holds the layer's Q/K/V and output (bf16 [B][H][N][D] each)
     int fused;        // single-launch pass for small maps: -1 by preference, 0 never, 1 wherever it fits
+    int ngroups;      // groups of kGroupRows block rows per head
+    int gchunk;       // union key blocks per tcgen05 work item (16, 32 or 64)
+    int gcap;         // tcgen05 work-item slots per head: ngroups + k / gchunk
 };
 
 struct Workspace {
@@ -75,7 +93,9 @@ struct Workspace {
     unsigned int *hist;      // [BH][3][kHistBins]
     unsigned int *arrive;    // [BH][4]
     int *row_arrive;         // [BH*nbr]
-    int *work_next;          // [4]: attention work-item counter
+    int *work_next;          // [4]: [0] attention work-item counter, [1] the tcgen05
+                             // kernel's counter, [2] most tcgen05 items of any head
+    int *group_arrive;       // [BH*ngroups]: split-group arrivals (tcgen05 kernel)
     size_t zero_bytes;       // the whole region
     size_t zero_bytes_no_hist;   // the region without the radix histograms
     void *zero_base;
@@ -95,7 +115,10 @@ struct Workspace {
     int *head_items;         // [BH]
     float *olo;              // [BH*nbr][D]
     float *llo;              // [BH*nbr]
-    float *partial;          // [BH*cap][32*(D+2)]
+    float *partial;          // [BH*cap][32*(D+2)], or [BH*gcap][128*(D+2)] for the tcgen05 kernel
+    int *ucols;              // [BH*k]: union entries of the groups (tcgen05 kernel)
+    GroupItem *gitems;       // [BH*gcap]
+    int *head_gitems;        // [BH]
     unsigned int *status;    // 1 word, persistent across calls
     // backward pass only (Problem::bwd)
     float *lse2, *delta;     // [BH*N]: base-2 log-sum-exp and dout . out per query
@@ -105,6 +128,9 @@ struct Workspace {
     void *lqkv;              // [3][B][H][N][D] bf16: projected, head-split Q, K, V
     void *lout;              // [B][H][N][D] bf16: attention output before the head merge
 };
+
+// Number of SMs of the current device (cached per device; thread-safe).
+int device_sm_count();
 
 // Planning and the launch sequence shared by the entry points (mra_api.cu).
 int validate_sizes(int B, int H, int N, int D, int bpr, int mode, int first_n, int diag_n);
@@ -198,10 +224,21 @@ cudaError_t launch_backward_items(const Problem &p, const Workspace &w, const vo
                                   float *dv, cudaStream_t s);
 cudaError_t launch_backward_lowres(const Problem &p, const Workspace &w, const float *mask, const void *dout,
                                    float *dq, float *dk, float *dv, cudaStream_t s);
-// tcgen05 / TMA attention (bf16, D = 64); used by launch_attention when supported.
+// tcgen05 / TMA attention (bf16, D = 64): groups of four block rows over the
+// union of their selected key blocks.  group_plan builds the unions and the
+// work items from the per-row items and column lists of the selection (or of
+// a block list); launch_attention runs the kernel when supported.
 bool attention_tc_supported(const Problem &p);
+// have_counts: the pool kernel's valid-token counts of this call are in the
+// workspace (not so for block lists).
+cudaError_t launch_group_plan(const Problem &p, const Workspace &w, const float *mask, bool have_counts,
+                              cudaStream_t s);
+// Whether launch_attention takes the tcgen05 kernel for this problem (gs: the
+// backward pass's statistics are wanted, which the warp-level kernels export).
+bool attention_uses_tc(const Problem &p, const GradStats *gs);
 cudaError_t launch_attention_tc(const Problem &p, const Workspace &w, const void *q, const void *k,
-                                const void *v, const float *mask, void *out, cudaStream_t s);
+                                const void *v, const float *mask, void *out, const OutLayout *ol,
+                                cudaStream_t s);
 // Block-sparse attention on caller-given block lists (mra_blocklist.cu): the
 // work items, column lists and per-call counters from lists [BH][cap_sel]
 // of ascending flat block indices padded with -1 (p.k == cap_sel).

@@ -397,16 +397,7 @@ __global__ void merge_heads_kernel(const __nv_bfloat16 *__restrict__ o, __nv_bfl
     }
 }
 
-int sm_count() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
-    return sms;
-}
+int sm_count() { return device_sm_count(); }
 
 }  // namespace
 

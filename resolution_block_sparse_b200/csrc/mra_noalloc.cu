@@ -77,3 +77,22 @@ extern "C" int mra_attention_fwd_noalloc(const void *q, const void *k, const voi
     return enqueue_forward(p, w, q, k, v, key_mask, out, nullptr, nullptr, nullptr, stream,
                            /*profile=*/false, &launches);
 }
+
+// The status word of the no-allocation calls on the current device: copied to
+// the host on `stream` (after the work already queued there), then cleared on
+// the same stream.  Neither step allocates.  0 when the entry point has not
+// run on this device yet.
+extern "C" int mra_get_noalloc_status(cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -MRA_ERR_CUDA;
+    unsigned char *base = g_scratch_ptr[dev];
+    if (!base) return 0;
+    unsigned int word = 0;
+    if (cudaMemcpyAsync(&word, base, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return -MRA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return -MRA_ERR_CUDA;
+    if (cudaMemsetAsync(base, 0, sizeof(word), stream) != cudaSuccess) return -MRA_ERR_CUDA;
+    return (int)word;
+}
+

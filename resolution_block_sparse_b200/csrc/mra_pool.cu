@@ -134,13 +134,7 @@ pool_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restric
 template <typename T, int D>
 cudaError_t launch_typed(const Problem &p, const Workspace &w, const void *q, const void *k,
                          const void *v, const float *mask, cudaStream_t s) {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
+    const int sms = device_sm_count();
     const int ntensors = (p.mode == 0) ? 3 : 2;
     const long long units = (long long)ntensors * p.BH * p.nbr;
     long long grid = (units + 7) / 8;   // one unit per warp, eight warps per CTA
