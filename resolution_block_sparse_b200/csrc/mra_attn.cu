@@ -441,14 +441,24 @@ attn_f32_kernel(const AttnArgs a) {
 
 }  // namespace
 
-// bf16 forward passes with head size 64 run on the tcgen05 kernel; fp32,
-// head size 32 and the backward pass's forward re-run (which exports per-row
-// statistics) on the warp-level kernels above.  MRA_ATTN_IMPL=mma (read once
-// per process) keeps every call on the warp-level kernels.
+// bf16 forward passes with head size 64 on dense maps (at least
+// kTcMinBlocksPerRow selected blocks per block row on average) run on the
+// tcgen05 kernel; sparse maps, fp32, head size 32 and the backward pass's
+// forward re-run (which exports per-row statistics) on the warp-level kernels
+// above.  On sparse maps a group's union holds few blocks per row and the
+// warp-level kernel, with ten CTAs per SM, is faster (measured: N=4096 with 4
+// blocks per row 40 against 78 us; N=16384 with 8 per row 113 against 286 us;
+// the BigBird pattern, 19 per row, 107 against 134 us; the saturated N=2048
+// map, 64 per row, 177 against 269 us on the tcgen05 kernel).
+// MRA_ATTN_IMPL=tc or =mma (read once per process) forces either kernel.
+constexpr int kTcMinBlocksPerRow = 32;
+
 bool attention_uses_tc(const Problem &p, const GradStats *gs) {
     static const char *impl = getenv("MRA_ATTN_IMPL");
-    const bool force_mma = impl && impl[0] == 'm';
-    return !force_mma && !gs && attention_tc_supported(p);
+    if (gs || !attention_tc_supported(p)) return false;
+    if (impl && impl[0] == 'm') return false;
+    if (impl && impl[0] == 't') return true;
+    return (long long)p.k >= (long long)kTcMinBlocksPerRow * p.nbr;
 }
 
 cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,

@@ -1,6 +1,8 @@
-"""Parity of the warp-level (mma.sync) attention kernel on the bf16, head size
-64 cases, where the default is the tcgen05 kernel: MRA_ATTN_IMPL=mma keeps
-every call on the warp-level kernels.
+"""Parity of both attention kernels on every bf16, head size 64 case: the
+tcgen05 kernel (groups of four block rows over the union of their selected
+blocks; the default on dense maps), forced with MRA_ATTN_IMPL=tc, and the
+warp-level mma.sync kernel (the default on sparse maps), forced with
+MRA_ATTN_IMPL=mma.
 
 The kernel choice is read once per process, so each case runs in a child
 process with the variable set; the child compares the CUDA output with the
@@ -50,12 +52,16 @@ CASES = [
     {"B": 2, "H": 3, "N": 288, "bpr": 2, "mode": 0, "f": 1, "g": 1, "seed": 5, "pad": [0, 70]},
     {"B": 1, "H": 1, "N": 8192, "bpr": 2, "mode": 0, "f": 1, "g": 0, "seed": 6},
     {"B": 2, "H": 1, "N": 256, "bpr": 2, "mode": 1, "f": 0, "g": 0, "seed": 7, "pad": [256, 0]},
+    {"B": 1, "H": 2, "N": 96, "bpr": 1, "mode": 0, "f": 0, "g": 0, "seed": 8},               # 3 rows: group past the end
+    {"B": 2, "H": 2, "N": 512, "bpr": 16, "mode": 0, "f": 0, "g": 0, "seed": 9, "pad": [0, 33]},   # saturated, padded keys
+    {"B": 1, "H": 2, "N": 800, "bpr": 3, "mode": 1, "f": 2, "g": 3, "seed": 10, "pad": [100]},
+    {"B": 1, "H": 1, "N": 8192, "bpr": 2, "mode": 1, "f": 1, "g": 0, "seed": 11, "pad": [300]},   # split groups, merge
 ]
 
 
-@pytest.mark.parametrize("impl", ["mma"])
+@pytest.mark.parametrize("impl", ["tc", "mma"])
 @pytest.mark.parametrize("case", CASES, ids=[json.dumps(c, sort_keys=True) for c in CASES])
-def test_warp_kernel_parity(case, impl):
+def test_attention_kernel_parity(case, impl):
     env = dict(os.environ, MRA_ATTN_IMPL=impl)
     r = subprocess.run([sys.executable, "-c", CHILD, ROOT, json.dumps(case)], env=env,
                        capture_output=True, text=True, timeout=600)

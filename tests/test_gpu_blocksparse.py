@@ -49,7 +49,8 @@ def _run(inputs, gpu_lists, ora_lists, *, skip_heads=()):
     idx = torch.from_numpy(_pad_lists(gpu_lists, -1)).to(dev)
     mra.mra_blocksparse_attention_fwd(qd, kd, vd, md, out, idx)
     torch.cuda.synchronize()
-    assert mra.mra_last_launch_count() == 2
+    # list kernel and attention, plus the group plan when the tcgen05 kernel runs
+    assert mra.mra_last_launch_count() in (2, 3)
     status = mra.mra_get_device_status()
     got = out.float().cpu().numpy()
     want = oracle.attend_with_selection(q.double().numpy(), k.double().numpy(), v.double().numpy(),
