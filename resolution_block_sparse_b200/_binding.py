@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libmra_b200.so")
 MRA_NOALLOC_SCRATCH_BYTES = 16 << 20
 MRA_FULL, MRA_SPARSE = 0, 1
 MRA_DTYPE_BF16, MRA_DTYPE_F32 = 0, 1
-MRA_DEV_KEY_RANGE, MRA_DEV_COUNT = 1, 2
+MRA_DEV_KEY_RANGE, MRA_DEV_COUNT, MRA_DEV_TIMEOUT = 1, 2, 4
 
 EXPORTED = (
     "mra_attention_fwd", "mra_attention_fwd_f32", "mra_attention_fwd_ex", "mra_attention_fwd_host",

@@ -236,6 +236,11 @@ int ensure_workspace(int dev, const Problem &p, Workspace *w) {
     }
     const size_t need = carve_workspace(p, nullptr, nullptr);
     if (need > ctx.ws_bytes) {
+        // MRA_TEST_FAIL_ALLOC=1 (read at every growth) makes the growth fail
+        // as an allocation failure would, before any CUDA call: the error path
+        // of every entry point can be tested without exhausting the device
+        const char *fail = getenv("MRA_TEST_FAIL_ALLOC");
+        if (fail && fail[0] == '1') return MRA_ERR_ALLOC;
         if (ctx.ws) {
             cudaDeviceSynchronize();
             cudaFree(ctx.ws);

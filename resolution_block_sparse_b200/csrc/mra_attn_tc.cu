@@ -42,6 +42,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstdlib>
 
 #include "mra_async.cuh"
 #include "mra_attn_common.cuh"
@@ -116,6 +117,7 @@ struct GArgs {
     long long ob;     // output element (b, h, n, e) at b * ob + h * oh + n * orow + e
     int oh, orow;
     unsigned int *status;
+    int expire_first_wait;   // test hook: the softmax's first wait gives up at once
 };
 
 struct Pending {   // a step whose PV is still to be issued
@@ -369,6 +371,11 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     }
                 }
                 const int sb = t & 1;
+                if (a.expire_first_wait && t == 0) {
+                    // a wait whose limit has run out (test hook, see the launcher)
+                    *abort_flag = 1;
+                    atomicOr(status, kDevTimeout);
+                }
                 waitb(&bar_sfull[sb], (t >> 1) & 1);
                 tc_fence_after();
                 float s[kStack][32];
@@ -690,6 +697,12 @@ cudaError_t launch_attention_tc(const Problem &p, const Workspace &w, const void
         a.orow = p.D;
     }
     a.status = w.status;
+    // MRA_TEST_EXPIRE_WAIT=1 (read at every launch) makes the first wait of
+    // every CTA's softmax report expiry without waiting, to test the kernel's
+    // timeout path: status bit, every role stopping, the copies and MMAs in
+    // flight drained, tensor memory freed
+    const char *expire = getenv("MRA_TEST_EXPIRE_WAIT");
+    a.expire_first_wait = (expire && expire[0] == '1') ? 1 : 0;
     const long long slots = (long long)p.BH * p.gcap;
     const int grid = (int)std::max<long long>(1, std::min<long long>(slots, 2LL * device_sm_count()));
     return launch_dependent(attn_group_kernel, dim3(grid), dim3(kThreads), kSmemAlloc, s, tq, tk, tv, a);

@@ -1,7 +1,8 @@
 """Parity of the CUDA backward pass (gradients of the forward output with the
 selection held fixed) with the fp64 oracle's backward on the same seeded
 inputs: both modes, key masks, priors, D = 32 and 64, fp32 and bf16 inputs,
-rows split across work items, and the full-mode low-resolution gradient.
+rows split across work items, and the full-mode low-resolution gradient, on
+maps of up to 512 x 512 blocks.
 
 Tolerance (max-abs error over each gradient, relative to max(1, its largest
 magnitude)): 1e-4 for fp32 inputs (all arithmetic fp32); 2e-2 for bf16
@@ -30,6 +31,11 @@ CASES = [
     (1, 1, 4096, 64, torch.bfloat16, 4, 1, 2, 3, None),        # 16-item first-n rows
     (2, 1, 256, 64, torch.bfloat16, 2, 0, 0, 0, [256, 10]),    # a fully padded sequence
     (1, 2, 512, 64, torch.float32, 16, 0, 0, 0, [17]),         # saturated budget
+    # maps above 128 x 128 blocks: the multi-kernel selection and the
+    # low-resolution gradient over long rows of unselected blocks
+    (1, 1, 8192, 64, torch.bfloat16, 4, 0, 1, 1, None),        # 256 x 256 blocks, full mode
+    (1, 1, 8192, 32, torch.float32, 2, 0, 2, 3, [300]),        # fp32, padded, 256 x 256
+    (1, 1, 16384, 64, torch.bfloat16, 8, 0, 1, 1, [500]),      # 512 x 512 blocks, full mode
 ]
 
 

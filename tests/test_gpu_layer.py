@@ -4,11 +4,14 @@ oracle's layer, and of its tcgen05 projection with an fp64 projection.
 The projection's bf16 output is compared with the fp64 projection of the same
 bf16 inputs within bf16 rounding (2^-8 relative, plus a small absolute term
 for the fp32 accumulation).  The layer's Q, K, V are bf16 on the GPU and
-fp64 in the oracle, so the two selections may differ on blocks whose oracle
-key lies within the logit perturbation of bf16 rounding of the k-th key:
-layer outputs are compared on every query row whose block row holds no such
-block (and everywhere when the budget selects every block), with the forward
-pass's bf16 tolerance of 2e-2.
+fp64 in the oracle's layer.  At a saturated budget the layer output is
+compared with the oracle's layer on every row.  At sparse budgets the
+expected value is the oracle's forward pass on the bf16-rounded heads (the
+layer's reading: the projected Q, K, V are bf16, as the kernels' inputs),
+computed here from the fp64 projection; the selections then differ only on
+blocks within fp32-accumulation noise of the k-th key, and at least 95 % of
+the rows are compared (rows with a block within 2e-3 of the k-th key are
+left out).  Tolerance: the forward pass's bf16 2e-2.
 """
 import numpy as np
 import pytest
@@ -20,7 +23,8 @@ import resolution_block_sparse_b200 as mra
 pytestmark = pytest.mark.gpu
 
 OUT_TOL = 2e-2
-KEY_MARGIN = 0.05
+KEY_MARGIN = 0.05          # fp64 projection against the GPU's bf16 heads
+KEY_MARGIN_BF16 = 2e-3     # bf16 heads on both sides: fp32 accumulation order only
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -89,7 +93,22 @@ def test_projection_parity(B, N, hidden, H, bias):
     assert np.all(err <= bound), float(np.max(err - bound))
 
 
-def _compare_layer(x, w, b, mask, H, *, bpr, mode, f=0, g=0, min_rows=0.5):
+def _bf16_heads_reference(x, w, b, mask, H, **kw):
+    """The layer on bf16 projected heads, computed here: the fp64 projection
+    of the bf16 inputs (padded heads, Q scaled by sqrt(Dp/d), as the layer
+    reads the page), rounded to bf16 through fp32 (the GPU rounds its fp32
+    accumulator once), then the oracle's forward pass per head and the head
+    merge.  Returns the merged output [B][N][hidden] and the oracle's keys."""
+    B, N, hidden = x.shape
+    d = hidden // H
+    ref, Dp = _ref_projection(x, w, b, H)
+    heads = torch.from_numpy(ref).float().to(torch.bfloat16).double().numpy()   # [3][B][H][N][Dp]
+    res = oracle.forward(heads[0], heads[1], heads[2], mask, **kw)
+    out = res["out"][..., :d].transpose(0, 2, 1, 3).reshape(B, N, hidden)
+    return out, res
+
+
+def _compare_layer(x, w, b, mask, H, *, bpr, mode, f=0, g=0, min_rows=0.5, bf16_heads=False):
     B, N, hidden = x.shape
     dev = torch.device("cuda:0")
     out = torch.full((B, N, hidden), float("nan"), dtype=torch.bfloat16, device=dev)
@@ -101,21 +120,29 @@ def _compare_layer(x, w, b, mask, H, *, bpr, mode, f=0, g=0, min_rows=0.5):
     assert np.all(np.isfinite(got))
     kw = dict(block_per_row=bpr, approx_mode=mode, first_n=f, diag_n=g)
     m = None if mask is None else mask.double().numpy()
-    want = oracle.self_attention(x.double().numpy(), w.double().numpy(), None if b is None else b.double().numpy(),
-                                 m, H, **kw)
-    # rows whose selection cannot differ: no block of the row within the margin of the k-th key
     d = hidden // H
     nbr = N // 32
-    proj = x.double().numpy() @ w.double().numpy().T + (0 if b is None else b.double().numpy())
-    heads = [proj[:, :, j * hidden:(j + 1) * hidden].reshape(B, N, H, d).transpose(0, 2, 1, 3) for j in range(2)]
-    res = oracle.forward(heads[0], heads[1], heads[0], m, **kw)
+    if bf16_heads:
+        # expected value on bf16 heads; only blocks within rounding noise of
+        # the k-th key can be selected differently
+        want, res = _bf16_heads_reference(x, w, b, m, H, **kw)
+        margin = KEY_MARGIN_BF16
+    else:
+        want = oracle.self_attention(x.double().numpy(), w.double().numpy(),
+                                     None if b is None else b.double().numpy(), m, H, **kw)
+        proj = x.double().numpy() @ w.double().numpy().T + (0 if b is None else b.double().numpy())
+        heads = [proj[:, :, j * hidden:(j + 1) * hidden].reshape(B, N, H, d).transpose(0, 2, 1, 3)
+                 for j in range(2)]
+        res = oracle.forward(heads[0], heads[1], heads[0], m, **kw)
+        margin = KEY_MARGIN
+    # rows whose selection cannot differ: no block of the row within the margin of the k-th key
     kk = res["k"]
     keep = np.ones((B, H, nbr), dtype=bool)
     if kk < nbr * nbr:
         key = res["key"].reshape(B * H, nbr, nbr)
         for bh in range(B * H):
             kth = np.sort(key[bh].ravel())[::-1][kk - 1]
-            near = np.abs(key[bh] - kth) <= KEY_MARGIN
+            near = np.abs(key[bh] - kth) <= margin
             keep[bh // H, bh % H] = ~near.any(axis=1)
     frac = float(keep.mean())
     assert frac >= min_rows, frac
@@ -139,21 +166,21 @@ def test_layer_saturated_budget(B, N, hidden, H, mode, pad):
     assert frac == 1.0
 
 
-@pytest.mark.parametrize("B,N,hidden,H,bpr,mode,f,g,pad", [
-    (1, 1024, 256, 4, 4, 1, 2, 3, None),     # the metric's pattern on a smaller layer
-    (1, 1024, 256, 4, 4, 0, 2, 3, [100]),
-    (2, 512, 128, 8, 2, 0, 1, 1, [0, 64]),   # d = 16
+@pytest.mark.parametrize("B,N,hidden,H,bpr,mode,f,g,pad,min_rows", [
+    (1, 1024, 256, 4, 4, 1, 2, 3, None, 0.95),     # the metric's pattern on a smaller layer
+    (1, 1024, 256, 4, 4, 0, 2, 3, [100], 0.95),
+    (2, 512, 128, 8, 2, 0, 1, 1, [0, 64], 0.9),    # d = 16; 16 rows per head: one near-tie row is 6 %
 ])
-def test_layer_sparse_budget(B, N, hidden, H, bpr, mode, f, g, pad):
+def test_layer_sparse_budget(B, N, hidden, H, bpr, mode, f, g, pad, min_rows):
     x, w, b, mask = _layer_inputs(B, N, hidden, seed=41 + N + hidden, pad=pad, blocky=True)
-    err, frac = _compare_layer(x, w, b, mask, H, bpr=bpr, mode=mode, f=f, g=g)
+    err, frac = _compare_layer(x, w, b, mask, H, bpr=bpr, mode=mode, f=f, g=g, min_rows=min_rows, bf16_heads=True)
     print(f"layer N={N} hidden={hidden}: max-abs {err:.3e} on {frac:.0%} of the rows")
 
 
 def test_layer_workload():
     """B=2, N=4096, hidden=768, H=12, sparse, 4 blocks per row, priors 2 and 3."""
     x, w, b, mask = _layer_inputs(2, 4096, 768, seed=4096, blocky=True)
-    err, frac = _compare_layer(x, w, b, mask, 12, bpr=4, mode=1, f=2, g=3, min_rows=0.6)
+    err, frac = _compare_layer(x, w, b, mask, 12, bpr=4, mode=1, f=2, g=3, min_rows=0.95, bf16_heads=True)
     print(f"layer workload: max-abs {err:.3e} on {frac:.0%} of the rows")
 
 
