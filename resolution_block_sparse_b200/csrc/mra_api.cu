@@ -71,8 +71,6 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
     p.diag_n = diag_n;
     p.dtype = dtype;
     set_budget(p, (int)std::min<long long>((long long)p.nbr * bpr, p.nbr2));
-    // low-res rows per CTA: at most 64 KB of logits per CTA, and enough CTAs
-    // to cover the SMs twice when the problem allows
     // low-res rows per CTA: the logits of a CTA's rows stay in shared memory
     // (at most 64 KB), so longer maps take fewer rows per CTA
     p.r_tile = p.nbr > 1024 ? 8 : (p.nbr > 512 ? 16 : 32);

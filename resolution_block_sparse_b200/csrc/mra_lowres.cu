@@ -38,9 +38,13 @@ __device__ __forceinline__ int in_band(int r, int c, int g) {
 
 constexpr int kLowresThreads = 256;
 
-// One CTA: R block rows of one (batch, head) against every block column.
-// Thread tile: 4 rows x 4 consecutive columns, fp32 FFMA; Q-hat rows and a
-// transposed K-hat column tile sit in shared memory and are read as float4.
+// One CTA: R block rows of one (batch, head) against every block column, in
+// tiles of kKeysCT columns.  Thread tile: R/8 rows x 2 consecutive columns,
+// fp32 FFMA; the Q-hat rows and a transposed K-hat column tile sit in shared
+// memory (a fixed 16 KB tile, so that short row strips leave room for several
+// CTAs per SM).
+constexpr int kKeysCT = 64;
+
 template <int D, int R>
 __global__ void __launch_bounds__(kLowresThreads)
 lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ khat,
@@ -50,9 +54,9 @@ lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ kha
                    unsigned int *__restrict__ hist, unsigned int *__restrict__ arrive,
                    SelState *__restrict__ state, unsigned int *__restrict__ status) {
     pdl_wait();
-    constexpr int RG = R / 4;                  // row groups
-    constexpr int CG = kLowresThreads / RG;    // column groups
-    constexpr int CT = 4 * CG;                 // columns per tile
+    constexpr int CT = kKeysCT;
+    constexpr int RPT = R / 8;                 // rows per thread (eight row groups)
+    static_assert(R % 8 == 0 && kLowresThreads == 256, "thread tiling: 8 row groups x 32 column pairs");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *qs = reinterpret_cast<float *>(smem_raw);                  // [R][D]
     float *kT = qs + R * D;                                            // [D][CT]
@@ -93,7 +97,7 @@ lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ kha
         }
     }
 
-    const int rg = t / CG, cg = t % CG;
+    const int rg = t >> 5, cg = t & 31;   // rows RPT*rg .., columns 2*cg, 2*cg + 1 of the tile
     for (int ct = 0; ct < nbr; ct += CT) {
         __syncthreads();
         // transposed column tile: kT[d][c] = khat[ct + c][d]
@@ -118,35 +122,31 @@ lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ kha
             }
         }
         __syncthreads();
-        float acc[4][4];
+        float acc[RPT][2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+        for (int i = 0; i < RPT; ++i) acc[i][0] = acc[i][1] = 0.0f;
 #pragma unroll 4
         for (int d = 0; d < D; d += 4) {
-            float4 qv[4];
+            float4 qv[RPT];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const float4 *>(qs + (4 * rg + i) * D + d);
+            for (int i = 0; i < RPT; ++i) qv[i] = *reinterpret_cast<const float4 *>(qs + (RPT * rg + i) * D + d);
 #pragma unroll
             for (int dd = 0; dd < 4; ++dd) {
-                const float4 kv = *reinterpret_cast<const float4 *>(kT + (d + dd) * CT + 4 * cg);
+                const float2 kv = *reinterpret_cast<const float2 *>(kT + (d + dd) * CT + 2 * cg);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < RPT; ++i) {
                     const float qd = dd == 0 ? qv[i].x : dd == 1 ? qv[i].y : dd == 2 ? qv[i].z : qv[i].w;
                     acc[i][0] = fmaf(qd, kv.x, acc[i][0]);
                     acc[i][1] = fmaf(qd, kv.y, acc[i][1]);
-                    acc[i][2] = fmaf(qd, kv.z, acc[i][2]);
-                    acc[i][3] = fmaf(qd, kv.w, acc[i][3]);
                 }
             }
         }
-        const int c0 = ct + 4 * cg;
+        const int c0 = ct + 2 * cg;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < RPT; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (c0 + j < nbr) lt[(size_t)(4 * rg + i) * nbr + c0 + j] = acc[i][j] * scale;
+            for (int j = 0; j < 2; ++j)
+                if (c0 + j < nbr) lt[(size_t)(RPT * rg + i) * nbr + c0 + j] = acc[i][j] * scale;
     }
     __syncthreads();
 
@@ -324,7 +324,7 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
 
 template <int D, int R>
 cudaError_t launch_keys_rt(const Problem &p, const Workspace &w, float *logit_out, cudaStream_t s) {
-    constexpr int CT = 4 * (kLowresThreads / (R / 4));
+    constexpr int CT = kKeysCT;
     const size_t smem = sizeof(float) * ((size_t)R * D + (size_t)D * CT + (size_t)R * p.nbr + R) +
                         sizeof(int) * (size_t)p.nbr + sizeof(unsigned int) * (1u << kHist0Bits);
     cudaError_t e = cudaFuncSetAttribute(lowres_keys_kernel<D, R>,
