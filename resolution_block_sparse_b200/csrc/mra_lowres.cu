@@ -221,13 +221,18 @@ lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ kha
 // Low-resolution part of full mode for R block rows of one (batch, head):
 //   w_rc = cnt_c * exp(l_rc - rowmax_r) for every unselected c with cnt_c > 0,
 //   olo_r = sum_c w_rc * vhat_c,   llo_r = sum_c w_rc.
+// block rows per CTA (every CTA reads the whole pooled V of its head, so
+// fewer rows per CTA cost more loads than they win in occupancy)
+template <int D>
+constexpr int pv_rows() { return 32; }
+
 template <int D>
 __global__ void __launch_bounds__(kLowresThreads)
 lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int *__restrict__ bitmap,
                  int wpr, const int *__restrict__ cnt, const float *__restrict__ vhat, int H,
                  int nbr, long long nbr2, float *__restrict__ olo, float *__restrict__ llo) {
     pdl_wait();
-    constexpr int R = 32;
+    constexpr int R = pv_rows<D>();
     constexpr int kCt = 32;
     constexpr int kVL = kCt * D / 4 / kLowresThreads;      // float4 loads of the V-hat tile
     constexpr int kWL = R * kCt / kLowresThreads;          // weights per thread and tile
@@ -252,9 +257,13 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
         lsum[i] = 0.0f;
     }
 
-    for (int ct = 0; ct < nbr; ct += kCt) {
-        // issue every global load of this tile before touching shared memory
-        float4 vv[kVL];
+    // the global loads of tile ct + kCt are issued before the products of
+    // tile ct, so that their latency overlaps the arithmetic
+    float4 vv[kVL];
+    unsigned long long kv[kWL];
+    unsigned int bw[kWL];
+    int cc[kWL];
+    auto load_tile = [&](int ct) {
 #pragma unroll
         for (int u = 0; u < kVL; ++u) {
             const int i = t + u * kLowresThreads;
@@ -262,9 +271,6 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
             vv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (ct + c < nbr) vv[u] = reinterpret_cast<const float4 *>(vh + (size_t)(ct + c) * D)[(4 * i) % D / 4];
         }
-        unsigned long long kv[kWL];
-        unsigned int bw[kWL];
-        int cc[kWL];
 #pragma unroll
         for (int u = 0; u < kWL; ++u) {
             const int e = t + u * kLowresThreads;
@@ -279,6 +285,9 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
                 kv[u] = keys[(size_t)bh * nbr2 + (size_t)gr * nbr + gc];
             }
         }
+    };
+    load_tile(0);
+    for (int ct = 0; ct < nbr; ct += kCt) {
         __syncthreads();   // previous tile fully consumed
 #pragma unroll
         for (int u = 0; u < kVL; ++u) {
@@ -297,6 +306,7 @@ lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int
             }
             ws[r][c] = wv;
         }
+        if (ct + kCt < nbr) load_tile(ct + kCt);
         __syncthreads();
 #pragma unroll 8
         for (int c = 0; c < kCt; ++c) {
@@ -356,13 +366,14 @@ cudaError_t launch_lowres_keys(const Problem &p, const Workspace &w, float *logi
 }
 
 cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t s) {
-    dim3 grid((p.nbr + 31) / 32, p.BH);
     const float *vhat = w.pooled + (size_t)2 * p.BH * p.nbr * p.D;
     if (p.D == 64)
-        return launch_dependent(lowres_pv_kernel<64>, grid, dim3(kLowresThreads), 0, s, w.keys, w.bitmap,
-                                w.words_per_row, w.cnt, vhat, p.H, p.nbr, p.nbr2, w.olo, w.llo);
-    return launch_dependent(lowres_pv_kernel<32>, grid, dim3(kLowresThreads), 0, s, w.keys, w.bitmap,
-                            w.words_per_row, w.cnt, vhat, p.H, p.nbr, p.nbr2, w.olo, w.llo);
+        return launch_dependent(lowres_pv_kernel<64>, dim3((p.nbr + pv_rows<64>() - 1) / pv_rows<64>(), p.BH),
+                                dim3(kLowresThreads), 0, s, w.keys, w.bitmap, w.words_per_row, w.cnt, vhat, p.H,
+                                p.nbr, p.nbr2, w.olo, w.llo);
+    return launch_dependent(lowres_pv_kernel<32>, dim3((p.nbr + pv_rows<32>() - 1) / pv_rows<32>(), p.BH),
+                            dim3(kLowresThreads), 0, s, w.keys, w.bitmap, w.words_per_row, w.cnt, vhat, p.H,
+                            p.nbr, p.nbr2, w.olo, w.llo);
 }
 
 }  // namespace mra
