@@ -115,6 +115,7 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     t.row_arrive = (int *)take(sizeof(int) * BH * nbr);
     t.work_next = (int *)take(sizeof(int) * 4);
     t.group_arrive = (int *)take(sizeof(int) * BH * (size_t)p.ngroups);
+    t.slot_arrive = (int *)take(sizeof(int) * BH * (size_t)p.cap);
     t.zero_bytes_no_hist = off;
     t.hist = (unsigned int *)take(sizeof(unsigned int) * BH * 3 * kHistBins);
     t.zero_base = t.arrive;

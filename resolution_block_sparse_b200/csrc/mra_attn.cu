@@ -44,6 +44,7 @@ struct AttnArgs {
     const float *mlo, *olo, *llo;
     unsigned char *partial;   // split-row partial slots
     int *row_arrive;
+    int *slot_arrive; // split rows: arrivals per group of items (at the group's first slot)
     int *work_next;   // items handed out beyond the first wave (zeroed per call)
     void *out;
     // output layout: element (b, h, n, e) at b * ob + h * oh + n * orow + e
@@ -322,7 +323,7 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
     gs.qbase = (size_t)bh * a.N + (size_t)r * 32;
     finish_item<D, kBf16Threads, __nv_bfloat16, __nv_bfloat16, SyncAll>(
         reinterpret_cast<const unsigned char *>(stage), slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
-        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, a.orow, sm, &s_last, gs);
+        a.llo, a.partial, a.row_arrive, a.slot_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, a.orow, sm, &s_last, gs);
 }
 
 // Persistent: the first wave takes items 0..gridDim.x-1, after that a CTA
@@ -436,7 +437,7 @@ attn_f32_kernel(const AttnArgs a) {
     gs.qbase = (size_t)bh * a.N + (size_t)r * 32;
     finish_item<D, kF32Threads, float, float, SyncAll>(
         reinterpret_cast<const unsigned char *>(stage), slot, chunk, nchunks, it.row, a.full, a.mlo, a.olo,
-        a.llo, a.partial, a.row_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, a.orow, sm, &s_last, gs);
+        a.llo, a.partial, a.row_arrive, a.slot_arrive, mrow ? mrow + r * 32 : nullptr, out_blk, a.orow, sm, &s_last, gs);
 }
 
 }  // namespace
@@ -493,6 +494,7 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
     a.llo = w.llo;
     a.partial = reinterpret_cast<unsigned char *>(w.partial);
     a.row_arrive = w.row_arrive;
+    a.slot_arrive = w.slot_arrive;
     a.work_next = w.work_next;
     a.out = out;
     const long long grid = (long long)p.BH * p.cap;

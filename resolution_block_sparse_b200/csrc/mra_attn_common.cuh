@@ -223,15 +223,89 @@ __device__ void merge_write(const unsigned char *src0, size_t slot_bytes, int nc
     }
 }
 
+// Partials of a split row are combined as a tree: the items of the row form
+// groups of kTreeGroup consecutive items; the last item of a group to finish
+// combines the group's partials into one (same slot format, in the group's
+// first slot), and the last group to finish merges the group partials into
+// the output.  Every hand-off is "the last to arrive continues" (arrival
+// counters, no waiting), and the critical path of a row is one item plus two
+// short merges instead of one merge over every partial.
+constexpr int kTreeGroup = 4;
+
+// Combines n <= kTreeGroup partials (slot layout of partial_slot_bytes, m in
+// log2 units, l and O relative to exp2(m)) at src0, src0 + slot_bytes, ...
+// into one partial of the same layout written over the first.  Run by the NT
+// threads that Sync synchronises; tid = 0..NT-1.
+template <int D, int NT, typename PartT, typename Sync>
+__device__ void combine_group(unsigned char *src0, size_t slot_bytes, int n, MergeSmem &sm, int tid) {
+    static_assert((8 * D) % NT == 0, "a partial's O tile must split evenly into quads per thread");
+    constexpr int F = 8 * D / NT;   // quads of the O tile per thread
+    constexpr int kRowQ = D / 4;
+    if (tid < 32) {
+        const int q = tid;
+        float mv[kTreeGroup], lv[kTreeGroup];
+#pragma unroll
+        for (int c = 0; c < kTreeGroup; ++c) {
+            const float *P = reinterpret_cast<const float *>(src0 + (size_t)c * slot_bytes);
+            mv[c] = c < n ? __ldcg(P + q) : -INFINITY;
+            lv[c] = c < n ? __ldcg(P + 32 + q) : 0.0f;
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kTreeGroup; ++c)
+            if (lv[c] > 0.0f) M = fmaxf(M, mv[c]);
+        float L = 0.0f;
+#pragma unroll
+        for (int c = 0; c < kTreeGroup; ++c) {
+            const float wgt = (lv[c] > 0.0f) ? exp2f(mv[c] - M) : 0.0f;
+            sm.w[c][q] = wgt;
+            L = fmaf(wgt, lv[c], L);
+        }
+        sm.M[q] = M;
+        sm.den[q] = L;
+    }
+    Sync::sync();
+    float4 acc[F];
+#pragma unroll
+    for (int i = 0; i < F; ++i) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int c = 0; c < kTreeGroup; ++c) {
+        if (c < n) {
+            const PartT *O = reinterpret_cast<const PartT *>(src0 + (size_t)c * slot_bytes + 64 * sizeof(float));
+#pragma unroll
+            for (int i = 0; i < F; ++i) {
+                const int f = tid + i * NT;
+                const float wgt = sm.w[c][f / kRowQ];
+                const float4 v = ld_quad<true>(O + 4 * f);
+                acc[i].x = fmaf(wgt, v.x, acc[i].x);
+                acc[i].y = fmaf(wgt, v.y, acc[i].y);
+                acc[i].z = fmaf(wgt, v.z, acc[i].z);
+                acc[i].w = fmaf(wgt, v.w, acc[i].w);
+            }
+        }
+    }
+    Sync::sync();   // every read of the group's slots is done before the first is overwritten
+    float *P0 = reinterpret_cast<float *>(src0);
+    if (tid < 32) {
+        P0[tid] = sm.M[tid];
+        P0[32 + tid] = sm.den[tid];
+    }
+    PartT *O0 = reinterpret_cast<PartT *>(src0 + 64 * sizeof(float));
+#pragma unroll
+    for (int i = 0; i < F; ++i) store4(O0 + 4 * (tid + i * NT), acc[i]);
+}
+
 // Shared epilogue: the item's (m, l, O) sit in `stage` (shared memory, slot
 // layout of partial_slot_bytes<D, PartT>).  A row that fits one item merges
 // and writes at once; otherwise the slot is copied to the partial buffer and
-// the last item of the row to arrive (counter, no waiting) merges them all.
+// the row's partials are combined as a tree (kTreeGroup above): slot_arrive
+// counts the arrivals of a group at its first slot, row_arrive the groups of
+// the row.
 template <int D, int NT, typename OutT, typename PartT, typename Sync>
 __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int nchunks, int row, int full,
                             const float *mlo, const float *olo, const float *llo,
-                            unsigned char *partial, int *row_arrive, const float *qmask, OutT *out_blk,
-                            int orow, MergeSmem &sm, int *s_last, const GradStats &gs) {
+                            unsigned char *partial, int *row_arrive, int *slot_arrive, const float *qmask,
+                            OutT *out_blk, int orow, MergeSmem &sm, int *s_last, const GradStats &gs) {
     constexpr size_t kSlot = partial_slot_bytes<D, PartT>();
     static_assert(kSlot % 16 == 0, "partial slots stay 16-byte aligned");
     const int tid = threadIdx.x;
@@ -248,13 +322,31 @@ __device__ void finish_item(const unsigned char *stage, int slot, int chunk, int
     for (int e = tid; e < (int)(kSlot / 16); e += NT) dst[e] = src[e];
     __threadfence();
     Sync::sync();
-    if (tid == 0) *s_last = (atomicAdd(&row_arrive[row], 1) == nchunks - 1);
-    Sync::sync();
-    if (!*s_last) return;
-    __threadfence();
-    merge_write<D, NT, true, OutT, PartT, Sync>(partial + (size_t)(slot - chunk) * kSlot, kSlot, nchunks, full,
-                                                m_lo2, l_lo, olo_row, qmask, out_blk, orow, sm, tid, gs);
-    if (tid == 0) row_arrive[row] = 0;
+    const int row_slot0 = slot - chunk;
+    const int first = (chunk / kTreeGroup) * kTreeGroup;
+    const int gsize = min(kTreeGroup, nchunks - first);
+    const int ngroups = (nchunks + kTreeGroup - 1) / kTreeGroup;
+    unsigned char *grp0 = partial + (size_t)(row_slot0 + first) * kSlot;
+    if (gsize > 1) {
+        if (tid == 0) *s_last = (atomicAdd(&slot_arrive[row_slot0 + first], 1) == gsize - 1);
+        Sync::sync();
+        if (!*s_last) return;
+        __threadfence();
+        combine_group<D, NT, PartT, Sync>(grp0, kSlot, gsize, sm, tid);
+        if (tid == 0) slot_arrive[row_slot0 + first] = 0;
+        __threadfence();
+        Sync::sync();
+    }
+    if (ngroups > 1) {
+        if (tid == 0) *s_last = (atomicAdd(&row_arrive[row], 1) == ngroups - 1);
+        Sync::sync();
+        if (!*s_last) return;
+        __threadfence();
+    }
+    // the group partials sit kTreeGroup slots apart from the row's first slot
+    merge_write<D, NT, true, OutT, PartT, Sync>(partial + (size_t)row_slot0 * kSlot, kTreeGroup * kSlot, ngroups,
+                                                full, m_lo2, l_lo, olo_row, qmask, out_blk, orow, sm, tid, gs);
+    if (tid == 0 && ngroups > 1) row_arrive[row] = 0;
 }
 
 }  // namespace attn

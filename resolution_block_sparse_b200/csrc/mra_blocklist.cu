@@ -56,7 +56,7 @@ __device__ int cta_exclusive_scan(int v, int *warp_sums, int *total) {
 }
 
 // One CTA per (batch, head): clears the attention kernel's per-call counters
-// (the head's row arrival counts; CTA 0 the work counter), validates the
+// (the head's row and item-group arrival counts; CTA 0 the work counter), validates the
 // head's list (entries in [0, nbr^2), strictly increasing, -1 padding only at
 // the end) while counting its entries per block row and writing the column
 // list, then builds the work items (row starts = exclusive scan of the row
@@ -66,7 +66,7 @@ __device__ int cta_exclusive_scan(int v, int *warp_sums, int *total) {
 __global__ void __launch_bounds__(kListThreads)
 blocklist_items_kernel(const int32_t *__restrict__ lists, int cap_sel, int nbr, int k, int cap, int chunk,
                        int *__restrict__ cols, WorkItem *__restrict__ items, int *__restrict__ head_items,
-                       int *__restrict__ row_arrive, int *__restrict__ work_next,
+                       int *__restrict__ row_arrive, int *__restrict__ slot_arrive, int *__restrict__ work_next,
                        unsigned int *__restrict__ status) {
     pdl_wait();
     __shared__ int warp_sums[33];
@@ -79,6 +79,7 @@ blocklist_items_kernel(const int32_t *__restrict__ lists, int cap_sel, int nbr, 
         row_arrive[(size_t)bh * nbr + r] = 0;
         s_cnt[r] = 0;
     }
+    for (int i = t; i < cap; i += kListThreads) slot_arrive[(size_t)bh * cap + i] = 0;
     if (bh == 0 && t < 4) work_next[t] = 0;
     if (t == 0) {
         s_len = cap_sel;
@@ -157,7 +158,7 @@ cudaError_t launch_blocklist_items(const Problem &p, const Workspace &w, const i
                                    cudaStream_t s) {
     return launch_dependent(blocklist_items_kernel, dim3((unsigned)p.BH), dim3(kListThreads), 0, s, lists, cap_sel,
                             p.nbr, p.k, p.cap, p.chunk, w.cols, w.items, w.head_items, w.row_arrive,
-                            w.work_next, w.status);
+                            w.slot_arrive, w.work_next, w.status);
 }
 
 // The BigBird pattern of one head as sorted flat 32-token block indices.

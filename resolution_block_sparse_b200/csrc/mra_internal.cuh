@@ -96,6 +96,7 @@ struct Workspace {
     int *work_next;          // [4]: [0] attention work-item counter, [1] the tcgen05
                              // kernel's counter, [2] most tcgen05 items of any head
     int *group_arrive;       // [BH*ngroups]: split-group arrivals (tcgen05 kernel)
+    int *slot_arrive;        // [BH*cap]: arrivals of a split row's item groups (warp-level kernels)
     size_t zero_bytes;       // the whole region
     size_t zero_bytes_no_hist;   // the region without the radix histograms
     void *zero_base;
