@@ -409,7 +409,11 @@ int backward_locked(const void *q, const void *k, const void *v, const float *ma
     rc = enqueue_forward(p, w, q, k, v, mask, dq, nullptr, nullptr, nullptr, s, true, &launches, &gs);
     if (rc != MRA_OK) return rc;
     const bool prof = g_prof;
-    {
+    if (mode == MRA_FULL) {
+        // the low-resolution pass writes every element of dq, dk and dv
+        PhaseScope ps("bwd_lowres", s, prof);
+        MRA_TRY(launch_backward_lowres(p, w, mask, dout, dq, dk, dv, s));
+    } else {
         PhaseScope ps("bwd_clear", s, prof);
         const size_t bytes = sizeof(float) * (size_t)B * H * N * D;
         MRA_TRY(cudaMemsetAsync(dq, 0, bytes, s));
@@ -420,11 +424,7 @@ int backward_locked(const void *q, const void *k, const void *v, const float *ma
         PhaseScope ps("bwd_items", s, prof);
         MRA_TRY(launch_backward_items(p, w, q, k, v, mask, dout, dq, dk, dv, s));
     }
-    if (mode == MRA_FULL) {
-        PhaseScope ps("bwd_lowres", s, prof);
-        MRA_TRY(launch_backward_lowres(p, w, mask, dout, dq, dk, dv, s));
-    }
-    g_last_launches = launches + (mode == MRA_FULL ? 5 : 1);
+    g_last_launches = launches + (mode == MRA_FULL ? 4 : 1);
     return MRA_OK;
 }
 

@@ -25,9 +25,10 @@
 // Kernels: bwd_item (one CTA per forward work item: dQ of its rows in
 // registers, dK and dV of its key blocks added with vector fp32 atomics, the
 // transposed index traversal being the atomics' addresses), and in full mode
-// lowres_bwd_prep (A, B, R per row block), lowres_bwd_rows (dqhat),
-// lowres_bwd_cols (dkhat, dvhat, a traversal of the map by key block) and
-// lowres_bwd_scatter (block means to tokens).  All arithmetic is fp32 (FFMA).
+// lowres_bwd_prep (A, B, R per row block), lowres_bwd_rows (dqhat) and
+// lowres_bwd_cols (dkhat, dvhat) on 32 x 32 tiles of (row block, key block)
+// pairs in shared memory, and lowres_bwd_scatter (block means to tokens).
+// All arithmetic is fp32 (FFMA).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -413,6 +414,11 @@ lowres_bwd_prep_kernel(const LoArgs a) {
     for (int i = 0; i < 32; ++i) acc = fmaf(w[i], ldf(g, (size_t)i * D + t), acc);
     float *out = a.ab + (size_t)rb * (D + 4);
     out[t] = acc;
+    // the block-mean gradient planes start at zero: the tile kernel adds into them
+    const size_t plane = (size_t)gridDim.x * D;
+    a.dxh[(size_t)rb * D + t] = 0.0f;
+    a.dxh[plane + (size_t)rb * D + t] = 0.0f;
+    a.dxh[2 * plane + (size_t)rb * D + t] = 0.0f;
     if (t == 0) {
         float bsum = 0.0f;
         for (int i = 0; i < 32; ++i) bsum = fmaf(w[i], a.delta[q0 + i], bsum);
@@ -422,105 +428,215 @@ lowres_bwd_prep_kernel(const LoArgs a) {
     }
 }
 
-// dl_bc and W_bc of one (row block b, key block c) pair, or 0 when the pair
-// takes no low-resolution weight (selected, empty column, or no query).
-// One warp: lane holds dims lane and lane + 32 (D = 64) or lane (D = 32).
+// The low-resolution gradient on 64 x 64 tiles of (row block b, key block c)
+// pairs, one CTA per tile.  The CTA stages Q-hat and A of its 64 row blocks
+// and K-hat and V-hat of its 64 key blocks in shared memory and forms
+//   lg_bc = qhat_b . khat_c,  va_bc = vhat_c . A_b
+//   W_bc  = cnt_c 2^(lg_bc scale log2e - R_b)  for an unselected pair with a
+//           valid column and a row block that has a query with terms, else 0
+//   dl_bc = W_bc (va_bc - B_b)
+// once, then the tile's shares of the three sums
+//   dqhat_b = scale sum_c dl_bc khat_c,  dkhat_c = scale sum_b dl_bc qhat_b,
+//   dvhat_c = sum_b W_bc A_b
+// which it adds into the block-mean gradient planes (zeroed by the prep
+// kernel) with vector atomics.  Every product is an outer product of 4 x 4
+// register tiles: thread (tx, ty) of 16 x 16 holds rows ty + 16 i and
+// columns tx + 16 j of the tile, so a warp's row loads are 16 consecutive
+// rows of a padded [64][D + 4] array (two wavefronts) and its column loads
+// broadcast.  fp32 FFMA throughout.
+constexpr int kLoT = 64;                 // blocks per tile side
+constexpr int kLoThreads = 256;
+constexpr int kLoP = kLoT + 4;           // padded row of the tile's pair arrays
+
 template <int D>
-__device__ __forceinline__ void lo_pair(const LoArgs &a, int bh, int b, int c, const float *qb,
-                                        const float *ab, int lane, float &W, float &dl) {
-    W = dl = 0.0f;
-    const int cntc = a.cnt[(size_t)(bh / a.H) * a.nbr + c];
-    const bool sel = (a.bitmap[((size_t)bh * a.nbr + b) * a.wpr + (c >> 5)] >> (c & 31)) & 1u;
-    if (cntc <= 0 || sel || ab[D + 2] == 0.0f) return;
-    const float *kc = a.khat + ((size_t)bh * a.nbr + c) * D;
-    const float *vc = a.vhat + ((size_t)bh * a.nbr + c) * D;
-    float lg = 0.0f, va = 0.0f;
-#pragma unroll
-    for (int d = lane; d < D; d += 32) {
-        lg = fmaf(qb[d], kc[d], lg);
-        va = fmaf(vc[d], ab[d], va);
+struct LoTileSmem {
+    float q[kLoT][D + 4];        // Q-hat of the tile's row blocks
+    float a[kLoT][D + 4];        // A of the row blocks
+    float k[kLoT][D + 4];        // K-hat of the key blocks
+    union {
+        float v[kLoT][D + 4];    // V-hat of the key blocks, then
+        float wt[kLoT][kLoP];    // W [c][b] once the weights are formed
+    };
+    float dl[kLoT][kLoP];        // dl [b][c]
+    float dlt[kLoT][kLoP];       // dl [c][b]
+    float rb[kLoT], rbb[kLoT], rvalid[kLoT];   // R, B and validity of the row blocks
+    float cntc[kLoT];                           // column counts (0 past nbr)
+    unsigned long long sel[kLoT];               // selected bits of each row over the tile's columns
+};
+
+// n = 64 rows of [nbr][stride] starting at row0 into dst (zeros past nbr).
+template <int D>
+__device__ __forceinline__ void lo_stage(float (*dst)[D + 4], const float *src, int row0, int nbr, size_t stride,
+                                         int t) {
+    for (int i = t; i < kLoT * D / 4; i += kLoThreads) {
+        const int r = i / (D / 4), d4 = i % (D / 4);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (row0 + r < nbr) v = *reinterpret_cast<const float4 *>(src + (size_t)(row0 + r) * stride + 4 * d4);
+        *reinterpret_cast<float4 *>(&dst[r][4 * d4]) = v;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        lg += __shfl_xor_sync(0xffffffffu, lg, o);
-        va += __shfl_xor_sync(0xffffffffu, va, o);
-    }
-    W = (float)cntc * exp2f(fmaf(lg * a.scale, kLog2eB, -ab[D + 1]));
-    dl = W * (va - ab[D]);
 }
 
-// dqhat_b = sum_c dl_bc khat_c / sqrt(D): one CTA of 4 warps per row block.
+// acc[i][*] += sum over u of x[ri][u] * y[u][d0..d0+DW), ri = ty + 16 i; x is
+// a [64][kLoP] pair array, y a [64][D + 4] operand; DW = D / 16 dims.
 template <int D>
-__global__ void __launch_bounds__(128)
-lowres_bwd_rows_kernel(const LoArgs a) {
-    pdl_wait();
-    __shared__ float qb[D], abs_[D + 4], red[4][D];
-    const int rb = blockIdx.x;
-    const int bh = rb / a.nbr, b = rb % a.nbr;
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    for (int d = t; d < D; d += 128) qb[d] = a.qhat[(size_t)rb * D + d];
-    for (int d = t; d < D + 4; d += 128) abs_[d] = a.ab[(size_t)rb * (D + 4) + d];
-    __syncthreads();
-    float acc[D / 32];
+__device__ __forceinline__ void lo_accumulate(float (&acc)[4][D / 16], const float (*x)[kLoP],
+                                              const float (*y)[D + 4], int ty, int d0) {
+    constexpr int DW = D / 16;
+#pragma unroll 2
+    for (int u = 0; u < kLoT; u += 4) {
+        float4 xr[4];
 #pragma unroll
-    for (int i = 0; i < D / 32; ++i) acc[i] = 0.0f;
-    for (int c = warp; c < a.nbr; c += 4) {
-        float W, dl;
-        lo_pair<D>(a, bh, b, c, qb, abs_, lane, W, dl);
-        if (dl != 0.0f) {
-            const float *kc = a.khat + ((size_t)bh * a.nbr + c) * D;
+        for (int i = 0; i < 4; ++i) xr[i] = *reinterpret_cast<const float4 *>(&x[ty + 16 * i][u]);
 #pragma unroll
-            for (int i = 0; i < D / 32; ++i) acc[i] = fmaf(dl * a.scale, kc[lane + 32 * i], acc[i]);
+        for (int uu = 0; uu < 4; ++uu) {
+            float yv[DW];
+            if constexpr (DW == 4) {
+                const float4 y4 = *reinterpret_cast<const float4 *>(&y[u + uu][d0]);
+                yv[0] = y4.x; yv[1] = y4.y; yv[2] = y4.z; yv[3] = y4.w;
+            } else {
+                const float2 y2 = *reinterpret_cast<const float2 *>(&y[u + uu][d0]);
+                yv[0] = y2.x; yv[1] = y2.y;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float xv = uu == 0 ? xr[i].x : (uu == 1 ? xr[i].y : (uu == 2 ? xr[i].z : xr[i].w));
+#pragma unroll
+                for (int e = 0; e < DW; ++e) acc[i][e] = fmaf(xv, yv[e], acc[i][e]);
+            }
         }
     }
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) red[warp][lane + 32 * i] = acc[i];
-    __syncthreads();
-    for (int d = t; d < D; d += 128)
-        a.dxh[(size_t)rb * D + d] = red[0][d] + red[1][d] + red[2][d] + red[3][d];
 }
 
-// dkhat_c = sum_b dl_bc qhat_b / sqrt(D) and dvhat_c = sum_b W_bc A_b: one CTA
-// of 4 warps per key block.
+// Adds scale * acc[i] to rows row0 + ty + 16 i (those below nbr) of the
+// plane [nbr][D] at dst.
 template <int D>
-__global__ void __launch_bounds__(128)
-lowres_bwd_cols_kernel(const LoArgs a, int BH) {
+__device__ __forceinline__ void lo_flush(float *dst, const float (&acc)[4][D / 16], int row0, int nbr, int ty,
+                                         int d0, float scale) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = row0 + ty + 16 * i;
+        if (r >= nbr) continue;
+        float *p = dst + (size_t)r * D + d0;
+        if constexpr (D / 16 == 4) {
+            atomic_add4(p, make_float4(acc[i][0] * scale, acc[i][1] * scale, acc[i][2] * scale, acc[i][3] * scale));
+        } else {
+            atomicAdd(reinterpret_cast<float2 *>(p), make_float2(acc[i][0] * scale, acc[i][1] * scale));
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kLoThreads, 2)
+lowres_bwd_tile_kernel(const LoArgs a, int BH) {
     pdl_wait();
-    __shared__ float rk[4][D], rv[4][D];
-    const int cb = blockIdx.x;   // bh * nbr + c
-    const int bh = cb / a.nbr, c = cb % a.nbr;
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    float ak[D / 32], av[D / 32];
+    extern __shared__ __align__(16) unsigned char lo_smem[];
+    LoTileSmem<D> &sh = *reinterpret_cast<LoTileSmem<D> *>(lo_smem);
+    const int col0 = blockIdx.x * kLoT, row0 = blockIdx.y * kLoT, bh = blockIdx.z;
+    const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
+    const size_t head = (size_t)bh * a.nbr * D;
+    lo_stage<D>(sh.q, a.qhat + head, row0, a.nbr, D, t);
+    lo_stage<D>(sh.a, a.ab + (size_t)bh * a.nbr * (D + 4), row0, a.nbr, D + 4, t);
+    lo_stage<D>(sh.k, a.khat + head, col0, a.nbr, D, t);
+    lo_stage<D>(sh.v, a.vhat + head, col0, a.nbr, D, t);
+    if (t < kLoT) {
+        const int r = row0 + t;
+        const bool ok = r < a.nbr;
+        const float *ab = a.ab + ((size_t)bh * a.nbr + (ok ? r : 0)) * (D + 4);
+        sh.rbb[t] = ok ? ab[D] : 0.0f;
+        sh.rb[t] = ok ? ab[D + 1] : 0.0f;
+        sh.rvalid[t] = ok ? ab[D + 2] : 0.0f;
+        unsigned long long bits = ~0ull;
+        if (ok) {
+            const unsigned int *row = a.bitmap + ((size_t)bh * a.nbr + r) * a.wpr;
+            const int w0 = col0 >> 5;   // col0 is a multiple of 64
+            bits = (unsigned long long)row[w0];
+            bits |= (unsigned long long)(w0 + 1 < a.wpr ? row[w0 + 1] : ~0u) << 32;
+        }
+        sh.sel[t] = bits;
+    } else if (t < 2 * kLoT) {
+        const int c = col0 + t - kLoT;
+        sh.cntc[t - kLoT] = c < a.nbr ? (float)a.cnt[(size_t)(bh / a.H) * a.nbr + c] : 0.0f;
+    }
+    __syncthreads();
+
+    // the weights: lg and va of rows ty + 16 i and columns tx + 16 j
+    float lg[4][4], va[4][4];
 #pragma unroll
-    for (int i = 0; i < D / 32; ++i) ak[i] = av[i] = 0.0f;
-    for (int b = warp; b < a.nbr; b += 4) {
-        const size_t rb = (size_t)bh * a.nbr + b;
-        const float *qb = a.qhat + rb * D;
-        const float *ab = a.ab + rb * (D + 4);
-        float W, dl;
-        lo_pair<D>(a, bh, b, c, qb, ab, lane, W, dl);
-        if (W != 0.0f) {
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int i = 0; i < D / 32; ++i) {
-                ak[i] = fmaf(dl * a.scale, qb[lane + 32 * i], ak[i]);
-                av[i] = fmaf(W, ab[lane + 32 * i], av[i]);
+        for (int j = 0; j < 4; ++j) lg[i][j] = va[i][j] = 0.0f;
+#pragma unroll 2
+    for (int d = 0; d < D; d += 4) {
+        float4 kc[4], vc[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            kc[j] = *reinterpret_cast<const float4 *>(&sh.k[tx + 16 * j][d]);
+            vc[j] = *reinterpret_cast<const float4 *>(&sh.v[tx + 16 * j][d]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 qr = *reinterpret_cast<const float4 *>(&sh.q[ty + 16 * i][d]);
+            const float4 ar = *reinterpret_cast<const float4 *>(&sh.a[ty + 16 * i][d]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                lg[i][j] = fmaf(qr.x, kc[j].x, fmaf(qr.y, kc[j].y, fmaf(qr.z, kc[j].z, fmaf(qr.w, kc[j].w, lg[i][j]))));
+                va[i][j] = fmaf(ar.x, vc[j].x, fmaf(ar.y, vc[j].y, fmaf(ar.z, vc[j].z, fmaf(ar.w, vc[j].w, va[i][j]))));
             }
         }
     }
 #pragma unroll
-    for (int i = 0; i < D / 32; ++i) {
-        rk[warp][lane + 32 * i] = ak[i];
-        rv[warp][lane + 32 * i] = av[i];
+    for (int i = 0; i < 4; ++i) {
+        const int r = ty + 16 * i;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = tx + 16 * j;
+            float W = 0.0f;
+            if (sh.rvalid[r] != 0.0f && sh.cntc[c] > 0.0f && !((sh.sel[r] >> c) & 1ull))
+                W = sh.cntc[c] * exp2f(fmaf(lg[i][j] * a.scale, kLog2eB, -sh.rb[r]));
+            const float dl = W * (va[i][j] - sh.rbb[r]);
+            sh.dl[r][c] = dl;
+            sh.dlt[c][r] = dl;
+            lg[i][j] = W;   // kept for the transposed store below
+        }
     }
+    __syncthreads();   // every thread is done reading V-hat
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sh.wt[tx + 16 * j][ty + 16 * i] = lg[i][j];
     __syncthreads();
+
+    constexpr int DW = D / 16;
+    const int d0 = DW * tx;
     const size_t plane = (size_t)BH * a.nbr * D;
-    for (int d = t; d < D; d += 128) {
-        a.dxh[plane + (size_t)cb * D + d] = rk[0][d] + rk[1][d] + rk[2][d] + rk[3][d];
-        a.dxh[2 * plane + (size_t)cb * D + d] = rv[0][d] + rv[1][d] + rv[2][d] + rv[3][d];
-    }
+    float acc[4][DW];
+    // dqhat of the row blocks: dl [b][c] times K-hat [c][d]
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < DW; ++e) acc[i][e] = 0.0f;
+    lo_accumulate<D>(acc, sh.dl, sh.k, ty, d0);
+    lo_flush<D>(a.dxh + head, acc, row0, a.nbr, ty, d0, a.scale);
+    // dkhat of the key blocks: dl [c][b] times Q-hat [b][d]
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < DW; ++e) acc[i][e] = 0.0f;
+    lo_accumulate<D>(acc, sh.dlt, sh.q, ty, d0);
+    lo_flush<D>(a.dxh + plane + head, acc, col0, a.nbr, ty, d0, a.scale);
+    // dvhat of the key blocks: W [c][b] times A [b][d]
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < DW; ++e) acc[i][e] = 0.0f;
+    lo_accumulate<D>(acc, sh.wt, sh.a, ty, d0);
+    lo_flush<D>(a.dxh + 2 * plane + head, acc, col0, a.nbr, ty, d0, 1.0f);
 }
 
-// Every valid token takes its block mean's gradient divided by the count.
+// Writes every token's low-resolution gradient: its block mean's gradient
+// divided by the count for a valid token of a non-empty block, zero for the
+// rest.  This is the first write of dq, dk and dv in a full-mode backward;
+// the per-item kernel adds the selected blocks' terms after it.
 template <int D>
 __global__ void __launch_bounds__(256)
 lowres_bwd_scatter_kernel(const float *__restrict__ dxh, const int *__restrict__ cnt,
@@ -536,23 +652,20 @@ lowres_bwd_scatter_kernel(const float *__restrict__ dxh, const int *__restrict__
         const int bh = (int)(tok / N), t = (int)(tok % N);
         const int b = t / 32;
         const int cb = cnt[(size_t)(bh / H) * nbr + b];
-        if (cb <= 0) continue;
-        if (mask && !(mask[(size_t)(bh / H) * N + t] > 0.0f)) continue;
-        const float inv = 1.0f / (float)cb;
-        const size_t src = ((size_t)bh * nbr + b) * D + d;
-        float4 x;
-        x = *reinterpret_cast<float4 *>(dq + i);
-        x.x = fmaf(dxh[src], inv, x.x); x.y = fmaf(dxh[src + 1], inv, x.y);
-        x.z = fmaf(dxh[src + 2], inv, x.z); x.w = fmaf(dxh[src + 3], inv, x.w);
-        *reinterpret_cast<float4 *>(dq + i) = x;
-        x = *reinterpret_cast<float4 *>(dk + i);
-        x.x = fmaf(dxh[plane + src], inv, x.x); x.y = fmaf(dxh[plane + src + 1], inv, x.y);
-        x.z = fmaf(dxh[plane + src + 2], inv, x.z); x.w = fmaf(dxh[plane + src + 3], inv, x.w);
-        *reinterpret_cast<float4 *>(dk + i) = x;
-        x = *reinterpret_cast<float4 *>(dv + i);
-        x.x = fmaf(dxh[2 * plane + src], inv, x.x); x.y = fmaf(dxh[2 * plane + src + 1], inv, x.y);
-        x.z = fmaf(dxh[2 * plane + src + 2], inv, x.z); x.w = fmaf(dxh[2 * plane + src + 3], inv, x.w);
-        *reinterpret_cast<float4 *>(dv + i) = x;
+        float4 xq = make_float4(0.f, 0.f, 0.f, 0.f), xk = xq, xv = xq;
+        if (cb > 0 && (!mask || mask[(size_t)(bh / H) * N + t] > 0.0f)) {
+            const float inv = 1.0f / (float)cb;
+            const size_t src = ((size_t)bh * nbr + b) * D + d;
+            const float4 hq = *reinterpret_cast<const float4 *>(dxh + src);
+            const float4 hk = *reinterpret_cast<const float4 *>(dxh + plane + src);
+            const float4 hv = *reinterpret_cast<const float4 *>(dxh + 2 * plane + src);
+            xq = make_float4(hq.x * inv, hq.y * inv, hq.z * inv, hq.w * inv);
+            xk = make_float4(hk.x * inv, hk.y * inv, hk.z * inv, hk.w * inv);
+            xv = make_float4(hv.x * inv, hv.y * inv, hv.z * inv, hv.w * inv);
+        }
+        *reinterpret_cast<float4 *>(dq + i) = xq;
+        *reinterpret_cast<float4 *>(dk + i) = xk;
+        *reinterpret_cast<float4 *>(dv + i) = xv;
     }
 }
 
@@ -607,12 +720,15 @@ cudaError_t launch_lowres_typed(const Problem &p, const Workspace &w, const floa
     const unsigned blocks = (unsigned)(p.BH * p.nbr);
     cudaError_t e = launch_dependent(lowres_bwd_prep_kernel<T, D>, dim3(blocks), dim3(D), 0, s, l);
     if (e != cudaSuccess) return e;
-    e = launch_dependent(lowres_bwd_rows_kernel<D>, dim3(blocks), dim3(128), 0, s, l);
+    const size_t lo_smem = sizeof(LoTileSmem<D>);
+    e = cudaFuncSetAttribute(lowres_bwd_tile_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lo_smem);
     if (e != cudaSuccess) return e;
-    e = launch_dependent(lowres_bwd_cols_kernel<D>, dim3(blocks), dim3(128), 0, s, l, p.BH);
+    const unsigned nt = (unsigned)((p.nbr + kLoT - 1) / kLoT);
+    e = launch_dependent(lowres_bwd_tile_kernel<D>, dim3(nt, nt, (unsigned)p.BH), dim3(kLoThreads), lo_smem, s, l,
+                         p.BH);
     if (e != cudaSuccess) return e;
     const size_t n4 = (size_t)p.BH * p.N * D / 4;
-    const unsigned grid = (unsigned)std::min<size_t>((n4 + 255) / 256, 148 * 16);
+    const unsigned grid = (unsigned)std::min<size_t>((n4 + 255) / 256, (size_t)device_sm_count() * 16);
     return launch_dependent(lowres_bwd_scatter_kernel<D>, dim3(grid), dim3(256), 0, s, w.lo_dxh, w.cnt, mask, p.H,
                             p.N, p.nbr, p.BH, dq, dk, dv);
 }
