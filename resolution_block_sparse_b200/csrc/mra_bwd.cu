@@ -389,42 +389,54 @@ struct LoArgs {
     float *dxh;                        // [3][BH][nbr][D]: dqhat, dkhat, dvhat
 };
 
-// A_b, B_b, R_b of one row block (one CTA of D threads).
+// A_b, B_b, R_b of one row block per warp (lane i holds query i of the
+// block for the weights, dims lane + 32 e for A), and the block's rows of
+// the three block-mean gradient planes set to zero.
+constexpr int kPrepWarps = 8;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(D)
-lowres_bwd_prep_kernel(const LoArgs a) {
+__global__ void __launch_bounds__(32 * kPrepWarps)
+lowres_bwd_prep_kernel(const LoArgs a, int nrb) {
     pdl_wait();
-    __shared__ float w[32];
-    __shared__ float s_r;
-    const int rb = blockIdx.x;   // bh * nbr + b
+    const int lane = threadIdx.x & 31;
+    const int rb = blockIdx.x * kPrepWarps + (threadIdx.x >> 5);   // bh * nbr + b
+    if (rb >= nrb) return;
     const int bh = rb / a.nbr, b = rb % a.nbr;
     const size_t q0 = (size_t)bh * a.N + (size_t)b * 32;
-    const int t = threadIdx.x;
-    if (t < 32) {
-        const float l = a.lse2[q0 + t];
-        float m = l;
+    const float l = a.lse2[q0 + lane];
+    const float dl = a.delta[q0 + lane];
+    float m = l;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fminf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        w[t] = (l == INFINITY) ? 0.0f : exp2f(m - l);
-        if (t == 0) s_r = m;
-    }
-    __syncthreads();
+    for (int o = 16; o > 0; o >>= 1) m = fminf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float wl = (l == INFINITY) ? 0.0f : exp2f(m - l);
+    float bsum = wl * dl;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bsum += __shfl_xor_sync(0xffffffffu, bsum, o);
+    constexpr int E = D / 32;
     const T *g = static_cast<const T *>(a.dout) + q0 * D;
-    float acc = 0.0f;
-    for (int i = 0; i < 32; ++i) acc = fmaf(w[i], ldf(g, (size_t)i * D + t), acc);
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {
+        const float wi = __shfl_sync(0xffffffffu, wl, i);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(wi, ldf(g, (size_t)i * D + lane + 32 * e), acc[e]);
+    }
     float *out = a.ab + (size_t)rb * (D + 4);
-    out[t] = acc;
-    // the block-mean gradient planes start at zero: the tile kernel adds into them
-    const size_t plane = (size_t)gridDim.x * D;
-    a.dxh[(size_t)rb * D + t] = 0.0f;
-    a.dxh[plane + (size_t)rb * D + t] = 0.0f;
-    a.dxh[2 * plane + (size_t)rb * D + t] = 0.0f;
-    if (t == 0) {
-        float bsum = 0.0f;
-        for (int i = 0; i < 32; ++i) bsum = fmaf(w[i], a.delta[q0 + i], bsum);
+    const size_t plane = (size_t)nrb * D;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int d = lane + 32 * e;
+        out[d] = acc[e];
+        a.dxh[(size_t)rb * D + d] = 0.0f;
+        a.dxh[plane + (size_t)rb * D + d] = 0.0f;
+        a.dxh[2 * plane + (size_t)rb * D + d] = 0.0f;
+    }
+    if (lane == 0) {
         out[D] = bsum;
-        out[D + 1] = s_r;
-        out[D + 2] = (s_r == INFINITY) ? 0.0f : 1.0f;   // the row block has a query with terms
+        out[D + 1] = m;
+        out[D + 2] = (m == INFINITY) ? 0.0f : 1.0f;   // the row block has a query with terms
     }
 }
 
@@ -464,15 +476,18 @@ struct LoTileSmem {
     unsigned long long sel[kLoT];               // selected bits of each row over the tile's columns
 };
 
-// n = 64 rows of [nbr][stride] starting at row0 into dst (zeros past nbr).
+// 64 rows of [nbr][stride] starting at row0 into dst by cp.async (zeros
+// past nbr); the caller commits and waits.
 template <int D>
 __device__ __forceinline__ void lo_stage(float (*dst)[D + 4], const float *src, int row0, int nbr, size_t stride,
                                          int t) {
+#pragma unroll
     for (int i = t; i < kLoT * D / 4; i += kLoThreads) {
         const int r = i / (D / 4), d4 = i % (D / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (row0 + r < nbr) v = *reinterpret_cast<const float4 *>(src + (size_t)(row0 + r) * stride + 4 * d4);
-        *reinterpret_cast<float4 *>(&dst[r][4 * d4]) = v;
+        if (row0 + r < nbr)
+            mma::cp_async16(&dst[r][4 * d4], src + (size_t)(row0 + r) * stride + 4 * d4);
+        else
+            *reinterpret_cast<float4 *>(&dst[r][4 * d4]) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 
@@ -538,6 +553,7 @@ lowres_bwd_tile_kernel(const LoArgs a, int BH) {
     lo_stage<D>(sh.a, a.ab + (size_t)bh * a.nbr * (D + 4), row0, a.nbr, D + 4, t);
     lo_stage<D>(sh.k, a.khat + head, col0, a.nbr, D, t);
     lo_stage<D>(sh.v, a.vhat + head, col0, a.nbr, D, t);
+    mma::cp_async_commit();
     if (t < kLoT) {
         const int r = row0 + t;
         const bool ok = r < a.nbr;
@@ -557,6 +573,7 @@ lowres_bwd_tile_kernel(const LoArgs a, int BH) {
         const int c = col0 + t - kLoT;
         sh.cntc[t - kLoT] = c < a.nbr ? (float)a.cnt[(size_t)(bh / a.H) * a.nbr + c] : 0.0f;
     }
+    mma::cp_async_wait<0>();
     __syncthreads();
 
     // the weights: lg and va of rows ty + 16 i and columns tx + 16 j
@@ -717,8 +734,9 @@ cudaError_t launch_lowres_typed(const Problem &p, const Workspace &w, const floa
     l.scale = 1.0f / sqrtf((float)D);
     l.ab = w.lo_ab;
     l.dxh = w.lo_dxh;
-    const unsigned blocks = (unsigned)(p.BH * p.nbr);
-    cudaError_t e = launch_dependent(lowres_bwd_prep_kernel<T, D>, dim3(blocks), dim3(D), 0, s, l);
+    const int nrb = p.BH * p.nbr;
+    cudaError_t e = launch_dependent(lowres_bwd_prep_kernel<T, D>, dim3((unsigned)((nrb + kPrepWarps - 1) / kPrepWarps)),
+                                     dim3(32 * kPrepWarps), 0, s, l, nrb);
     if (e != cudaSuccess) return e;
     const size_t lo_smem = sizeof(LoTileSmem<D>);
     e = cudaFuncSetAttribute(lowres_bwd_tile_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lo_smem);
