@@ -73,7 +73,7 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
     set_budget(p, (int)std::min<long long>((long long)p.nbr * bpr, p.nbr2));
     // low-res rows per CTA: the logits of a CTA's rows stay in shared memory
     // (at most 64 KB), so longer maps take fewer rows per CTA
-    p.r_tile = p.nbr > 1024 ? 8 : (p.nbr > 512 ? 16 : 32);
+    p.r_tile = p.nbr > 1024 ? 8 : 16;
     p.lowres_ctas = (p.nbr + p.r_tile - 1) / p.r_tile;
     long long ctas = (p.nbr2 + 4095) / 4096;
     if (ctas < 1) ctas = 1;
@@ -123,6 +123,8 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     t.cnt = (int *)take(sizeof(int) * (size_t)p.B * nbr);
     t.pooled = (float *)take(sizeof(float) * 3 * BH * nbr * D);
     t.keys = (unsigned long long *)take(sizeof(unsigned long long) * BH * (size_t)p.nbr2);
+    t.lo_logits = (float *)take(sizeof(float) * BH * (size_t)p.nbr2);
+    t.lo_pmax = (float *)take(sizeof(float) * BH * nbr * ((nbr + 63) / 64));
     t.mlo = (float *)take(sizeof(float) * BH * nbr);
     t.state = (SelState *)take(sizeof(SelState) * BH);
     t.gt = (int *)take(sizeof(int) * BH * nbr);
@@ -327,7 +329,7 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
     }
     if (p.mode == MRA_FULL) {
         PhaseScope ps("lowres_pv", s, prof);
-        MRA_TRY(launch_lowres_pv(p, w, s));
+        MRA_TRY(launch_lowres_pv(p, w, logit_out, s));
         ++launches;
     }
     if (attention_uses_tc(p, gs)) {

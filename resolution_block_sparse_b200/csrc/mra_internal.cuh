@@ -104,6 +104,8 @@ struct Workspace {
     int *cnt;                // [B][nbr]
     float *pooled;           // [3][BH][nbr][D]
     unsigned long long *keys;// [BH][nbr2]
+    float *lo_logits;        // [BH][nbr2] low-resolution logit map (full mode, maps over 128 x 128)
+    float *lo_pmax;          // [BH][nbr][ceil(nbr / 64)] per-tile row maxima of the logit map
     float *mlo;              // [BH][nbr]
     SelState *state;         // [BH]
     int *gt, *eq;            // [BH*nbr]
@@ -209,7 +211,7 @@ cudaError_t launch_lowres_select_fused(const Problem &p, const Workspace &w, flo
 // per head, for nbr <= kSmallMaxRows.
 cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *sel_out,
                                 cudaStream_t s);
-cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t s);
+cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, const float *logit_out, cudaStream_t s);
 // Output layout of the attention kernels: element (b, h, n, e) of the
 // [B][H][N][D] result at out[b * ob + h * oh + n * orow + e] (null: the
 // contiguous [B][H][N][D] layout).

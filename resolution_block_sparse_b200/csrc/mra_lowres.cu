@@ -21,6 +21,8 @@
 // raises MRA_DEV_KEY_RANGE in the device status word.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "mra_internal.cuh"
 #include "mra_select_common.cuh"
 
@@ -38,124 +40,152 @@ __device__ __forceinline__ int in_band(int r, int c, int g) {
 
 constexpr int kLowresThreads = 256;
 
-// One CTA: R block rows of one (batch, head) against every block column, in
-// tiles of kKeysCT columns.  Thread tile: R/8 rows x 2 consecutive columns,
-// fp32 FFMA; the Q-hat rows and a transposed K-hat column tile sit in shared
-// memory (a fixed 16 KB tile, so that short row strips leave room for several
-// CTAs per SM).
-constexpr int kKeysCT = 64;
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"((unsigned)__cvta_generic_to_shared(dst)),
+                 "l"(src));
+}
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"((unsigned)__cvta_generic_to_shared(dst)),
+                 "l"(src));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
 
-template <int D, int R>
+// Logit map of maps above 128 x 128 blocks on 64 x 64 tiles:
+// l_rc = scale * qhat_r . khat_c in fp32 (FFMA, d ascending), written to
+// L [BH][nbr][nbr], and the maximum over the tile's valid columns (cnt > 0) of
+// each row to pmax [BH][nbr][ntiles] (-inf when none).  Persistent CTAs walk
+// the tiles with a stride of the grid; the next tile's Q-hat and K-hat rows
+// arrive by cp.async into the other of two buffers while the current tile is
+// multiplied.  Thread (tx, ty) of 16 x 16 holds rows ty + 16 i and columns
+// tx + 16 j (4 x 4 register tile): a warp's column loads are 16 consecutive
+// rows of a padded [64][D + 4] tile and its row loads broadcast.
+constexpr int kLgT = 64;
+
+template <int D>
+struct LgSmem {
+    float q[2][kLgT][D + 4];
+    float k[2][kLgT][D + 4];
+};
+
+template <int D>
+__global__ void __launch_bounds__(kLowresThreads, 3)
+lowres_logits_kernel(const float *__restrict__ qhat, const float *__restrict__ khat,
+                     const int *__restrict__ cnt, int H, int nbr, float scale, float *__restrict__ L,
+                     float *__restrict__ pmax, int total_tiles) {
+    pdl_wait();
+    extern __shared__ __align__(16) unsigned char lg_smem[];
+    LgSmem<D> &sh = *reinterpret_cast<LgSmem<D> *>(lg_smem);
+    const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
+    const int nt = (nbr + kLgT - 1) / kLgT;
+    auto stage = [&](int tile, int bf) {
+        const int bh = tile / (nt * nt), rem = tile - bh * nt * nt;
+        const int row0 = (rem / nt) * kLgT, col0 = (rem % nt) * kLgT;
+        const float *qh = qhat + (size_t)bh * nbr * D;
+        const float *kh = khat + (size_t)bh * nbr * D;
+        for (int i = t; i < kLgT * D / 4; i += kLowresThreads) {
+            const int r = i / (D / 4), d4 = i % (D / 4);
+            if (row0 + r < nbr) cp_async16(&sh.q[bf][r][4 * d4], qh + (size_t)(row0 + r) * D + 4 * d4);
+            else *reinterpret_cast<float4 *>(&sh.q[bf][r][4 * d4]) = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (col0 + r < nbr) cp_async16(&sh.k[bf][r][4 * d4], kh + (size_t)(col0 + r) * D + 4 * d4);
+            else *reinterpret_cast<float4 *>(&sh.k[bf][r][4 * d4]) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    int tile = blockIdx.x;
+    if (tile < total_tiles) stage(tile, 0);
+    cp_async_commit();
+    for (int it = 0; tile < total_tiles; ++it, tile += gridDim.x) {
+        const int bf = it & 1;
+        if (tile + (int)gridDim.x < total_tiles) stage(tile + gridDim.x, bf ^ 1);
+        cp_async_commit();
+        const int bh = tile / (nt * nt), rem = tile - bh * nt * nt;
+        const int ct = rem % nt;
+        const int row0 = (rem / nt) * kLgT, col0 = ct * kLgT;
+        int cv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = col0 + tx + 16 * j;
+            cv[j] = c < nbr ? cnt[(size_t)(bh / H) * nbr + c] : 0;
+        }
+        cp_async_wait<1>();
+        __syncthreads();   // this tile landed and is visible
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+#pragma unroll 2
+        for (int d = 0; d < D; d += 4) {
+            float4 kc[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) kc[j] = *reinterpret_cast<const float4 *>(&sh.k[bf][tx + 16 * j][d]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 qr = *reinterpret_cast<const float4 *>(&sh.q[bf][ty + 16 * i][d]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[i][j] = fmaf(qr.x, kc[j].x, acc[i][j]);
+                    acc[i][j] = fmaf(qr.y, kc[j].y, acc[i][j]);
+                    acc[i][j] = fmaf(qr.z, kc[j].z, acc[i][j]);
+                    acc[i][j] = fmaf(qr.w, kc[j].w, acc[i][j]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = row0 + ty + 16 * i;
+            float m = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = col0 + tx + 16 * j;
+                const float l = acc[i][j] * scale;
+                if (r < nbr && c < nbr) L[((size_t)bh * nbr + r) * nbr + c] = l;
+                if (cv[j] > 0) m = fmaxf(m, l);
+            }
+            // maximum over the 16 lanes of this row (a half warp)
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (tx == 0 && r < nbr) pmax[((size_t)bh * nbr + r) * nt + ct] = m;
+        }
+        __syncthreads();   // every thread is done with this buffer before it is staged again
+    }
+}
+
+// Selection keys of R block rows of one (batch, head) from the logit map: the
+// row maximum over valid columns from the tile maxima (0 when the row has
+// none), x = l - rowmax, the key (tier, order bits of x), and the first radix
+// histogram; the last CTA of the head locates the bucket of the k-th key.
+template <int R>
 __global__ void __launch_bounds__(kLowresThreads)
-lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ khat,
-                   const int *__restrict__ cnt, int H, int nbr, long long nbr2, float scale,
+lowres_keys_kernel(const float *__restrict__ L, const float *__restrict__ pmax,
+                   const int *__restrict__ cnt, int H, int nbr, long long nbr2,
                    int first_n, int diag_n, int k, unsigned long long *__restrict__ keys,
-                   float *__restrict__ mlo, float *__restrict__ logit_out,
-                   unsigned int *__restrict__ hist, unsigned int *__restrict__ arrive,
+                   float *__restrict__ mlo, unsigned int *__restrict__ hist, unsigned int *__restrict__ arrive,
                    SelState *__restrict__ state, unsigned int *__restrict__ status) {
     pdl_wait();
-    constexpr int CT = kKeysCT;
-    constexpr int RPT = R / 8;                 // rows per thread (eight row groups)
-    static_assert(R % 8 == 0 && kLowresThreads == 256, "thread tiling: 8 row groups x 32 column pairs");
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    float *qs = reinterpret_cast<float *>(smem_raw);                  // [R][D]
-    float *kT = qs + R * D;                                            // [D][CT]
-    float *lt = kT + D * CT;                                           // [R][nbr]
-    float *rmax = lt + (size_t)R * nbr;                                // [R]
-    int *cnts = reinterpret_cast<int *>(rmax + R);                     // [nbr]
+    int *cnts = reinterpret_cast<int *>(smem_raw);                     // [nbr]
     unsigned int *h0 = reinterpret_cast<unsigned int *>(cnts + nbr);   // [2048]
+    __shared__ float rmax[R];
     __shared__ unsigned int s_tmp[256];
     __shared__ int s_flag, s_last, s_bin;
     __shared__ unsigned int s_need;
 
-    const int t = threadIdx.x;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int bh = blockIdx.y;
     const int b = bh / H;
     const int r0 = blockIdx.x * R;
-    const float *qh = qhat + (size_t)bh * nbr * D;
-    const float *kh = khat + (size_t)bh * nbr * D;
-
     if (t == 0) s_flag = 0;
     for (int c = t; c < nbr; c += kLowresThreads) cnts[c] = cnt[(size_t)b * nbr + c];
     for (int i = t; i < (1 << kHist0Bits); i += kLowresThreads) h0[i] = 0u;
-    {
-        // all loads in flight before the first shared-memory store
-        constexpr int kQ = (R * D / 4 + kLowresThreads - 1) / kLowresThreads;
-        float4 v[kQ];
-#pragma unroll
-        for (int u = 0; u < kQ; ++u) {
-            const int i = t + u * kLowresThreads;
-            const int r = (4 * i) / D;
-            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < R * D / 4 && r0 + r < nbr)
-                v[u] = reinterpret_cast<const float4 *>(qh + (size_t)(r0 + r) * D)[(4 * i) % D / 4];
-        }
-#pragma unroll
-        for (int u = 0; u < kQ; ++u) {
-            const int i = t + u * kLowresThreads;
-            if (i < R * D / 4) reinterpret_cast<float4 *>(qs)[i] = v[u];
-        }
-    }
-
-    const int rg = t >> 5, cg = t & 31;   // rows RPT*rg .., columns 2*cg, 2*cg + 1 of the tile
-    for (int ct = 0; ct < nbr; ct += CT) {
-        __syncthreads();
-        // transposed column tile: kT[d][c] = khat[ct + c][d]
-        {
-            constexpr int kL = CT * D / 4 / kLowresThreads;   // float4 loads per thread
-            float4 v[kL];
-#pragma unroll
-            for (int u = 0; u < kL; ++u) {
-                const int e = t + u * kLowresThreads;
-                const int c = e % CT, d4 = e / CT;
-                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (ct + c < nbr) v[u] = reinterpret_cast<const float4 *>(kh + (size_t)(ct + c) * D)[d4];
-            }
-#pragma unroll
-            for (int u = 0; u < kL; ++u) {
-                const int e = t + u * kLowresThreads;
-                const int c = e % CT, d4 = e / CT;
-                kT[(4 * d4 + 0) * CT + c] = v[u].x;
-                kT[(4 * d4 + 1) * CT + c] = v[u].y;
-                kT[(4 * d4 + 2) * CT + c] = v[u].z;
-                kT[(4 * d4 + 3) * CT + c] = v[u].w;
-            }
-        }
-        __syncthreads();
-        float acc[RPT][2];
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) acc[i][0] = acc[i][1] = 0.0f;
-#pragma unroll 4
-        for (int d = 0; d < D; d += 4) {
-            float4 qv[RPT];
-#pragma unroll
-            for (int i = 0; i < RPT; ++i) qv[i] = *reinterpret_cast<const float4 *>(qs + (RPT * rg + i) * D + d);
-#pragma unroll
-            for (int dd = 0; dd < 4; ++dd) {
-                const float2 kv = *reinterpret_cast<const float2 *>(kT + (d + dd) * CT + 2 * cg);
-#pragma unroll
-                for (int i = 0; i < RPT; ++i) {
-                    const float qd = dd == 0 ? qv[i].x : dd == 1 ? qv[i].y : dd == 2 ? qv[i].z : qv[i].w;
-                    acc[i][0] = fmaf(qd, kv.x, acc[i][0]);
-                    acc[i][1] = fmaf(qd, kv.y, acc[i][1]);
-                }
-            }
-        }
-        const int c0 = ct + 2 * cg;
-#pragma unroll
-        for (int i = 0; i < RPT; ++i)
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-                if (c0 + j < nbr) lt[(size_t)(RPT * rg + i) * nbr + c0 + j] = acc[i][j] * scale;
-    }
-    __syncthreads();
-
-    // row max over valid columns (0 when the row has none)
-    const int warp = t >> 5, lane = t & 31;
+    const int ntiles = (nbr + kLgT - 1) / kLgT;
     for (int r = warp; r < R; r += kLowresThreads / 32) {
         float m = -INFINITY;
-        for (int c = lane; c < nbr; c += 32)
-            if (cnts[c] > 0) m = fmaxf(m, lt[(size_t)r * nbr + c]);
+        if (r0 + r < nbr)
+            for (int j = lane; j < ntiles; j += 32) m = fmaxf(m, pmax[((size_t)bh * nbr + r0 + r) * ntiles + j]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (m == -INFINITY) m = 0.0f;
@@ -166,33 +196,43 @@ lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ kha
     }
     __syncthreads();
 
-    // keys, exported logits, first radix histogram (bits 24..34)
+    // keys and the first radix histogram (bits 24..34): one warp per row, the
+    // row's terms hoisted, kU loads of the row in flight per lane
     const int rows_here = min(R, nbr - r0);
-    const int n_here = rows_here * nbr;
-    unsigned long long *kout = keys + (size_t)bh * nbr2 + (size_t)r0 * nbr;
     int flag = 0;
-    // warp-uniform trip count so that the histogram update can aggregate lanes
-    for (int e0 = (t & ~31); e0 < n_here; e0 += kLowresThreads) {
-        const int e = e0 + lane;
-        const bool act = e < n_here;
-        unsigned long long key = 0;
-        if (act) {
-            const int r = e / nbr, c = e - r * nbr;
-            const int gr = r0 + r;
-            const float l = lt[e];
-            float x = l - rmax[r];
-            if (x == 0.0f) x = 0.0f;  // canonical +0
-            if (!(fabsf(x) < 2500.0f)) flag = 1;
-            int tier = 0;
-            if (first_n > 0 && (gr < first_n || c < first_n)) ++tier;
-            tier += in_band(gr, c, diag_n);
-            if (cnts[gr] <= 0) tier -= 2;
-            if (cnts[c] <= 0) tier -= 2;
-            key = ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
-            kout[e] = key;
-            if (logit_out) logit_out[(size_t)bh * nbr2 + (size_t)gr * nbr + c] = l;
+    constexpr int kU = 4;
+    for (int r = warp; r < rows_here; r += kLowresThreads / 32) {
+        const int gr = r0 + r;
+        const float m = rmax[r];
+        const float *lrow = L + ((size_t)bh * nbr + gr) * nbr;
+        unsigned long long *krow = keys + (size_t)bh * nbr2 + (size_t)gr * nbr;
+        const bool row_first = first_n > 0 && gr < first_n;
+        const int row_tier = cnts[gr] <= 0 ? -2 : 0;
+        for (int c0 = 0; c0 < nbr; c0 += 32 * kU) {
+            float lv[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int c = c0 + 32 * u + lane;
+                lv[u] = c < nbr ? lrow[c] : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int c = c0 + 32 * u + lane;
+                const bool act = c < nbr;
+                unsigned long long key = 0;
+                if (act) {
+                    float x = lv[u] - m;
+                    if (x == 0.0f) x = 0.0f;  // canonical +0
+                    if (!(fabsf(x) < 2500.0f)) flag = 1;
+                    int tier = row_tier + ((row_first || (first_n > 0 && c < first_n)) ? 1 : 0);
+                    tier += in_band(gr, c, diag_n);
+                    if (cnts[c] <= 0) tier -= 2;
+                    key = ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
+                    krow[c] = key;
+                }
+                warp_hist_add(h0, (unsigned)(key >> 24), act);
+            }
         }
-        warp_hist_add(h0, (unsigned)(key >> 24), act);
     }
     if (flag) s_flag = 1;
     __syncthreads();
@@ -218,162 +258,183 @@ lowres_keys_kernel(const float *__restrict__ qhat, const float *__restrict__ kha
     }
 }
 
-// Low-resolution part of full mode for R block rows of one (batch, head):
+// Low-resolution part of full mode for kPvR block rows of one (batch, head):
 //   w_rc = cnt_c * exp(l_rc - rowmax_r) for every unselected c with cnt_c > 0,
-//   olo_r = sum_c w_rc * vhat_c,   llo_r = sum_c w_rc.
-// block rows per CTA (every CTA reads the whole pooled V of its head, so
-// fewer rows per CTA cost more loads than they win in occupancy)
+//   olo_r = sum_c w_rc * vhat_c,   llo_r = sum_c w_rc,
+// over tiles of kPvC columns.  Each tile's logits, V-hat rows, counts and
+// selection words arrive by cp.async into one of two buffers while the
+// previous tile is multiplied; the weights are formed once per tile (stored
+// [c][r]), then a register-tiled product: thread (tx, ty) of 16 x 16 holds
+// rows 2 ty, 2 ty + 1 and dims D/16 * tx ...
+constexpr int kPvR = 32, kPvC = 64;
+
 template <int D>
-constexpr int pv_rows() { return 32; }
+struct PvSmem {
+    float v[2][kPvC][D + 4];
+    float l[2][kPvR][kPvC + 4];
+    float wt[kPvC][kPvR + 4];
+    unsigned int selw[2][kPvR][2];
+    int cntc[2][kPvC];
+    float m[kPvR];
+};
 
 template <int D>
 __global__ void __launch_bounds__(kLowresThreads)
-lowres_pv_kernel(const unsigned long long *__restrict__ keys, const unsigned int *__restrict__ bitmap,
-                 int wpr, const int *__restrict__ cnt, const float *__restrict__ vhat, int H,
-                 int nbr, long long nbr2, float *__restrict__ olo, float *__restrict__ llo) {
+lowres_pv_kernel(const float *__restrict__ L, const float *__restrict__ mlo, const unsigned int *__restrict__ bitmap,
+                 int wpr, const int *__restrict__ cnt, const float *__restrict__ vhat, int H, int nbr,
+                 float *__restrict__ olo, float *__restrict__ llo) {
     pdl_wait();
-    constexpr int R = pv_rows<D>();
-    constexpr int kCt = 32;
-    constexpr int kVL = kCt * D / 4 / kLowresThreads;      // float4 loads of the V-hat tile
-    constexpr int kWL = R * kCt / kLowresThreads;          // weights per thread and tile
-    __shared__ __align__(16) float vs[kCt][D];
-    __shared__ float ws[R][kCt + 1];
-    const int t = threadIdx.x;
+    constexpr int DW = D / 16;
+    extern __shared__ __align__(16) unsigned char pv_smem[];
+    PvSmem<D> &sh = *reinterpret_cast<PvSmem<D> *>(pv_smem);
+    const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
     const int bh = blockIdx.y;
     const int b = bh / H;
-    const int r0 = blockIdx.x * R;
+    const int r0 = blockIdx.x * kPvR;
     const float *vh = vhat + (size_t)bh * nbr * D;
-    // thread tile: kRpt rows x 4 head dims
-    constexpr int kDG = D / 4;                    // dim groups
-    constexpr int kRG = kLowresThreads / kDG;     // row groups
-    constexpr int kRpt = R / kRG;                 // rows per thread
-    static_assert(kRpt >= 1 && kRG * kRpt == R, "tile shape");
-    const int dg = t % kDG, rg = t / kDG;
-    float4 acc[kRpt];
-    float lsum[kRpt];
-#pragma unroll
-    for (int i = 0; i < kRpt; ++i) {
-        acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        lsum[i] = 0.0f;
-    }
-
-    // the global loads of tile ct + kCt are issued before the products of
-    // tile ct, so that their latency overlaps the arithmetic
-    float4 vv[kVL];
-    unsigned long long kv[kWL];
-    unsigned int bw[kWL];
-    int cc[kWL];
-    auto load_tile = [&](int ct) {
-#pragma unroll
-        for (int u = 0; u < kVL; ++u) {
-            const int i = t + u * kLowresThreads;
-            const int c = (4 * i) / D;
-            vv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (ct + c < nbr) vv[u] = reinterpret_cast<const float4 *>(vh + (size_t)(ct + c) * D)[(4 * i) % D / 4];
+    const float *lh = L + (size_t)bh * nbr * nbr;
+    const bool l16 = (nbr & 3) == 0;   // logit rows 16-byte aligned
+    // issues the copies of the tile at column c0 into buffer bf; out-of-range
+    // entries are written as zeros (counts 0: no weight)
+    auto stage = [&](int c0, int bf) {
+        for (int i = t; i < kPvC * D / 4; i += kLowresThreads) {
+            const int c = i / (D / 4), d4 = i % (D / 4);
+            if (c0 + c < nbr) cp_async16(&sh.v[bf][c][4 * d4], vh + (size_t)(c0 + c) * D + 4 * d4);
+            else *reinterpret_cast<float4 *>(&sh.v[bf][c][4 * d4]) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-#pragma unroll
-        for (int u = 0; u < kWL; ++u) {
-            const int e = t + u * kLowresThreads;
-            const int r = e / kCt, c = e % kCt;
-            const int gr = r0 + r, gc = ct + c;
-            kv[u] = 0ull;
-            bw[u] = 0xffffffffu;
-            cc[u] = 0;
-            if (gr < nbr && gc < nbr) {
-                cc[u] = cnt[(size_t)b * nbr + gc];
-                bw[u] = bitmap[((size_t)bh * nbr + gr) * wpr + (gc >> 5)];
-                kv[u] = keys[(size_t)bh * nbr2 + (size_t)gr * nbr + gc];
+        if (l16) {
+            for (int i = t; i < kPvR * kPvC / 4; i += kLowresThreads) {
+                const int r = i / (kPvC / 4), c4 = 4 * (i % (kPvC / 4));
+                if (r0 + r < nbr && c0 + c4 < nbr)
+                    cp_async16(&sh.l[bf][r][c4], lh + (size_t)(r0 + r) * nbr + c0 + c4);
             }
+        } else {
+            for (int i = t; i < kPvR * kPvC; i += kLowresThreads) {
+                const int r = i / kPvC, c = i % kPvC;
+                if (r0 + r < nbr && c0 + c < nbr) cp_async4(&sh.l[bf][r][c], lh + (size_t)(r0 + r) * nbr + c0 + c);
+            }
+        }
+        if (t < kPvC) {
+            if (c0 + t < nbr) cp_async4(&sh.cntc[bf][t], cnt + (size_t)b * nbr + c0 + t);
+            else sh.cntc[bf][t] = 0;
+        } else if (t < kPvC + 2 * kPvR) {
+            const int r = (t - kPvC) >> 1, wsel = (t - kPvC) & 1;
+            const int w = (c0 >> 5) + wsel;   // c0 is a multiple of 64
+            if (r0 + r < nbr && w < wpr) cp_async4(&sh.selw[bf][r][wsel], bitmap + ((size_t)bh * nbr + r0 + r) * wpr + w);
+            else sh.selw[bf][r][wsel] = ~0u;
         }
     };
-    load_tile(0);
-    for (int ct = 0; ct < nbr; ct += kCt) {
-        __syncthreads();   // previous tile fully consumed
+    if (t < kPvR) sh.m[t] = r0 + t < nbr ? mlo[(size_t)bh * nbr + r0 + t] : 0.0f;
+    float acc[2][DW], ls[2] = {0.0f, 0.0f};
 #pragma unroll
-        for (int u = 0; u < kVL; ++u) {
-            const int i = t + u * kLowresThreads;
-            reinterpret_cast<float4 *>(&vs[0][0])[i] = vv[u];
-        }
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
-        for (int u = 0; u < kWL; ++u) {
+        for (int e = 0; e < DW; ++e) acc[i][e] = 0.0f;
+    const int ntiles = (nbr + kPvC - 1) / kPvC;
+    stage(0, 0);
+    cp_async_commit();
+    for (int it = 0; it < ntiles; ++it) {
+        const int bf = it & 1, c0 = it * kPvC;
+        if (it + 1 < ntiles) stage(c0 + kPvC, bf ^ 1);   // that buffer was last read before the barrier below
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();   // tile it landed (every thread's copies) and is visible
+        // weights: thread t forms (r, c) = (e % 32, e / 32) for e = t + 256 u
+#pragma unroll
+        for (int u = 0; u < kPvR * kPvC / kLowresThreads; ++u) {
             const int e = t + u * kLowresThreads;
-            const int r = e / kCt, c = e % kCt;
-            const int gc = ct + c;
-            float wv = 0.0f;
-            if (cc[u] > 0 && !((bw[u] >> (gc & 31)) & 1u)) {
-                const float x = float_from_order_bits((unsigned int)(kv[u] & 0xffffffffull));
-                wv = (float)cc[u] * expf(x);
-            }
-            ws[r][c] = wv;
+            const int r = e % kPvR, c = e / kPvR;
+            float w = 0.0f;
+            const int cc = sh.cntc[bf][c];
+            if (cc > 0 && !((sh.selw[bf][r][c >> 5] >> (c & 31)) & 1u))
+                w = (float)cc * expf(sh.l[bf][r][c] - sh.m[r]);
+            sh.wt[c][r] = w;
         }
-        if (ct + kCt < nbr) load_tile(ct + kCt);
         __syncthreads();
 #pragma unroll 8
-        for (int c = 0; c < kCt; ++c) {
-            const float4 v4 = *reinterpret_cast<const float4 *>(&vs[c][4 * dg]);
-#pragma unroll
-            for (int i = 0; i < kRpt; ++i) {
-                const float wv = ws[rg * kRpt + i][c];
-                acc[i].x = fmaf(wv, v4.x, acc[i].x);
-                acc[i].y = fmaf(wv, v4.y, acc[i].y);
-                acc[i].z = fmaf(wv, v4.z, acc[i].z);
-                acc[i].w = fmaf(wv, v4.w, acc[i].w);
-                lsum[i] += wv;
+        for (int c = 0; c < kPvC; ++c) {
+            const float2 w2 = *reinterpret_cast<const float2 *>(&sh.wt[c][2 * ty]);
+            float vv[DW];
+            if constexpr (DW == 4) {
+                const float4 v4 = *reinterpret_cast<const float4 *>(&sh.v[bf][c][4 * tx]);
+                vv[0] = v4.x; vv[1] = v4.y; vv[2] = v4.z; vv[3] = v4.w;
+            } else {
+                const float2 v2 = *reinterpret_cast<const float2 *>(&sh.v[bf][c][2 * tx]);
+                vv[0] = v2.x; vv[1] = v2.y;
             }
+#pragma unroll
+            for (int e = 0; e < DW; ++e) {
+                acc[0][e] = fmaf(w2.x, vv[e], acc[0][e]);
+                acc[1][e] = fmaf(w2.y, vv[e], acc[1][e]);
+            }
+            ls[0] += w2.x;
+            ls[1] += w2.y;
         }
+        __syncthreads();   // wt and this tile's buffers are free
     }
 #pragma unroll
-    for (int i = 0; i < kRpt; ++i) {
-        const int gr = r0 + rg * kRpt + i;
-        if (gr < nbr) {
-            *reinterpret_cast<float4 *>(olo + ((size_t)bh * nbr + gr) * D + 4 * dg) = acc[i];
-            if (dg == 0) llo[(size_t)bh * nbr + gr] = lsum[i];
-        }
+    for (int i = 0; i < 2; ++i) {
+        const int gr = r0 + 2 * ty + i;
+        if (gr >= nbr) continue;
+        float *dst = olo + ((size_t)bh * nbr + gr) * D + DW * tx;
+#pragma unroll
+        for (int e = 0; e < DW; ++e) dst[e] = acc[i][e];
+        if (tx == 0) llo[(size_t)bh * nbr + gr] = ls[i];
     }
 }
 
-template <int D, int R>
-cudaError_t launch_keys_rt(const Problem &p, const Workspace &w, float *logit_out, cudaStream_t s) {
-    constexpr int CT = kKeysCT;
-    const size_t smem = sizeof(float) * ((size_t)R * D + (size_t)D * CT + (size_t)R * p.nbr + R) +
-                        sizeof(int) * (size_t)p.nbr + sizeof(unsigned int) * (1u << kHist0Bits);
-    cudaError_t e = cudaFuncSetAttribute(lowres_keys_kernel<D, R>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int R>
+cudaError_t launch_keys_rt(const Problem &p, const Workspace &w, const float *L, cudaStream_t s) {
+    const size_t smem = sizeof(int) * (size_t)p.nbr + sizeof(unsigned int) * (1u << kHist0Bits);
+    cudaError_t e = cudaFuncSetAttribute(lowres_keys_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((p.nbr + R - 1) / R, p.BH);
-    const float scale = 1.0f / sqrtf((float)p.D);
-    const float *qhat = w.pooled;
-    const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;
-    return launch_dependent(lowres_keys_kernel<D, R>, dim3(grid), dim3(kLowresThreads), smem, s, 
-        qhat, khat, w.cnt, p.H, p.nbr, p.nbr2, scale, p.first_n, p.diag_n, p.k, w.keys, w.mlo,
-        logit_out, w.hist, w.arrive, w.state, w.status);
+    return launch_dependent(lowres_keys_kernel<R>, dim3((p.nbr + R - 1) / R, p.BH), dim3(kLowresThreads), smem, s,
+                            L, (const float *)w.lo_pmax, (const int *)w.cnt, p.H, p.nbr, p.nbr2, p.first_n,
+                            p.diag_n, p.k, w.keys, w.mlo, w.hist, w.arrive, w.state, w.status);
 }
 
 template <int D>
-cudaError_t launch_keys_typed(const Problem &p, const Workspace &w, float *logit_out,
-                              cudaStream_t s) {
-    if (p.r_tile == 32) return launch_keys_rt<D, 32>(p, w, logit_out, s);
-    if (p.r_tile == 16) return launch_keys_rt<D, 16>(p, w, logit_out, s);
-    return launch_keys_rt<D, 8>(p, w, logit_out, s);
+cudaError_t launch_logits_typed(const Problem &p, const Workspace &w, float *L, cudaStream_t s) {
+    const long long nt = (p.nbr + kLgT - 1) / kLgT;
+    const long long total = nt * nt * p.BH;
+    const float scale = 1.0f / sqrtf((float)p.D);
+    const float *qhat = w.pooled;
+    const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;
+    const size_t smem = sizeof(LgSmem<D>);
+    cudaError_t e = cudaFuncSetAttribute(lowres_logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long grid = std::min<long long>(total, 3LL * device_sm_count());
+    return launch_dependent(lowres_logits_kernel<D>, dim3((unsigned)grid), dim3(kLowresThreads), smem, s, qhat, khat,
+                            (const int *)w.cnt, p.H, p.nbr, scale, L, w.lo_pmax, (int)total);
 }
 
 }  // namespace
 
-cudaError_t launch_lowres_keys(const Problem &p, const Workspace &w, float *logit_out,
-                               cudaStream_t s) {
-    return p.D == 64 ? launch_keys_typed<64>(p, w, logit_out, s)
-                     : launch_keys_typed<32>(p, w, logit_out, s);
+float *lowres_logit_map(const Workspace &w, float *logit_out) { return logit_out ? logit_out : w.lo_logits; }
+
+cudaError_t launch_lowres_keys(const Problem &p, const Workspace &w, float *logit_out, cudaStream_t s) {
+    float *L = lowres_logit_map(w, logit_out);
+    cudaError_t e = p.D == 64 ? launch_logits_typed<64>(p, w, L, s) : launch_logits_typed<32>(p, w, L, s);
+    if (e != cudaSuccess) return e;
+    if (p.r_tile == 32) return launch_keys_rt<32>(p, w, L, s);
+    if (p.r_tile == 16) return launch_keys_rt<16>(p, w, L, s);
+    return launch_keys_rt<8>(p, w, L, s);
 }
 
-cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, cudaStream_t s) {
+cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, const float *logit_out, cudaStream_t s) {
+    const float *L = logit_out ? logit_out : w.lo_logits;
     const float *vhat = w.pooled + (size_t)2 * p.BH * p.nbr * p.D;
-    if (p.D == 64)
-        return launch_dependent(lowres_pv_kernel<64>, dim3((p.nbr + pv_rows<64>() - 1) / pv_rows<64>(), p.BH),
-                                dim3(kLowresThreads), 0, s, w.keys, w.bitmap, w.words_per_row, w.cnt, vhat, p.H,
-                                p.nbr, p.nbr2, w.olo, w.llo);
-    return launch_dependent(lowres_pv_kernel<32>, dim3((p.nbr + pv_rows<32>() - 1) / pv_rows<32>(), p.BH),
-                            dim3(kLowresThreads), 0, s, w.keys, w.bitmap, w.words_per_row, w.cnt, vhat, p.H,
-                            p.nbr, p.nbr2, w.olo, w.llo);
+    const dim3 grid((unsigned)((p.nbr + kPvR - 1) / kPvR), (unsigned)p.BH);
+    auto run = [&](auto kern, size_t smem) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_dependent(kern, grid, dim3(kLowresThreads), smem, s, L, (const float *)w.mlo,
+                                (const unsigned int *)w.bitmap, w.words_per_row, (const int *)w.cnt, vhat, p.H,
+                                p.nbr, w.olo, w.llo);
+    };
+    return p.D == 64 ? run(lowres_pv_kernel<64>, sizeof(PvSmem<64>)) : run(lowres_pv_kernel<32>, sizeof(PvSmem<32>));
 }
 
 }  // namespace mra

@@ -99,7 +99,6 @@ __global__ void __launch_bounds__(kThreads)
 lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__restrict__ khat,
                              const int *__restrict__ cnt, int H, int nbr, float scale, int first_n,
                              int diag_n, int k, int cap, int chunk,
-                             unsigned long long *__restrict__ keys_out,
                              float *__restrict__ mlo, float *__restrict__ logit_out,
                              int *__restrict__ cols, int32_t *__restrict__ sel_out,
                              unsigned int *__restrict__ bitmap, int wpr, WorkItem *__restrict__ items,
@@ -256,7 +255,6 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                     key = ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
                     sk[rr * nbr + c] = key;
                     const size_t gi = (size_t)bh * nbr2 + (size_t)gr * nbr + c;
-                    if (keys_out) keys_out[gi] = key;
                     if (logit_out) logit_out[gi] = lv[j];
                 }
                 warp_hist_add(cs.lh, (unsigned)(key >> (kHist1Bits + kHist2Bits)) & ((1u << kHist0Bits) - 1u), ok);
@@ -592,9 +590,10 @@ cudaError_t launch_typed(const Problem &p, const Workspace &w, float *logit_out,
     const float scale = 1.0f / sqrtf((float)p.D);
     const float *qhat = w.pooled;
     const float *khat = w.pooled + (size_t)p.BH * p.nbr * p.D;
+    // full mode keeps the logit map for the low-resolution part
+    float *lmap = logit_out ? logit_out : (p.mode == 0 ? w.lo_logits : nullptr);
     e = cudaLaunchKernelEx(&cfg, kern, qhat, khat, (const int *)w.cnt, p.H, p.nbr, scale, p.first_n,
-                           p.diag_n, p.k, p.cap, p.chunk, p.mode == 0 ? w.keys : (unsigned long long *)nullptr,
-                           w.mlo, logit_out, w.cols, sel_out,
+                           p.diag_n, p.k, p.cap, p.chunk, w.mlo, lmap, w.cols, sel_out,
                            p.mode == 0 ? w.bitmap : (unsigned int *)nullptr, w.words_per_row, w.items,
                            w.head_items, w.state, w.status);
     if (e != cudaSuccess) return e;
