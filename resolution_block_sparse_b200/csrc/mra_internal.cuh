@@ -172,11 +172,11 @@ struct GradStats {
 // programmatic stream serialization: it may be scheduled while the kernel
 // before it drains, and it calls pdl_wait() (which returns once every earlier
 // kernel of the stream has completed and its writes are visible) before it
-// touches their results.  Kernels call pdl_trigger() early so that the next
-// launch is not held back until they exit.  Without the launch attribute both
-// instructions are no-ops.
+// touches their results.  No kernel triggers its dependents early: dependents
+// made resident early took SM space from the running kernel (the N=4096
+// graph-replayed pass 3 us slower).  Without the launch attribute the wait is
+// a no-op.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
