@@ -119,20 +119,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def traffic_for(kernel_phase: str, src_file: str):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel source changed since the counters were taken."""
+def traffic_for(kernel_phase: str, src_file: str, workload: int):
+    """DRAM bytes per launch from the committed ncu record of this workload,
+    or None when there is none or the kernel source changed since the
+    counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel_phase)
-    except (OSError, ValueError):
+            rec = json.load(f).get(str(workload), {}).get(kernel_phase)
+    except (OSError, ValueError, AttributeError):
         return None
     if not rec:
         return None
     with open(os.path.join(ROOT, "resolution_block_sparse_b200", "csrc", src_file), "rb") as f:
         h = hashlib.sha256(f.read()).hexdigest()[:16]
-    if rec.get("source_sha256_16") != h:
+    if rec.get("source") != src_file or rec.get("source_sha256_16") != h:
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -840,8 +841,11 @@ def main():
     dom_s = phases[dom]["avg_us"] * 1e-6
     esz = 2 if w.dtype == "bf16" else 4
     BH = w.B * w.H
-    # bf16 head size 64 runs the tcgen05 kernel unless MRA_ATTN_IMPL=mma
-    tc_attn = w.dtype == "bf16" and w.D == 64 and not os.environ.get("MRA_ATTN_IMPL", "").startswith("m")
+    # bf16 head size 64 runs the tcgen05 kernel on maps with at least 32
+    # selected blocks per block row (MRA_ATTN_IMPL=tc / =mma force either)
+    impl = os.environ.get("MRA_ATTN_IMPL", "")
+    tc_attn = w.dtype == "bf16" and w.D == 64 and (
+        impl.startswith("t") or (not impl.startswith("m") and min(w.block_per_row, w.nbr) >= 32))
     kernel_src = {"attention": "mra_attn_tc.cu" if tc_attn else "mra_attn.cu", "pool": "mra_pool.cu",
                   "lowres_keys": "mra_lowres.cu", "lowres_pv": "mra_lowres.cu", "select": "mra_select.cu",
                   "lowres_select": "mra_lowres_select.cu", "group_plan": "mra_group_plan.cu"}
@@ -860,7 +864,7 @@ def main():
     roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "peak_source": f"{peak_src} (burst)",
                 "algorithmic_bytes_per_launch": bytes_,
-                "traffic": traffic_for(dom, kernel_src.get(dom, "mra_attn.cu"))}
+                "traffic": traffic_for(dom, kernel_src.get(dom, "mra_attn.cu"), w.index)}
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
