@@ -75,11 +75,6 @@ Problem make_problem(int B, int H, int N, int D, int bpr, int mode, int first_n,
     // (at most 64 KB), so longer maps take fewer rows per CTA
     p.r_tile = p.nbr > 1024 ? 8 : 16;
     p.lowres_ctas = (p.nbr + p.r_tile - 1) / p.r_tile;
-    long long ctas = (p.nbr2 + 4095) / 4096;
-    if (ctas < 1) ctas = 1;
-    if (ctas > 1024) ctas = 1024;
-    p.radix_ctas = (int)ctas;
-    p.radix_chunk = (p.nbr2 + ctas - 1) / ctas;
     return p;
 }
 
@@ -118,6 +113,7 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     t.slot_arrive = (int *)take(sizeof(int) * BH * (size_t)p.cap);
     t.zero_bytes_no_hist = off;
     t.hist = (unsigned int *)take(sizeof(unsigned int) * BH * 3 * kHistBins);
+    t.ccount = (int *)take(sizeof(int) * BH);
     t.zero_base = t.arrive;
     t.zero_bytes = off;
     t.cnt = (int *)take(sizeof(int) * (size_t)p.B * nbr);
@@ -127,13 +123,17 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     t.lo_pmax = (float *)take(sizeof(float) * BH * nbr * ((nbr + 63) / 64));
     t.mlo = (float *)take(sizeof(float) * BH * nbr);
     t.state = (SelState *)take(sizeof(SelState) * BH);
-    t.gt = (int *)take(sizeof(int) * BH * nbr);
-    t.eq = (int *)take(sizeof(int) * BH * nbr);
-    t.row_start = (int *)take(sizeof(int) * BH * nbr);
-    t.take_eq = (int *)take(sizeof(int) * BH * nbr);
     t.cols = (int *)take(sizeof(int) * BH * (size_t)p.k);
     t.words_per_row = (p.nbr + 31) / 32;
     t.bitmap = (unsigned int *)take(sizeof(unsigned int) * BH * nbr * (size_t)t.words_per_row);
+    if (!lowres_select_fused_supported(p)) {   // the multi-kernel selection
+        t.cand_key = (unsigned long long *)take(sizeof(unsigned long long) * BH * (size_t)p.nbr2);
+        t.cand_idx = (int *)take(sizeof(int) * BH * (size_t)p.nbr2);
+        t.tiebits = (unsigned int *)take(sizeof(unsigned int) * BH * nbr * (size_t)t.words_per_row);
+        t.above_cnt = (int *)take(sizeof(int) * BH * nbr);
+        t.row_start = (int *)take(sizeof(int) * BH * nbr);
+        t.row_take = (int *)take(sizeof(int) * BH * nbr);
+    }
     t.items = (WorkItem *)take(sizeof(WorkItem) * BH * (size_t)p.cap);
     t.head_items = (int *)take(sizeof(int) * BH);
     t.olo = (float *)take(sizeof(float) * BH * nbr * D);
@@ -315,17 +315,9 @@ int enqueue_forward(const Problem &p, const Workspace &w, const void *q, const v
             ++launches;
         }
         PhaseScope ps("select", s, prof);
-        if (p.nbr <= kSmallMaxRows) {
-            MRA_TRY(launch_select_small(p, w, sel_out, s));
-            launches += 1;
-        } else {
-            MRA_TRY(launch_radix_pass(p, w, 1, s));
-            MRA_TRY(launch_radix_pass(p, w, 2, s));
-            MRA_TRY(launch_row_counts(p, w, s));
-            MRA_TRY(launch_row_scan(p, w, s));
-            MRA_TRY(launch_cols(p, w, sel_out, s));
-            launches += 5;
-        }
+        MRA_TRY(launch_select_scan(p, w, s));
+        MRA_TRY(launch_select_finalize(p, w, sel_out, s));
+        launches += 3;
     }
     if (p.mode == MRA_FULL) {
         PhaseScope ps("lowres_pv", s, prof);

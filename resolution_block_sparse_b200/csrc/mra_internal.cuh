@@ -31,8 +31,6 @@ constexpr int kHist1Bits = 12;
 constexpr int kHist2Bits = 12;
 constexpr int kHistBins = 4096;       // per-pass histogram stride per head
 constexpr int kMaxN = 65536;
-constexpr int kSmallMaxRows = 128;               // one-CTA selection up to 128 x 128 blocks
-constexpr int kSmallMaxKeys = kSmallMaxRows * kSmallMaxRows;
 
 // Device status bits (mirrors of the public MRA_DEV_* values).
 constexpr unsigned kDevKeyRange = 1u;
@@ -78,8 +76,6 @@ struct Problem {
     int cap;          // work-item slots per head: nbr + k / chunk
     int r_tile;       // rows per CTA of the low-res kernels
     int lowres_ctas;  // CTAs per head of the low-res key kernel
-    int radix_ctas;   // CTAs per head of a radix pass
-    long long radix_chunk;  // keys per radix CTA
     int bwd;          // the workspace also holds the backward pass's buffers
     int layer;        // the workspace also holds the layer's Q/K/V and output (bf16 [B][H][N][D] each)
     int fused;        // single-launch pass for small maps: -1 by preference, 0 never, 1 wherever it fits
@@ -98,7 +94,7 @@ struct Workspace {
     int *group_arrive;       // [BH*ngroups]: split-group arrivals (tcgen05 kernel)
     int *slot_arrive;        // [BH*cap]: arrivals of a split row's item groups (warp-level kernels)
     size_t zero_bytes;       // the whole region
-    size_t zero_bytes_no_hist;   // the region without the radix histograms
+    size_t zero_bytes_no_hist;   // the region without the radix histograms and the candidate counts
     void *zero_base;
     // written before read every call
     int *cnt;                // [B][nbr]
@@ -108,9 +104,13 @@ struct Workspace {
     float *lo_pmax;          // [BH][nbr][ceil(nbr / 64)] per-tile row maxima of the logit map
     float *mlo;              // [BH][nbr]
     SelState *state;         // [BH]
-    int *gt, *eq;            // [BH*nbr]
-    int *row_start;          // [BH*nbr]
-    int *take_eq;            // [BH*nbr]
+    int *ccount;             // [BH] candidates of the first digit's bucket (zeroed region)
+    unsigned long long *cand_key;   // [BH][nbr2] the bucket's keys (maps over 128 x 128)
+    int *cand_idx;           // [BH][nbr2] their flat indices r * nbr + c
+    unsigned int *tiebits;   // [BH*nbr][words_per_row] keys equal to the threshold
+    int *above_cnt;          // [BH*nbr] per row: keys above the first digit's bucket
+    int *row_start;          // [BH*nbr] CSR offset of each row's columns in cols[]
+    int *row_take;           // [BH*nbr] keys equal to the threshold that each row takes
     int *cols;               // [BH*k]
     unsigned int *bitmap;    // [BH*nbr][words_per_row]
     int words_per_row;
@@ -198,19 +198,18 @@ cudaError_t launch_pool(const Problem &p, const Workspace &w, const void *q, con
                         const void *v, const float *mask, cudaStream_t s);
 cudaError_t launch_lowres_keys(const Problem &p, const Workspace &w, float *logit_out,
                                cudaStream_t s);
-cudaError_t launch_radix_pass(const Problem &p, const Workspace &w, int pass, cudaStream_t s);
-cudaError_t launch_row_counts(const Problem &p, const Workspace &w, cudaStream_t s);
-cudaError_t launch_row_scan(const Problem &p, const Workspace &w, cudaStream_t s);
-cudaError_t launch_cols(const Problem &p, const Workspace &w, int32_t *sel_out, cudaStream_t s);
+// Selection of maps above 128 x 128 after the keys kernel: one pass over the
+// keys (certain selections into the bitmap, the first digit's bucket into a
+// candidate list); then one CTA per head (threshold, row counts, scan, work
+// list) followed by the column lists, one warp per row (both launched by
+// launch_select_finalize).
+cudaError_t launch_select_scan(const Problem &p, const Workspace &w, cudaStream_t s);
+cudaError_t launch_select_finalize(const Problem &p, const Workspace &w, int32_t *sel_out, cudaStream_t s);
 // Low-resolution logits, keys and the whole selection in one kernel: one
 // thread-block cluster per head (nbr <= 128).
 bool lowres_select_fused_supported(const Problem &p);
 cudaError_t launch_lowres_select_fused(const Problem &p, const Workspace &w, float *logit_out,
                                        int32_t *sel_out, cudaStream_t s);
-// Whole selection (radix passes 2-3, counts, scan, work list, cols) in one CTA
-// per head, for nbr <= kSmallMaxRows.
-cudaError_t launch_select_small(const Problem &p, const Workspace &w, int32_t *sel_out,
-                                cudaStream_t s);
 cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, const float *logit_out, cudaStream_t s);
 // Output layout of the attention kernels: element (b, h, n, e) of the
 // [B][H][N][D] result at out[b * ob + h * oh + n * orow + e] (null: the
