@@ -136,6 +136,13 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     }
     t.items = (WorkItem *)take(sizeof(WorkItem) * BH * (size_t)p.cap);
     t.head_items = (int *)take(sizeof(int) * BH);
+    {
+        const int sp = lowres_pv_splits(p);
+        if (sp > 1) {
+            t.lo_opart = (float *)take(sizeof(float) * (size_t)sp * BH * nbr * D);
+            t.lo_lpart = (float *)take(sizeof(float) * (size_t)sp * BH * nbr);
+        }
+    }
     t.olo = (float *)take(sizeof(float) * BH * nbr * D);
     t.llo = (float *)take(sizeof(float) * BH * nbr);
     t.partial = (float *)take(sizeof(float) * BH * (D + 2) *

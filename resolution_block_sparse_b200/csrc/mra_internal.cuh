@@ -116,6 +116,8 @@ struct Workspace {
     int words_per_row;
     WorkItem *items;         // [BH*cap]
     int *head_items;         // [BH]
+    float *lo_opart;         // [splits][BH*nbr][D] partial low-resolution outputs (tensor-core kernel)
+    float *lo_lpart;         // [splits][BH*nbr] partial normalisers
     float *olo;              // [BH*nbr][D]
     float *llo;              // [BH*nbr]
     float *partial;          // [BH*cap][32*(D+2)], or [BH*gcap][128*(D+2)] for the tcgen05 kernel
@@ -211,6 +213,8 @@ bool lowres_select_fused_supported(const Problem &p);
 cudaError_t launch_lowres_select_fused(const Problem &p, const Workspace &w, float *logit_out,
                                        int32_t *sel_out, cudaStream_t s);
 cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, const float *logit_out, cudaStream_t s);
+// column splits of the low-resolution kernel (1: no partials)
+int lowres_pv_splits(const Problem &p);
 // Output layout of the attention kernels: element (b, h, n, e) of the
 // [B][H][N][D] result at out[b * ob + h * oh + n * orow + e] (null: the
 // contiguous [B][H][N][D] layout).

@@ -383,6 +383,185 @@ lowres_pv_kernel(const float *__restrict__ L, const float *__restrict__ mlo, con
     }
 }
 
+// The same low-resolution part on the tensor cores for bf16 problems:
+// O_lo = W V-hat as mma.sync m16n8k8 with tf32 operands (W and V-hat rounded
+// to tf32, 2^-11 relative, far inside the bf16 output's rounding) and fp32
+// accumulation; the normaliser llo sums the fp32 weights.  A CTA covers
+// kPtR = 32 block rows with four warps: warp w takes rows 16 (w & 1) ..
+// + 15 and head dims (w >> 1) D/2 .. + D/2 - 1, forming the weights of its A
+// fragments itself (cnt_c exp(l - rowmax) for unselected valid blocks) from
+// the logit tile; 64-column tiles of the logits and V-hat arrive by
+// double-buffered cp.async.  The column tiles of a row block split over
+// gridDim.z CTAs (so that a small number of heads still fills the SMs); with
+// more than one split each writes fp32 partials of O and of the normaliser
+// at opart / lpart [split][row], which lowres_pv_merge adds in split order.
+constexpr int kPtR = 32, kPtC = 64, kPtThreads = 128;
+constexpr int kPtMaxSplits = 4;
+
+template <int D>
+struct PtSmem {
+    float l[2][kPtR][kPtC + 4];        // rows: 8 g + tq spread over the banks
+    float v[2][kPtC][D + 8];           // rows 4 apart in distinct banks
+    int cntc[2][kPtC];
+    unsigned int selw[2][kPtR][2];
+};
+
+__device__ __forceinline__ unsigned int to_tf32(float x) {
+    unsigned int r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void mma_tf32(float (&c)[4], const unsigned int (&a)[4], unsigned int b0, unsigned int b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPtThreads)
+lowres_pv_tf32_kernel(const float *__restrict__ L, const float *__restrict__ mlo,
+                      const unsigned int *__restrict__ bitmap, int wpr, const int *__restrict__ cnt,
+                      const float *__restrict__ vhat, int H, int nbr, float *__restrict__ olo,
+                      float *__restrict__ llo, float *__restrict__ opart, float *__restrict__ lpart) {
+    pdl_wait();
+    constexpr int NT = D / 16;   // n-tiles of 8 dims per warp
+    extern __shared__ __align__(16) unsigned char pt_smem[];
+    PtSmem<D> &sh = *reinterpret_cast<PtSmem<D> *>(pt_smem);
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int g = lane >> 2, tq = lane & 3;
+    const int bh = blockIdx.y, b = bh / H;
+    const int r0 = blockIdx.x * kPtR;
+    const int wr = 16 * (warp & 1), wd = (warp >> 1) * (D / 2);
+    const float *vh = vhat + (size_t)bh * nbr * D;
+    const float *lh = L + (size_t)bh * nbr * nbr;
+    const bool l16 = (nbr & 3) == 0;
+    auto stage = [&](int c0, int bf) {
+        for (int i = t; i < kPtC * D / 4; i += kPtThreads) {
+            const int c = i / (D / 4), d4 = i % (D / 4);
+            if (c0 + c < nbr) cp_async16(&sh.v[bf][c][4 * d4], vh + (size_t)(c0 + c) * D + 4 * d4);
+            else *reinterpret_cast<float4 *>(&sh.v[bf][c][4 * d4]) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (l16) {
+            for (int i = t; i < kPtR * kPtC / 4; i += kPtThreads) {
+                const int r = i / (kPtC / 4), c4 = 4 * (i % (kPtC / 4));
+                if (r0 + r < nbr && c0 + c4 < nbr)
+                    cp_async16(&sh.l[bf][r][c4], lh + (size_t)(r0 + r) * nbr + c0 + c4);
+                else
+                    *reinterpret_cast<float4 *>(&sh.l[bf][r][c4]) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else {
+            for (int i = t; i < kPtR * kPtC; i += kPtThreads) {
+                const int r = i / kPtC, c = i % kPtC;
+                if (r0 + r < nbr && c0 + c < nbr) cp_async4(&sh.l[bf][r][c], lh + (size_t)(r0 + r) * nbr + c0 + c);
+                else sh.l[bf][r][c] = 0.0f;
+            }
+        }
+        if (t < kPtC) {
+            if (c0 + t < nbr) cp_async4(&sh.cntc[bf][t], cnt + (size_t)b * nbr + c0 + t);
+            else sh.cntc[bf][t] = 0;
+        } else if (t < kPtC + 2 * kPtR) {
+            const int r = (t - kPtC) >> 1, ws = (t - kPtC) & 1;
+            const int w = (c0 >> 5) + ws;   // c0 is a multiple of 64
+            if (r0 + r < nbr && w < wpr) cp_async4(&sh.selw[bf][r][ws], bitmap + ((size_t)bh * nbr + r0 + r) * wpr + w);
+            else sh.selw[bf][r][ws] = ~0u;
+        }
+    };
+    // this thread's two rows: wr + g and wr + g + 8 of the CTA
+    const int ra = r0 + wr + g, rb = ra + 8;
+    const float ma = ra < nbr ? mlo[(size_t)bh * nbr + ra] : 0.0f;
+    const float mb = rb < nbr ? mlo[(size_t)bh * nbr + rb] : 0.0f;
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+    float la = 0.0f, lb = 0.0f;
+    const int ntiles_all = (nbr + kPtC - 1) / kPtC;
+    const int split = blockIdx.z, nsplit = gridDim.z;
+    const int t_begin = split * ntiles_all / nsplit, t_end = (split + 1) * ntiles_all / nsplit;
+    const int ntiles = t_end - t_begin;
+    if (ntiles > 0) stage(t_begin * kPtC, 0);
+    cp_async_commit();
+    for (int it = 0; it < ntiles; ++it) {
+        const int bf = it & 1;
+        if (it + 1 < ntiles) stage((t_begin + it + 1) * kPtC, bf ^ 1);   // that buffer was last read before the barrier below
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();   // tile it landed and is visible
+        const unsigned long long sa = (unsigned long long)sh.selw[bf][wr + g][0] |
+                                      ((unsigned long long)sh.selw[bf][wr + g][1] << 32);
+        const unsigned long long sb = (unsigned long long)sh.selw[bf][wr + g + 8][0] |
+                                      ((unsigned long long)sh.selw[bf][wr + g + 8][1] << 32);
+#pragma unroll 2
+        for (int ks = 0; ks < kPtC / 8; ++ks) {
+            const int c = 8 * ks + tq;
+            const int cc0 = sh.cntc[bf][c], cc1 = sh.cntc[bf][c + 4];
+            float w[4];
+            w[0] = (cc0 > 0 && !((sa >> c) & 1ull)) ? (float)cc0 * expf(sh.l[bf][wr + g][c] - ma) : 0.0f;
+            w[1] = (cc0 > 0 && !((sb >> c) & 1ull)) ? (float)cc0 * expf(sh.l[bf][wr + g + 8][c] - mb) : 0.0f;
+            w[2] = (cc1 > 0 && !((sa >> (c + 4)) & 1ull)) ? (float)cc1 * expf(sh.l[bf][wr + g][c + 4] - ma) : 0.0f;
+            w[3] = (cc1 > 0 && !((sb >> (c + 4)) & 1ull)) ? (float)cc1 * expf(sh.l[bf][wr + g + 8][c + 4] - mb) : 0.0f;
+            la += w[0] + w[2];
+            lb += w[1] + w[3];
+            const unsigned int af[4] = {to_tf32(w[0]), to_tf32(w[1]), to_tf32(w[2]), to_tf32(w[3])};
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const unsigned int b0 = to_tf32(sh.v[bf][c][wd + 8 * n + g]);
+                const unsigned int b1 = to_tf32(sh.v[bf][c + 4][wd + 8 * n + g]);
+                mma_tf32(acc[n], af, b0, b1);
+            }
+        }
+        __syncthreads();   // this tile's buffers are free
+    }
+    // row sums over the four lanes of a row
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+        la += __shfl_xor_sync(0xffffffffu, la, o);
+        lb += __shfl_xor_sync(0xffffffffu, lb, o);
+    }
+    const size_t plane = (size_t)gridDim.y * nbr;   // rows of all heads
+    float *od = nsplit == 1 ? olo : opart + (size_t)split * plane * D;
+    float *ld = nsplit == 1 ? llo : lpart + (size_t)split * plane;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const int d = wd + 8 * n + 2 * tq;
+        if (ra < nbr) *reinterpret_cast<float2 *>(od + ((size_t)bh * nbr + ra) * D + d) = make_float2(acc[n][0], acc[n][1]);
+        if (rb < nbr) *reinterpret_cast<float2 *>(od + ((size_t)bh * nbr + rb) * D + d) = make_float2(acc[n][2], acc[n][3]);
+    }
+    if (tq == 0 && (warp >> 1) == 0) {
+        if (ra < nbr) ld[(size_t)bh * nbr + ra] = la;
+        if (rb < nbr) ld[(size_t)bh * nbr + rb] = lb;
+    }
+}
+
+// Sums the split partials of the low-resolution part in split order: one
+// thread per four elements of O (and per row of the normaliser).
+template <int D>
+__global__ void __launch_bounds__(256)
+lowres_pv_merge_kernel(const float *__restrict__ opart, const float *__restrict__ lpart, int nsplit, int rows,
+                       float *__restrict__ olo, float *__restrict__ llo) {
+    pdl_wait();
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;   // float4 index
+    const int n4 = rows * (D / 4);
+    if (i < n4) {
+        float4 a = reinterpret_cast<const float4 *>(opart)[i];
+        for (int sp = 1; sp < nsplit; ++sp) {
+            const float4 b = reinterpret_cast<const float4 *>(opart + (size_t)sp * rows * D)[i];
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+        }
+        reinterpret_cast<float4 *>(olo)[i] = a;
+    }
+    if (i < rows) {
+        float l = lpart[i];
+        for (int sp = 1; sp < nsplit; ++sp) l += lpart[(size_t)sp * rows + i];
+        llo[i] = l;
+    }
+}
+
 template <int R>
 cudaError_t launch_keys_rt(const Problem &p, const Workspace &w, const float *L, cudaStream_t s) {
     const size_t smem = sizeof(int) * (size_t)p.nbr + sizeof(unsigned int) * (1u << kHist0Bits);
@@ -423,6 +602,16 @@ cudaError_t launch_lowres_keys(const Problem &p, const Workspace &w, float *logi
     return launch_keys_rt<8>(p, w, L, s);
 }
 
+// Column splits of the tensor-core low-resolution kernel: enough CTAs for
+// about four per SM, at most kPtMaxSplits and one 64-column tile per split.
+int lowres_pv_splits(const Problem &p) {
+    if (p.dtype != 0) return 1;
+    const long long ctas = (long long)((p.nbr + kPtR - 1) / kPtR) * p.BH;
+    const long long want = (4LL * device_sm_count() + ctas - 1) / ctas;
+    const int ntiles = (p.nbr + kPtC - 1) / kPtC;
+    return (int)std::max<long long>(1, std::min<long long>({want, (long long)kPtMaxSplits, (long long)ntiles}));
+}
+
 cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, const float *logit_out, cudaStream_t s) {
     const float *L = logit_out ? logit_out : w.lo_logits;
     const float *vhat = w.pooled + (size_t)2 * p.BH * p.nbr * p.D;
@@ -434,6 +623,28 @@ cudaError_t launch_lowres_pv(const Problem &p, const Workspace &w, const float *
                                 (const unsigned int *)w.bitmap, w.words_per_row, (const int *)w.cnt, vhat, p.H,
                                 p.nbr, w.olo, w.llo);
     };
+    if (p.dtype == 0) {   // bf16 problems: tf32 tensor-core products
+        const int nsplit = lowres_pv_splits(p);
+        const dim3 tgrid((unsigned)((p.nbr + kPtR - 1) / kPtR), (unsigned)p.BH, (unsigned)nsplit);
+        auto run_tc = [&](auto kern, size_t smem) -> cudaError_t {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            return launch_dependent(kern, tgrid, dim3(kPtThreads), smem, s, L, (const float *)w.mlo,
+                                    (const unsigned int *)w.bitmap, w.words_per_row, (const int *)w.cnt, vhat, p.H,
+                                    p.nbr, w.olo, w.llo, w.lo_opart, w.lo_lpart);
+        };
+        cudaError_t e = p.D == 64 ? run_tc(lowres_pv_tf32_kernel<64>, sizeof(PtSmem<64>))
+                                  : run_tc(lowres_pv_tf32_kernel<32>, sizeof(PtSmem<32>));
+        if (e != cudaSuccess || nsplit == 1) return e;
+        const int rows = p.BH * p.nbr;
+        const int mgrid = (rows * (p.D / 4) + 255) / 256;
+        return p.D == 64 ? launch_dependent(lowres_pv_merge_kernel<64>, dim3(mgrid), dim3(256), 0, s,
+                                            (const float *)w.lo_opart, (const float *)w.lo_lpart, nsplit, rows, w.olo,
+                                            w.llo)
+                         : launch_dependent(lowres_pv_merge_kernel<32>, dim3(mgrid), dim3(256), 0, s,
+                                            (const float *)w.lo_opart, (const float *)w.lo_lpart, nsplit, rows, w.olo,
+                                            w.llo);
+    }
     return p.D == 64 ? run(lowres_pv_kernel<64>, sizeof(PvSmem<64>)) : run(lowres_pv_kernel<32>, sizeof(PvSmem<32>));
 }
 

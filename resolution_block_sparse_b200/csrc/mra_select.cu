@@ -33,8 +33,11 @@ namespace {
 constexpr int kScanWarps = 8;
 constexpr int kShift0 = kHist1Bits + kHist2Bits;
 
-// One warp per block row.  The row's candidates are counted first so that one
-// atomic per row reserves their slots.
+// One warp per block row, in groups of kScanChunks 32-column chunks: all of a
+// group's loads are issued before any is used, the group's keys stay in
+// registers, and one atomic per group reserves its candidates' slots.
+constexpr int kScanChunks = 16;
+
 __global__ void __launch_bounds__(32 * kScanWarps)
 select_scan_kernel(const unsigned long long *__restrict__ keys, const SelState *__restrict__ state, int nbr,
                    long long nbr2, int rows, int wpr, unsigned int *__restrict__ bitmap,
@@ -48,39 +51,48 @@ select_scan_kernel(const unsigned long long *__restrict__ keys, const SelState *
     const int bh = row / nbr, r = row - bh * nbr;
     const unsigned long long b0 = state[bh].prefix >> kShift0;   // the bucket's first digit
     const unsigned long long *kr = keys + (size_t)bh * nbr2 + (size_t)r * nbr;
-    const unsigned int lt_mask = (1u << lane) - 1u;
-    int ncand = 0, nabove = 0;
-    for (int c0 = 0; c0 < nbr; c0 += 32) {
-        const int c = c0 + lane;
-        const unsigned long long d0 = c < nbr ? (__ldcg(kr + c) >> kShift0) : 0ull;
-        const unsigned int above = __ballot_sync(0xffffffffu, c < nbr && d0 > b0);
-        const unsigned int inb = __ballot_sync(0xffffffffu, c < nbr && d0 == b0);
-        if (lane == 0) {
-            bitmap[(size_t)row * wpr + (c0 >> 5)] = above;
-            tiebits[(size_t)row * wpr + (c0 >> 5)] = 0u;
-        }
-        ncand += __popc(inb);
-        nabove += __popc(above);
-    }
-    if (lane == 0) above_cnt[row] = nabove;
-    if (ncand == 0) return;
-    int base = 0;
-    if (lane == 0) base = atomicAdd(&ccount[bh], ncand);
-    base = __shfl_sync(0xffffffffu, base, 0);
     unsigned long long *ck = cand_key + (size_t)bh * nbr2;
     int *ci = cand_idx + (size_t)bh * nbr2;
-    for (int c0 = 0; c0 < nbr; c0 += 32) {
-        const int c = c0 + lane;
-        const unsigned long long key = c < nbr ? __ldcg(kr + c) : 0ull;
-        const bool m = c < nbr && (key >> kShift0) == b0;
-        const unsigned int inb = __ballot_sync(0xffffffffu, m);
-        if (m) {
-            const int pos = base + __popc(inb & lt_mask);
-            ck[pos] = key;
-            ci[pos] = r * nbr + c;
+    const unsigned int lt_mask = (1u << lane) - 1u;
+    int nabove = 0;
+    for (int g0 = 0; g0 < nbr; g0 += 32 * kScanChunks) {
+        unsigned long long kv[kScanChunks];
+#pragma unroll
+        for (int j = 0; j < kScanChunks; ++j) {
+            const int c = g0 + 32 * j + lane;
+            kv[j] = c < nbr ? __ldcg(kr + c) : 0ull;
         }
-        base += __popc(inb);
+        unsigned int inb[kScanChunks];
+        int ncand = 0;
+#pragma unroll
+        for (int j = 0; j < kScanChunks; ++j) {
+            const int c0 = g0 + 32 * j;
+            const int c = c0 + lane;
+            const unsigned long long d0 = kv[j] >> kShift0;
+            const unsigned int above = __ballot_sync(0xffffffffu, c < nbr && d0 > b0);
+            inb[j] = __ballot_sync(0xffffffffu, c < nbr && d0 == b0);
+            if (lane == 0 && c0 < nbr) {
+                bitmap[(size_t)row * wpr + (c0 >> 5)] = above;
+                tiebits[(size_t)row * wpr + (c0 >> 5)] = 0u;
+            }
+            ncand += __popc(inb[j]);
+            nabove += __popc(above);
+        }
+        if (ncand == 0) continue;
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&ccount[bh], ncand);
+        base = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+        for (int j = 0; j < kScanChunks; ++j) {
+            if ((inb[j] >> lane) & 1u) {
+                const int pos = base + __popc(inb[j] & lt_mask);
+                ck[pos] = kv[j];
+                ci[pos] = r * nbr + g0 + 32 * j + lane;
+            }
+            base += __popc(inb[j]);
+        }
     }
+    if (lane == 0) above_cnt[row] = nabove;
 }
 
 constexpr int kFinThreads = 1024;
@@ -165,7 +177,7 @@ select_finalize_kernel(SelState *__restrict__ state, const unsigned long long *_
             warp_hist_add(h, (unsigned)(key >> shift) & 0xfffu, i < n && (key >> hi) == want);
         }
         __syncthreads();
-        find_bucket<kFinThreads>([h](int i) { return h[i]; }, kHistBins, need, s_tmp, &s_bin, &s_need);
+        find_bucket_smem<kFinThreads, kHistBins>(h, need, s_tmp, &s_bin, &s_need);
         const int bin = s_bin;
         const unsigned int bneed = s_need;
         const bool whole = bneed == h[bin];
