@@ -145,3 +145,24 @@ def test_invalid_arguments_do_not_launch():
     with pytest.raises(mra.MraError) as e:
         mra.mra_attention_fwd(q48, q48, q48, None, torch.empty_like(q48), 1, 0, 0, 0)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("N", [4096, 8192])
+def test_exact_ties_take_smallest_indices(N, mode):
+    """Every token has the same Q and the same K, so every low-resolution logit
+    is equal, every key's x is exactly 0 and the keys differ only by the
+    priors' tier: the k-th key sits among hundreds of exactly equal keys.  The
+    selection takes the equal keys of smallest flat index r * nbr + c, on the
+    single-kernel selection (N=4096, 128 x 128 blocks) and on the multi-kernel
+    one (N=8192).  Near-tie tolerance does not apply: the sets must be equal."""
+    d = random_inputs(1, 2, N, 64, dtype=torch.bfloat16, seed=77 + N + mode, v_scale=1.0)
+    base = torch.linspace(-1.0, 1.0, 64)
+    d["q"] = base.expand(1, 2, N, 64).to(torch.bfloat16).contiguous()
+    d["k"] = (0.5 * base.flip(0)).expand(1, 2, N, 64).to(torch.bfloat16).contiguous()
+    kw = dict(block_per_row=2, approx_mode=mode, first_n=1, diag_n=1)
+    gpu = tl.run_gpu(d, **kw)
+    ora = tl.run_oracle(d, **kw)
+    for bh in range(2):
+        np.testing.assert_array_equal(gpu["sel"][bh], ora["sel"][bh], err_msg=f"head {bh}")
+    tl.compare(d, gpu, ora)
