@@ -384,9 +384,11 @@ lowres_pv_kernel(const float *__restrict__ L, const float *__restrict__ mlo, con
 }
 
 // The same low-resolution part on the tensor cores for bf16 problems:
-// O_lo = W V-hat as mma.sync m16n8k8 with tf32 operands (W and V-hat rounded
-// to tf32, 2^-11 relative, far inside the bf16 output's rounding) and fp32
-// accumulation; the normaliser llo sums the fp32 weights.  A CTA covers
+// O_lo = W V-hat as mma.sync m16n8k8 with tf32 operands (the fp32 bits of W
+// and V-hat are passed as they are; the tensor core reads their top 19 bits,
+// 2^-10 relative, far inside the bf16 output's rounding) and fp32
+// accumulation; the weights use the special-function unit's 2^x (about 2 ulp)
+// and the normaliser llo sums the fp32 weights.  A CTA covers
 // kPtR = 32 block rows with four warps: warp w takes rows 16 (w & 1) ..
 // + 15 and head dims (w >> 1) D/2 .. + D/2 - 1, forming the weights of its A
 // fragments itself (cnt_c exp(l - rowmax) for unselected valid blocks) from
@@ -406,10 +408,12 @@ struct PtSmem {
     unsigned int selw[2][kPtR][2];
 };
 
-__device__ __forceinline__ unsigned int to_tf32(float x) {
-    unsigned int r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+constexpr float kLog2eLo = 1.4426950408889634f;
+// 2^x on the special-function unit (ex2.approx.ftz, about 2 ulp)
+__device__ __forceinline__ float sfu_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ void mma_tf32(float (&c)[4], const unsigned int (&a)[4], unsigned int b0, unsigned int b1) {
@@ -471,8 +475,9 @@ lowres_pv_tf32_kernel(const float *__restrict__ L, const float *__restrict__ mlo
     };
     // this thread's two rows: wr + g and wr + g + 8 of the CTA
     const int ra = r0 + wr + g, rb = ra + 8;
-    const float ma = ra < nbr ? mlo[(size_t)bh * nbr + ra] : 0.0f;
-    const float mb = rb < nbr ? mlo[(size_t)bh * nbr + rb] : 0.0f;
+    // exp(l - m) = 2^(l log2e - m log2e)
+    const float ma = (ra < nbr ? mlo[(size_t)bh * nbr + ra] : 0.0f) * kLog2eLo;
+    const float mb = (rb < nbr ? mlo[(size_t)bh * nbr + rb] : 0.0f) * kLog2eLo;
     float acc[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
@@ -498,17 +503,18 @@ lowres_pv_tf32_kernel(const float *__restrict__ L, const float *__restrict__ mlo
             const int c = 8 * ks + tq;
             const int cc0 = sh.cntc[bf][c], cc1 = sh.cntc[bf][c + 4];
             float w[4];
-            w[0] = (cc0 > 0 && !((sa >> c) & 1ull)) ? (float)cc0 * expf(sh.l[bf][wr + g][c] - ma) : 0.0f;
-            w[1] = (cc0 > 0 && !((sb >> c) & 1ull)) ? (float)cc0 * expf(sh.l[bf][wr + g + 8][c] - mb) : 0.0f;
-            w[2] = (cc1 > 0 && !((sa >> (c + 4)) & 1ull)) ? (float)cc1 * expf(sh.l[bf][wr + g][c + 4] - ma) : 0.0f;
-            w[3] = (cc1 > 0 && !((sb >> (c + 4)) & 1ull)) ? (float)cc1 * expf(sh.l[bf][wr + g + 8][c + 4] - mb) : 0.0f;
+            w[0] = (cc0 > 0 && !((sa >> c) & 1ull)) ? (float)cc0 * sfu_exp2(fmaf(sh.l[bf][wr + g][c], kLog2eLo, -ma)) : 0.0f;
+            w[1] = (cc0 > 0 && !((sb >> c) & 1ull)) ? (float)cc0 * sfu_exp2(fmaf(sh.l[bf][wr + g + 8][c], kLog2eLo, -mb)) : 0.0f;
+            w[2] = (cc1 > 0 && !((sa >> (c + 4)) & 1ull)) ? (float)cc1 * sfu_exp2(fmaf(sh.l[bf][wr + g][c + 4], kLog2eLo, -ma)) : 0.0f;
+            w[3] = (cc1 > 0 && !((sb >> (c + 4)) & 1ull)) ? (float)cc1 * sfu_exp2(fmaf(sh.l[bf][wr + g + 8][c + 4], kLog2eLo, -mb)) : 0.0f;
             la += w[0] + w[2];
             lb += w[1] + w[3];
-            const unsigned int af[4] = {to_tf32(w[0]), to_tf32(w[1]), to_tf32(w[2]), to_tf32(w[3])};
+            const unsigned int af[4] = {__float_as_uint(w[0]), __float_as_uint(w[1]), __float_as_uint(w[2]),
+                                        __float_as_uint(w[3])};
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
-                const unsigned int b0 = to_tf32(sh.v[bf][c][wd + 8 * n + g]);
-                const unsigned int b1 = to_tf32(sh.v[bf][c + 4][wd + 8 * n + g]);
+                const unsigned int b0 = __float_as_uint(sh.v[bf][c][wd + 8 * n + g]);
+                const unsigned int b1 = __float_as_uint(sh.v[bf][c + 4][wd + 8 * n + g]);
                 mma_tf32(acc[n], af, b0, b1);
             }
         }

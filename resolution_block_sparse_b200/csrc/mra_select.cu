@@ -97,6 +97,7 @@ select_scan_kernel(const unsigned long long *__restrict__ keys, const SelState *
 
 constexpr int kFinThreads = 1024;
 constexpr int kFinWarps = kFinThreads / 32;
+constexpr int kFinStage = 4096;   // candidates kept in shared memory (the rest are read from L2)
 
 // Exclusive scan of one int per thread over the block; returns the prefix and
 // writes the block total to *total.
@@ -147,10 +148,12 @@ select_finalize_kernel(SelState *__restrict__ state, const unsigned long long *_
                        int *__restrict__ row_start, int *__restrict__ row_take, WorkItem *__restrict__ items,
                        int *__restrict__ head_items, unsigned int *__restrict__ status) {
     pdl_wait();
-    extern __shared__ __align__(16) int fin_smem[];
-    unsigned int *h = reinterpret_cast<unsigned int *>(fin_smem);   // [kHistBins]
-    int *s_gt = fin_smem + kHistBins;                                // [nbr] keys above T per row
-    int *s_eq = s_gt + nbr;                                          // [nbr] keys equal to T per row
+    extern __shared__ __align__(16) unsigned long long fin_smem[];
+    unsigned long long *s_ck = fin_smem;                                           // [kFinStage] candidate keys
+    int *s_ci = reinterpret_cast<int *>(s_ck + kFinStage);                          // [kFinStage] their indices
+    unsigned int *h = reinterpret_cast<unsigned int *>(s_ci + kFinStage);          // [kHistBins]
+    int *s_gt = reinterpret_cast<int *>(h + kHistBins);                             // [nbr] keys above T per row
+    int *s_eq = s_gt + nbr;                                                         // [nbr] keys equal to T per row
     __shared__ unsigned int s_tmp[kFinThreads];
     __shared__ int s_warp[32];
     __shared__ int s_bin;
@@ -158,11 +161,23 @@ select_finalize_kernel(SelState *__restrict__ state, const unsigned long long *_
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int bh = blockIdx.x;
     const int n = ccount[bh];
-    const unsigned long long *ck = cand_key + (size_t)bh * nbr2;
-    const int *ci = cand_idx + (size_t)bh * nbr2;
+    const unsigned long long *gck = cand_key + (size_t)bh * nbr2;
+    const int *gci = cand_idx + (size_t)bh * nbr2;
     unsigned long long prefix = state[bh].prefix;
     unsigned int need = state[bh].need;
     int sh = kShift0;
+    // the row counts of the scan and the candidates, all loads issued at once
+    for (int r = t; r < nbr; r += kFinThreads) {
+        s_gt[r] = __ldcg(above_cnt + (size_t)bh * nbr + r);
+        s_eq[r] = 0;
+    }
+    for (int i = t; i < min(n, kFinStage); i += kFinThreads) {
+        s_ck[i] = __ldcg(gck + i);
+        s_ci[i] = __ldcg(gci + i);
+    }
+    __syncthreads();
+    auto cand_key_at = [&](int i) { return i < kFinStage ? s_ck[i] : __ldcg(gck + i); };
+    auto cand_idx_at = [&](int i) { return i < kFinStage ? s_ci[i] : __ldcg(gci + i); };
     // the two lower digits over the candidates (every candidate matches the
     // first digit); a digit whose bucket is taken whole ends the search
     for (int pass = 1; pass <= 2; ++pass) {
@@ -173,7 +188,7 @@ select_finalize_kernel(SelState *__restrict__ state, const unsigned long long *_
         __syncthreads();
         for (int i0 = warp * 32; i0 < n; i0 += kFinThreads) {
             const int i = i0 + lane;
-            const unsigned long long key = i < n ? __ldcg(ck + i) : ~0ull;
+            const unsigned long long key = i < n ? cand_key_at(i) : ~0ull;
             warp_hist_add(h, (unsigned)(key >> shift) & 0xfffu, i < n && (key >> hi) == want);
         }
         __syncthreads();
@@ -200,14 +215,9 @@ select_finalize_kernel(SelState *__restrict__ state, const unsigned long long *_
     // cleared by the scan)
     unsigned int *bm = bitmap + (size_t)bh * nbr * wpr;
     unsigned int *tb = tiebits + (size_t)bh * nbr * wpr;
-    for (int r = t; r < nbr; r += kFinThreads) {
-        s_gt[r] = __ldcg(above_cnt + (size_t)bh * nbr + r);
-        s_eq[r] = 0;
-    }
-    __syncthreads();
     for (int i = t; i < n; i += kFinThreads) {
-        const unsigned long long kk = __ldcg(ck + i) >> sh;
-        const int idx = __ldcg(ci + i);
+        const unsigned long long kk = cand_key_at(i) >> sh;
+        const int idx = cand_idx_at(i);
         const int r = idx / nbr, c = idx - r * nbr;
         if (kk > Tsh) {
             atomicOr(&bm[r * wpr + (c >> 5)], 1u << (c & 31));
@@ -322,7 +332,8 @@ cudaError_t launch_select_scan(const Problem &p, const Workspace &w, cudaStream_
 }
 
 cudaError_t launch_select_finalize(const Problem &p, const Workspace &w, int32_t *sel_out, cudaStream_t s) {
-    const size_t smem = sizeof(int) * ((size_t)kHistBins + 2 * (size_t)p.nbr);
+    const size_t smem = (sizeof(unsigned long long) + sizeof(int)) * kFinStage +
+                        sizeof(int) * ((size_t)kHistBins + 2 * (size_t)p.nbr);
     cudaError_t e = cudaFuncSetAttribute(select_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
