@@ -55,12 +55,6 @@ struct FusedSmem {
     int flag;
 };
 
-__device__ __forceinline__ int band(int r, int c, int g) {
-    if (g <= 0) return 0;
-    const int off = c - r;
-    return (off >= -(g / 2) && off <= (g + 1) / 2 - 1) ? 1 : 0;
-}
-
 // element (t, d) of a head tensor in shared memory: bf16 tensors are stored
 // as swizzled [32][D] tiles (the layout the tensor-core fragments read),
 // fp32 tensors row-major
@@ -370,15 +364,10 @@ fused_small_kernel(FusedArgs a) {
             if (fs.cntf[cc] > 0.0f) m = fmaxf(m, fs.lg[r * nbr + cc]);
         if (m == -INFINITY) m = 0.0f;
         if (c == 0) fs.mlo[r] = m;
-        float x = fs.lg[tid] - m;
-        if (x == 0.0f) x = 0.0f;   // canonical +0
-        if (!(fabsf(x) < 2500.0f)) fs.flag = 1;
-        int tier = 0;
-        if (a.first_n > 0 && (r < a.first_n || c < a.first_n)) ++tier;
-        tier += band(r, c, a.diag_n);
-        if (!(fs.cntf[r] > 0.0f)) tier -= 2;
-        if (!(fs.cntf[c] > 0.0f)) tier -= 2;
-        fs.keys[tid] = ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
+        int range_err = 0;
+        fs.keys[tid] = selection_key(fs.lg[tid], m, r, c, a.first_n, a.diag_n, !(fs.cntf[r] > 0.0f),
+                                     !(fs.cntf[c] > 0.0f), range_err);
+        if (range_err) fs.flag = 1;
     }
     __syncthreads();
     // ------------------------------------------------ global top-k: rank count, ties to the smaller index

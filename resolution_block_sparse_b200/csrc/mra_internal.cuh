@@ -280,6 +280,30 @@ __device__ __forceinline__ unsigned int float_order_bits(float x) {
 __device__ __forceinline__ float float_from_order_bits(unsigned int u) {
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
+// Diagonal prior of width g: key-block offsets c - r in -(g/2) .. (g+1)/2 - 1.
+__device__ __forceinline__ int prior_band(int r, int c, int g) {
+    if (g <= 0) return 0;
+    const int off = c - r;
+    return (off >= -(g / 2) && off <= (g + 1) / 2 - 1) ? 1 : 0;
+}
+// Selection key of block (r, c) (page "深入解析 Transformers 中的 MRA 模型",
+// section "源码级原理", step two): the additive priors as the exact pair
+// (tier, x), x = l - rowmax in fp32 (canonical +0), packed as
+// (tier + 4) << 32 | order bits of x.  range_err is set when |x| >= 2500,
+// where the pair's order could differ from the order of the biased sums.
+__device__ __forceinline__ unsigned long long selection_key(float l, float rowmax, int r, int c, int first_n,
+                                                            int diag_n, bool row_empty, bool col_empty,
+                                                            int &range_err) {
+    float x = l - rowmax;
+    if (x == 0.0f) x = 0.0f;
+    if (!(fabsf(x) < 2500.0f)) range_err = 1;
+    int tier = 0;
+    if (first_n > 0 && (r < first_n || c < first_n)) ++tier;
+    tier += prior_band(r, c, diag_n);
+    if (row_empty) tier -= 2;
+    if (col_empty) tier -= 2;
+    return ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
+}
 #endif
 
 }  // namespace mra

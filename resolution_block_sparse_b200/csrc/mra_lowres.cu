@@ -30,14 +30,6 @@ namespace mra {
 
 namespace {
 
-__device__ __forceinline__ int in_band(int r, int c, int g) {
-    if (g <= 0) return 0;
-    const int lo = -(g / 2);
-    const int hi = (g + 1) / 2 - 1;
-    const int off = c - r;
-    return (off >= lo && off <= hi) ? 1 : 0;
-}
-
 constexpr int kLowresThreads = 256;
 
 __device__ __forceinline__ void cp_async4(void *dst, const void *src) {
@@ -206,8 +198,7 @@ lowres_keys_kernel(const float *__restrict__ L, const float *__restrict__ pmax,
         const float m = rmax[r];
         const float *lrow = L + ((size_t)bh * nbr + gr) * nbr;
         unsigned long long *krow = keys + (size_t)bh * nbr2 + (size_t)gr * nbr;
-        const bool row_first = first_n > 0 && gr < first_n;
-        const int row_tier = cnts[gr] <= 0 ? -2 : 0;
+        const bool row_empty = cnts[gr] <= 0;
         for (int c0 = 0; c0 < nbr; c0 += 32 * kU) {
             float lv[kU];
 #pragma unroll
@@ -219,17 +210,9 @@ lowres_keys_kernel(const float *__restrict__ L, const float *__restrict__ pmax,
             for (int u = 0; u < kU; ++u) {
                 const int c = c0 + 32 * u + lane;
                 const bool act = c < nbr;
-                unsigned long long key = 0;
-                if (act) {
-                    float x = lv[u] - m;
-                    if (x == 0.0f) x = 0.0f;  // canonical +0
-                    if (!(fabsf(x) < 2500.0f)) flag = 1;
-                    int tier = row_tier + ((row_first || (first_n > 0 && c < first_n)) ? 1 : 0);
-                    tier += in_band(gr, c, diag_n);
-                    if (cnts[c] <= 0) tier -= 2;
-                    key = ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
-                    krow[c] = key;
-                }
+                const unsigned long long key =
+                    act ? selection_key(lv[u], m, gr, c, first_n, diag_n, row_empty, cnts[c] <= 0, flag) : 0ull;
+                if (act) krow[c] = key;
                 warp_hist_add(h0, (unsigned)(key >> 24), act);
             }
         }

@@ -62,14 +62,6 @@ __host__ __device__ constexpr int region_floats() {
     return ks_stride<D>() * kCT > kSelWords ? ks_stride<D>() * kCT : kSelWords;
 }
 
-__device__ __forceinline__ int band_of(int r, int c, int g) {
-    if (g <= 0) return 0;
-    const int lo = -(g / 2);
-    const int hi = (g + 1) / 2 - 1;
-    const int off = c - r;
-    return (off >= lo && off <= hi) ? 1 : 0;
-}
-
 __device__ __forceinline__ void cluster_arrive() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
 }
@@ -244,15 +236,7 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                 const bool ok = row_ok && c < nbr;
                 unsigned long long key = 0ull;
                 if (ok) {
-                    float x = lv[j] - m;
-                    if (x == 0.0f) x = 0.0f;   // canonical +0
-                    if (!(fabsf(x) < 2500.0f)) flag = 1;
-                    int tier = 0;
-                    if (first_n > 0 && (gr < first_n || c < first_n)) ++tier;
-                    tier += band_of(gr, c, diag_n);
-                    if (row_empty) tier -= 2;
-                    if (cnts[c] <= 0) tier -= 2;
-                    key = ((unsigned long long)(tier + 4) << 32) | (unsigned long long)float_order_bits(x);
+                    key = selection_key(lv[j], m, gr, c, first_n, diag_n, row_empty, cnts[c] <= 0, flag);
                     sk[rr * nbr + c] = key;
                     const size_t gi = (size_t)bh * nbr2 + (size_t)gr * nbr + c;
                     if (logit_out) logit_out[gi] = lv[j];
