@@ -63,6 +63,11 @@ SMALL = [
     (1, 1, 8192, 64, torch.bfloat16, 2, 0, 1, 0, None, 1.0),       # 32-item row: grouped merge
     (1, 1, 8192, 64, torch.bfloat16, 2, 1, 1, 0, [300], 1.0),
     (1, 1, 8192, 32, torch.float32, 2, 0, 1, 0, [300], 1.0),
+    # 130 x 130 blocks: ragged 64-column tiles of the logit map and of the
+    # low-resolution part (rows not 16-byte aligned), 5-word bitmap rows
+    (1, 2, 4160, 64, torch.bfloat16, 3, 0, 1, 1, [333], 1.0),
+    (1, 2, 4160, 64, torch.bfloat16, 3, 1, 2, 3, [333], 1.0),
+    (1, 1, 4160, 32, torch.float32, 3, 0, 1, 1, [70], 1.0),
 ]
 
 
