@@ -24,11 +24,13 @@
 //
 // Kernels: bwd_item (one CTA per forward work item: dQ of its rows in
 // registers, dK and dV of its key blocks added with vector fp32 atomics, the
-// transposed index traversal being the atomics' addresses), and in full mode
-// lowres_bwd_prep (A, B, R per row block), lowres_bwd_rows (dqhat) and
-// lowres_bwd_cols (dkhat, dvhat) on 32 x 32 tiles of (row block, key block)
-// pairs in shared memory, and lowres_bwd_scatter (block means to tokens).
-// All arithmetic is fp32 (FFMA).
+// transposed index traversal being the atomics' addresses), and in full mode,
+// launched before bwd_item, lowres_bwd_prep (A, B, R per row block; clears
+// the block-mean gradient planes), lowres_bwd_tile (one CTA per 64 x 64 tile
+// of (row block, key block) pairs: dl in shared memory, dqhat, dkhat and
+// dvhat partial sums from 4 x 4 register tiles added with fp32 atomics) and
+// lowres_bwd_scatter (block means to tokens; writes dQ, dK, dV, which the
+// item kernel then adds to). All arithmetic is fp32 (FFMA).
 #include <cuda_bf16.h>
 
 #include <algorithm>

@@ -36,6 +36,9 @@ CASES = [
     (1, 1, 8192, 64, torch.bfloat16, 4, 0, 1, 1, None),        # 256 x 256 blocks, full mode
     (1, 1, 8192, 32, torch.float32, 2, 0, 2, 3, [300]),        # fp32, padded, 256 x 256
     (1, 1, 16384, 64, torch.bfloat16, 8, 0, 1, 1, [500]),      # 512 x 512 blocks, full mode
+    # 130 x 130 blocks: ragged last 64 x 64 pair tile in both directions
+    (1, 2, 4160, 64, torch.bfloat16, 3, 0, 1, 1, [333]),
+    (1, 1, 4160, 32, torch.float32, 3, 0, 2, 3, [70]),
 ]
 
 
