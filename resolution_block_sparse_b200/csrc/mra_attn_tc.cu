@@ -12,17 +12,21 @@
 // i of the tile on tensor-memory lane i, so each softmax thread owns one query
 // row and its max and sum need no exchange between threads.  The tile runs
 // over the union of the four rows' selected key blocks (built by the group
-// plan), four key blocks per step:
-//   S = Q_128 . K_stack^T          (M = 128, N = 32 * blocks <= 128, K = 64)
-//   O += P . V_stack               (M = 128, N = 64, K = 32 * blocks; P read
-//                                   from tensor memory, V from the TMA tile)
-// A (row, key block) pair outside that row's selection gets no weight: the
-// warp owning the row (warp w of the softmax warps holds block row 4g+w, one
-// of the four TMEM lane quarters) skips the block entirely and writes zero P
-// there, so the exponentials computed are exactly those of the selected
-// blocks.  The row maximum is kept lazily (the exponent reference moves only
-// when the maximum grows by more than 2^8), so the accumulator in tensor
-// memory is rescaled rarely.
+// plan), two key blocks per step:
+//   S = Q_128 . K_stack^T          (M = 128, N = 32 * blocks <= 64, K = 64)
+//   O_j += P_j . V_j               (M = 128, N = 64, K = 32, for block j of
+//                                   the step; P read from tensor memory, V
+//                                   from the TMA tile)
+// Two softmax warps share each tensor-memory lane quarter: warp (w, j) owns
+// the 32 rows of block row 4g+w and key block j of every step, keeps its own
+// running maximum and sum for that half of the keys, and accumulates into its
+// own O_j; the halves are merged under a common maximum in the epilogue.  A
+// (row, key block) pair outside that row's selection gets no weight: its warp
+// skips the block and writes zero P there, so the exponentials computed are
+// exactly those of the selected blocks.  P (bf16) is written over the S
+// columns it was computed from.  The row maximum is kept lazily (the exponent
+// reference moves only when the maximum grows by more than 2^8), so the
+// accumulators in tensor memory are rescaled rarely.
 //
 // Work item = (group, chunk of at most gchunk union entries).  A group whose
 // union is longer is split over several items; each writes (max, sum, O) for
@@ -31,9 +35,9 @@
 // from a per-call counter and passes it to the other roles through a ring in
 // shared memory.
 //
-// Warp roles (two CTAs per SM, 256 tensor-memory columns each: S 128, P 64,
-// O 64): warps 0-3 softmax and epilogue, warp 4 TMA producer (Q per item, K
-// and V per step, two stages), warp 5 MMA issuer.  Every mbarrier wait is
+// Warp roles (two CTAs per SM, 256 tensor-memory columns each: S 2 x 64, O
+// 2 x 64): warps 0-7 softmax and epilogue, warp 8 TMA producer (Q per item, K
+// and V per step, four stages), warp 9 MMA issuer.  Every mbarrier wait is
 // bounded: on expiry the kernel raises MRA_DEV_TIMEOUT in the status word,
 // every role stops, the kernel waits (bounded) for its own loads and MMAs in
 // flight, frees its tensor memory and returns.
@@ -56,9 +60,10 @@ using namespace async;
 using namespace tc;
 using attn::kLog2e;
 
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 8;                    // two per tensor-memory lane quarter
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 32 * (kSoftWarps + 2);
 constexpr int kStack = 2;                        // key blocks per step (N = 64 keys)
 constexpr int kStages = 4;                       // K and V steps in flight
 constexpr int kRing = 4;                         // work items in flight
@@ -71,10 +76,11 @@ constexpr int kOffV = kOffK + kStages * kStackBytes;
 constexpr int kSmemBytes = kOffV + kStages * kStackBytes;   // 96 KB
 constexpr int kSmemAlloc = kSmemBytes + 1024;               // room to align the base to 1 KB
 constexpr uint32_t kTmemCols = 256;
-// S double-buffered (64 fp32 columns each), P double-buffered (64 bf16 keys
-// packed in 32 columns each), O (64 columns)
-constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
-constexpr uint32_t kSCols = 32 * kStack, kPCols = 16 * kStack;
+// S double-buffered (64 fp32 columns each; block j of a step in columns
+// 32j..32j+31, its P in bf16 over the first 16 of them), O_0 and O_1 (64
+// columns each)
+constexpr uint32_t kColS = 0, kColO = 128;
+constexpr uint32_t kSCols = 32 * kStack;
 constexpr float kRescale = 8.0f;                 // lazy-rescale threshold (log2 units)
 constexpr int kRows = 32 * kGroupRows;           // 128
 constexpr int kPartialFloats = kRows * (2 + 64); // m[128], l[128], O[128][64]
@@ -89,12 +95,12 @@ __host__ __device__ constexpr uint32_t idesc_s(int nblocks) {
 // O += P V: B = V read MN-major (d contiguous in the tile), N = 64
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
 
-__device__ __forceinline__ void named_sync() { asm volatile("bar.sync 1, 128;\n" ::: "memory"); }
-// Barrier over the 128 softmax threads that also ANDs a predicate.
+__device__ __forceinline__ void named_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+// Barrier over the 256 softmax threads that also ANDs a predicate.
 __device__ __forceinline__ bool named_sync_and(bool v) {
     uint32_t out;
     asm volatile(
-        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, 1, 128, p;\n"
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, 1, 256, p;\n"
         " selp.u32 %0, 1, 0, q;\n}\n"
         : "=r"(out)
         : "r"((uint32_t)v)
@@ -129,8 +135,9 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                   const __grid_constant__ CUtensorMap tv, const GArgs a) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) unsigned long long bar_qfull[2], bar_qempty[2], bar_kfull[kStages],
-        bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages], bar_sfull[2], bar_sfree[2], bar_pfull[2], bar_pvdone[2],
+        bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages], bar_sfull[2], bar_pfull[2], bar_pvdone[2],
         bar_ofull, bar_oempty, bar_ifull[kRing], bar_iempty[kRing], bar_fin;
+    __shared__ float2 s_ml[kStack][kRows];   // (max, sum) of each row's key-block halves
     __shared__ int s_ring[kRing];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort, s_last;
@@ -154,16 +161,15 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         }
         for (int i = 0; i < kRing; ++i) {
             mbar_init(saddr(&bar_ifull[i]), 1);
-            mbar_init(saddr(&bar_iempty[i]), 1 + kGroupRows);   // MMA thread + softmax warps
+            mbar_init(saddr(&bar_iempty[i]), 1 + kSoftWarps);   // MMA thread + softmax warps
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(saddr(&bar_sfull[i]), 1);
-            mbar_init(saddr(&bar_sfree[i]), kGroupRows);
-            mbar_init(saddr(&bar_pfull[i]), kGroupRows);
+            mbar_init(saddr(&bar_pfull[i]), kSoftWarps);
             mbar_init(saddr(&bar_pvdone[i]), 1);
         }
         mbar_init(saddr(&bar_ofull), 1);
-        mbar_init(saddr(&bar_oempty), kGroupRows);
+        mbar_init(saddr(&bar_oempty), kSoftWarps);
         mbar_init(saddr(&bar_fin), 1);
         s_iss_q = s_iss_k = s_iss_v = s_con_q = s_con_k = s_con_v = 0;
         s_abort = 0;
@@ -272,9 +278,12 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 if (p.first && npv > 0 && !waitb(&bar_oempty, (npv - 1) & 1)) return false;
                 tc_fence_after();
                 const uint32_t vb = sV + p.sg * kStackBytes;
-                for (int kk = 0; kk < 2 * p.nv; ++kk)
-                    mma_f16_ts(tmem + kColO, tmem + kColP + pb * kPCols + 8 * kk, sdesc(vb + kk * 2048, 16, 1024), kIdescPV,
-                               (p.first && kk == 0) ? 0u : 1u);
+                for (int j = 0; j < p.nv; ++j)
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk)
+                        mma_f16_ts(tmem + kColO + 64 * j, tmem + kColS + pb * kSCols + 32 * j + 8 * kk,
+                                   sdesc(vb + j * kTile + kk * 2048, 16, 1024), kIdescPV,
+                                   (p.first && kk == 0) ? 0u : 1u);
                 mma_commit(saddr(&bar_vempty[p.sg]));
                 mma_commit(saddr(&bar_pvdone[pb]));
                 if (p.last) {
@@ -302,9 +311,10 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     const int nv = min(kStack, it.ucount - st * kStack);
                     if (!(ok = waitb(&bar_kfull[sg], (t / kStages) & 1))) break;
                     s_con_k = t + 1;
-                    // S buffer t & 1 was last read by the softmax of step t - 2
+                    // S buffer t & 1 holds the P of step t - 2 until that
+                    // step's PV is done
                     const int sb = t & 1;
-                    if (t >= 2 && !(ok = waitb(&bar_sfree[sb], ((t >> 1) - 1) & 1))) break;
+                    if (t >= 2 && !(ok = waitb(&bar_pvdone[sb], ((t >> 1) - 1) & 1))) break;
                     if (st == 0) {
                         if (!(ok = waitb(&bar_qfull[qs], (qn >> 1) & 1))) break;
                         s_con_q = qn + 1;
@@ -333,11 +343,12 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             mbar_wait(saddr(&bar_fin), 0);
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else if (warp < kSoftWarps) {
         // ------------------------------------------------------------ softmax + epilogue
-        const uint32_t lq = (uint32_t)(warp * 32) << 16;   // this warp's TMEM lane quarter
-        const uint32_t tS = tmem + lq + kColS, tP = tmem + lq + kColP, tO = tmem + lq + kColO;
-        const int row = warp * 32 + lane;                   // row of the 128-row tile
+        const int wq = warp & 3, hh = warp >> 2;            // lane quarter, key-block half
+        const uint32_t lq = (uint32_t)(wq * 32) << 16;     // this warp's TMEM lane quarter
+        const uint32_t tS = tmem + lq + kColS + 32 * hh, tO = tmem + lq + kColO;
+        const int row = wq * 32 + lane;                     // row of the 128-row tile
         int n = 0, t = 0, on = 0;
         while (true) {
             const int slot = n % kRing;
@@ -350,7 +361,7 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             const GroupItem it = a.gitems[sidx];
             const int bh = it.group / a.ngroups, g = it.group - bh * a.ngroups;
             const int b = bh / a.H, h = bh - b * a.H;
-            const int r = g * kGroupRows + warp;   // this warp's block row
+            const int r = g * kGroupRows + wq;   // this warp's block row
             const bool row_ok = r < a.nbr;
             const int nst = (it.ucount + kStack - 1) / kStack;
             const int e0 = lane < it.ucount ? a.ucols[it.ustart + lane] : 0;
@@ -359,17 +370,10 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             float mref = -INFINITY, lsum = 0.0f;
             for (int st = 0; st < nst; ++st, ++t) {
                 const int nv = min(kStack, it.ucount - st * kStack);
-                int act = 0, part = 0, cb[kStack];
-#pragma unroll
-                for (int j = 0; j < kStack; ++j) {
-                    const int u = st * kStack + j;
-                    const int e = __shfl_sync(0xffffffffu, u < 32 ? e0 : e1, u & 31);
-                    cb[j] = e & 0xffff;
-                    if (j < nv && row_ok && ((e >> (kUnionRowShift + warp)) & 1)) {
-                        act |= 1 << j;
-                        if (e & kUnionPartial) part |= 1 << j;
-                    }
-                }
+                const int u = st * kStack + hh;
+                const int e = __shfl_sync(0xffffffffu, u < 32 ? e0 : e1, u & 31);
+                const bool act = hh < nv && row_ok && ((e >> (kUnionRowShift + wq)) & 1);
+                const bool part = act && (e & kUnionPartial);
                 const int sb = t & 1;
                 if (a.expire_first_wait && t == 0) {
                     // a wait whose limit has run out (test hook, see the launcher)
@@ -378,134 +382,133 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 }
                 waitb(&bar_sfull[sb], (t >> 1) & 1);
                 tc_fence_after();
-                float s[kStack][32];
+                float s[32];
+                if (act) {
+                    uint32_t raw[32];
+                    tmem_ld32(tS + sb * kSCols, raw);
+                    tmem_wait_ld_regs(raw);
 #pragma unroll
-                for (int j = 0; j < kStack; ++j) {
-                    if ((act >> j) & 1) {
-                        uint32_t raw[32];
-                        tmem_ld32(tS + sb * kSCols + 32 * j, raw);
-                        tmem_wait_ld_regs(raw);
+                    for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(raw[i]);
+                    // padded keys of partly padded key blocks take no weight
+                    if (part) {
+                        const unsigned kv = __ballot_sync(0xffffffffu, mrow[(e & 0xffff) * 32 + lane] > 0.0f);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) s[j][i] = __uint_as_float(raw[i]);
+                        for (int i = 0; i < 32; ++i)
+                            if (!((kv >> i) & 1u)) s[i] = -INFINITY;
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(saddr(&bar_sfree[sb]));
-                // padded keys of partly padded key blocks take no weight
-                if (part) {
-#pragma unroll
-                    for (int j = 0; j < kStack; ++j) {
-                        if ((part >> j) & 1) {
-                            const unsigned kv = __ballot_sync(0xffffffffu, mrow[cb[j] * 32 + lane] > 0.0f);
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (!((kv >> i) & 1u)) s[j][i] = -INFINITY;
-                        }
-                    }
-                }
-                float mx = -INFINITY;
-#pragma unroll
-                for (int j = 0; j < kStack; ++j)
-                    if ((act >> j) & 1)
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, s[j][i]);
-                const float mxs = mx * a.scale_log2;
-                float alpha = 1.0f;
+                float alpha = 1.0f, ls = 0.0f;
                 bool resc = false;
-                if (mxs > mref + kRescale) {
-                    if (mref != -INFINITY) {
-                        alpha = fast_exp2(mref - mxs);
-                        resc = true;
-                    }
-                    mref = mxs;
-                }
-                const float ref = (mref == -INFINITY) ? 0.0f : mref;
-                uint32_t pk[kStack][16];
-                float ls = 0.0f;
+                uint32_t pk[16];
+                if (act) {
+                    float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-                for (int j = 0; j < kStack; ++j) {
-                    if ((act >> j) & 1) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float p0 = fast_exp2(fmaf(s[j][2 * i], a.scale_log2, -ref));
-                            const float p1 = fast_exp2(fmaf(s[j][2 * i + 1], a.scale_log2, -ref));
-                            const __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
-                            pk[j][i] = *reinterpret_cast<const uint32_t *>(&hp);
-                            ls += p0 + p1;
+                    for (int i = 4; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], s[i]);
+                    const float mxs = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
+                    if (mxs > mref + kRescale) {
+                        if (mref != -INFINITY) {
+                            alpha = fast_exp2(mref - mxs);
+                            resc = true;
                         }
+                        mref = mxs;
                     }
+                    const float ref = (mref == -INFINITY) ? 0.0f : mref;
+                    float ls2 = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = fast_exp2(fmaf(s[2 * i], a.scale_log2, -ref));
+                        const float p1 = fast_exp2(fmaf(s[2 * i + 1], a.scale_log2, -ref));
+                        const __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
+                        pk[i] = *reinterpret_cast<const uint32_t *>(&hp);
+                        ls += p0;
+                        ls2 += p1;
+                    }
+                    ls += ls2;
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
                 }
                 lsum = fmaf(lsum, alpha, ls);
-                // P buffer sb is free once the PV of step t - 2 is done; O may
-                // be rescaled once every earlier PV (that of step t - 1) is done
-                if (t >= 2) waitb(&bar_pvdone[sb], ((t >> 1) - 1) & 1);
+                // O_j may be rescaled once every earlier PV (that of step t - 1)
+                // is done
                 const bool any_resc = __any_sync(0xffffffffu, resc);
-                if (any_resc && t >= 1) waitb(&bar_pvdone[sb ^ 1], ((t - 1) >> 1) & 1);
-                tc_fence_after();
                 if (any_resc) {
+                    if (t >= 1) waitb(&bar_pvdone[sb ^ 1], ((t - 1) >> 1) & 1);
+                    tc_fence_after();
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         uint32_t o[32];
-                        tmem_ld32(tO + 32 * half, o);
+                        tmem_ld32(tO + 64 * hh + 32 * half, o);
                         tmem_wait_ld_regs(o);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(tO + 32 * half, o);
+                        tmem_st32(tO + 64 * hh + 32 * half, o);
                     }
                 }
-#pragma unroll
-                for (int j = 0; j < kStack; ++j) {
-                    if (j < nv) {
-                        if ((act >> j) & 1) {
-                            tmem_st16(tP + sb * kPCols + 16 * j, pk[j]);
-                        } else {
-                            const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-                            tmem_st16(tP + sb * kPCols + 16 * j, z);
-                        }
-                    }
-                }
+                if (hh < nv) tmem_st16(tS + sb * kSCols, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(saddr(&bar_pfull[sb]));
             }
             // ---------------------------------------------------- epilogue
-            // O is read from tensor memory (or the partial slots) 32 columns
-            // at a time, so that at most half a row is held in registers
+            // the row's two key-block halves under one maximum; this warp then
+            // produces output columns 32*hh .. 32*hh+31 of its 32 rows
             const int chunk = it.chunk_info & 0xffff, nch = it.chunk_info >> 16;
+            s_ml[hh][row] = make_float2(mref, lsum);
+            named_sync();
+            const float2 oth = s_ml[hh ^ 1][row];
+            const float m0 = hh ? oth.x : mref, l0 = hh ? oth.y : lsum;
+            const float m1 = hh ? mref : oth.x, l1 = hh ? lsum : oth.y;
+            float m_hi = -INFINITY, l_hi = 0.0f, w0 = 0.0f, w1 = 0.0f;
+            if (l0 > 0.0f) m_hi = m0;
+            if (l1 > 0.0f) m_hi = fmaxf(m_hi, m1);
+            if (m_hi != -INFINITY) {
+                w0 = l0 > 0.0f ? fast_exp2(m0 - m_hi) : 0.0f;
+                w1 = l1 > 0.0f ? fast_exp2(m1 - m_hi) : 0.0f;
+                l_hi = fmaf(w0, l0, w1 * l1);
+            }
+            float o[32];
             if (nst > 0) {
                 waitb(&bar_ofull, on & 1);
                 ++on;
                 tc_fence_after();
+                {
+                    uint32_t raw[32];
+                    tmem_ld32(tO + 32 * hh, raw);
+                    tmem_wait_ld_regs(raw);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = w0 * __uint_as_float(raw[i]);
+                }
+                if (it.ucount >= 2) {   // O_1 holds a term only when the item has a second block
+                    uint32_t raw[32];
+                    tmem_ld32(tO + 64 + 32 * hh, raw);
+                    tmem_wait_ld_regs(raw);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = fmaf(w1, __uint_as_float(raw[i]), o[i]);
+                }
+                // both accumulators are free for the next item's first PV
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(saddr(&bar_oempty));
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = 0.0f;
             }
-            float m_hi = mref, l_hi = lsum;
             bool write = true;
             if (nch > 1) {
                 // split group: this item's (max, sum, O) to its slot; the last
                 // item of the group to arrive merges the slots
                 float *P = a.partial + (size_t)sidx * kPartialFloats;
-                P[row] = mref;
-                P[kRows + row] = lsum;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t o[32];
-                    if (nst > 0) {
-                        tmem_ld32(tO + 32 * half, o);
-                        tmem_wait_ld_regs(o);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = 0u;
-                    }
-                    uint4 *Po = reinterpret_cast<uint4 *>(P + 2 * kRows + row * 64 + 32 * half);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) Po[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+                if (hh == 0) {
+                    P[row] = m_hi;
+                    P[kRows + row] = l_hi;
                 }
-                if (nst > 0) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(saddr(&bar_oempty));
-                }
+                uint4 *Po = reinterpret_cast<uint4 *>(P + 2 * kRows + row * 64 + 32 * hh);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    Po[i] = make_uint4(__float_as_uint(o[4 * i]), __float_as_uint(o[4 * i + 1]),
+                                       __float_as_uint(o[4 * i + 2]), __float_as_uint(o[4 * i + 3]));
                 __threadfence();
                 named_sync();
                 if (tid == 0) s_last = (atomicAdd(&a.group_arrive[it.group], 1) == nch - 1);
@@ -539,6 +542,26 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     }
                     m_hi = M;
                     l_hi = L;
+                    // merged high-resolution part: this warp's 32 columns of
+                    // every item's O
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = 0.0f;
+                    for (int c = 0; c < nch; ++c) {
+                        const float *Pc = P0 + (size_t)c * kPartialFloats;
+                        const float lc = __ldcg(Pc + kRows + row);
+                        const float wc = (lc > 0.0f) ? fast_exp2(__ldcg(Pc + row) - m_hi) : 0.0f;
+                        const float4 *Oc = reinterpret_cast<const float4 *>(Pc + 2 * kRows + row * 64 + 32 * hh);
+                        float4 x[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) x[i] = __ldcg(Oc + i);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            o[4 * i] = fmaf(wc, x[i].x, o[4 * i]);
+                            o[4 * i + 1] = fmaf(wc, x[i].y, o[4 * i + 1]);
+                            o[4 * i + 2] = fmaf(wc, x[i].z, o[4 * i + 2]);
+                            o[4 * i + 3] = fmaf(wc, x[i].w, o[4 * i + 3]);
+                        }
+                    }
                     if (tid == 0) a.group_arrive[it.group] = 0;
                 }
             }
@@ -563,77 +586,27 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                         fb = be / den;
                     }
                 }
-                const float *olo_row = a.olo + (size_t)rg * 64;
-                __nv_bfloat16 *op = a.out + (size_t)b * a.ob + (size_t)h * a.oh + (size_t)(r * 32 + lane) * a.orow;
+                const float *olo_row = a.olo + (size_t)rg * 64 + 32 * hh;
+                __nv_bfloat16 *op = a.out + (size_t)b * a.ob + (size_t)h * a.oh + (size_t)(r * 32 + lane) * a.orow + 32 * hh;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float o[32];
-                    if (nch > 1) {
-                        // merged high-resolution part of the split group: the
-                        // O halves of two items in flight at once
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = 0.0f;
-                        const float *P0 = a.partial + (size_t)(sidx - chunk) * kPartialFloats;
-                        for (int c = 0; c < nch; c += 2) {
-                            float wc[2];
-                            float4 x[2][8];
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const float *Pc = P0 + (size_t)(c + u) * kPartialFloats;
-                                const bool in = c + u < nch;
-                                const float lc = in ? __ldcg(Pc + kRows + row) : 0.0f;
-                                const float mc = in ? __ldcg(Pc + row) : -INFINITY;
-                                wc[u] = (lc > 0.0f) ? fast_exp2(mc - m_hi) : 0.0f;
-                                const float4 *Oc = reinterpret_cast<const float4 *>(Pc + 2 * kRows + row * 64 + 32 * half);
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) x[u][i] = in ? __ldcg(Oc + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-                            }
-#pragma unroll
-                            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) {
-                                    o[4 * i] = fmaf(wc[u], x[u][i].x, o[4 * i]);
-                                    o[4 * i + 1] = fmaf(wc[u], x[u][i].y, o[4 * i + 1]);
-                                    o[4 * i + 2] = fmaf(wc[u], x[u][i].z, o[4 * i + 2]);
-                                    o[4 * i + 3] = fmaf(wc[u], x[u][i].w, o[4 * i + 3]);
-                                }
-                        }
-                    } else if (nst > 0) {
-                        uint32_t raw[32];
-                        tmem_ld32(tO + 32 * half, raw);
-                        tmem_wait_ld_regs(raw);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(raw[i]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = 0.0f;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float lo_v = lo ? __ldg(olo_row + 32 * half + i) : 0.0f;
-                        o[i] = fmaf(o[i], fa, lo_v * fb);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(op + 32 * half);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const __nv_bfloat162 h0 = __floats2bfloat162_rn(o[8 * i], o[8 * i + 1]);
-                        const __nv_bfloat162 h1 = __floats2bfloat162_rn(o[8 * i + 2], o[8 * i + 3]);
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[8 * i + 4], o[8 * i + 5]);
-                        const __nv_bfloat162 h3 = __floats2bfloat162_rn(o[8 * i + 6], o[8 * i + 7]);
-                        uint4 u;
-                        u.x = *reinterpret_cast<const uint32_t *>(&h0);
-                        u.y = *reinterpret_cast<const uint32_t *>(&h1);
-                        u.z = *reinterpret_cast<const uint32_t *>(&h2);
-                        u.w = *reinterpret_cast<const uint32_t *>(&h3);
-                        dst[i] = u;
-                    }
+                for (int i = 0; i < 32; ++i) {
+                    const float lo_v = lo ? __ldg(olo_row + i) : 0.0f;
+                    o[i] = fmaf(o[i], fa, lo_v * fb);
                 }
-            }
-            if (nch == 1 && nst > 0) {
-                // the accumulator is free for the next item's first PV
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(saddr(&bar_oempty));
+                uint4 *dst = reinterpret_cast<uint4 *>(op);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __nv_bfloat162 h0 = __floats2bfloat162_rn(o[8 * i], o[8 * i + 1]);
+                    const __nv_bfloat162 h1 = __floats2bfloat162_rn(o[8 * i + 2], o[8 * i + 3]);
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[8 * i + 4], o[8 * i + 5]);
+                    const __nv_bfloat162 h3 = __floats2bfloat162_rn(o[8 * i + 6], o[8 * i + 7]);
+                    uint4 u;
+                    u.x = *reinterpret_cast<const uint32_t *>(&h0);
+                    u.y = *reinterpret_cast<const uint32_t *>(&h1);
+                    u.z = *reinterpret_cast<const uint32_t *>(&h2);
+                    u.w = *reinterpret_cast<const uint32_t *>(&h3);
+                    dst[i] = u;
+                }
             }
         }
     }
