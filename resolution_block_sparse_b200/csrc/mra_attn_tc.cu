@@ -64,8 +64,9 @@ constexpr int kSoftWarps = 8;                    // two per tensor-memory lane q
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 32 * (kSoftWarps + 2);
-constexpr int kStack = 2;                        // key blocks per step (N = 64 keys)
-constexpr int kStages = 4;                       // K and V steps in flight
+constexpr int kStack = 4;                        // key blocks per step (N = 128 keys)
+constexpr int kHalf = kStack / 2;                // key blocks of a step per softmax warp
+constexpr int kStages = 2;                       // K and V steps in flight
 constexpr int kRing = 4;                         // work items in flight
 constexpr int kTile = 32 * 64 * 2;               // one 32-token block, bf16, 4 KB
 constexpr int kQBytes = kGroupRows * kTile;      // 128 query rows, 16 KB
@@ -76,11 +77,9 @@ constexpr int kOffV = kOffK + kStages * kStackBytes;
 constexpr int kSmemBytes = kOffV + kStages * kStackBytes;   // 96 KB
 constexpr int kSmemAlloc = kSmemBytes + 1024;               // room to align the base to 1 KB
 constexpr uint32_t kTmemCols = 256;
-// S double-buffered (64 fp32 columns each; block j of a step in columns
-// 32j..32j+31, its P in bf16 over the first 16 of them), O_0 and O_1 (64
-// columns each)
-constexpr uint32_t kColS = 0, kColO = 128;
-constexpr uint32_t kSCols = 32 * kStack;
+// S (128 fp32 columns, block j of a step in columns 32j..32j+31), P (the
+// step's 128 keys in bf16, two per column) and O (64 columns)
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
 constexpr float kRescale = 8.0f;                 // lazy-rescale threshold (log2 units)
 constexpr int kRows = 32 * kGroupRows;           // 128
 constexpr int kPartialFloats = kRows * (2 + 64); // m[128], l[128], O[128][64]
@@ -96,6 +95,22 @@ __host__ __device__ constexpr uint32_t idesc_s(int nblocks) {
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
 
 __device__ __forceinline__ void named_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+// Barrier over the two softmax warps of tensor-memory lane quarter wq
+// (barrier ids 2-5, named as immediates).
+__device__ __forceinline__ void pair_sync(int wq) {
+    switch (wq) {
+        case 0: asm volatile("bar.sync 2, 64;\n" ::: "memory"); break;
+        case 1: asm volatile("bar.sync 3, 64;\n" ::: "memory"); break;
+        case 2: asm volatile("bar.sync 4, 64;\n" ::: "memory"); break;
+        default: asm volatile("bar.sync 5, 64;\n" ::: "memory"); break;
+    }
+}
+// a bf16 pair times f (rounded to nearest)
+__device__ __forceinline__ uint32_t scale_bf16_pair(uint32_t v, float f) {
+    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v));
+    const __nv_bfloat162 y = __floats2bfloat162_rn(x.x * f, x.y * f);
+    return *reinterpret_cast<const uint32_t *>(&y);
+}
 // Barrier over the 256 softmax threads that also ANDs a predicate.
 __device__ __forceinline__ bool named_sync_and(bool v) {
     uint32_t out;
@@ -126,18 +141,15 @@ struct GArgs {
     int expire_first_wait;   // test hook: the softmax's first wait gives up at once
 };
 
-struct Pending {   // a step whose PV is still to be issued
-    int t, sg, nv, first, last;
-};
-
 __global__ void __launch_bounds__(kThreads, 2)
 attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const GArgs a) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) unsigned long long bar_qfull[2], bar_qempty[2], bar_kfull[kStages],
-        bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages], bar_sfull[2], bar_pfull[2], bar_pvdone[2],
+        bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages], bar_sfull, bar_sfree, bar_pfull, bar_pvdone,
         bar_ofull, bar_oempty, bar_ifull[kRing], bar_iempty[kRing], bar_fin;
-    __shared__ float2 s_ml[kStack][kRows];   // (max, sum) of each row's key-block halves
+    __shared__ float s_sum[2][kRows];       // each row's sums over its two key-block halves
+    __shared__ float s_ref[2][2][kRows];    // (step parity, half, row): each half's reference after a step
     __shared__ int s_ring[kRing];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort, s_last;
@@ -163,11 +175,10 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             mbar_init(saddr(&bar_ifull[i]), 1);
             mbar_init(saddr(&bar_iempty[i]), 1 + kSoftWarps);   // MMA thread + softmax warps
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(saddr(&bar_sfull[i]), 1);
-            mbar_init(saddr(&bar_pfull[i]), kSoftWarps);
-            mbar_init(saddr(&bar_pvdone[i]), 1);
-        }
+        mbar_init(saddr(&bar_sfull), 1);
+        mbar_init(saddr(&bar_sfree), kSoftWarps);
+        mbar_init(saddr(&bar_pfull), kSoftWarps);
+        mbar_init(saddr(&bar_pvdone), 1);
         mbar_init(saddr(&bar_ofull), 1);
         mbar_init(saddr(&bar_oempty), kSoftWarps);
         mbar_init(saddr(&bar_fin), 1);
@@ -267,26 +278,34 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            // shared-memory descriptors of the first Q, K and V tiles; a tile at
+            // byte offset d from one of them is its descriptor + d / 16 (every
+            // address stays below 256 KB, inside the descriptor's 14-bit field)
+            const uint64_t dQ = sdesc(sQ, 16, 1024), dK = sdesc(sK, 16, 1024), dV = sdesc(sV, 16, 1024);
             int n = 0, qn = 0, t = 0, npv = 0;
             bool ok = true, have = false;
-            Pending pend{0, 0, 0, 0, 0};
-            auto issue_pv = [&](const Pending &p) -> bool {
-                if (!waitb(&bar_vfull[p.sg], (p.t / kStages) & 1)) return false;
-                s_con_v = p.t + 1;
-                const int pb = p.t & 1;
-                if (!waitb(&bar_pfull[pb], (p.t >> 1) & 1)) return false;
-                if (p.first && npv > 0 && !waitb(&bar_oempty, (npv - 1) & 1)) return false;
+            int p_t = 0, p_sg = 0, p_nv = 0, p_first = 0, p_last = 0;   // the step whose PV is pending
+            // O += P V for the pending step, once its softmax wrote P
+            auto issue_pv = [&]() -> bool {
+                if (!waitb(&bar_vfull[p_sg], (p_t / kStages) & 1)) return false;
+                s_con_v = p_t + 1;
+                if (!waitb(&bar_pfull, p_t & 1)) return false;
+                if (p_first && npv > 0 && !waitb(&bar_oempty, (npv - 1) & 1)) return false;
                 tc_fence_after();
-                const uint32_t vb = sV + p.sg * kStackBytes;
-                for (int j = 0; j < p.nv; ++j)
+                const uint64_t dv = dV + (uint64_t)((p_sg * kStackBytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < 2; ++kk)
-                        mma_f16_ts(tmem + kColO + 64 * j, tmem + kColS + pb * kSCols + 32 * j + 8 * kk,
-                                   sdesc(vb + j * kTile + kk * 2048, 16, 1024), kIdescPV,
-                                   (p.first && kk == 0) ? 0u : 1u);
-                mma_commit(saddr(&bar_vempty[p.sg]));
-                mma_commit(saddr(&bar_pvdone[pb]));
-                if (p.last) {
+                for (int j = 0; j < kStack; ++j) {
+                    if (j < p_nv) {
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk)
+                            mma_f16_ts(tmem + kColO, tmem + kColP + 16 * j + 8 * kk,
+                                       dv + (uint64_t)((j * kTile + kk * 2048) >> 4), kIdescPV,
+                                       (p_first && j == 0 && kk == 0) ? 0u : 1u);
+                    }
+                }
+                mma_commit(saddr(&bar_vempty[p_sg]));
+                mma_commit(saddr(&bar_pvdone));
+                if (p_last) {
                     mma_commit(saddr(&bar_ofull));
                     ++npv;
                 }
@@ -306,38 +325,39 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 const int nst = (it.ucount + kStack - 1) / kStack;
                 if (nst == 0) continue;
                 const int qs = qn & 1;
-                for (int st = 0; st < nst; ++st) {
+                for (int st = 0; st < nst; ++st, ++t) {
                     const int sg = t % kStages;
                     const int nv = min(kStack, it.ucount - st * kStack);
                     if (!(ok = waitb(&bar_kfull[sg], (t / kStages) & 1))) break;
                     s_con_k = t + 1;
-                    // S buffer t & 1 holds the P of step t - 2 until that
-                    // step's PV is done
-                    const int sb = t & 1;
-                    if (t >= 2 && !(ok = waitb(&bar_pvdone[sb], ((t >> 1) - 1) & 1))) break;
+                    // S is rewritten once the softmax of step t - 1 has read it
+                    if (t >= 1 && !(ok = waitb(&bar_sfree, (t - 1) & 1))) break;
                     if (st == 0) {
                         if (!(ok = waitb(&bar_qfull[qs], (qn >> 1) & 1))) break;
                         s_con_q = qn + 1;
                     }
                     tc_fence_after();
                     const uint32_t idesc = idesc_s(nv);
+                    const uint64_t dq = dQ + (uint64_t)((qs * kQBytes) >> 4), dk = dK + (uint64_t)((sg * kStackBytes) >> 4);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + kColS + sb * kSCols, sdesc(sQ + qs * kQBytes + ks * 32, 16, 1024),
-                                sdesc(sK + sg * kStackBytes + ks * 32, 16, 1024), idesc, ks > 0 ? 1u : 0u);
-                    mma_commit(saddr(&bar_sfull[sb]));
+                        mma_f16(tmem + kColS, dq + 2 * ks, dk + 2 * ks, idesc, ks > 0 ? 1u : 0u);
+                    mma_commit(saddr(&bar_sfull));
                     mma_commit(saddr(&bar_kempty[sg]));
                     if (st == nst - 1) mma_commit(saddr(&bar_qempty[qs]));
                     // the PV of the previous step goes after this step's S, so
                     // that the softmax of this step overlaps it
-                    if (have && !(ok = issue_pv(pend))) break;
-                    pend = Pending{t, sg, nv, st == 0, st == nst - 1};
+                    if (have && !(ok = issue_pv())) break;
+                    p_t = t;
+                    p_sg = sg;
+                    p_nv = nv;
+                    p_first = st == 0;
+                    p_last = st == nst - 1;
                     have = true;
-                    ++t;
                 }
                 ++qn;
             }
-            if (ok && have) ok = issue_pv(pend);
+            if (ok && have) ok = issue_pv();
             // every MMA issued by this thread completes before TMEM is freed
             mma_commit(saddr(&bar_fin));
             mbar_wait(saddr(&bar_fin), 0);
@@ -347,7 +367,8 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         // ------------------------------------------------------------ softmax + epilogue
         const int wq = warp & 3, hh = warp >> 2;            // lane quarter, key-block half
         const uint32_t lq = (uint32_t)(wq * 32) << 16;     // this warp's TMEM lane quarter
-        const uint32_t tS = tmem + lq + kColS + 32 * hh, tO = tmem + lq + kColO;
+        const uint32_t tS = tmem + lq + kColS + 32 * kHalf * hh, tP = tmem + lq + kColP + 16 * kHalf * hh,
+                       tO = tmem + lq + kColO;
         const int row = wq * 32 + lane;                     // row of the 128-row tile
         int n = 0, t = 0, on = 0;
         while (true) {
@@ -370,124 +391,151 @@ attn_group_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             float mref = -INFINITY, lsum = 0.0f;
             for (int st = 0; st < nst; ++st, ++t) {
                 const int nv = min(kStack, it.ucount - st * kStack);
-                const int u = st * kStack + hh;
-                const int e = __shfl_sync(0xffffffffu, u < 32 ? e0 : e1, u & 31);
-                const bool act = hh < nv && row_ok && ((e >> (kUnionRowShift + wq)) & 1);
-                const bool part = act && (e & kUnionPartial);
-                const int sb = t & 1;
+                int act = 0, part = 0, cb[kHalf];
+#pragma unroll
+                for (int jj = 0; jj < kHalf; ++jj) {
+                    const int u = st * kStack + kHalf * hh + jj;
+                    const int e = __shfl_sync(0xffffffffu, u < 32 ? e0 : e1, u & 31);
+                    cb[jj] = e & 0xffff;
+                    if (kHalf * hh + jj < nv && row_ok && ((e >> (kUnionRowShift + wq)) & 1)) {
+                        act |= 1 << jj;
+                        if (e & kUnionPartial) part |= 1 << jj;
+                    }
+                }
                 if (a.expire_first_wait && t == 0) {
                     // a wait whose limit has run out (test hook, see the launcher)
                     *abort_flag = 1;
                     atomicOr(status, kDevTimeout);
                 }
-                waitb(&bar_sfull[sb], (t >> 1) & 1);
+                waitb(&bar_sfull, t & 1);
                 tc_fence_after();
-                float s[32];
-                if (act) {
-                    uint32_t raw[32];
-                    tmem_ld32(tS + sb * kSCols, raw);
-                    tmem_wait_ld_regs(raw);
+                // this warp's blocks of S one at a time into registers (S is
+                // free for the next step's scores once both are read), each
+                // turned into P against this half's lazy reference; P of the
+                // first block is rescaled in registers when the second moves it
+                const float mstart = mref;
+                float ls = 0.0f, ls2 = 0.0f;
+                uint32_t pk[kHalf][16];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(raw[i]);
-                    // padded keys of partly padded key blocks take no weight
-                    if (part) {
-                        const unsigned kv = __ballot_sync(0xffffffffu, mrow[(e & 0xffff) * 32 + lane] > 0.0f);
+                for (int jj = 0; jj < kHalf; ++jj) {
+                    if ((act >> jj) & 1) {
+                        float x[32];
+                        {
+                            uint32_t r[32];
+                            tmem_ld32(tS + 32 * jj, r);
+                            tmem_wait_ld_regs(r);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (!((kv >> i) & 1u)) s[i] = -INFINITY;
-                    }
-                }
-                float alpha = 1.0f, ls = 0.0f;
-                bool resc = false;
-                uint32_t pk[16];
-                if (act) {
-                    float m4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-                    for (int i = 4; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], s[i]);
-                    const float mxs = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
-                    if (mxs > mref + kRescale) {
-                        if (mref != -INFINITY) {
-                            alpha = fast_exp2(mref - mxs);
-                            resc = true;
+                            for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
                         }
-                        mref = mxs;
-                    }
-                    const float ref = (mref == -INFINITY) ? 0.0f : mref;
-                    float ls2 = 0.0f;
+                        if (jj == kHalf - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(saddr(&bar_sfree));
+                        }
+                        // padded keys of partly padded key blocks take no weight
+                        if ((part >> jj) & 1) {
+                            const unsigned kv = __ballot_sync(0xffffffffu, mrow[cb[jj] * 32 + lane] > 0.0f);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float p0 = fast_exp2(fmaf(s[2 * i], a.scale_log2, -ref));
-                        const float p1 = fast_exp2(fmaf(s[2 * i + 1], a.scale_log2, -ref));
-                        const __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
-                        pk[i] = *reinterpret_cast<const uint32_t *>(&hp);
-                        ls += p0;
-                        ls2 += p1;
-                    }
-                    ls += ls2;
-                } else {
+                            for (int i = 0; i < 32; ++i)
+                                if (!((kv >> i) & 1u)) x[i] = -INFINITY;
+                        }
+                        float m4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                        for (int i = 4; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], x[i]);
+                        const float mxs = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
+                        if (mxs > mref + kRescale) {
+                            if (jj > 0 && mref != -INFINITY) {
+                                const float aj = fast_exp2(mref - mxs);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) pk[0][i] = scale_bf16_pair(pk[0][i], aj);
+                                ls *= aj;
+                                ls2 *= aj;
+                            }
+                            mref = mxs;
+                        }
+                        const float ref = (mref == -INFINITY) ? 0.0f : mref;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float p0 = fast_exp2(fmaf(x[2 * i], a.scale_log2, -ref));
+                            const float p1 = fast_exp2(fmaf(x[2 * i + 1], a.scale_log2, -ref));
+                            const __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
+                            pk[jj][i] = *reinterpret_cast<const uint32_t *>(&hp);
+                            ls += p0;
+                            ls2 += p1;
+                        }
+                    } else {
+                        if (jj == kHalf - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(saddr(&bar_sfree));
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pk[jj][i] = 0u;
+                    }
                 }
-                lsum = fmaf(lsum, alpha, ls);
-                // O_j may be rescaled once every earlier PV (that of step t - 1)
+                // both halves of the row take the larger reference, so that
+                // they share one O; the half whose reference was lower
+                // rescales its P in registers
+                s_ref[t & 1][hh][row] = mref;
+                pair_sync(wq);
+                const float mo = s_ref[t & 1][hh ^ 1][row];
+                if (mo > mref) {
+                    if (mref != -INFINITY) {
+                        const float aj = fast_exp2(mref - mo);
+#pragma unroll
+                        for (int jj = 0; jj < kHalf; ++jj)
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) pk[jj][i] = scale_bf16_pair(pk[jj][i], aj);
+                        ls *= aj;
+                        ls2 *= aj;
+                    }
+                    mref = mo;
+                }
+                const bool resc = mstart != -INFINITY && mref != mstart;
+                const float alpha = resc ? fast_exp2(mstart - mref) : 1.0f;
+                lsum = fmaf(lsum, alpha, ls + ls2);
+                // P (and O, for a rescale) are free once the PV of step t - 1
                 // is done
-                const bool any_resc = __any_sync(0xffffffffu, resc);
-                if (any_resc) {
-                    if (t >= 1) waitb(&bar_pvdone[sb ^ 1], ((t - 1) >> 1) & 1);
-                    tc_fence_after();
+                if (t >= 1) waitb(&bar_pvdone, (t - 1) & 1);
+                tc_fence_after();
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + 64 * hh + 32 * half, o);
-                        tmem_wait_ld_regs(o);
+                for (int jj = 0; jj < kHalf; ++jj)
+                    if (kHalf * hh + jj < nv) tmem_st16(tP + 16 * jj, pk[jj]);
+                // both warps of the quarter took the same decision; each
+                // rescales its 32 columns of O
+                if (__any_sync(0xffffffffu, resc)) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + 32 * hh, o);
+                    tmem_wait_ld_regs(o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(tO + 64 * hh + 32 * half, o);
-                    }
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + 32 * hh, o);
                 }
-                if (hh < nv) tmem_st16(tS + sb * kSCols, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(saddr(&bar_pfull[sb]));
+                if (lane == 0) mbar_arrive(saddr(&bar_pfull));
             }
             // ---------------------------------------------------- epilogue
             // the row's two key-block halves under one maximum; this warp then
             // produces output columns 32*hh .. 32*hh+31 of its 32 rows
             const int chunk = it.chunk_info & 0xffff, nch = it.chunk_info >> 16;
-            s_ml[hh][row] = make_float2(mref, lsum);
+            s_sum[hh][row] = lsum;
             named_sync();
-            const float2 oth = s_ml[hh ^ 1][row];
-            const float m0 = hh ? oth.x : mref, l0 = hh ? oth.y : lsum;
-            const float m1 = hh ? mref : oth.x, l1 = hh ? lsum : oth.y;
-            float m_hi = -INFINITY, l_hi = 0.0f, w0 = 0.0f, w1 = 0.0f;
-            if (l0 > 0.0f) m_hi = m0;
-            if (l1 > 0.0f) m_hi = fmaxf(m_hi, m1);
-            if (m_hi != -INFINITY) {
-                w0 = l0 > 0.0f ? fast_exp2(m0 - m_hi) : 0.0f;
-                w1 = l1 > 0.0f ? fast_exp2(m1 - m_hi) : 0.0f;
-                l_hi = fmaf(w0, l0, w1 * l1);
-            }
+            // both halves share the reference mref; O holds both
+            float l_hi = lsum + s_sum[hh ^ 1][row];
+            float m_hi = l_hi > 0.0f ? mref : -INFINITY;
             float o[32];
             if (nst > 0) {
                 waitb(&bar_ofull, on & 1);
                 ++on;
                 tc_fence_after();
-                {
-                    uint32_t raw[32];
-                    tmem_ld32(tO + 32 * hh, raw);
-                    tmem_wait_ld_regs(raw);
+                uint32_t raw[32];
+                tmem_ld32(tO + 32 * hh, raw);
+                tmem_wait_ld_regs(raw);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = w0 * __uint_as_float(raw[i]);
-                }
-                if (it.ucount >= 2) {   // O_1 holds a term only when the item has a second block
-                    uint32_t raw[32];
-                    tmem_ld32(tO + 64 + 32 * hh, raw);
-                    tmem_wait_ld_regs(raw);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = fmaf(w1, __uint_as_float(raw[i]), o[i]);
-                }
-                // both accumulators are free for the next item's first PV
+                for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(raw[i]);
+                // the accumulator is free for the next item's first PV
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(saddr(&bar_oempty));
