@@ -841,11 +841,12 @@ def main():
     dom_s = phases[dom]["avg_us"] * 1e-6
     esz = 2 if w.dtype == "bf16" else 4
     BH = w.B * w.H
-    # bf16 head size 64 runs the tcgen05 kernel on maps with at least 32
-    # selected blocks per block row (MRA_ATTN_IMPL=tc / =mma force either)
+    # bf16 head size 64 runs the tcgen05 kernel on maps with at least 45 % of
+    # the block map selected (MRA_ATTN_IMPL=tc / =mma force either)
     impl = os.environ.get("MRA_ATTN_IMPL", "")
     tc_attn = w.dtype == "bf16" and w.D == 64 and (
-        impl.startswith("t") or (not impl.startswith("m") and min(w.block_per_row, w.nbr) >= 32))
+        impl.startswith("t") or (not impl.startswith("m") and
+                                 20 * min(w.block_per_row, w.nbr) * w.nbr >= 9 * w.nbr * w.nbr))
     kernel_src = {"attention": "mra_attn_tc.cu" if tc_attn else "mra_attn.cu", "pool": "mra_pool.cu",
                   "lowres_keys": "mra_lowres.cu", "lowres_pv": "mra_lowres.cu", "select": "mra_select.cu",
                   "lowres_select": "mra_lowres_select.cu", "group_plan": "mra_group_plan.cu"}

@@ -456,24 +456,28 @@ attn_f32_kernel(const AttnArgs a) {
 
 }  // namespace
 
-// bf16 forward passes with head size 64 on dense maps (at least
-// kTcMinBlocksPerRow selected blocks per block row on average) run on the
-// tcgen05 kernel; sparse maps, fp32, head size 32 and the backward pass's
-// forward re-run (which exports per-row statistics) on the warp-level kernels
-// above.  On sparse maps a group's union holds few blocks per row and the
-// warp-level kernel, with ten CTAs per SM, is faster (measured: N=4096 with 4
-// blocks per row 40 against 78 us; N=16384 with 8 per row 113 against 286 us;
-// the BigBird pattern, 19 per row, 107 against 134 us; the saturated N=2048
-// map, 64 per row, 177 against 269 us on the tcgen05 kernel).
+// bf16 forward passes with head size 64 on dense maps (at least 45 % of the
+// block map selected: kTcMinShare20 / 20) run on the tcgen05 kernel; sparser
+// maps, fp32, head size 32 and the backward pass's forward re-run (which
+// exports per-row statistics) on the warp-level kernels above.  The tcgen05
+// kernel works over the union of four block rows' selections, which on
+// sparse maps is mostly disjoint, while the warp-level kernel (ten CTAs per
+// SM) touches the selected blocks only.  Measured, whole forward step,
+// tcgen05 against warp-level: N=2048 (64 x 64 blocks) with 16 blocks per row
+// 133 against 99 us, 24 per row 106.5 against 130, 64 per row 128.6 against
+// 273.5 (attention alone); N=4096 (128 x 128) with 32 per row 276.5 against
+// 216.7, 48 per row 309 against 279, 64 per row 326 against 332, 80 per row
+// 339 against 385; the sparse N=4096 and N=16384 maps (4 and 8 per row) and
+// the BigBird pattern (19 per row) stay well below the line.
 // MRA_ATTN_IMPL=tc or =mma (read once per process) forces either kernel.
-constexpr int kTcMinBlocksPerRow = 32;
+constexpr int kTcMinShare20 = 9;
 
 bool attention_uses_tc(const Problem &p, const GradStats *gs) {
     static const char *impl = getenv("MRA_ATTN_IMPL");
     if (gs || !attention_tc_supported(p)) return false;
     if (impl && impl[0] == 'm') return false;
     if (impl && impl[0] == 't') return true;
-    return (long long)p.k >= (long long)kTcMinBlocksPerRow * p.nbr;
+    return 20LL * p.k >= (long long)kTcMinShare20 * p.nbr * p.nbr;
 }
 
 cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q, const void *k,
