@@ -32,10 +32,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRows = 16;                 // block rows per CTA
-constexpr int kRG = 8, kCG = 32;          // row groups x column lanes of the GEMM
-constexpr int kMR = kRows / kRG;          // rows per thread tile (2)
 constexpr int kCT = 128;                  // columns of the map (at most)
-constexpr int kCPT = kCT / kCG;           // columns per thread (4), strided by 32
+constexpr int kCPT = kCT / 32;            // columns per lane in the per-row passes (4), strided by 32
 constexpr int kMaxCta = 8;                // portable cluster size
 constexpr int kHistBits12 = 12;           // the two lower digits
 constexpr unsigned int kMask12 = (1u << kHistBits12) - 1u;
@@ -168,37 +166,34 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
     }
     __syncthreads();
     {
-        // thread tile: rows kMR*rg + i, columns cg_ + 32*j
-        const int rg = t / kCG, cg_ = t % kCG;
-        float acc[kMR][kCPT];
+        // thread tile: one column c of the map (its K-hat row in registers)
+        // and kRPT rows (Q-hat read as loads that every lane of the warp
+        // shares); the sum over d runs in the same order as a plain dot
+        // product
+        constexpr int kHalves = kThreads / kCT;
+        constexpr int kRPT = kRows / kHalves;
+        const int c = t % kCT, half = t / kCT;
+        if (c < nbr) {
+            float4 kr[kF4];
 #pragma unroll
-        for (int i = 0; i < kMR; ++i)
+            for (int d4 = 0; d4 < kF4; ++d4) kr[d4] = *reinterpret_cast<const float4 *>(ks + c * KS + 4 * d4);
+            float acc[kRPT];
 #pragma unroll
-            for (int j = 0; j < kCPT; ++j) acc[i][j] = 0.0f;
-#pragma unroll 4
-        for (int d = 0; d < D; d += 4) {
-            float4 q4[kMR], k4[kCPT];
+            for (int i = 0; i < kRPT; ++i) acc[i] = 0.0f;
 #pragma unroll
-            for (int i = 0; i < kMR; ++i) q4[i] = *reinterpret_cast<const float4 *>(qs + (kMR * rg + i) * D + d);
+            for (int d4 = 0; d4 < kF4; ++d4) {
 #pragma unroll
-            for (int j = 0; j < kCPT; ++j) k4[j] = *reinterpret_cast<const float4 *>(ks + (cg_ + 32 * j) * KS + d);
-#pragma unroll
-            for (int i = 0; i < kMR; ++i)
-#pragma unroll
-                for (int j = 0; j < kCPT; ++j) {
-                    acc[i][j] = fmaf(q4[i].x, k4[j].x, acc[i][j]);
-                    acc[i][j] = fmaf(q4[i].y, k4[j].y, acc[i][j]);
-                    acc[i][j] = fmaf(q4[i].z, k4[j].z, acc[i][j]);
-                    acc[i][j] = fmaf(q4[i].w, k4[j].w, acc[i][j]);
+                for (int i = 0; i < kRPT; ++i) {
+                    const float4 q4 = *reinterpret_cast<const float4 *>(qs + (kRPT * half + i) * D + 4 * d4);
+                    acc[i] = fmaf(q4.x, kr[d4].x, acc[i]);
+                    acc[i] = fmaf(q4.y, kr[d4].y, acc[i]);
+                    acc[i] = fmaf(q4.z, kr[d4].z, acc[i]);
+                    acc[i] = fmaf(q4.w, kr[d4].w, acc[i]);
                 }
-        }
-#pragma unroll
-        for (int i = 0; i < kMR; ++i)
-#pragma unroll
-            for (int j = 0; j < kCPT; ++j) {
-                const int c = cg_ + 32 * j;
-                if (c < nbr) lt[(kMR * rg + i) * nbr + c] = acc[i][j] * scale;
             }
+#pragma unroll
+            for (int i = 0; i < kRPT; ++i) lt[(kRPT * half + i) * nbr + c] = acc[i] * scale;
+        }
     }
     __syncthreads();
     // the K-hat tile is dead: it becomes the cluster histograms, cleared
