@@ -120,7 +120,7 @@ size_t carve_workspace(const Problem &p, char *base, Workspace *w) {
     t.pooled = (float *)take(sizeof(float) * 3 * BH * nbr * D);
     t.keys = (unsigned long long *)take(sizeof(unsigned long long) * BH * (size_t)p.nbr2);
     t.lo_logits = (float *)take(sizeof(float) * BH * (size_t)p.nbr2);
-    t.lo_pmax = (float *)take(sizeof(float) * BH * nbr * ((nbr + 63) / 64));
+    t.lo_pmax = (float *)take(sizeof(float) * BH * nbr * ((nbr + 127) / 128));
     t.mlo = (float *)take(sizeof(float) * BH * nbr);
     t.state = (SelState *)take(sizeof(SelState) * BH);
     t.cols = (int *)take(sizeof(int) * BH * (size_t)p.k);

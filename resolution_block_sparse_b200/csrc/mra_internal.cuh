@@ -101,7 +101,7 @@ struct Workspace {
     float *pooled;           // [3][BH][nbr][D]
     unsigned long long *keys;// [BH][nbr2]
     float *lo_logits;        // [BH][nbr2] low-resolution logit map (full mode, maps over 128 x 128)
-    float *lo_pmax;          // [BH][nbr][ceil(nbr / 64)] per-tile row maxima of the logit map
+    float *lo_pmax;          // [BH][nbr][ceil(nbr / 128)] per-tile row maxima of the logit map
     float *mlo;              // [BH][nbr]
     SelState *state;         // [BH]
     int *ccount;             // [BH] candidates of the first digit's bucket (zeroed region)

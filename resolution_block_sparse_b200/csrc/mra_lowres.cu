@@ -46,25 +46,27 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
 }
 
-// Logit map of maps above 128 x 128 blocks on 64 x 64 tiles:
+// Logit map of maps above 128 x 128 blocks on 128 x 128 tiles:
 // l_rc = scale * qhat_r . khat_c in fp32 (FFMA, d ascending), written to
 // L [BH][nbr][nbr], and the maximum over the tile's valid columns (cnt > 0) of
-// each row to pmax [BH][nbr][ntiles] (-inf when none).  Persistent CTAs walk
-// the tiles with a stride of the grid; the next tile's Q-hat and K-hat rows
-// arrive by cp.async into the other of two buffers while the current tile is
-// multiplied.  Thread (tx, ty) of 16 x 16 holds rows ty + 16 i and columns
-// tx + 16 j (4 x 4 register tile): a warp's column loads are 16 consecutive
-// rows of a padded [64][D + 4] tile and its row loads broadcast.
-constexpr int kLgT = 64;
+// each row to pmax [BH][nbr][ntiles] (-inf when none).  CTAs walk the tiles
+// with a stride of the grid, two CTAs per SM, so that one CTA's cp.async
+// loads of Q-hat and K-hat rows overlap the other's products.  Thread (tx, ty)
+// of 16 x 16 holds rows ty + 16 i and columns tx + 16 j (8 x 8 register tile:
+// 256 FMAs per 16 shared-memory loads of 16 bytes); a warp's column loads are
+// 16 consecutive rows of a padded [128][D + 4] tile and its row loads
+// broadcast.
+constexpr int kLgT = 128;
+constexpr int kLgR = kLgT / 16;   // rows (and columns) per thread
 
 template <int D>
 struct LgSmem {
-    float q[2][kLgT][D + 4];
-    float k[2][kLgT][D + 4];
+    float q[kLgT][D + 4];
+    float k[kLgT][D + 4];
 };
 
 template <int D>
-__global__ void __launch_bounds__(kLowresThreads, 3)
+__global__ void __launch_bounds__(kLowresThreads, 2)
 lowres_logits_kernel(const float *__restrict__ qhat, const float *__restrict__ khat,
                      const int *__restrict__ cnt, int H, int nbr, float scale, float *__restrict__ L,
                      float *__restrict__ pmax, int total_tiles) {
@@ -73,52 +75,39 @@ lowres_logits_kernel(const float *__restrict__ qhat, const float *__restrict__ k
     LgSmem<D> &sh = *reinterpret_cast<LgSmem<D> *>(lg_smem);
     const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
     const int nt = (nbr + kLgT - 1) / kLgT;
-    auto stage = [&](int tile, int bf) {
-        const int bh = tile / (nt * nt), rem = tile - bh * nt * nt;
-        const int row0 = (rem / nt) * kLgT, col0 = (rem % nt) * kLgT;
-        const float *qh = qhat + (size_t)bh * nbr * D;
-        const float *kh = khat + (size_t)bh * nbr * D;
-        for (int i = t; i < kLgT * D / 4; i += kLowresThreads) {
-            const int r = i / (D / 4), d4 = i % (D / 4);
-            if (row0 + r < nbr) cp_async16(&sh.q[bf][r][4 * d4], qh + (size_t)(row0 + r) * D + 4 * d4);
-            else *reinterpret_cast<float4 *>(&sh.q[bf][r][4 * d4]) = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (col0 + r < nbr) cp_async16(&sh.k[bf][r][4 * d4], kh + (size_t)(col0 + r) * D + 4 * d4);
-            else *reinterpret_cast<float4 *>(&sh.k[bf][r][4 * d4]) = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    };
-    int tile = blockIdx.x;
-    if (tile < total_tiles) stage(tile, 0);
-    cp_async_commit();
-    for (int it = 0; tile < total_tiles; ++it, tile += gridDim.x) {
-        const int bf = it & 1;
-        if (tile + (int)gridDim.x < total_tiles) stage(tile + gridDim.x, bf ^ 1);
-        cp_async_commit();
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
         const int bh = tile / (nt * nt), rem = tile - bh * nt * nt;
         const int ct = rem % nt;
         const int row0 = (rem / nt) * kLgT, col0 = ct * kLgT;
-        int cv[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c = col0 + tx + 16 * j;
-            cv[j] = c < nbr ? cnt[(size_t)(bh / H) * nbr + c] : 0;
+        {
+            const float *qh = qhat + (size_t)bh * nbr * D;
+            const float *kh = khat + (size_t)bh * nbr * D;
+            for (int i = t; i < kLgT * D / 4; i += kLowresThreads) {
+                const int r = i / (D / 4), d4 = i % (D / 4);
+                if (row0 + r < nbr) cp_async16(&sh.q[r][4 * d4], qh + (size_t)(row0 + r) * D + 4 * d4);
+                else *reinterpret_cast<float4 *>(&sh.q[r][4 * d4]) = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (col0 + r < nbr) cp_async16(&sh.k[r][4 * d4], kh + (size_t)(col0 + r) * D + 4 * d4);
+                else *reinterpret_cast<float4 *>(&sh.k[r][4 * d4]) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
         }
-        cp_async_wait<1>();
         __syncthreads();   // this tile landed and is visible
-        float acc[4][4];
+        float acc[kLgR][kLgR];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < kLgR; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-#pragma unroll 2
+            for (int j = 0; j < kLgR; ++j) acc[i][j] = 0.0f;
+#pragma unroll 1
         for (int d = 0; d < D; d += 4) {
-            float4 kc[4];
+            float4 kc[kLgR];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) kc[j] = *reinterpret_cast<const float4 *>(&sh.k[bf][tx + 16 * j][d]);
+            for (int j = 0; j < kLgR; ++j) kc[j] = *reinterpret_cast<const float4 *>(&sh.k[tx + 16 * j][d]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float4 qr = *reinterpret_cast<const float4 *>(&sh.q[bf][ty + 16 * i][d]);
+            for (int i = 0; i < kLgR; ++i) {
+                const float4 qr = *reinterpret_cast<const float4 *>(&sh.q[ty + 16 * i][d]);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < kLgR; ++j) {
                     acc[i][j] = fmaf(qr.x, kc[j].x, acc[i][j]);
                     acc[i][j] = fmaf(qr.y, kc[j].y, acc[i][j]);
                     acc[i][j] = fmaf(qr.z, kc[j].z, acc[i][j]);
@@ -126,23 +115,24 @@ lowres_logits_kernel(const float *__restrict__ qhat, const float *__restrict__ k
                 }
             }
         }
+        __syncthreads();   // every thread is done with the tiles before the next are staged
+        const int *crow = cnt + (size_t)(bh / H) * nbr;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kLgR; ++i) {
             const int r = row0 + ty + 16 * i;
             float m = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < kLgR; ++j) {
                 const int c = col0 + tx + 16 * j;
                 const float l = acc[i][j] * scale;
                 if (r < nbr && c < nbr) L[((size_t)bh * nbr + r) * nbr + c] = l;
-                if (cv[j] > 0) m = fmaxf(m, l);
+                if (c < nbr && __ldg(crow + c) > 0) m = fmaxf(m, l);
             }
             // maximum over the 16 lanes of this row (a half warp)
 #pragma unroll
             for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             if (tx == 0 && r < nbr) pmax[((size_t)bh * nbr + r) * nt + ct] = m;
         }
-        __syncthreads();   // every thread is done with this buffer before it is staged again
     }
 }
 
@@ -213,7 +203,7 @@ lowres_keys_kernel(const float *__restrict__ L, const float *__restrict__ pmax,
                 const unsigned long long key =
                     act ? selection_key(lv[u], m, gr, c, first_n, diag_n, row_empty, cnts[c] <= 0, flag) : 0ull;
                 if (act) krow[c] = key;
-                warp_hist_add(h0, (unsigned)(key >> 24), act);
+                hist_add(h0, (unsigned)(key >> 24), act);
             }
         }
     }
@@ -573,7 +563,7 @@ cudaError_t launch_logits_typed(const Problem &p, const Workspace &w, float *L, 
     cudaError_t e = cudaFuncSetAttribute(lowres_logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const long long grid = std::min<long long>(total, 3LL * device_sm_count());
+    const long long grid = std::min<long long>(total, 2LL * device_sm_count());
     return launch_dependent(lowres_logits_kernel<D>, dim3((unsigned)grid), dim3(kLowresThreads), smem, s, qhat, khat,
                             (const int *)w.cnt, p.H, p.nbr, scale, L, w.lo_pmax, (int)total);
 }

@@ -236,7 +236,7 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                     const size_t gi = (size_t)bh * nbr2 + (size_t)gr * nbr + c;
                     if (logit_out) logit_out[gi] = lv[j];
                 }
-                warp_hist_add(cs.lh, (unsigned)(key >> (kHist1Bits + kHist2Bits)) & ((1u << kHist0Bits) - 1u), ok);
+                hist_add(cs.lh, (unsigned)(key >> (kHist1Bits + kHist2Bits)) & ((1u << kHist0Bits) - 1u), ok);
             }
         }
         if (flag) atomicOr(&cs.flag, 1);
@@ -313,7 +313,7 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                     for (int e0 = warp * 32; e0 < n; e0 += kThreads) {
                         const int e = e0 + lane;
                         const unsigned long long key = e < n ? cand[e] : ~0ull;
-                        warp_hist_add(cs.lh, (unsigned)(key >> shift) & kMask12, e < n && (key >> hi) == want);
+                        hist_add(cs.lh, (unsigned)(key >> shift) & kMask12, e < n && (key >> hi) == want);
                     }
                     __syncthreads();
                     find_bucket_smem<kThreads, kHistBins>(cs.lh, need, cs.s_tot, &cs.bin, &cs.bin_need);
@@ -386,7 +386,7 @@ lowres_select_cluster_kernel(const float *__restrict__ qhat, const float *__rest
                 for (int e0 = warp * 32; e0 < n_here; e0 += kThreads) {
                     const int e = e0 + lane;
                     const unsigned long long key = e < n_here ? sk[e] : ~0ull;
-                    warp_hist_add(cs.lh, (unsigned)(key >> shift) & dmask, e < n_here && (key >> hi) == want);
+                    hist_add(cs.lh, (unsigned)(key >> shift) & dmask, e < n_here && (key >> hi) == want);
                 }
                 __syncthreads();
                 unsigned int *hp = hist0 + (1 << kHist0Bits) + (pass - 1) * kHistBins;

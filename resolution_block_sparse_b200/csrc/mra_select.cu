@@ -189,7 +189,7 @@ select_finalize_kernel(SelState *__restrict__ state, const unsigned long long *_
         for (int i0 = warp * 32; i0 < n; i0 += kFinThreads) {
             const int i = i0 + lane;
             const unsigned long long key = i < n ? cand_key_at(i) : ~0ull;
-            warp_hist_add(h, (unsigned)(key >> shift) & 0xfffu, i < n && (key >> hi) == want);
+            hist_add(h, (unsigned)(key >> shift) & 0xfffu, i < n && (key >> hi) == want);
         }
         __syncthreads();
         find_bucket_smem<kFinThreads, kHistBins>(h, need, s_tmp, &s_bin, &s_need);
