@@ -10,23 +10,22 @@
 //
 // Tile = four adjacent query block rows of one head: M = 128 query rows, row
 // i of the tile on tensor-memory lane i, so each softmax thread owns one query
-// row and its max and sum need no exchange between threads.  The tile runs
-// over the union of the four rows' selected key blocks (built by the group
-// plan), two key blocks per step:
-//   S = Q_128 . K_stack^T          (M = 128, N = 32 * blocks <= 64, K = 64)
-//   O_j += P_j . V_j               (M = 128, N = 64, K = 32, for block j of
-//                                   the step; P read from tensor memory, V
-//                                   from the TMA tile)
-// Two softmax warps share each tensor-memory lane quarter: warp (w, j) owns
-// the 32 rows of block row 4g+w and key block j of every step, keeps its own
-// running maximum and sum for that half of the keys, and accumulates into its
-// own O_j; the halves are merged under a common maximum in the epilogue.  A
-// (row, key block) pair outside that row's selection gets no weight: its warp
-// skips the block and writes zero P there, so the exponentials computed are
-// exactly those of the selected blocks.  P (bf16) is written over the S
-// columns it was computed from.  The row maximum is kept lazily (the exponent
-// reference moves only when the maximum grows by more than 2^8), so the
-// accumulators in tensor memory are rescaled rarely.
+// row.  The tile runs over the union of the four rows' selected key blocks
+// (built by the group plan), four key blocks (128 keys) per step:
+//   S = Q_128 . K_step^T           (M = 128, N = 32 * blocks <= 128, K = 64)
+//   O += P . V_step                (M = 128, N = 64, K = 32 per block; P read
+//                                   from tensor memory, V from the TMA tile)
+// Two softmax warps share each tensor-memory lane quarter: warp (w, h) holds
+// the 32 rows of block row 4g+w and key blocks 2h, 2h+1 of every step.  It
+// turns each of its blocks into P against a lazy reference (the exponent
+// reference moves only when the maximum grows by more than 2^8), then both
+// warps of the quarter take the larger of their two references (one value
+// per row through shared memory), so that they share one O; the one whose
+// reference was lower rescales its P in registers.  A (row, key block) pair
+// outside that row's selection gets no weight: its warp skips the block and
+// writes zero P there, so the exponentials computed are exactly those of the
+// selected blocks.  P has a tensor-memory buffer of its own, so S of the next
+// step is computed while the softmax of this one runs.
 //
 // Work item = (group, chunk of at most gchunk union entries).  A group whose
 // union is longer is split over several items; each writes (max, sum, O) for
@@ -35,12 +34,13 @@
 // from a per-call counter and passes it to the other roles through a ring in
 // shared memory.
 //
-// Warp roles (two CTAs per SM, 256 tensor-memory columns each: S 2 x 64, O
-// 2 x 64): warps 0-7 softmax and epilogue, warp 8 TMA producer (Q per item, K
-// and V per step, four stages), warp 9 MMA issuer.  Every mbarrier wait is
-// bounded: on expiry the kernel raises MRA_DEV_TIMEOUT in the status word,
-// every role stops, the kernel waits (bounded) for its own loads and MMAs in
-// flight, frees its tensor memory and returns.
+// Warp roles (two CTAs per SM, 256 tensor-memory columns each: S 128, P 64,
+// O 64): warps 0-7 softmax and epilogue (each writes 32 of the 64 output
+// columns of its rows), warp 8 TMA producer (Q per item, K and V per step, two
+// stages), warp 9 MMA issuer.  Every mbarrier wait is bounded: on expiry the
+// kernel raises MRA_DEV_TIMEOUT in the status word, every role stops, the
+// kernel waits (bounded) for its own loads and MMAs in flight, frees its
+// tensor memory and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
