@@ -16,16 +16,20 @@
 // counter, no waiting) merges them.  Padded queries (mask 0) output 0.
 //
 // bf16 kernel: two warps, each owning 16 query rows, mma.sync m16n8k16 with
-// fp32 accumulation; K/V blocks in a ring of XOR-swizzled shared-memory buffers
-// by cp.async.  fp32 kernel: FFMA only (no TF32).
+// fp32 accumulation; Q and K/V blocks in a ring of XOR-swizzled shared-memory
+// buffers, loaded by TMA (one 4 KB tile per copy, 128-byte swizzle, completion
+// on an mbarrier per buffer) for head size 64 and by cp.async for 32.  fp32
+// kernel: FFMA only (no TF32).
 #include <cuda_bf16.h>
 
 #include <algorithm>
 #include <cstdlib>
 
+#include "mra_async.cuh"
 #include "mra_attn_common.cuh"
 #include "mra_internal.cuh"
 #include "mra_mma.cuh"
+#include "mra_tcgen05.cuh"
 
 namespace mra {
 namespace {
@@ -51,6 +55,7 @@ struct AttnArgs {
     long long ob;
     int oh, orow;
     GradStats gs;     // backward-pass statistics (gs.lse2 == nullptr: forward only)
+    unsigned int *status;   // device status word (a bounded wait that expired)
 };
 
 constexpr int kBf16Threads = 64;
@@ -69,10 +74,13 @@ struct Bf16Smem {
     static constexpr int kTile = 32 * D;
     static constexpr size_t kKvBytes = sizeof(__nv_bfloat16) * 2 * kBf16Stages * kTile;
     static constexpr size_t kMergeBytes = partial_slot_bytes<D, __nv_bfloat16>() + sizeof(MergeSmem);
-    __nv_bfloat16 q[kTile];
-    // K/V ring; after the block loop the same bytes hold the output staging
-    // or, for split rows, the partial and the merge scratch
-    alignas(128) unsigned char kv_raw[kKvBytes > kMergeBytes ? kKvBytes : kMergeBytes];
+    // Q and the K/V ring first, 1024-byte aligned (the 128-byte swizzle of the
+    // TMA copies repeats every 1024 bytes); after the block loop the ring's
+    // bytes hold the output staging or, for split rows, the partial and the
+    // merge scratch
+    alignas(1024) __nv_bfloat16 q[kTile];
+    alignas(1024) unsigned char kv_raw[kKvBytes > kMergeBytes ? kKvBytes : kMergeBytes];
+    unsigned long long bar[kBf16Stages];   // TMA completion per buffer (Q rides on buffer 0's)
     float km[kBf16Stages][32];   // key mask per buffer
     int cols[kChunk];
     int last;
@@ -81,7 +89,8 @@ struct Bf16Smem {
 
 // One work item (block row, chunk of selected columns) on a 64-thread CTA.
 template <int D>
-__device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<D> &sh) {
+__device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<D> &sh, const CUtensorMap *map_q,
+                                          const CUtensorMap *map_k, const CUtensorMap *map_v, uint32_t &ph) {
     constexpr int kTile = 32 * D;
     __nv_bfloat16 *sQ = sh.q;
     auto sKV = reinterpret_cast<__nv_bfloat16(*)[2][kTile]>(sh.kv_raw);   // [buffer][K or V]
@@ -101,23 +110,40 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, tq = lane & 3;
 
-    load_tile_async<D, kBf16Threads>(sQ, qg + (size_t)r * kTile, tid);
+    if constexpr (D != 64) load_tile_async<D, kBf16Threads>(sQ, qg + (size_t)r * kTile, tid);
     const int ncols = it.ncols;
     // the item's column list, read once (the loads below depend on it)
     int *s_cols = sh.cols;
     for (int j = tid; j < ncols; j += kBf16Threads) s_cols[j] = a.cols[it.col_start + j];
     __syncthreads();
-    // one commit group per block (the first also holds Q); empty groups keep
-    // the count uniform
+    // the first blocks' loads: head size 64 by TMA on the buffers' mbarriers
+    // (Q on the first one), head size 32 by cp.async, one commit group per
+    // block (the first also holds Q; empty groups keep the count uniform).
+    // Rows of this head in the [B*H*N][D] tensor maps:
+    const int row0 = bh * a.N;
 #pragma unroll
     for (int st = 0; st < kBf16Stages - 1; ++st) {
         if (st < ncols) {
             const int c0 = s_cols[st];
-            load_tile_async<D, kBf16Threads>(sKV[st][0], kg + (size_t)c0 * kTile, tid);
-            load_tile_async<D, kBf16Threads>(sKV[st][1], vg + (size_t)c0 * kTile, tid);
+            if constexpr (D == 64) {
+                if (tid == 0) {
+                    // the previous item's epilogue wrote these bytes through
+                    // the generic proxy; the copies go through the async one
+                    if (st == 0) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+                    // Q rides on the first buffer's barrier
+                    const uint32_t bar = async::saddr(&sh.bar[st]);
+                    async::mbar_expect_tx(bar, (st == 0 ? 3 : 2) * kTile * 2);
+                    if (st == 0) tc::tma_load_2d(async::saddr(sQ), map_q, 0, row0 + r * 32, bar);
+                    tc::tma_load_2d(async::saddr(sKV[st][0]), map_k, 0, row0 + c0 * 32, bar);
+                    tc::tma_load_2d(async::saddr(sKV[st][1]), map_v, 0, row0 + c0 * 32, bar);
+                }
+            } else {
+                load_tile_async<D, kBf16Threads>(sKV[st][0], kg + (size_t)c0 * kTile, tid);
+                load_tile_async<D, kBf16Threads>(sKV[st][1], vg + (size_t)c0 * kTile, tid);
+            }
             if (tid < 32) sKm[st][tid] = mrow ? mrow[c0 * 32 + tid] : 1.0f;
         }
-        cp_async_commit();
+        if constexpr (D != 64) cp_async_commit();
     }
 
     float o[D / 8][4];
@@ -132,12 +158,33 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
         if (jn < ncols) {
             const int c1 = s_cols[jn];
             const int nb = jn % kBf16Stages;
-            load_tile_async<D, kBf16Threads>(sKV[nb][0], kg + (size_t)c1 * kTile, tid);
-            load_tile_async<D, kBf16Threads>(sKV[nb][1], vg + (size_t)c1 * kTile, tid);
+            if constexpr (D == 64) {
+                if (tid == 0) {
+                    const uint32_t bar = async::saddr(&sh.bar[nb]);
+                    async::mbar_expect_tx(bar, 2 * kTile * 2);
+                    tc::tma_load_2d(async::saddr(sKV[nb][0]), map_k, 0, row0 + c1 * 32, bar);
+                    tc::tma_load_2d(async::saddr(sKV[nb][1]), map_v, 0, row0 + c1 * 32, bar);
+                }
+            } else {
+                load_tile_async<D, kBf16Threads>(sKV[nb][0], kg + (size_t)c1 * kTile, tid);
+                load_tile_async<D, kBf16Threads>(sKV[nb][1], vg + (size_t)c1 * kTile, tid);
+            }
             if (tid < 32) sKm[nb][tid] = mrow ? mrow[c1 * 32 + tid] : 1.0f;
         }
-        cp_async_commit();
-        cp_async_wait<kBf16Stages - 1>();   // block j's group is complete
+        if constexpr (D == 64) {
+            // block j's copies (and, for j = 0, Q's) have landed; a wait that
+            // runs out is reported and waited once more, so that no copy is
+            // left in flight
+            const uint32_t bar = async::saddr(&sh.bar[buf]);
+            if (!async::mbar_wait(bar, (ph >> buf) & 1u)) {
+                atomicOr(a.status, kDevTimeout);
+                async::mbar_wait(bar, (ph >> buf) & 1u);
+            }
+            ph ^= 1u << buf;
+        } else {
+            cp_async_commit();
+            cp_async_wait<kBf16Stages - 1>();   // block j's group is complete
+        }
         __syncthreads();
         if (j == 0) {
 #pragma unroll
@@ -349,14 +396,23 @@ __device__ __forceinline__ void bf16_item(const AttnArgs &a, int slot, Bf16Smem<
 // of an item, so the atomic's round trip hides behind the item's work.
 template <int D>
 __global__ void __launch_bounds__(kBf16Threads, kBf16CtasPerSm)
-attn_bf16_kernel(const AttnArgs a, int total_slots, int heads) {
+attn_bf16_kernel(const AttnArgs a, int total_slots, int heads, const __grid_constant__ CUtensorMap tq,
+                 const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
     pdl_wait();
-    __shared__ __align__(128) Bf16Smem<D> sh;
+    __shared__ __align__(1024) Bf16Smem<D> sh;
+    if constexpr (D == 64) {
+        if (threadIdx.x == 0) {
+            for (int b = 0; b < kBf16Stages; ++b) async::mbar_init(async::saddr(&sh.bar[b]), 1);
+            async::mbar_init_fence();
+        }
+        __syncthreads();
+    }
+    uint32_t ph = 0;   // parity of the next completion of each buffer's barrier
     int i = blockIdx.x;
     for (int t = 0; i < total_slots; ++t) {
         if (threadIdx.x == 0) sh.next[t & 1] = (int)gridDim.x + atomicAdd(a.work_next, 1);
         const int slot = (i % heads) * a.cap + i / heads;
-        bf16_item<D>(a, slot, sh);
+        bf16_item<D>(a, slot, sh, &tq, &tk, &tv, ph);
         __syncthreads();   // shared buffers are free for the next item; next[] is visible
         i = sh.next[t & 1];
     }
@@ -515,15 +571,23 @@ cudaError_t launch_attention(const Problem &p, const Workspace &w, const void *q
     a.slot_arrive = w.slot_arrive;
     a.work_next = w.work_next;
     a.out = out;
+    a.status = w.status;
     const long long grid = (long long)p.BH * p.cap;
     if (attention_uses_tc(p, gs)) return launch_attention_tc(p, w, q, k, v, mask, out, ol, s);
     if (p.dtype == 0) {
         const long long pgrid = std::min<long long>(grid, (long long)kBf16CtasPerSm * device_sm_count());
-        if (p.D == 64)
+        // [B*H*N][64] tensor maps of Q, K and V, 32-row boxes with the
+        // 128-byte swizzle that the shared-memory tiles use (head size 64)
+        CUtensorMap tq{}, tk{}, tv{};
+        if (p.D == 64) {
+            const unsigned long long rows = (unsigned long long)p.BH * p.N;
+            if (!tc::make_map(&tq, q, rows) || !tc::make_map(&tk, k, rows) || !tc::make_map(&tv, v, rows))
+                return cudaErrorInvalidValue;
             return launch_dependent(attn_bf16_kernel<64>, dim3((unsigned)pgrid), dim3(kBf16Threads), 0, s, a,
-                                    (int)grid, p.BH);
+                                    (int)grid, p.BH, tq, tk, tv);
+        }
         return launch_dependent(attn_bf16_kernel<32>, dim3((unsigned)pgrid), dim3(kBf16Threads), 0, s, a,
-                                (int)grid, p.BH);
+                                (int)grid, p.BH, tq, tk, tv);
     }
     if (p.D == 64) return launch_dependent(attn_f32_kernel<64>, dim3((unsigned)grid), dim3(kF32Threads), 0, s, a);
     return launch_dependent(attn_f32_kernel<32>, dim3((unsigned)grid), dim3(kF32Threads), 0, s, a);
