@@ -61,9 +61,10 @@ struct AttnArgs {
 constexpr int kBf16Threads = 64;
 // K/V blocks of an item in flight: a ring of kBf16Stages buffers, the loads
 // of block j + kBf16Stages - 1 issued before block j is computed.  Two (ten
-// CTAs per SM) measured best: three stages (seven CTAs) 39.4 against 39.1 us
-// on the N=4096 map and 138 against 119 us on the N=16384 map, four stages
-// (six CTAs) 37.4 and 130 us.
+// CTAs per SM) measured best: with cp.async loads three stages (seven CTAs)
+// took 39.4 against 39.1 us on the N=4096 map and 138 against 119 us on the
+// N=16384 map, four stages (six CTAs) 37.4 and 130 us; with the TMA loads
+// three stages took 35.3 against 35.9 us and 121.8 against 106.5 us.
 constexpr int kBf16Stages = 2;
 // CTAs per SM that the ring's shared memory leaves room for (the launch
 // bound and the persistent grid)
