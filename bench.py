@@ -138,6 +138,17 @@ def traffic_for(kernel_phase: str, src_file: str, workload: int):
     return rec.get("dram_bytes_per_launch")
 
 
+def attention_source(w, impl: str = "") -> str:
+    """Source file of the attention kernel the library runs on workload w (the
+    library's dispatch rule): the tcgen05 kernel for bf16 with head size 64
+    when at least 45 % of the block map is selected, the warp-level kernel
+    otherwise; MRA_ATTN_IMPL=tc / =mma (impl) forces either."""
+    tc_attn = w.dtype == "bf16" and w.D == 64 and (
+        impl.startswith("t") or (not impl.startswith("m") and
+                                 20 * min(w.block_per_row, w.nbr) * w.nbr >= 9 * w.nbr * w.nbr))
+    return "mra_attn_tc.cu" if tc_attn else "mra_attn.cu"
+
+
 def algorithmic(w):
     """Selected-block FLOPs and compulsory bytes of one step (per workload)."""
     esz = 2 if w.dtype == "bf16" else 4
@@ -841,13 +852,7 @@ def main():
     dom_s = phases[dom]["avg_us"] * 1e-6
     esz = 2 if w.dtype == "bf16" else 4
     BH = w.B * w.H
-    # bf16 head size 64 runs the tcgen05 kernel on maps with at least 45 % of
-    # the block map selected (MRA_ATTN_IMPL=tc / =mma force either)
-    impl = os.environ.get("MRA_ATTN_IMPL", "")
-    tc_attn = w.dtype == "bf16" and w.D == 64 and (
-        impl.startswith("t") or (not impl.startswith("m") and
-                                 20 * min(w.block_per_row, w.nbr) * w.nbr >= 9 * w.nbr * w.nbr))
-    kernel_src = {"attention": "mra_attn_tc.cu" if tc_attn else "mra_attn.cu", "pool": "mra_pool.cu",
+    kernel_src = {"attention": attention_source(w, os.environ.get("MRA_ATTN_IMPL", "")), "pool": "mra_pool.cu",
                   "lowres_keys": "mra_lowres.cu", "lowres_pv": "mra_lowres.cu", "select": "mra_select.cu",
                   "lowres_select": "mra_lowres_select.cu", "group_plan": "mra_group_plan.cu"}
     if dom == "attention":
