@@ -46,3 +46,37 @@ def test_attention_source_follows_the_dispatch_rule_and_the_traffic_records():
         if key.startswith("_") or "attention" not in entry:
             continue
         assert entry["attention"]["source"] == bench.attention_source(WORKLOADS[int(key)]), key
+
+
+def test_cuda_arm_line_from_a_stubbed_run(monkeypatch, capsys):
+    """The CUDA arm's JSON line, assembled on the CPU from a stubbed device
+    run of the N=4096 workload: every key the benchmark contract asks for,
+    the attention phase as the roofline kernel with the recorded DRAM
+    traffic, and the throughput computed from the stubbed step time."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    def fake_run(args, w, world, rank, local):
+        return {"ms": 0.0625, "e2e_ms": 1.0, "eager_ms": 0.19, "h2d": 37748736, "d2h": 12582912,
+                "phases": {"pool": (1, 0.0124), "lowres_select": (1, 0.0214), "attention": (1, 0.0359)},
+                "status": 0, "launches_per_step": 3,
+                "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 4}}
+
+    monkeypatch.setattr(bench, "run_cuda", fake_run)
+    monkeypatch.delenv("MRA_ATTN_IMPL", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--no-cpu-baseline"])
+    bench.main()
+    lines = [line for line in capsys.readouterr().out.splitlines() if line.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches",
+                "clocks"):
+        assert key in d, key
+    assert abs(d["value"] - 2 * 4096 / 0.0625e-3) < 1e-3 * d["value"]
+    assert d["roofline"]["kernel"] == "attention" and d["roofline"]["bound"] == "hbm"
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        recorded = json.load(f)["4"]["attention"]["dram_bytes_per_launch"]
+    assert d["roofline"]["traffic"] == recorded
+    assert d["gpu_launches"] == 3 * d["steps"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 37748736
